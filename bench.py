@@ -1,0 +1,400 @@
+"""Benchmark of the INT4 weight-only path on B200.
+
+One step is one pass of the whole path over one weight matrix
+W [28672, 8192] (bf16, heavy-tailed Student-t(3) * 0.02 with 1% all-zero
+groups, group 128):
+
+  quantize  W -> packed [28672, 4096] uint8 + scales [28672, 64] fp16
+  unpack    packed -> int8 [28672, 8192]
+  decode    y = x @ dequant(W)^T with x [1, 8192] bf16         (M = 1)
+  prefill   y = x @ dequant(W)^T with x [8192, 8192] bf16      (M = 8192)
+
+Every kernel is timed with CUDA events on the stream it runs on, and L2 is
+flushed (a 256 MiB write) before each kernel, outside its events.  The
+headline ``value`` is the decode throughput on packed-weight bytes
+(N * ceil(K/2) / time); the other rows are reported under ``rows``.
+
+Launch: ``python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]``
+(under torchrun for N > 1: every rank runs the same step on its own GPU,
+"replicas only"; value is the sum over ranks with the max time over ranks).
+``--impl reference`` times the CPU oracle on a bounded sample on this host.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+N_W, K_W, GROUP = 28672, 8192, 128
+M_DECODE, M_PREFILL = 1, 8192
+METRIC = "int4_matmul decode GB/s & prefill TFLOP/s vs B200 roofline; quantize GB/s"
+WORKLOAD = "W[28672,8192] bf16 g128: quantize+unpack, decode M=1, prefill M=8192"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def _row_units():
+    Kp = (K_W + 1) // 2
+    G = -(-K_W // GROUP)
+    packed = N_W * Kp
+    scales = 2 * N_W * G
+    return {
+        "quantize": {"bytes": N_W * K_W * 2 + packed + scales, "bound": "hbm"},
+        "unpack": {"bytes": packed + N_W * K_W, "bound": "hbm"},
+        "decode": {"bytes": packed, "bytes_total": packed + scales + M_DECODE * K_W * 2 + 4 * M_DECODE * N_W,
+                   "bound": "hbm"},
+        "prefill": {"flops": 2 * M_PREFILL * N_W * K_W, "bound": "tensor"},
+    }
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    return world, rank, local
+
+
+def _max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_baseline(rows: int = 8192):
+    """Time the CPU oracle on bounded row samples of the same workload."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from workloads import make_activations, make_weights
+
+    threads = torch.get_num_threads()
+    w = make_weights(rows, K_W, seed=5, device="cpu", dtype=torch.bfloat16, dist="student_t3",
+                     zero_group_frac=0.01, group=GROUP).float().numpy()
+    out = {}
+    t0 = time.perf_counter()
+    packed, scales, K = oracle.quantize_int4(w, GROUP)
+    tq = time.perf_counter() - t0
+    out["quantize_gbs"] = (rows * K_W * 2 + packed.nbytes + scales.nbytes) / tq / 1e9
+    t0 = time.perf_counter()
+    oracle.unpack_int4(packed, K)
+    tu = time.perf_counter() - t0
+    out["unpack_gbs"] = (packed.nbytes + rows * K_W) / tu / 1e9
+    x1 = make_activations(1, K_W, seed=11, device="cpu").float().numpy()
+    t0 = time.perf_counter()
+    oracle.int4_matmul_ref(x1, packed, scales, K, GROUP)
+    td = time.perf_counter() - t0
+    out["decode_gbs"] = packed.nbytes / td / 1e9
+    xm = make_activations(64, K_W, seed=12, device="cpu").float().numpy()
+    t0 = time.perf_counter()
+    oracle.int4_matmul_ref(xm, packed, scales, K, GROUP)
+    tp = time.perf_counter() - t0
+    out["prefill_tflops"] = 2 * 64 * rows * K_W / tp / 1e12
+    out["seconds"] = tq + tu + td + tp
+    out["threads"] = threads
+    out["sample"] = (f"{rows} rows of W [{N_W},{K_W}] bf16 g{GROUP}: quantize, unpack, decode M=1, "
+                     f"prefill M=64 slice (fp64 BLAS); throughput per the full-size byte/flop counts")
+    return out
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed on this host's cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    times = []
+    res = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        res = cpu_baseline(rows=4096)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": res["decode_gbs"], "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD + " (row sample)"},
+        "rows": {k: res[k] for k in ("quantize_gbs", "unpack_gbs", "decode_gbs", "prefill_tflops")},
+        "cpu_baseline": {"value": res["decode_gbs"], "unit": "GB/s", "cores": res["threads"],
+                         "kind": "oracle", "sample": res["sample"]},
+        "e2e": {"value": res["decode_gbs"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+    from workloads import make_activations, make_weights
+
+    world, rank, local = _dist_setup(args)
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    q4.lib()
+    stream = torch.cuda.current_stream(dev)
+
+    w = make_weights(N_W, K_W, seed=5, device=dev, dtype=torch.bfloat16, dist="student_t3",
+                     zero_group_frac=0.01, group=GROUP)
+    xd = make_activations(M_DECODE, K_W, seed=7, device=dev, dtype=torch.bfloat16)
+    xp = make_activations(M_PREFILL, K_W, seed=8, device=dev, dtype=torch.bfloat16)
+    packed = torch.empty((N_W, K_W // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N_W, K_W // GROUP), dtype=torch.float16, device=dev)
+    unpacked = torch.empty((N_W, K_W), dtype=torch.int8, device=dev)
+    yd = torch.empty((M_DECODE, N_W), dtype=torch.float32, device=dev)
+    yp = torch.empty((M_PREFILL, N_W), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = q4.lib()
+    sp = lambda: stream.cuda_stream  # noqa: E731
+
+    def call(rc):
+        if rc != 0:
+            raise RuntimeError(f"INT4 library error {rc}: {L.int4_last_error()}")
+
+    kernels = {
+        "quantize": lambda: call(L.int4_quantize(w.data_ptr(), 1, N_W, K_W, GROUP, packed.data_ptr(),
+                                                 scales.data_ptr(), sp())),
+        "unpack": lambda: call(L.int4_unpack(packed.data_ptr(), K_W, N_W, unpacked.data_ptr(), sp())),
+        "decode": lambda: call(L.int4_matmul(xd.data_ptr(), 1, packed.data_ptr(), scales.data_ptr(),
+                                             K_W, GROUP, M_DECODE, N_W, yd.data_ptr(), sp())),
+        "prefill": lambda: call(L.int4_matmul(xp.data_ptr(), 1, packed.data_ptr(), scales.data_ptr(),
+                                              K_W, GROUP, M_PREFILL, N_W, yp.data_ptr(), sp())),
+    }
+    order = ["quantize", "unpack", "decode", "prefill"]
+    launches_per_step = {
+        "quantize": 1, "unpack": 1, "decode": 1,
+        "prefill": 1,
+    }
+
+    def step(events=None):
+        for name in order:
+            flush.fill_(1)
+            if events is not None:
+                events[name][0].record(stream)
+            kernels[name]()
+            if events is not None:
+                events[name][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    ev = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for n in order} for _ in range(args.steps)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    _barrier(world)
+    clocks = clk.summary()
+    per = {n: statistics.mean(e[n][0].elapsed_time(e[n][1]) for e in ev) for n in order}
+    per = {n: _max_over_ranks(v, world) for n, v in per.items()}
+    wall_ms = _max_over_ranks(t_start.elapsed_time(t_end), world)
+    units = _row_units()
+    peaks = _peaks()
+    rows = {}
+    for n in order:
+        t = per[n] * 1e-3
+        u = units[n]
+        if u["bound"] == "hbm":
+            ach = u["bytes"] / t / 1e9
+            rows[n] = {"ms": per[n], "GB/s": ach * world, "frac": ach / peaks["hbm_gbs"]}
+            if "bytes_total" in u:
+                rows[n]["GB/s_total_bytes"] = u["bytes_total"] / t / 1e9 * world
+        else:
+            ach = u["flops"] / t / 1e12
+            rows[n] = {"ms": per[n], "TFLOP/s": ach * world, "frac": ach / peaks["bf16_tflops"]}
+        rows[n]["path"] = (q4.matmul_select(torch.bfloat16, K_W, GROUP, M_DECODE if n == "decode" else M_PREFILL, N_W)
+                           if n in ("decode", "prefill") else None)
+    dom = max(order, key=lambda n: per[n])
+    du = units[dom]
+    if du["bound"] == "hbm":
+        roof = {"kernel": dom, "bound": "hbm", "achieved": du["bytes"] / (per[dom] * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"kernel": dom, "bound": "tensor", "achieved": du["flops"] / (per[dom] * 1e-3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = peaks["source"] + (" bf16 burst" if roof["bound"] == "tensor" else " copy")
+    roof["traffic"] = None
+
+    # End to end through the public Python API: pinned host x in, y out.
+    e2e = None
+    if not args.no_e2e:
+        import dequant_gemm_int4_b200 as api
+        xh = xd.cpu().pin_memory()
+        yh = torch.empty((M_DECODE, N_W), dtype=torch.float32).pin_memory()
+        for _ in range(args.warmup):
+            y = api.int4_matmul(xh.to(dev, non_blocking=True), packed, scales, K_W, GROUP)
+            yh.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0.record(stream)
+            y = api.int4_matmul(xh.to(dev, non_blocking=True), packed, scales, K_W, GROUP)
+            yh.copy_(y, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        t = _max_over_ranks(tot / args.steps, world) * 1e-3
+        e2e = {"value": units["decode"]["bytes"] / t / 1e9 * world, "unit": "GB/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": yh.numel() * yh.element_size(),
+               "scope": "decode row via the Python API: H2D of x, int4_matmul, D2H of y"}
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline()
+        cpu = {"value": cb["decode_gbs"], "unit": "GB/s", "cores": cb["threads"], "kind": "oracle",
+               "sample": cb["sample"], "rows": {k: cb[k] for k in ("quantize_gbs", "unpack_gbs",
+                                                                    "decode_gbs", "prefill_tflops")}}
+    line = {
+        "metric": METRIC, "value": rows["decode"]["GB/s"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(per.values()), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "l2": "flushed (256 MiB write) before every kernel",
+                   "parallelism": f"replicas x{world}"},
+        "rows": rows, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": args.steps * sum(launches_per_step.values()),
+        "wall_ms_timed_region": wall_ms,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

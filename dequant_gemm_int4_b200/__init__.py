@@ -1,0 +1,188 @@
+"""B200 (sm_100a) INT4 weight-only quantization and dequantizing matmul.
+
+Thin Python binding over the C-ABI library ``libint4.so`` (declared in
+``include/int4.h``).  It only marshals arguments: it allocates the output
+tensors with PyTorch on the input's CUDA device, passes raw device pointers
+and the current CUDA stream, and raises on a non-zero status.  Every step of
+the computation runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback, and a missing library is an error.
+
+The three functions keep the names, argument order and layouts of the page
+"Implement INT4 group quantization, nibble packing and a dequantizing
+matmul" (problem statement):
+
+* ``quantize_int4(w, group=128) -> (packed, scales, K)``
+* ``unpack_int4(packed, K) -> int8 [N, K]``
+* ``int4_matmul(x, packed, scales, K, group=128) -> float32 [M, N]``
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "quantize_int4", "unpack_int4", "int4_matmul", "matmul_select", "device_status",
+    "selftest_wait_timeout", "lib", "library_path", "Int4Error",
+    "PATH_AUTO", "PATH_SIMT", "PATH_DECODE", "PATH_PREFILL",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libint4.so")
+
+OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
+DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
+PATH_AUTO, PATH_SIMT, PATH_DECODE, PATH_PREFILL = 0, 1, 2, 3
+
+_DTYPE_CODE = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Int4Error(RuntimeError):
+    """A non-zero status from the INT4 library."""
+
+    def __init__(self, code: int, message: str):
+        super().__init__(f"INT4 library error {code}: {message}")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libint4.so once and declare its C signatures."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m dequant_gemm_int4_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64, u32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
+        L.int4_quantize.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp]
+        L.int4_unpack.argtypes = [vp, i64, i64, vp, vp]
+        L.int4_matmul.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
+        L.int4_matmul_path.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, i32, vp]
+        L.int4_matmul_select.argtypes = [i32, i64, i32, i64, i64]
+        L.int4_device_status.argtypes = [vp]
+        L.int4_selftest_wait_timeout.argtypes = [u32, vp]
+        L.int4_last_error.restype = ctypes.c_char_p
+        L.int4_last_error.argtypes = []
+        L.int4_version.argtypes = []
+        for name in ("int4_quantize", "int4_unpack", "int4_matmul", "int4_matmul_path",
+                     "int4_matmul_select", "int4_device_status", "int4_selftest_wait_timeout",
+                     "int4_version"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+        return L
+
+
+def _check(rc: int) -> None:
+    if rc != OK:
+        msg = lib().int4_last_error()
+        raise Int4Error(rc, msg.decode() if msg else "")
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major, no padding)")
+
+
+def quantize_int4(w: torch.Tensor, group: int = 128):
+    """Quantize w [N, K] (fp32/bf16/fp16) -> (packed uint8 [N, ceil(K/2)], scales fp16 [N, G], K)."""
+    _need_cuda("w", w)
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    if w.dtype not in _DTYPE_CODE:
+        raise TypeError("w must be float32, bfloat16 or float16")
+    N, K = w.shape
+    G = -(-K // group) if group >= 1 else 0
+    packed = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((N, max(G, 0)), dtype=torch.float16, device=w.device)
+    with torch.cuda.device(w.device):
+        _check(lib().int4_quantize(w.data_ptr(), _DTYPE_CODE[w.dtype], N, K, int(group),
+                                   packed.data_ptr(), scales.data_ptr(), _stream(w)))
+    return packed, scales, K
+
+
+def unpack_int4(packed: torch.Tensor, K: int) -> torch.Tensor:
+    """Unpack packed [N, ceil(K/2)] -> sign-extended int8 [N, K]."""
+    _need_cuda("packed", packed)
+    if packed.dtype != torch.uint8 or packed.dim() != 2 or packed.shape[1] != (K + 1) // 2:
+        raise ValueError("packed must be uint8 [N, ceil(K/2)]")
+    N = packed.shape[0]
+    out = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    with torch.cuda.device(packed.device):
+        _check(lib().int4_unpack(packed.data_ptr(), K, N, out.data_ptr(), _stream(packed)))
+    return out
+
+
+def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: int,
+                group: int = 128, *, path: int = PATH_AUTO, out: torch.Tensor | None = None):
+    """y = x @ dequantize(W).T as float32 [M, N]; x is [M, K] fp32/bf16/fp16."""
+    _need_cuda("x", x)
+    _need_cuda("packed", packed)
+    _need_cuda("scales", scales)
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M, K]")
+    if x.dtype not in _DTYPE_CODE:
+        raise TypeError("x must be float32, bfloat16 or float16")
+    N = packed.shape[0]
+    G = -(-K // group)
+    if packed.dtype != torch.uint8 or tuple(packed.shape) != (N, (K + 1) // 2):
+        raise ValueError("packed must be uint8 [N, ceil(K/2)]")
+    if scales.dtype != torch.float16 or tuple(scales.shape) != (N, G):
+        raise ValueError("scales must be float16 [N, ceil(K/group)]")
+    M = x.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    else:
+        _need_cuda("out", out)
+        if out.dtype != torch.float32 or tuple(out.shape) != (M, N):
+            raise ValueError("out must be float32 [M, N]")
+    with torch.cuda.device(x.device):
+        _check(lib().int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
+                                      scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
+                                      int(path), _stream(x)))
+    return out
+
+
+def matmul_select(x_dtype: torch.dtype, K: int, group: int, M: int, N: int) -> int:
+    """The kernel path int4_matmul takes for this problem (PATH_SIMT/DECODE/PREFILL)."""
+    rc = lib().int4_matmul_select(_DTYPE_CODE[x_dtype], K, group, M, N)
+    if rc < 0:
+        _check(-rc)
+    return rc
+
+
+def device_status(device=None) -> int:
+    """Synchronize the current stream and read/clear the device status word.
+
+    Returns OK (0) or ERR_TIMEOUT (5); raises on a CUDA error."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        rc = lib().int4_device_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
+    if rc not in (OK, ERR_TIMEOUT):
+        _check(rc)
+    return rc
+
+
+def selftest_wait_timeout(spins: int, device=None) -> None:
+    """Launch the bounded-wait self-test kernel (its wait can never be satisfied)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib().int4_selftest_wait_timeout(
+            int(spins), ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))

@@ -1,0 +1,47 @@
+// Internal launcher interface between the C-ABI layer (int4_abi.cu) and the
+// kernels.  Each launcher assumes its arguments were validated by the ABI
+// layer and returns a cudaError_t from the launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace int4lib {
+
+enum class DType : int { F32 = 0, BF16 = 1, F16 = 2 };
+
+inline int dtype_size(DType t) { return t == DType::F32 ? 4 : 2; }
+
+// Device-side status word: kernels whose bounded waits give up set a bit.
+constexpr uint32_t kStatusTimeout = 1u;
+cudaError_t read_and_clear_status(uint32_t* out, cudaStream_t stream);
+// Device address of the status word on the current device (nullptr on error).
+uint32_t* status_word();
+cudaError_t launch_wait_timeout_selftest(uint32_t spins, cudaStream_t stream);
+
+// quantize.cu
+cudaError_t launch_quantize(const void* w, DType wt, int64_t N, int64_t K, int group,
+                            uint8_t* packed, uint16_t* scales, cudaStream_t stream);
+// unpack.cu
+cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out,
+                          cudaStream_t stream);
+// matmul_simt.cu
+cudaError_t launch_matmul_simt(const void* x, DType xt, const uint8_t* packed,
+                               const uint16_t* scales, int64_t K, int group, int64_t M,
+                               int64_t N, float* y, cudaStream_t stream);
+// matmul_decode.cu
+bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
+                      const uint8_t* packed);
+cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
+                                 const uint16_t* scales, int64_t K, int group, int64_t M,
+                                 int64_t N, float* y, cudaStream_t stream);
+// matmul_prefill.cu
+bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
+                       const uint8_t* packed);
+cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
+                                  const uint16_t* scales, int64_t K, int group, int64_t M,
+                                  int64_t N, float* y, cudaStream_t stream);
+
+int num_sms();  // SM count of the current device (cached per device)
+
+}  // namespace int4lib

@@ -1,0 +1,254 @@
+// Group-wise INT4 quantization and nibble packing (sm_100a).
+//
+// Follows the quantize_int4 function of the page "Implement INT4 group
+// quantization, nibble packing and a dequantizing matmul" (problem
+// statement): per row and per K-group, scale = absmax / 7 stored as fp16,
+// q = round(w / scale) clamped to [-8, 7], two's-complement nibbles with
+// element 2j in the low nibble of byte j, a zero pad nibble for odd K and
+// scale 0 for an all-zero group.  Rounding convention: fp32 IEEE division
+// absmax / 7, then round-to-nearest-even to fp16; q = rint_half_even of the
+// IEEE fp32 quotient w / float(scale).
+//
+// HBM-bound: every weight is read once (fp32/bf16/fp16) and the packed codes
+// and scales written once.  The fast kernel gives each warp a window of 32
+// consecutive 8-element chunks of one row (one 16-byte load per lane for
+// 16-bit weights), reduces the group absmax with warp shuffles across the
+// group/8 lanes of each group, and stores 4 packed bytes per lane.
+#include "common.cuh"
+#include "internal.h"
+
+namespace int4lib {
+
+namespace {
+
+struct ScaleInfo {
+  uint32_t bits;  // fp16 bit pattern of the scale
+  float sf;       // the scale widened to fp32
+  float r;        // fp32(1 / sf), or 0 when sf is 0 (or +inf)
+};
+
+__device__ __forceinline__ ScaleInfo scale_from_bits(uint32_t bits) {
+  ScaleInfo si;
+  si.bits = bits;
+  si.sf = f16_bits_to_float(bits);
+  si.r = (si.sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, si.sf);
+  return si;
+}
+
+// s = fp16_RNE(fp32(m) / 7), with the IEEE-exact division.
+__device__ __forceinline__ ScaleInfo scale_from_absmax(float m) {
+  const __half h = __float2half_rn(__fdiv_rn(m, 7.0f));
+  return scale_from_bits(__half_as_ushort(h));
+}
+
+// The 4-bit code of v: clamp(rint(fp32(v / sf)), -8, 7), 0 when sf == 0.
+//
+// The quotient is first approximated as t = v * r with r = fp32(1/sf).  With
+// x the exact quotient, |t - x| <= |x| * 2^-23 (two roundings), and the
+// correctly rounded fp32(x) lies within another half ulp of x, so for
+// |x| < 16 the two differ from t by less than 2^-19.  rint(fp32(x)) can only
+// differ from rint(t) if a half-integer lies within that distance of t; t is
+// then recomputed with the IEEE division.  Half-integers beyond +-7.5 never
+// change the clamped result.  Hence the result equals the IEEE-division
+// result for every finite v; the slow path runs for about 1 element in 10^5.
+__device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
+  float t = v * si.r;
+  float rt = rintf(t);
+  if (fabsf(t - rt) >= 0.5f - 0x1p-18f && si.sf != 0.0f) {
+    t = __fdiv_rn(v, si.sf);
+    rt = rintf(t);
+  }
+  rt = fminf(fmaxf(rt, -8.0f), 7.0f);
+  return static_cast<uint32_t>(static_cast<int>(rt)) & 0xFu;
+}
+
+// Load 8 consecutive elements starting at p (16-byte aligned) as fp32.
+template <typename T>
+struct Load8;
+template <>
+struct Load8<float> {
+  __device__ __forceinline__ static void run(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+template <>
+struct Load8<__nv_bfloat16> {
+  __device__ __forceinline__ static void run(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <>
+struct Load8<__half> {
+  __device__ __forceinline__ static void run(const __half* p, float (&v)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = f16_bits_to_float(w[i] & 0xFFFFu);
+      v[2 * i + 1] = f16_bits_to_float(w[i] >> 16);
+    }
+  }
+};
+
+constexpr int kUnroll = 2;  // windows in flight per warp
+
+// Fast path: K % 8 == 0, group = 8 * LPG with LPG a power of two <= 32,
+// w 16-byte aligned, packed 4-byte aligned.  One warp window = 32 chunks of 8
+// elements of one row; windows are numbered row-major over (row, window).
+template <typename T, int LPG>
+__global__ void __launch_bounds__(256) quantize_aligned_kernel(
+    const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
+    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t chunks_per_row = K >> 3;
+  const int64_t Kp = K >> 1;
+
+  for (int64_t base = warp0; base < total_windows; base += nwarps * kUnroll) {
+    float v[kUnroll][8];
+    int64_t row[kUnroll], chunk[kUnroll];
+    bool valid[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t wi = base + u * nwarps;
+      row[u] = wi / windows_per_row;
+      chunk[u] = (wi - row[u] * windows_per_row) * 32 + lane;
+      valid[u] = (wi < total_windows) && (chunk[u] < chunks_per_row);
+      if (valid[u]) {
+        Load8<T>::run(w + row[u] * K + chunk[u] * 8, v[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[u][i]));
+#pragma unroll
+      for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const ScaleInfo si = scale_from_absmax(m);
+      if (valid[u]) {
+        if ((lane & (LPG - 1)) == 0)
+          scales[row[u] * G + chunk[u] / LPG] = static_cast<uint16_t>(si.bits);
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= code_of(v[u][i], si) << (4 * i);
+        *reinterpret_cast<uint32_t*>(packed + row[u] * Kp + chunk[u] * 4) = word;
+      }
+    }
+  }
+}
+
+// General path, step 1: one thread per (row, group) computes the scale.
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_scales_general_kernel(
+    const T* __restrict__ w, int64_t N, int64_t K, int group, int G, uint16_t* __restrict__ scales) {
+  const int64_t total = N * G;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx / G;
+    const int64_t g = idx - n * G;
+    const int64_t k0 = g * group;
+    const int64_t k1 = (k0 + group < K) ? k0 + group : K;
+    float m = 0.0f;
+    for (int64_t k = k0; k < k1; ++k) m = fmaxf(m, fabsf(Elem<T>::load(w + n * K + k)));
+    scales[idx] = static_cast<uint16_t>(scale_from_absmax(m).bits);
+  }
+}
+
+// General path, step 2: one thread per packed byte, using the stored scales.
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_pack_general_kernel(
+    const T* __restrict__ w, int64_t N, int64_t K, int group, int G,
+    const uint16_t* __restrict__ scales, uint8_t* __restrict__ packed) {
+  const int64_t Kp = (K + 1) >> 1;
+  const int64_t total = N * Kp;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx / Kp;
+    const int64_t k = 2 * (idx - n * Kp);
+    const ScaleInfo s0 = scale_from_bits(scales[n * G + k / group]);
+    uint32_t byte = code_of(Elem<T>::load(w + n * K + k), s0);
+    if (k + 1 < K) {
+      const ScaleInfo s1 = scale_from_bits(scales[n * G + (k + 1) / group]);
+      byte |= code_of(Elem<T>::load(w + n * K + k + 1), s1) << 4;
+    }
+    packed[idx] = static_cast<uint8_t>(byte);
+  }
+}
+
+int grid_for(int64_t work_items, int per_block, int max_blocks_per_sm) {
+  const int64_t want = (work_items + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * max_blocks_per_sm;
+  const int64_t g = want < cap ? want : cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+template <typename T>
+cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* packed,
+                         uint16_t* scales, cudaStream_t stream) {
+  const int G = static_cast<int>((K + group - 1) / group);
+  const bool aligned = (K % 8 == 0) && (reinterpret_cast<uintptr_t>(w) % 16 == 0) &&
+                       (reinterpret_cast<uintptr_t>(packed) % 4 == 0);
+  const int lpg = group / 8;
+  const bool pow2_group = (group % 8 == 0) && lpg >= 1 && lpg <= 32 && (lpg & (lpg - 1)) == 0;
+  if (aligned && pow2_group) {
+    const int64_t wpr = (K / 8 + 31) / 32;
+    const int64_t total = N * wpr;
+    const int grid = grid_for(total, 8 * kUnroll, 16);
+    switch (lpg) {
+#define INT4_Q_CASE(L)                                                                       \
+  case L:                                                                                    \
+    quantize_aligned_kernel<T, L><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed, scales); \
+    break;
+      INT4_Q_CASE(1)
+      INT4_Q_CASE(2)
+      INT4_Q_CASE(4)
+      INT4_Q_CASE(8)
+      INT4_Q_CASE(16)
+      INT4_Q_CASE(32)
+#undef INT4_Q_CASE
+      default:
+        break;
+    }
+    return cudaGetLastError();
+  }
+  quantize_scales_general_kernel<T><<<grid_for(N * G, 256, 16), 256, 0, stream>>>(w, N, K, group, G,
+                                                                                    scales);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t Kp = (K + 1) / 2;
+  quantize_pack_general_kernel<T><<<grid_for(N * Kp, 256, 16), 256, 0, stream>>>(w, N, K, group, G,
+                                                                                   scales, packed);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* w, DType wt, int64_t N, int64_t K, int group,
+                            uint8_t* packed, uint16_t* scales, cudaStream_t stream) {
+  switch (wt) {
+    case DType::F32:
+      return launch_typed(static_cast<const float*>(w), N, K, group, packed, scales, stream);
+    case DType::BF16:
+      return launch_typed(static_cast<const __nv_bfloat16*>(w), N, K, group, packed, scales,
+                          stream);
+    case DType::F16:
+      return launch_typed(static_cast<const __half*>(w), N, K, group, packed, scales, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace int4lib

@@ -1,0 +1,184 @@
+/*
+ * int4.h - C ABI of the B200 (sm_100a) INT4 weight-only quantization library.
+ *
+ * Symmetric group-wise INT4 quantization with two's-complement nibble packing
+ * and the weight-only dequantizing matmul, as stated by the web page
+ * "Implement INT4 group quantization, nibble packing and a dequantizing
+ * matmul" (inferenceinterviews.com drill), problem statement: three functions
+ * quantize_int4(w, group) -> (packed, scales, K), unpack_int4(packed, K) and
+ * int4_matmul(x, packed, scales, K, group).  The entry points below keep that
+ * argument order: inputs in the page's order, then derived shapes, then the
+ * outputs, then the CUDA stream.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller.  The
+ *   library allocates no device or host memory and keeps no reference to the
+ *   buffers after the call returns.
+ * - All tensors are dense and row-major with no padding between rows:
+ *     w       [N, K]         fp32, bf16 or fp16 (w_dtype)
+ *     packed  [N, ceil(K/2)] uint8; row stride ceil(K/2) bytes
+ *     scales  [N, G]         fp16 bit patterns, G = ceil(K / group)
+ *     unpack  [N, K]         int8
+ *     x       [M, K]         fp32, bf16 or fp16 (x_dtype)
+ *     y       [M, N]         fp32
+ * - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL means
+ *   the legacy default stream), like a kernel launch.  A zero return means
+ *   the work was launched, not that it has finished.
+ * - Buffers must not overlap, except that nothing is written to an input.
+ * - Return value: INT4_OK (0) or one of the INT4_ERR_* codes.  Arguments are
+ *   validated on the host before anything is launched; on a non-zero return
+ *   nothing was launched and no output was touched, except INT4_ERR_CUDA,
+ *   which reports a launch failure (its message is in int4_last_error()).
+ * - Thread safety: entry points may be called from several host threads; the
+ *   last-error message is kept per host thread.
+ * - Sizes: N, M >= 1, K >= 1, group >= 1.  (N or M == 0, an empty problem,
+ *   returns INT4_OK and launches nothing.)  N * K, M * K and M * N must each
+ *   be below 2^62.
+ */
+#ifndef INT4_B200_H
+#define INT4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define INT4_OK             0
+#define INT4_ERR_ARG        1  /* null pointer, negative size, group < 1, size overflow */
+#define INT4_ERR_DTYPE      2  /* unknown dtype code */
+#define INT4_ERR_ALIGN      3  /* a pointer not aligned to its element size */
+#define INT4_ERR_CUDA       4  /* a CUDA launch or runtime call failed */
+#define INT4_ERR_TIMEOUT    5  /* a bounded device-side wait gave up (see int4_device_status) */
+#define INT4_ERR_UNSUPPORTED 6 /* a forced kernel path cannot run this shape */
+
+/* Element type codes for w_dtype and x_dtype. */
+#define INT4_DTYPE_F32   0
+#define INT4_DTYPE_BF16  1
+#define INT4_DTYPE_F16   2
+
+/*
+ * int4_quantize - group absmax, fp16 scale, INT4 codes and nibble packing.
+ *
+ * Page: the drill's quantize_int4 ("scale = absmax of the group / 7", "q =
+ * round(w / scale) clipped to [-8, 7], as a two's-complement nibble; element
+ * 2j in the low nibble of byte j (an odd K pads one zero nibble; a group of
+ * zeros gets scale 0)"), with the per-row blocks along K of the page
+ * "Building a pure-Python INT4 transformer weight quantizer with block-wise
+ * per-channel scaling", sections 3 and 4.
+ *
+ * For row n and group g (columns [g*group, min((g+1)*group, K))):
+ *   m      = max |w[n, k]| over the group's real columns (exact)
+ *   s      = fp16_RNE( fp32(m) / 7 )   (IEEE fp32 division, then RNE to fp16)
+ *   q[n,k] = clamp( rint_half_even( fp32(w[n,k]) / fp32(s) ), -8, 7 )
+ *            (IEEE fp32 division), and q = 0 for the whole group when s == 0
+ *   packed[n, j] = (q[n,2j] & 0xF) | ((q[n,2j+1] & 0xF) << 4), q[n,K] := 0
+ *   scales[n, g] = bit pattern of s
+ * The outputs are bit-exact functions of w under this convention.
+ * Precondition: w is finite (NaN/Inf input gives unspecified codes).
+ *
+ * w       [N, K] device buffer of w_dtype; alignment: its element size.
+ * w_dtype INT4_DTYPE_F32 / _BF16 / _F16.
+ * packed  [N, ceil(K/2)] device output; any alignment.
+ * scales  [N, ceil(K/group)] device output (fp16 bits); 2-byte aligned.
+ */
+int int4_quantize(const void* w, int32_t w_dtype, int64_t N, int64_t K, int32_t group,
+                  uint8_t* packed, uint16_t* scales, void* stream);
+
+/*
+ * int4_unpack - nibbles to sign-extended int8.
+ *
+ * Page: the drill's unpack_int4(packed, K) -> int8 [N, K], sign-extended
+ * (its hidden suite names "sign extension of -8").  out[n, k] is the low
+ * nibble of packed[n, k/2] for even k and the high nibble for odd k, read as
+ * a 4-bit two's-complement value in [-8, 7].  The pad nibble of an odd K is
+ * not read.  Bit-exact.
+ *
+ * packed [N, ceil(K/2)] device input; any alignment.
+ * out    [N, K] int8 device output; any alignment.
+ */
+int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* stream);
+
+/*
+ * int4_matmul - weight-only dequantizing matmul y = x @ dequantize(W)^T.
+ *
+ * Page: the drill's int4_matmul(x, packed, scales, K, group) -> float32
+ * [M, N]: "computed one group at a time: multiply x by the group's integer
+ * weights first, then apply the group's scale to each output column".
+ *   y[m, n] = sum_g s[n, g] * ( sum_{k in g} x[m, k] * q[n, k] )
+ * Integer weights enter the arithmetic exactly (-8..7 is exact in bf16, fp16
+ * and fp32); group partial sums are accumulated in fp32 (fp64 across groups
+ * for fp32 x); the group's scale is applied to each partial before it joins
+ * the running sum.  Accuracy: |y - y_exact| <= c * sum_k |x[m,k]| |w_hat[n,k]|
+ * with c = 1e-5 for fp32 x and c = 4e-3 for bf16 / fp16 x.  Summation order
+ * differs between kernels; results are deterministic for a given shape,
+ * dtype and device.
+ *
+ * x       [M, K] device input of x_dtype; alignment: its element size.
+ * packed  [N, ceil(K/2)] device input; any alignment.
+ * scales  [N, ceil(K/group)] fp16 bits; 2-byte aligned.
+ * y       [M, N] fp32 device output; 4-byte aligned.
+ *
+ * Kernel choice (automatic): bf16/fp16 x with M <= 16 takes the streaming
+ * decode kernel; bf16/fp16 x with larger M takes the tcgen05 tensor-core
+ * kernel; fp32 x, and shapes the fast kernels do not cover (K or group not a
+ * multiple of 32, unaligned rows), take the general CUDA-core kernel.
+ */
+int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* stream);
+
+/* Kernel selectors for int4_matmul_path. */
+#define INT4_PATH_AUTO     0
+#define INT4_PATH_SIMT     1  /* general CUDA-core kernel (any shape, any dtype) */
+#define INT4_PATH_DECODE   2  /* skinny decode kernel (bf16/fp16 x, M <= 16) */
+#define INT4_PATH_PREFILL  3  /* tcgen05 tensor-core kernel (bf16/fp16 x) */
+
+/*
+ * int4_matmul_path - int4_matmul with the kernel chosen by the caller.
+ *
+ * Same contract as int4_matmul; `path` is one of INT4_PATH_*.  A forced path
+ * that cannot run the given shape or dtype returns INT4_ERR_UNSUPPORTED and
+ * launches nothing.  Used to test every kernel on every shape it accepts.
+ */
+int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                     int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
+                     void* stream);
+
+/*
+ * int4_matmul_select - the path int4_matmul would take for this problem
+ * (one of INT4_PATH_SIMT / _DECODE / _PREFILL), or a negative status if the
+ * arguments are invalid.  Host-only; launches nothing.
+ */
+int int4_matmul_select(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N);
+
+/*
+ * int4_device_status - synchronize `stream`, then read and clear the
+ * library's device-side status word of the current device.  Returns INT4_OK,
+ * or INT4_ERR_TIMEOUT if a kernel's bounded wait on an mbarrier gave up since
+ * the last call (that kernel wrote no output and returned), or INT4_ERR_CUDA.
+ */
+int int4_device_status(void* stream);
+
+/*
+ * int4_selftest_wait_timeout - launch one small kernel whose mbarrier wait is
+ * never satisfied, with an iteration limit of `spins`, so that the bounded
+ * wait gives up and sets the device status word; used by the tests of the
+ * failure path.  No other kernel state is touched.  Returns INT4_OK if the
+ * launch succeeded (call int4_device_status to read the outcome).
+ */
+int int4_selftest_wait_timeout(uint32_t spins, void* stream);
+
+/* Message for the last non-zero status returned on this host thread. */
+const char* int4_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int int4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT4_B200_H */

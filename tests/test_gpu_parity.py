@@ -1,0 +1,323 @@
+"""GPU parity: the CUDA library against the CPU oracle, through the C ABI.
+
+Packed bytes, fp16 scale bits and unpacked int8 must be bit-exact; the matmul
+must meet |y - y_ref| <= c * sum|x||w_hat| with c = 1e-5 (fp32 x) or 4e-3
+(bf16/fp16 x).  Every kernel path is exercised on the shapes it accepts,
+including ragged tails, odd K, partial last groups, all-zero groups, -8
+codes and the degenerate sizes.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import dequant_gemm_int4_b200 as q4
+import oracle
+from gpu_util import (TOL_F32, TOL_HALF, assert_matmul_close, assert_quantize_exact,
+                      oracle_quantize, to_np)
+from workloads import (DISTILGPT2_LINEARS, LLAMA7B_DECODE_LINEARS, make_activations,
+                       make_weights, tiny_case)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    q4.lib()
+    yield
+    torch.cuda.synchronize()
+    assert q4.device_status() == q4.OK
+
+
+def _tol(dtype):
+    return TOL_F32 if dtype == torch.float32 else TOL_HALF
+
+
+# ---------------------------------------------------------------------------
+# quantize_int4
+# ---------------------------------------------------------------------------
+def test_quantize_tiny_case_matches_golden_and_oracle():
+    case = tiny_case()
+    w = torch.from_numpy(case["w"]).to(DEV)
+    packed, scales, K = q4.quantize_int4(w, case["group"])
+    assert K == 259 and tuple(packed.shape) == (16, 130) and tuple(scales.shape) == (16, 3)
+    assert_quantize_exact(w, packed, scales, case["group"])
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "tiny_case_expected.json")))
+    assert packed.cpu().numpy().tobytes().hex() == g["packed_hex"]
+    assert scales.cpu().view(torch.int16).numpy().view(np.uint16).tolist() == g["scales_fp16_bits"]
+
+
+def test_quantize_drill_byte_layout():
+    w = torch.tensor([[1.0, -1.0, 7.0, -7.0]], device=DEV)
+    packed, scales, K = q4.quantize_int4(w, 4)
+    assert float(scales[0, 0]) == 1.0
+    assert packed.cpu().tolist() == [[0xF1, 0x97]]
+    # The same row on the fast path (K multiple of 8, group 8).
+    w8 = torch.tensor([[1.0, -1.0, 7.0, -7.0, 0.0, 0.0, 0.0, 0.0]], device=DEV)
+    packed8, scales8, _ = q4.quantize_int4(w8, 8)
+    assert packed8.cpu().tolist() == [[0xF1, 0x97, 0x00, 0x00]]
+
+
+def _special_rows():
+    t = 2.0 ** -24
+    rows = [
+        [7.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5, -3.5],
+        [0.0] * 8,
+        [7 * 2.0 ** -25, 0, 0, 0, 0, 0, 0, 0],
+        [7 * 1.49 * t, -7 * 1.49 * t, 0.5 * t, 0, 0, 0, 0, 0],
+        [1e-5, -3e-6, 2e-6, 0, 0, 0, 0, 0],
+        [-0.0, 0.0, -0.0, 0, 0, 0, 0, 0],
+        [3.0, -3.0, 1.0, 2.0, -1.5, 0.75, 0.2, -0.1],
+        [458000.0, -1.0, 1.0, 0, 0, 0, 0, 0],
+        [7 * 65520.0, 1.0, -5.0, 0, 0, 0, 0, 0],   # scale overflows to +inf
+    ]
+    return torch.tensor(rows, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("K_pad", [0, 1])
+def test_quantize_special_values(K_pad):
+    w = _special_rows()
+    if K_pad:  # odd K forces the general kernels
+        w = torch.cat([w, torch.zeros(w.shape[0], 1)], dim=1)
+    w = w.to(DEV)
+    packed, scales, K = q4.quantize_int4(w, 8)
+    assert_quantize_exact(w, packed, scales, 8)
+
+
+def test_quantize_half_integer_quotients():
+    """Weights placed exactly on and next to half-integer multiples of the
+    scale: the fast path must agree with the IEEE division on every tie."""
+    rng = np.random.default_rng(21)
+    s = (rng.uniform(0.01, 2.0, size=(4096, 1))).astype(np.float16).astype(np.float32)
+    half = rng.integers(-7, 7, size=(4096, 7)) + 0.5     # -6.5 .. 6.5
+    w = (half * s).astype(np.float32)
+    nudge = rng.integers(-2, 3, size=w.shape).astype(np.int32)
+    w = (w.view(np.int32) + nudge).view(np.float32)
+    w = np.concatenate([w, 7 * s], axis=1)          # absmax = 7 s -> scale s
+    wt = torch.from_numpy(w.astype(np.float32)).to(DEV)
+    for dtype in (torch.float32, torch.float16, torch.bfloat16):
+        wd = wt.to(dtype)
+        packed, scales, K = q4.quantize_int4(wd, 8)
+        assert_quantize_exact(wd, packed, scales, 8)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("N, K, group", [
+    (1, 8, 8), (3, 256, 32), (17, 1024, 128), (5, 1000, 64), (64, 4096, 256),
+    (7, 264, 128),            # partial last group on the fast path
+    (9, 259, 128), (4, 33, 32), (6, 1, 4), (2, 3, 2), (11, 515, 96), (8, 300, 300),
+    (3, 100, 1000),           # one partial group larger than K
+])
+def test_quantize_shapes(dtype, N, K, group):
+    w = make_weights(N, K, seed=N * 1000 + K, device=DEV, dtype=dtype, dist="student_t3",
+                     zero_group_frac=0.1, group=group)
+    packed, scales, Kout = q4.quantize_int4(w, group)
+    assert Kout == K
+    assert_quantize_exact(w, packed, scales, group)
+
+
+@pytest.mark.parametrize("layer", DISTILGPT2_LINEARS, ids=lambda l: l.name)
+def test_quantize_distilgpt2_full(layer):
+    w = make_weights(layer.N, layer.K, seed=2, device=DEV, dtype=torch.float32, std=0.02)
+    packed, scales, _ = q4.quantize_int4(w, layer.group)
+    assert_quantize_exact(w, packed, scales, layer.group)
+
+
+@pytest.mark.parametrize("N, K", [(28672, 8192), (8192, 28673)])
+@pytest.mark.parametrize("group", [32, 64, 128])
+def test_quantize_bulk_full_size_sampled_rows(N, K, group):
+    w = make_weights(N, K, seed=5, device=DEV, dtype=torch.bfloat16, dist="student_t3",
+                     zero_group_frac=0.01, group=group)
+    packed, scales, _ = q4.quantize_int4(w, group)
+    rng = np.random.default_rng(N + K + group)
+    rows = np.unique(np.concatenate([[0, 1, N - 1], rng.integers(0, N, size=61)]))
+    assert_quantize_exact(w, packed, scales, group, rows=rows)
+    # Unpack at full size, same rows.
+    q = q4.unpack_int4(packed, K)
+    q_ref = oracle.unpack_int4(packed[torch.as_tensor(rows, device=DEV)].cpu().numpy(), K)
+    assert np.array_equal(q[torch.as_tensor(rows, device=DEV)].cpu().numpy(), q_ref)
+
+
+def test_quantize_unaligned_pointers_take_the_general_path():
+    base = make_weights(8, 1025, seed=3, device=DEV, dtype=torch.bfloat16).reshape(-1)
+    w = base[1:1 + 8 * 1024].view(8, 1024)     # 2-byte aligned only
+    assert w.data_ptr() % 16 != 0
+    packed, scales, _ = q4.quantize_int4(w, 128)
+    assert_quantize_exact(w, packed, scales, 128)
+
+
+def test_quantize_is_deterministic():
+    w = make_weights(512, 2048, seed=4, device=DEV, dtype=torch.bfloat16, dist="student_t3")
+    a = q4.quantize_int4(w, 64)
+    b = q4.quantize_int4(w, 64)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1].view(torch.int16), b[1].view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# unpack_int4
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N, K", [(1, 2), (1, 1), (3, 5), (16, 259), (7, 512), (33, 1000),
+                                  (5, 31), (1000, 34)])
+def test_unpack_random_bytes(N, K):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(N * 7 + K)
+    Kp = (K + 1) // 2
+    packed = torch.randint(0, 256, (N, Kp), generator=g, device=DEV, dtype=torch.int32).to(torch.uint8)
+    if K % 2:
+        packed[:, -1] &= 0x0F
+    q = q4.unpack_int4(packed, K)
+    assert q.dtype == torch.int8 and tuple(q.shape) == (N, K)
+    assert np.array_equal(q.cpu().numpy(), oracle.unpack_int4(packed.cpu().numpy(), K))
+
+
+def test_unpack_all_256_bytes_and_minus_eight():
+    packed = torch.arange(256, device=DEV, dtype=torch.int32).to(torch.uint8).view(1, 256)
+    q = q4.unpack_int4(packed, 512).cpu().numpy()[0]
+    assert np.array_equal(q, oracle.unpack_int4(packed.cpu().numpy(), 512)[0])
+    assert q[2 * 0x88] == -8 and q[2 * 0x88 + 1] == -8
+    assert q[2 * 0x80] == 0 and q[2 * 0x80 + 1] == -8
+
+
+def test_unpack_unaligned_pointer():
+    buf = torch.randint(0, 256, (8 * 64 + 1,), device=DEV, dtype=torch.int32).to(torch.uint8)
+    packed = buf[1:].view(8, 64)
+    q = q4.unpack_int4(packed, 128)
+    assert np.array_equal(q.cpu().numpy(), oracle.unpack_int4(packed.cpu().numpy(), 128))
+
+
+# ---------------------------------------------------------------------------
+# int4_matmul
+# ---------------------------------------------------------------------------
+def _quantized(N, K, group, seed, std=0.02, dist="normal", zero_group_frac=0.0):
+    w = make_weights(N, K, seed=seed, device=DEV, dtype=torch.float32, std=std, dist=dist,
+                     zero_group_frac=zero_group_frac, group=group)
+    return q4.quantize_int4(w, group)
+
+
+def test_matmul_tiny_case_fp32():
+    case = tiny_case()
+    w = torch.from_numpy(case["w"]).to(DEV)
+    x = torch.from_numpy(case["x"]).to(DEV)
+    packed, scales, K = q4.quantize_int4(w, 128)
+    y = q4.int4_matmul(x, packed, scales, K, 128)
+    assert tuple(y.shape) == (4, 16) and y.dtype == torch.float32
+    assert_matmul_close(y, x, packed, scales, K, 128, TOL_F32)
+    assert q4.matmul_select(torch.float32, K, 128, 4, 16) == q4.PATH_SIMT
+
+
+@pytest.mark.parametrize("path", [q4.PATH_SIMT, q4.PATH_DECODE])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M, N, K, group", [
+    (1, 128, 128, 128), (1, 4096, 4096, 128), (4, 11008, 4096, 128), (16, 4096, 11008, 128),
+    (3, 300, 4096, 64), (9, 200, 1024, 32), (1, 2304, 768, 32), (1, 768, 3072, 64),
+    (16, 77, 8224, 128), (5, 1000, 2048, 256), (2, 64, 96, 32), (7, 129, 160, 32),
+    (12, 33, 640, 64), (1, 1, 32, 32),
+])
+def test_matmul_paths(path, dtype, M, N, K, group):
+    packed, scales, _ = _quantized(N, K, group, seed=M + N + K)
+    x = make_activations(M, K, seed=M * 31 + K, device=DEV, dtype=dtype)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=path)
+    torch.cuda.synchronize()
+    cols = None
+    if N > 2048:
+        cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(N).integers(0, N, 1500)]))
+    assert_matmul_close(y, x, packed, scales, K, group, _tol(dtype), cols=cols)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M, N, K, group", [(4, 16, 259, 128), (33, 70, 1000, 96), (2, 5, 3, 2),
+                                            (20, 64, 512, 4), (1, 3, 1, 1), (64, 257, 4096, 128)])
+def test_matmul_simt_general_shapes(dtype, M, N, K, group):
+    packed, scales, _ = _quantized(N, K, group, seed=K, dist="student_t3", zero_group_frac=0.05)
+    x = make_activations(M, K, seed=M + K, device=DEV, dtype=dtype)
+    y = q4.int4_matmul(x, packed, scales, K, group)
+    assert_matmul_close(y, x, packed, scales, K, group, _tol(dtype))
+
+
+@pytest.mark.parametrize("path", [q4.PATH_SIMT, q4.PATH_DECODE])
+def test_matmul_one_hot_x_is_exact(path):
+    N, K, group = 96, 512, 128
+    packed, scales, _ = _quantized(N, K, group, seed=9, dist="student_t3", zero_group_frac=0.2)
+    w_hat = oracle.dequantize_int4(packed.cpu().numpy(), scales.cpu().numpy(), K, group)
+    ks = [0, 1, 127, 128, 300, 511]
+    x = torch.zeros(len(ks), K, device=DEV, dtype=torch.bfloat16)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    y = q4.int4_matmul(x, packed, scales, K, group, path=path).cpu().numpy().astype(np.float64)
+    for i, k in enumerate(ks):
+        assert np.array_equal(y[i], w_hat[:, k]), (path, k)
+
+
+@pytest.mark.parametrize("path", [q4.PATH_SIMT, q4.PATH_DECODE])
+def test_matmul_hand_made_bytes_row_sums(path):
+    N, K, group = 40, 256, 64
+    packed = torch.full((N, K // 2), 0x11, dtype=torch.uint8, device=DEV)
+    scales = torch.ones((N, K // group), dtype=torch.float16, device=DEV)
+    x = make_activations(3, K, seed=12, device=DEV, dtype=torch.bfloat16)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=path)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF)
+    # All bytes 0x88 (every weight -8) with scale 1: y = -8 * row sums.
+    packed.fill_(0x88)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=path)
+    expect = -8.0 * to_np(x).astype(np.float64).sum(1)
+    np.testing.assert_allclose(y.cpu().numpy(), np.repeat(expect[:, None], N, 1), rtol=1e-5, atol=1e-4)
+
+
+def test_matmul_decode_is_deterministic_and_matches_simt():
+    packed, scales, _ = _quantized(4096, 4096, 128, seed=1)
+    x = make_activations(4, 4096, seed=2, device=DEV, dtype=torch.bfloat16)
+    a = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_DECODE)
+    b = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_DECODE)
+    c = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_SIMT)
+    assert torch.equal(a, b)
+    rel = ((a - c).abs().max() / c.abs().max()).item()
+    assert rel < 1e-4
+
+
+@pytest.mark.parametrize("layer", LLAMA7B_DECODE_LINEARS, ids=lambda l: l.name)
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_matmul_llama7b_decode_full_size(layer, M):
+    packed, scales, _ = _quantized(layer.N, layer.K, layer.group, seed=3)
+    x = make_activations(M, layer.K, seed=3 + M, device=DEV, dtype=torch.bfloat16)
+    assert q4.matmul_select(torch.bfloat16, layer.K, layer.group, M, layer.N) == q4.PATH_DECODE
+    y = q4.int4_matmul(x, packed, scales, layer.K, layer.group)
+    assert_matmul_close(y, x, packed, scales, layer.K, layer.group, TOL_HALF)
+
+
+@pytest.mark.parametrize("layer", DISTILGPT2_LINEARS, ids=lambda l: l.name)
+@pytest.mark.parametrize("M", [1, 1024])
+def test_matmul_distilgpt2(layer, M):
+    packed, scales, _ = _quantized(layer.N, layer.K, layer.group, seed=2)
+    x = make_activations(M, layer.K, seed=2 + M, device=DEV, dtype=torch.float16)
+    y = q4.int4_matmul(x, packed, scales, layer.K, layer.group)
+    rows = None if M == 1 else np.random.default_rng(M).choice(M, 48, replace=False)
+    assert_matmul_close(y, x, packed, scales, layer.K, layer.group, TOL_HALF, rows=rows)
+
+
+def test_matmul_zero_group_contributes_nothing():
+    case = tiny_case()
+    w = torch.from_numpy(case["w"]).to(DEV)
+    packed, scales, K = q4.quantize_int4(w, 128)
+    x = torch.zeros(1, K, device=DEV)
+    x[0, 128:256] = 1.0                         # only row 3's zero group is hit
+    y = q4.int4_matmul(x, packed, scales, K, 128)
+    assert float(y[0, 3]) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# Failure path: a bounded device-side wait gives up and reports it.
+# ---------------------------------------------------------------------------
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert q4.device_status() == q4.OK
+    q4.selftest_wait_timeout(2000)
+    assert q4.device_status() == q4.ERR_TIMEOUT
+    assert q4.device_status() == q4.OK          # cleared by the read
+    packed, scales, _ = _quantized(64, 256, 64, seed=1)
+    x = make_activations(2, 256, seed=1, device=DEV, dtype=torch.bfloat16)
+    y = q4.int4_matmul(x, packed, scales, 256, 64)
+    assert_matmul_close(y, x, packed, scales, 256, 64, TOL_HALF)
