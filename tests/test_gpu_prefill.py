@@ -1,0 +1,100 @@
+"""GPU parity of the tcgen05 tensor-core matmul (the prefill path) against
+the CPU oracle: |y - y_ref| <= 4e-3 * sum|x||w_hat| for bf16/fp16 x, on
+shapes with ragged M, N and K tails, partial last groups, zero groups and
+the full-size prefill workloads (sampled outputs)."""
+
+import numpy as np
+import pytest
+import torch
+
+import dequant_gemm_int4_b200 as q4
+import oracle
+from gpu_util import TOL_HALF, assert_matmul_close
+from workloads import PREFILL_LINEARS, make_activations, make_weights
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    q4.lib()
+    assert q4.device_status() == q4.OK
+    yield
+    assert q4.device_status() == q4.OK
+
+
+def _quantized(N, K, group, seed, dist="normal", zero_group_frac=0.0):
+    w = make_weights(N, K, seed=seed, device=DEV, dtype=torch.float32, std=0.02, dist=dist,
+                     zero_group_frac=zero_group_frac, group=group)
+    return q4.quantize_int4(w, group)
+
+
+def _run(M, N, K, group, dtype, seed=0, dist="normal", zero_group_frac=0.0, rows=None, cols=None):
+    packed, scales, _ = _quantized(N, K, group, seed + 1, dist, zero_group_frac)
+    x = make_activations(M, K, seed=seed + 2, device=DEV, dtype=dtype)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL)
+    assert q4.device_status() == q4.OK, "a bounded wait in the tensor-core kernel timed out"
+    return assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF, rows=rows, cols=cols)
+
+
+def test_prefill_smallest_tile():
+    _run(256, 128, 64, 64, torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M, N, K, group", [
+    (256, 128, 128, 128), (256, 128, 1024, 128), (512, 256, 512, 64), (300, 200, 256, 128),
+    (17, 130, 192, 64), (1000, 77, 4096, 128), (256, 128, 96, 64), (256, 128, 8224, 128),
+    (513, 385, 640, 128), (64, 1000, 2048, 256), (257, 129, 3072, 3072),
+])
+def test_prefill_shapes(dtype, M, N, K, group):
+    _run(M, N, K, group, dtype, seed=M + N + K)
+
+
+def test_prefill_heavy_tailed_with_zero_groups():
+    _run(384, 256, 2048, 64, torch.bfloat16, dist="student_t3", zero_group_frac=0.05)
+
+
+def test_prefill_one_hot_x_is_exact():
+    N, K, group = 256, 512, 128
+    packed, scales, _ = _quantized(N, K, group, 9, "student_t3", 0.2)
+    w_hat = oracle.dequantize_int4(packed.cpu().numpy(), scales.cpu().numpy(), K, group)
+    ks = [0, 1, 63, 64, 127, 128, 300, 511]
+    x = torch.zeros(256, K, device=DEV, dtype=torch.bfloat16)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL).cpu().numpy()
+    for i, k in enumerate(ks):
+        assert np.array_equal(y[i].astype(np.float64), w_hat[:, k]), k
+    assert not y[len(ks):].any()
+
+
+def test_prefill_matches_decode_and_simt():
+    packed, scales, _ = _quantized(1024, 4096, 128, 3)
+    x = make_activations(64, 4096, seed=4, device=DEV, dtype=torch.bfloat16)
+    a = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_PREFILL)
+    b = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_SIMT)
+    c = q4.int4_matmul(x[:16], packed, scales, 4096, 128, path=q4.PATH_DECODE)
+    scale = b.abs().max().item()
+    assert (a - b).abs().max().item() < 1e-4 * scale
+    assert (a[:16] - c).abs().max().item() < 1e-4 * scale
+    d = q4.int4_matmul(x, packed, scales, 4096, 128, path=q4.PATH_PREFILL)
+    assert torch.equal(a, d)                    # deterministic
+
+
+def test_prefill_is_the_automatic_choice_for_large_m():
+    assert q4.matmul_select(torch.bfloat16, 8192, 128, 2048, 8192) == q4.PATH_PREFILL
+    assert q4.matmul_select(torch.float16, 768, 64, 1024, 2304) == q4.PATH_PREFILL
+
+
+@pytest.mark.parametrize("layer", PREFILL_LINEARS, ids=lambda l: l.name)
+@pytest.mark.parametrize("M", [2048, 8192])
+def test_prefill_full_size_sampled(layer, M):
+    rng = np.random.default_rng(M + layer.N)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 14)]))
+    cols = np.unique(np.concatenate([[0, layer.N - 1], rng.integers(0, layer.N, 254)]))
+    _run(M, layer.N, layer.K, layer.group, torch.bfloat16, seed=4, rows=rows, cols=cols)
