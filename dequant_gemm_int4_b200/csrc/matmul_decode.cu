@@ -5,33 +5,38 @@
 // and a dequantizing matmul" (problem statement), integer weights times x
 // first, then the group's scale per output column.
 //
-// The kernel is bound by HBM: every packed weight byte is read once, and at
-// M <= 16 each byte feeds at most 32 multiply-adds.  The design keeps the
-// dequantization in registers:
-//   * a warp owns 16 weight rows; each lane streams its share of every
-//     128-wide K block with 16-byte (or, for group 64/32, 8/4-byte) loads
-//     straight from HBM into registers;
-//   * nibbles are sign-extended to bf16/fp16 with two integer ops per pair
-//     ((w >> 4i) & 0x000F000F) ^ magic, then one packed subtract: the
-//     magic 0x4300 / 0x6400 makes 128 + u (bf16) or 1024 + u (fp16) exactly,
-//     u = q + 8, so every integer weight is exact;
+// The kernel is bound by HBM: every packed weight byte is read once and at
+// M <= 16 feeds at most 32 multiply-adds.  Design:
+//   * a producer warp streams the CTA's 128 weight rows through a 4-stage
+//     shared-memory ring with TMA (each stage: 128 rows x 256 k = 16 KB of
+//     packed nibbles, 128-byte swizzle, plus x [M x 256] bf16/fp16), so about
+//     64 KB per CTA are in flight;
+//   * eight consumer warps own 16 rows each; per 128-wide K block a lane reads
+//     its 16 (or 2 x 8, 4 x 4 for group 64/32) bytes of two rows from shared
+//     memory and sign-extends nibble pairs to bf16/fp16 exactly in registers:
+//     byte j -> ((byte_j | byte_j >> 4 << 16) & 0x000F000F) ^ magic, then one
+//     packed subtract (magic = 128 + 8 (bf16) or 1024 + 8 (fp16) in each half,
+//     the XOR flips the nibble's sign bit so that the value is q + 136 or
+//     q + 1032 before the subtract);
 //   * the 16 x 8 x 16 warp MMA (mma.sync, fp32 accumulate) multiplies them by
-//     x, which sits in shared memory already permuted into fragment order, so
-//     no multiply-add runs on the CUDA cores;
-//   * each K group gets its own fp32 accumulator; its scale is applied with
-//     one FMA per output into the fp32 running sum, per the page's order.
-// Within one MMA the 16 k-slots of the four lanes of a quad are a
-// permutation of the natural k order (pairs (e_i, e_{i+4}) of a 32-bit word);
-// x is staged with the same permutation, and every MMA only sees k of one
-// group.
-// Split-K: when N is small the K range is split over the CTAs of a thread
-// block cluster (up to 8); partial sums are reduced in a fixed order through
-// distributed shared memory, so the result is deterministic and the kernel
-// needs no memory beyond its inputs and outputs.
+//     x straight from shared memory (natural k order, no permutation), so no
+//     multiply-add runs on the CUDA cores;
+//   * each K group gets its own fp32 accumulator, which is scaled by its
+//     group's scale and added into the fp32 running sum, per the page's order.
+// All four lanes of a quad read the same group for a given word, so each MMA
+// only sums k of one group.  Split-K: when N is small the K range is split
+// over the CTAs of a cluster (up to 8); partial sums are reduced in rank order
+// through distributed shared memory, so the result is deterministic.  Every
+// mbarrier wait is bounded in time; a wait that gives up aborts the CTA (the
+// status word records it), drains its copies and skips the output.
 #include <cooperative_groups.h>
+#include <cuda.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -39,22 +44,23 @@ namespace int4lib {
 
 namespace {
 
-constexpr int kWarps = 8;                 // warps per CTA, one 16-row tile each
-constexpr int kRowsPerCta = 16 * kWarps;  // 128 weight rows per CTA
-constexpr int kPrefetch = 4;              // K blocks loaded ahead per warp
-constexpr int kChunkBlocks = 16;          // K blocks of x staged per pass
+constexpr int kConsumers = 8;               // consumer warps, 16 weight rows each
+constexpr int kRowsPerCta = 16 * kConsumers;
+constexpr int kThreads = 32 * (kConsumers + 1);
+constexpr int kSK = 2;                      // 128-wide K blocks per stage
+constexpr int kStages = 4;
 constexpr int kMaxCluster = 8;
+constexpr int kWBytes = kRowsPerCta * kSK * 64;  // 16 KB per stage
+constexpr uint64_t kTimeoutNs = 250000000ull;
 
 template <typename TX>
 struct Cvt;
-// bf16: (w & 0x000F000F) ^ 0x43084308 = bf16x2(128 + u_lo, 128 + u_hi), u = q + 8.
 template <>
 struct Cvt<__nv_bfloat16> {
   static constexpr uint32_t kMagic = 0x43084308u;
-  static constexpr uint32_t kBias = 0x43084308u;  // bf16x2(136, 136)
   __device__ __forceinline__ static uint32_t sub(uint32_t a) {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(kBias));
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x43084308u));
     return d;
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -66,14 +72,12 @@ struct Cvt<__nv_bfloat16> {
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
   }
 };
-// fp16: (w & 0x000F000F) ^ 0x64086408 = f16x2(1024 + u_lo, 1024 + u_hi).
 template <>
 struct Cvt<__half> {
   static constexpr uint32_t kMagic = 0x64086408u;
-  static constexpr uint32_t kBias = 0x64086408u;  // f16x2(1032, 1032)
   __device__ __forceinline__ static uint32_t sub(uint32_t a) {
     uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(kBias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x64086408u));
     return d;
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -86,24 +90,23 @@ struct Cvt<__half> {
   }
 };
 
-// Word w holds nibbles e0..e7 (k = 8*widx + 0..7).  p[i] = (e_i, e_{i+4}).
+// Word w = 8 consecutive k (nibbles e0..e7).  p[i] = (e_{2i}, e_{2i+1}).
 template <typename TX>
 __device__ __forceinline__ void expand(uint32_t w, uint32_t (&p)[4]) {
-  uint32_t t;
-  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
-  p[0] = Cvt<TX>::sub(t);
+  const uint32_t ws = w >> 4;
 #pragma unroll
-  for (int i = 1; i < 4; ++i) {
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;"
-        : "=r"(t)
-        : "r"(w >> (4 * i)), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
-    p[i] = Cvt<TX>::sub(t);
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t sel = static_cast<uint32_t>(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
+    const uint32_t t = __byte_perm(w, ws, sel);
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(t), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
+    p[i] = Cvt<TX>::sub(r);
   }
 }
 
-// Which 8-k group (0..15 inside a 128-k block) lane c uses as its word j,
-// for GPB groups per block (1: group >= 128, 2: group 64, 4: group 32), so
-// that all four lanes of a quad read the same group for word j.
+// The 8-k word (0..15 of a 128-k block) that lane c of a quad uses as its
+// word j, for GPB groups per block (1: group multiple of 128, 2: group 64,
+// 4: group 32); all four lanes of a quad then read the same group for word j.
 template <int GPB>
 __device__ __forceinline__ int word_index(int c, int j) {
   if (GPB == 1) return 4 * c + j;
@@ -111,81 +114,88 @@ __device__ __forceinline__ int word_index(int c, int j) {
   return 4 * j + c;
 }
 
-template <int GPB>
-__device__ __forceinline__ void word_owner(int kk, int& c, int& j) {
-  if (GPB == 1) {
-    c = kk >> 2;
-    j = kk & 3;
-  } else if (GPB == 2) {
-    j = (kk >> 3) * 2 + (kk & 1);
-    c = (kk & 7) >> 1;
-  } else {
-    j = kk >> 2;
-    c = kk & 3;
+// Byte offset of `off` (0..127) within row r of a 128-byte-swizzled W tile.
+__device__ __forceinline__ uint32_t swz(int r, int off) {
+  return static_cast<uint32_t>(r * 128 + ((((off >> 4) ^ (r & 7))) << 4) + (off & 15));
+}
+
+struct WaitCtx {
+  volatile uint32_t* abort;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t i = 1; i != 0; ++i) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((i & 127u) == 0u) {
+      if (*w.abort) return false;
+      if (ptx::globaltimer() - t0 > kTimeoutNs) break;
+    }
+  }
+  *w.abort = 1u;
+  report_status(w.status, kStatusTimeout);
+  return false;
+}
+
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer();
+  for (uint32_t i = 0; i != 0xFFFFFFFFu; ++i) {
+    if (ptx::mbar_try_wait(bar, parity)) return;
+    if ((i & 127u) == 0u && ptx::globaltimer() - t0 > kTimeoutNs) return;
   }
 }
 
-// Loads this lane's four words of one 128-k block of row `rowp` (row start).
-template <int GPB>
-__device__ __forceinline__ void load_words(const uint8_t* rowp, bool row_ok, int64_t kb, int c,
-                                           int64_t K, uint32_t (&w)[4]) {
-  const uint8_t* bp = rowp + kb * 64;
-  const int64_t kbase = kb * 128;
-  if (GPB == 1) {
-    if (row_ok && kbase + 32 * c < K) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(bp + 16 * c));
-      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else {
-      w[0] = w[1] = w[2] = w[3] = 0x88888888u & 0u;
-    }
-  } else if (GPB == 2) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (row_ok && kbase + 64 * h + 16 * c < K) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(bp + 32 * h + 8 * c));
-        w[2 * h] = v.x; w[2 * h + 1] = v.y;
-      } else {
-        w[2 * h] = w[2 * h + 1] = 0u;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      w[j] = (row_ok && kbase + 32 * j + 8 * c < K)
-                 ? __ldg(reinterpret_cast<const uint32_t*>(bp + 16 * j + 4 * c))
-                 : 0u;
-    }
-  }
-}
+template <int NT>
+struct DLayout {
+  // Per stage: W tile (1024-aligned for the swizzle), then the x tile.
+  static constexpr int kXBytesMax = 16 * kSK * 128 * 2;  // M <= 16 rows
+  static constexpr int kStageBytes = kWBytes + kXBytesMax;     // multiple of 1024
+  static constexpr int offRed = kStages * kStageBytes;
+  static constexpr int kRedBytes = kConsumers * NT * 4 * 32 * 4;
+  static constexpr int offBar = offRed + kRedBytes;
+  static constexpr int offMisc = offBar + 2 * kStages * 8;
+  static constexpr int kBytes = offMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
 
-// Shared memory: x chunk in fragment order, then the split-K partials.
-//   xs[((kbl * 4 + j) * NT + nt) * 32 + lane] : uint4 = 8 x values of
-//   batch row nt*8 + lane/4, k8-group word_index(lane%4, j) of block kbl,
-//   as (x0,x4) (x1,x5) (x2,x6) (x3,x7).
 template <typename TX, int NT, int GPB>
-__global__ void __launch_bounds__(256, 2) decode_kernel(
-    const TX* __restrict__ x, const uint8_t* __restrict__ packed,
-    const uint16_t* __restrict__ scales, int64_t K, int group, int G, int M, int64_t N,
-    float* __restrict__ y, int kblocks_per_slice, int S) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint4* xs = reinterpret_cast<uint4*>(smem);
-  float* red = reinterpret_cast<float*>(smem + kChunkBlocks * 16 * NT * 8 * 16);
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+    const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
+    int64_t N, int kblocks_per_slice, int S, uint32_t* status) {
+  using L = DLayout<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::offBar);
+  uint64_t* empty = full + kStages;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::offMisc);
+  float* red = reinterpret_cast<float*>(smem + L::offRed);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int c = lane & 3;
-  const int g = lane >> 2;
-  const int slice = blockIdx.x;  // == rank in the cluster when S > 1
+  const int slice = blockIdx.x;  // rank in the cluster when S > 1
   const int64_t KB = (K + 127) / 128;
   const int64_t kb0 = static_cast<int64_t>(slice) * kblocks_per_slice;
-  int64_t kb1 = kb0 + kblocks_per_slice;
-  if (kb1 > KB) kb1 = KB;
-  const int64_t Kp = K >> 1;
-  const int64_t ra = static_cast<int64_t>(blockIdx.y) * kRowsPerCta + warp * 16 + g;
-  const int64_t rb = ra + 8;
-  const bool va = ra < N, vb = rb < N;
-  const uint8_t* rowa = packed + (va ? ra : 0) * Kp;
-  const uint8_t* rowb = packed + (vb ? rb : 0) * Kp;
+  const int64_t kb1 = (kb0 + kblocks_per_slice < KB) ? kb0 + kblocks_per_slice : KB;
+  const int nst = static_cast<int>((kb1 - kb0 + kSK - 1) / kSK);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kRowsPerCta;
+  const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;
+  const WaitCtx wc{abort_flag, status};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&empty[s]), kConsumers);
+    }
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_w);
+    ptx::prefetch_tmap(&tm_x);
+  }
+  __syncthreads();
 
   float tot[NT][4];
 #pragma unroll
@@ -193,44 +203,47 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) tot[nt][i] = 0.0f;
 
-  for (int64_t cb0 = kb0; cb0 < kb1; cb0 += kChunkBlocks) {
-    const int64_t cb1 = (cb0 + kChunkBlocks < kb1) ? cb0 + kChunkBlocks : kb1;
-    const int nblk = static_cast<int>(cb1 - cb0);
-    // Stage x[:, cb0*128 : cb1*128] in fragment order (zeros past M and K).
-    __syncthreads();
-    const int entries = nblk * 16 * NT * 8;
-    for (int e = threadIdx.x; e < entries; e += blockDim.x) {
-      const int m = e % (NT * 8);
-      const int kk = (e / (NT * 8)) % 16;
-      const int kbl = e / (NT * 8 * 16);
-      const int64_t k = (cb0 + kbl) * 128 + kk * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (m < M && k < K) {
-        const uint4 r = __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k));
-        v.x = __byte_perm(r.x, r.z, 0x5410);
-        v.y = __byte_perm(r.x, r.z, 0x7632);
-        v.z = __byte_perm(r.y, r.w, 0x5410);
-        v.w = __byte_perm(r.y, r.w, 0x7632);
-      }
-      int cc, jj;
-      word_owner<GPB>(kk, cc, jj);
-      xs[((kbl * 4 + jj) * NT + (m >> 3)) * 32 + (m & 7) * 4 + cc] = v;
-    }
-    __syncthreads();
+  const int c = lane & 3;
+  const int g = lane >> 2;
+  const int cw = warp - 1;                       // consumer index
+  const int64_t ra = row0 + cw * 16 + g;
+  const int64_t rb = ra + 8;
 
-    for (int64_t kb = cb0; kb < cb1; kb += kPrefetch) {
-      uint32_t wa[kPrefetch][4], wb[kPrefetch][4];
-#pragma unroll
-      for (int p = 0; p < kPrefetch; ++p) {
-        if (kb + p < cb1) {
-          load_words<GPB>(rowa, va, kb + p, c, K, wa[p]);
-          load_words<GPB>(rowb, vb, kb + p, c, K, wb[p]);
-        }
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int it = 0;
+      for (; it < nst; ++it) {
+        const int s = it % kStages;
+        if (!wait_bar(ptx::smem_u32(&empty[s]), ((it / kStages) & 1) ^ 1u, wc)) break;
+        uint8_t* st = smem + s * L::kStageBytes;
+        const int64_t kb = kb0 + static_cast<int64_t>(it) * kSK;
+        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + xbytes);
+        ptx::tma_load_2d(ptx::smem_u32(st), &tm_w, static_cast<int32_t>(kb * 64),
+                         static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
+        ptx::tma_load_2d(ptx::smem_u32(st + kWBytes), &tm_x, static_cast<int32_t>(kb * 128), 0,
+                         ptx::smem_u32(&full[s]));
       }
+      if (*abort_flag) {
+        const int first = it - kStages > 0 ? it - kStages : 0;
+        for (int j = first; j < it; ++j) drain_bar(ptx::smem_u32(&full[j % kStages]), (j / kStages) & 1);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const bool va = ra < N, vb = rb < N;
+    const uint16_t* sra = scales + (va ? ra : 0) * G;
+    const uint16_t* srb = scales + (vb ? rb : 0) * G;
+    const int la = cw * 16 + g, lb = la + 8;      // rows within the W tile
+    for (int it = 0; it < nst; ++it) {
+      const int s = it % kStages;
+      if (!wait_bar(ptx::smem_u32(&full[s]), (it / kStages) & 1, wc)) break;
+      const uint8_t* wt = smem + s * L::kStageBytes;
+      const uint8_t* xt = wt + kWBytes;
 #pragma unroll
-      for (int p = 0; p < kPrefetch; ++p) {
-        if (kb + p >= cb1) break;
-        const int kbl = static_cast<int>(kb + p - cb0);
+      for (int b = 0; b < kSK; ++b) {
+        const int64_t kb = kb0 + static_cast<int64_t>(it) * kSK + b;
+        if (kb >= kb1) break;
         float acc[GPB][NT][4];
 #pragma unroll
         for (int a = 0; a < GPB; ++a)
@@ -238,26 +251,49 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[a][nt][i] = 0.0f;
+        uint32_t wa[4], wb[4];
+        if (GPB == 1) {
+          const uint4 u = *reinterpret_cast<const uint4*>(wt + swz(la, b * 64 + 16 * c));
+          const uint4 v = *reinterpret_cast<const uint4*>(wt + swz(lb, b * 64 + 16 * c));
+          wa[0] = u.x; wa[1] = u.y; wa[2] = u.z; wa[3] = u.w;
+          wb[0] = v.x; wb[1] = v.y; wb[2] = v.z; wb[3] = v.w;
+        } else if (GPB == 2) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint2 u = *reinterpret_cast<const uint2*>(wt + swz(la, b * 64 + 32 * h + 8 * c));
+            const uint2 v = *reinterpret_cast<const uint2*>(wt + swz(lb, b * 64 + 32 * h + 8 * c));
+            wa[2 * h] = u.x; wa[2 * h + 1] = u.y;
+            wb[2 * h] = v.x; wb[2 * h + 1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            wa[j] = *reinterpret_cast<const uint32_t*>(wt + swz(la, b * 64 + 16 * j + 4 * c));
+            wb[j] = *reinterpret_cast<const uint32_t*>(wt + swz(lb, b * 64 + 16 * j + 4 * c));
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t pa[4], pb[4];
-          expand<TX>(wa[p][j], pa);
-          expand<TX>(wb[p][j], pb);
+          expand<TX>(wa[j], pa);
+          expand<TX>(wb[j], pb);
           const int a = (GPB == 1) ? 0 : (GPB == 2 ? (j >> 1) : j);
+          const int kx = b * 128 + 8 * word_index<GPB>(c, j);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const uint4 xf = xs[((kbl * 4 + j) * NT + nt) * 32 + lane];
+            const int m = nt * 8 + g;
+            uint4 xf = make_uint4(0u, 0u, 0u, 0u);
+            if (m < M) xf = *reinterpret_cast<const uint4*>(xt + (m * kSK * 128 + kx) * 2);
             Cvt<TX>::mma(acc[a][nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
             Cvt<TX>::mma(acc[a][nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
           }
         }
-        // Apply each group's scale per output row, then add to the running sum.
-        const int64_t kbase = (kb + p) * 128;
+        const int64_t kbase = kb * 128;
 #pragma unroll
         for (int a = 0; a < GPB; ++a) {
           const int64_t gi = (kbase + a * (128 / GPB)) / group;
-          const float sa = (va && gi < G) ? f16_bits_to_float(__ldg(scales + ra * G + gi)) : 0.0f;
-          const float sb = (vb && gi < G) ? f16_bits_to_float(__ldg(scales + rb * G + gi)) : 0.0f;
+          const float sa = (va && gi < G) ? f16_bits_to_float(__ldg(sra + gi)) : 0.0f;
+          const float sb = (vb && gi < G) ? f16_bits_to_float(__ldg(srb + gi)) : 0.0f;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             tot[nt][0] = fmaf(acc[a][nt][0], sa, tot[nt][0]);
@@ -267,71 +303,124 @@ __global__ void __launch_bounds__(256, 2) decode_kernel(
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
     }
   }
 
+  const bool ok = (*abort_flag == 0u);
   // Output (m, row) of register i of n-tile nt: m = nt*8 + 2c + (i & 1),
   // row = (i < 2) ? ra : rb.
   if (S == 1) {
+    if (warp > 0 && ok) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = nt * 8 + 2 * c + (i & 1);
-        const int64_t row = (i < 2) ? ra : rb;
-        if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = tot[nt][i];
-      }
+        for (int i = 0; i < 4; ++i) {
+          const int m = nt * 8 + 2 * c + (i & 1);
+          const int64_t row = (i < 2) ? ra : rb;
+          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = tot[nt][i];
+        }
+    }
     return;
   }
 
-  // Split-K: partials to shared memory, reduce across the cluster in rank order.
+  // Split-K: partials to shared memory, reduced across the cluster in rank order.
+  if (warp > 0) {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) red[((warp * NT + nt) * 4 + i) * 32 + lane] = tot[nt][i];
+      for (int i = 0; i < 4; ++i) red[((cw * NT + nt) * 4 + i) * 32 + lane] = tot[nt][i];
+  }
   cg::cluster_group cluster = cg::this_cluster();
   cluster.sync();
-  const int total = kWarps * NT * 4 * 32;
+  const int total = kConsumers * NT * 4 * 32;
   for (int e = slice * blockDim.x + threadIdx.x; e < total; e += S * blockDim.x) {
-    float s = 0.0f;
-    for (int r = 0; r < S; ++r) s += cluster.map_shared_rank(red, r)[e];
+    float sum = 0.0f;
+    bool all_ok = ok;
+    for (int r = 0; r < S; ++r) sum += cluster.map_shared_rank(red, r)[e];
+    for (int r = 0; r < S; ++r)
+      all_ok = all_ok && (*cluster.map_shared_rank(const_cast<uint32_t*>(abort_flag), r) == 0u);
     const int ln = e & 31;
     const int i = (e >> 5) & 3;
     const int nt = (e >> 7) % NT;
     const int wp = (e >> 7) / NT;
     const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
-    const int64_t row = static_cast<int64_t>(blockIdx.y) * kRowsPerCta + wp * 16 + (ln >> 2) +
-                        ((i < 2) ? 0 : 8);
-    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = s;
+    const int64_t row = row0 + wp * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
+    if (all_ok && m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
   }
   cluster.sync();  // keep this CTA's partials alive until every rank has read them
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
 }
 
 template <typename TX, int NT, int GPB>
 cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                            int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  using L = DLayout<NT>;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
   const int G = static_cast<int>((K + group - 1) / group);
   const int64_t KB = (K + 127) / 128;
   const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
-  if (R > 65535) return cudaErrorInvalidConfiguration;
-  // Enough CTAs to cover the SMs about twice; at most 8 K slices.
-  const int64_t target = 2LL * num_sms();
-  int64_t S = (target + R - 1) / R;
+  // One wave of CTAs (two per SM), at most 8 K slices per cluster.
+  const int64_t slots = 2LL * num_sms();
+  int64_t S = slots / R;
   if (S > kMaxCluster) S = kMaxCluster;
   if (S > KB) S = KB;
   if (S < 1) S = 1;
   const int kbps = static_cast<int>((KB + S - 1) / S);
   S = (KB + kbps - 1) / kbps;  // no empty slices
-  const size_t smem = static_cast<size_t>(kChunkBlocks) * 16 * NT * 8 * 16 +
-                      static_cast<size_t>(kWarps) * NT * 4 * 32 * sizeof(float);
+
+  CUtensorMap tw, tx;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {kSK * 64, kRowsPerCta};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {kSK * 128, static_cast<cuuint32_t>(M)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
+                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   auto kern = decode_kernel<TX, NT, GPB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(R), 1);
-  cfg.blockDim = dim3(32 * kWarps, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kAlloc;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -340,8 +429,8 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, x, packed, scales, K, group, G, static_cast<int>(M), N, y,
-                            kbps, static_cast<int>(S));
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, scales, y, K, group, G, static_cast<int>(M), N, kbps,
+                            static_cast<int>(S), status);
 }
 
 template <typename TX, int NT>
@@ -365,7 +454,7 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
                       const uint8_t* packed) {
   if (xt == DType::F32) return false;
   if (M < 1 || M > 16 || N < 1) return false;
-  if (K % 32 != 0) return false;
+  if (K % 32 != 0 || K > (1LL << 31)) return false;
   if (!(group == 32 || group == 64 || group % 128 == 0)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return false;
   if (reinterpret_cast<uintptr_t>(packed) % 16 != 0) return false;

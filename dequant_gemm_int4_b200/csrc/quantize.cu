@@ -41,25 +41,40 @@ __device__ __forceinline__ ScaleInfo scale_from_absmax(float m) {
   return scale_from_bits(__half_as_ushort(h));
 }
 
-// The 4-bit code of v: clamp(rint(fp32(v / sf)), -8, 7), 0 when sf == 0.
-//
-// The quotient is first approximated as t = v * r with r = fp32(1/sf).  With
-// x the exact quotient, |t - x| <= |x| * 2^-23 (two roundings), and the
-// correctly rounded fp32(x) lies within another half ulp of x, so for
-// |x| < 16 the two differ from t by less than 2^-19.  rint(fp32(x)) can only
-// differ from rint(t) if a half-integer lies within that distance of t; t is
-// then recomputed with the IEEE division.  Half-integers beyond +-7.5 never
-// change the clamped result.  Hence the result equals the IEEE-division
-// result for every finite v; the slow path runs for about 1 element in 10^5.
-__device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
-  float t = v * si.r;
-  float rt = rintf(t);
-  if (fabsf(t - rt) >= 0.5f - 0x1p-18f && si.sf != 0.0f) {
-    t = __fdiv_rn(v, si.sf);
-    rt = rintf(t);
-  }
+// The 4-bit code of v: clamp(rint(fp32(v / sf)), -8, 7), 0 when sf == 0,
+// with the IEEE division (used on the rare path and by the general kernels).
+__device__ __forceinline__ uint32_t code_exact(float v, const ScaleInfo& si) {
+  if (si.sf == 0.0f) return 0u;
+  float rt = rintf(__fdiv_rn(v, si.sf));
   rt = fminf(fmaxf(rt, -8.0f), 7.0f);
   return static_cast<uint32_t>(static_cast<int>(rt)) & 0xFu;
+}
+
+// Fast path of the same code.  The quotient is approximated as t = v * r
+// with r = fp32(1/sf).  With x the exact quotient, |t - x| <= |x| * 2^-23
+// (two roundings), and the correctly rounded fp32(x) lies within another half
+// ulp of x, so for |x| < 16 the two differ from t by less than 2^-19.
+// rint(fp32(x)) can only differ from rint(t) if a half-integer lies within
+// that distance of t; `near` is then set and the caller recomputes with the
+// IEEE division.  Clamping before rounding is the same as after (the bounds
+// are integers), and a clamped t is far from every half-integer that can
+// change the result (+-7.5 and beyond never do).  Rounding uses the exact
+// magic-number addition t + 1.5 * 2^23, whose fp32 result is rint(t) (ties to
+// even) in the low mantissa bits, so the nibble is read from its bit pattern
+// and no conversion instruction is needed.
+__device__ __forceinline__ uint32_t code_fast(float v, float r, bool& near) {
+  const float t = fminf(fmaxf(v * r, -8.0f), 7.0f);
+  const float yv = __fadd_rn(t, 12582912.0f);
+  const float d = __fsub_rn(t, __fsub_rn(yv, 12582912.0f));
+  near = near || (fabsf(d) >= 0.5f - 0x1p-18f);
+  return __float_as_uint(yv) & 0xFu;
+}
+
+// Kept for the general kernels: the exact code via the fast path and its check.
+__device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
+  bool near = false;
+  const uint32_t q = code_fast(v, si.r, near);
+  return near ? code_exact(v, si) : q;
 }
 
 // Load 8 consecutive elements starting at p (16-byte aligned) as fp32.
@@ -99,7 +114,7 @@ struct Load8<__half> {
   }
 };
 
-constexpr int kUnroll = 2;  // windows in flight per warp
+constexpr int kUnroll = 4;  // windows in flight per warp
 
 // Fast path: K % 8 == 0, group = 8 * LPG with LPG a power of two <= 32,
 // w 16-byte aligned, packed 4-byte aligned.  One warp window = 32 chunks of 8
@@ -143,8 +158,14 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
         if ((lane & (LPG - 1)) == 0)
           scales[row[u] * G + chunk[u] / LPG] = static_cast<uint16_t>(si.bits);
         uint32_t word = 0;
+        bool near = false;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= code_of(v[u][i], si) << (4 * i);
+        for (int i = 0; i < 8; ++i) word |= code_fast(v[u][i], si.r, near) << (4 * i);
+        if (near) {
+          word = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) word |= code_exact(v[u][i], si) << (4 * i);
+        }
         *reinterpret_cast<uint32_t*>(packed + row[u] * Kp + chunk[u] * 4) = word;
       }
     }
