@@ -10,10 +10,12 @@
 //   * a producer warp streams the CTA's 128 weight rows through a 4-stage
 //     shared-memory ring with TMA (each stage: 128 rows x 256 k = 16 KB of
 //     packed nibbles, 128-byte swizzle, plus x [M x 256] bf16/fp16), so about
-//     64 KB per CTA are in flight;
-//   * eight consumer warps own 16 rows each; per 128-wide K block a lane reads
-//     its 16 (or 2 x 8, 4 x 4 for group 64/32) bytes of two rows from shared
-//     memory and sign-extends nibble pairs to bf16/fp16 exactly in registers:
+//     64 KB per CTA are in flight, with up to three CTAs per SM;
+//   * four consumer warps own 32 rows (two 16-row tiles) each, so every x
+//     fragment feeds two independent MMA chains; per 128-wide K block a lane
+//     reads its 16 (or 2 x 8, 4 x 4 for group 64/32) bytes of four rows from
+//     shared memory and sign-extends nibble pairs to bf16/fp16 exactly in
+//     registers:
 //     byte j -> ((byte_j | byte_j >> 4 << 16) & 0x000F000F) ^ magic, then one
 //     packed subtract (magic = 128 + 8 (bf16) or 1024 + 8 (fp16) in each half,
 //     the XOR flips the nibble's sign bit so that the value is q + 136 or
@@ -23,7 +25,8 @@
 //     multiply-add runs on the CUDA cores;
 //   * each K group gets its own fp32 accumulator, which is scaled by its
 //     group's scale and added into the fp32 running sum, per the page's order.
-// All four lanes of a quad read the same group for a given word, so each MMA
+// x rows M..15 of every stage are zeroed once, so lanes of padding batch rows
+// need no predicate.  All four lanes of a quad read the same group for a given word, so each MMA
 // only sums k of one group.  Split-K: when N is small the K range is split
 // over the CTAs of a cluster (up to 8); partial sums are reduced in rank order
 // through distributed shared memory, so the result is deterministic.  Every
@@ -44,11 +47,12 @@ namespace int4lib {
 
 namespace {
 
-constexpr int kConsumers = 8;               // consumer warps, 16 weight rows each
-constexpr int kRowsPerCta = 16 * kConsumers;
+constexpr int kConsumers = 4;               // consumer warps, 2 x 16 weight rows each
+constexpr int kTiles = 2;                   // 16-row tiles per consumer warp
+constexpr int kRowsPerCta = 16 * kTiles * kConsumers;
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kSK = 2;                      // 128-wide K blocks per stage
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kMaxCluster = 8;
 constexpr int kWBytes = kRowsPerCta * kSK * 64;  // 16 KB per stage
 constexpr uint64_t kTimeoutNs = 250000000ull;
@@ -114,11 +118,6 @@ __device__ __forceinline__ int word_index(int c, int j) {
   return 4 * j + c;
 }
 
-// Byte offset of `off` (0..127) within row r of a 128-byte-swizzled W tile.
-__device__ __forceinline__ uint32_t swz(int r, int off) {
-  return static_cast<uint32_t>(r * 128 + ((((off >> 4) ^ (r & 7))) << 4) + (off & 15));
-}
-
 struct WaitCtx {
   volatile uint32_t* abort;
   uint32_t* status;
@@ -149,11 +148,12 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
 
 template <int NT>
 struct DLayout {
-  // Per stage: W tile (1024-aligned for the swizzle), then the x tile.
-  static constexpr int kXBytesMax = 16 * kSK * 128 * 2;  // M <= 16 rows
-  static constexpr int kStageBytes = kWBytes + kXBytesMax;     // multiple of 1024
+  // Per stage: W tile (1024-aligned for the swizzle), then the x tile with
+  // NT * 8 rows (rows M.. stay zero).
+  static constexpr int kXBytes = NT * 8 * kSK * 128 * 2;  // 4 KB per n-tile
+  static constexpr int kStageBytes = kWBytes + kXBytes;   // multiple of 1024
   static constexpr int offRed = kStages * kStageBytes;
-  static constexpr int kRedBytes = kConsumers * NT * 4 * 32 * 4;
+  static constexpr int kRedBytes = kConsumers * kTiles * NT * 4 * 32 * 4;
   static constexpr int offBar = offRed + kRedBytes;
   static constexpr int offMisc = offBar + 2 * kStages * 8;
   static constexpr int kBytes = offMisc + 16;
@@ -161,7 +161,7 @@ struct DLayout {
 };
 
 template <typename TX, int NT, int GPB>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
     int64_t N, int kblocks_per_slice, int S, uint32_t* status) {
@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::offBar);
   uint64_t* empty = full + kStages;
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::offMisc);
@@ -177,14 +178,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int slice = blockIdx.x;  // rank in the cluster when S > 1
-  const int64_t KB = (K + 127) / 128;
-  const int64_t kb0 = static_cast<int64_t>(slice) * kblocks_per_slice;
-  const int64_t kb1 = (kb0 + kblocks_per_slice < KB) ? kb0 + kblocks_per_slice : KB;
-  const int nst = static_cast<int>((kb1 - kb0 + kSK - 1) / kSK);
+  const int KB = static_cast<int>((K + 127) / 128);
+  const int kb0 = slice * kblocks_per_slice;
+  const int kb1 = (kb0 + kblocks_per_slice < KB) ? kb0 + kblocks_per_slice : KB;
+  const int nst = (kb1 - kb0 + kSK - 1) / kSK;
   const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kRowsPerCta;
   const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;
   const WaitCtx wc{abort_flag, status};
 
+  // x rows M.. of every stage stay zero (the copies only write M rows).
+  for (int i = threadIdx.x; i < kStages * (L::kXBytes / 16); i += blockDim.x) {
+    const int st = i / (L::kXBytes / 16);
+    const int off = (i % (L::kXBytes / 16)) * 16;
+    if (off >= M * kSK * 128 * 2)
+      ptx::sts128(sbase + st * L::kStageBytes + kWBytes + off, make_uint4(0u, 0u, 0u, 0u));
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
@@ -197,17 +205,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   }
   __syncthreads();
 
-  float tot[NT][4];
+  float tot[kTiles][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tot[nt][i] = 0.0f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tot[t][nt][i] = 0.0f;
 
   const int c = lane & 3;
   const int g = lane >> 2;
-  const int cw = warp - 1;                       // consumer index
-  const int64_t ra = row0 + cw * 16 + g;
-  const int64_t rb = ra + 8;
+  const int cw = warp - 1;  // consumer index
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -216,13 +224,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
       for (; it < nst; ++it) {
         const int s = it % kStages;
         if (!wait_bar(ptx::smem_u32(&empty[s]), ((it / kStages) & 1) ^ 1u, wc)) break;
-        uint8_t* st = smem + s * L::kStageBytes;
-        const int64_t kb = kb0 + static_cast<int64_t>(it) * kSK;
+        const uint32_t st = sbase + s * L::kStageBytes;
+        const int kb = kb0 + it * kSK;
         ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + xbytes);
-        ptx::tma_load_2d(ptx::smem_u32(st), &tm_w, static_cast<int32_t>(kb * 64),
-                         static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
-        ptx::tma_load_2d(ptx::smem_u32(st + kWBytes), &tm_x, static_cast<int32_t>(kb * 128), 0,
-                         ptx::smem_u32(&full[s]));
+        ptx::tma_load_2d(st, &tm_w, kb * 64, static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
+        ptx::tma_load_2d(st + kWBytes, &tm_x, kb * 128, 0, ptx::smem_u32(&full[s]));
       }
       if (*abort_flag) {
         const int first = it - kStages > 0 ? it - kStages : 0;
@@ -231,75 +237,104 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     }
   } else {
     // ---------------- consumers ----------------
-    const bool va = ra < N, vb = rb < N;
-    const uint16_t* sra = scales + (va ? ra : 0) * G;
-    const uint16_t* srb = scales + (vb ? rb : 0) * G;
-    const int la = cw * 16 + g, lb = la + 8;      // rows within the W tile
+    // Rows of this lane within the W tile: tile t covers rows cw*32 + 16t .. +15.
+    int lr[kTiles][2];
+    const uint16_t* sp[kTiles][2];
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        lr[t][h] = cw * 16 * kTiles + 16 * t + g + 8 * h;
+        int64_t r = row0 + lr[t][h];
+        if (r >= N) r = N - 1;  // never written; keeps the scale load in bounds
+        sp[t][h] = scales + r * G;
+      }
+    const int bpg = group / 128;  // K blocks per group when GPB == 1
     for (int it = 0; it < nst; ++it) {
       const int s = it % kStages;
       if (!wait_bar(ptx::smem_u32(&full[s]), (it / kStages) & 1, wc)) break;
-      const uint8_t* wt = smem + s * L::kStageBytes;
-      const uint8_t* xt = wt + kWBytes;
+      const uint32_t wt = sbase + s * L::kStageBytes;
+      const uint32_t xt = wt + kWBytes;
 #pragma unroll
       for (int b = 0; b < kSK; ++b) {
-        const int64_t kb = kb0 + static_cast<int64_t>(it) * kSK + b;
+        const int kb = kb0 + it * kSK + b;
         if (kb >= kb1) break;
-        float acc[GPB][NT][4];
+        // This lane's four 8-k words of each of its rows in block b.
+        uint32_t wv[kTiles][2][4];
 #pragma unroll
-        for (int a = 0; a < GPB; ++a)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[a][nt][i] = 0.0f;
-        uint32_t wa[4], wb[4];
-        if (GPB == 1) {
-          const uint4 u = *reinterpret_cast<const uint4*>(wt + swz(la, b * 64 + 16 * c));
-          const uint4 v = *reinterpret_cast<const uint4*>(wt + swz(lb, b * 64 + 16 * c));
-          wa[0] = u.x; wa[1] = u.y; wa[2] = u.z; wa[3] = u.w;
-          wb[0] = v.x; wb[1] = v.y; wb[2] = v.z; wb[3] = v.w;
-        } else if (GPB == 2) {
+        for (int t = 0; t < kTiles; ++t)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const uint2 u = *reinterpret_cast<const uint2*>(wt + swz(la, b * 64 + 32 * h + 8 * c));
-            const uint2 v = *reinterpret_cast<const uint2*>(wt + swz(lb, b * 64 + 32 * h + 8 * c));
-            wa[2 * h] = u.x; wa[2 * h + 1] = u.y;
-            wb[2 * h] = v.x; wb[2 * h + 1] = v.y;
-          }
-        } else {
+            const int r = lr[t][h];
+            const uint32_t rb = wt + r * 128;
+            const int sw = r & 7;
+            if (GPB == 1) {
+              const uint4 u = ptx::lds128(rb + ((((b * 64 + 16 * c) >> 4) ^ sw) << 4));
+              wv[t][h][0] = u.x; wv[t][h][1] = u.y; wv[t][h][2] = u.z; wv[t][h][3] = u.w;
+            } else if (GPB == 2) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            wa[j] = *reinterpret_cast<const uint32_t*>(wt + swz(la, b * 64 + 16 * j + 4 * c));
-            wb[j] = *reinterpret_cast<const uint32_t*>(wt + swz(lb, b * 64 + 16 * j + 4 * c));
+              for (int q = 0; q < 2; ++q) {
+                const int off = b * 64 + 32 * q + 8 * c;
+                const uint2 u = ptx::lds64(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
+                wv[t][h][2 * q] = u.x; wv[t][h][2 * q + 1] = u.y;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int off = b * 64 + 16 * j + 4 * c;
+                wv[t][h][j] = ptx::lds32(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
+              }
+            }
           }
-        }
+        float acc[kTiles][NT][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          uint32_t pa[4], pb[4];
-          expand<TX>(wa[j], pa);
-          expand<TX>(wb[j], pb);
-          const int a = (GPB == 1) ? 0 : (GPB == 2 ? (j >> 1) : j);
-          const int kx = b * 128 + 8 * word_index<GPB>(c, j);
+          // Group a of word j; the accumulator restarts at the group's first word.
+          const bool first = (GPB == 1) ? (j == 0) : (GPB == 2 ? (j % 2 == 0) : true);
+          const bool last = (GPB == 1) ? (j == 3) : (GPB == 2 ? (j % 2 == 1) : true);
+          if (first) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int m = nt * 8 + g;
-            uint4 xf = make_uint4(0u, 0u, 0u, 0u);
-            if (m < M) xf = *reinterpret_cast<const uint4*>(xt + (m * kSK * 128 + kx) * 2);
-            Cvt<TX>::mma(acc[a][nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
-            Cvt<TX>::mma(acc[a][nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
+            for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[t][nt][i] = 0.0f;
           }
-        }
-        const int64_t kbase = kb * 128;
+          const int kx = b * 128 + 8 * word_index<GPB>(c, j);
+          uint4 xf[NT];
 #pragma unroll
-        for (int a = 0; a < GPB; ++a) {
-          const int64_t gi = (kbase + a * (128 / GPB)) / group;
-          const float sa = (va && gi < G) ? f16_bits_to_float(__ldg(sra + gi)) : 0.0f;
-          const float sb = (vb && gi < G) ? f16_bits_to_float(__ldg(srb + gi)) : 0.0f;
+          for (int nt = 0; nt < NT; ++nt) xf[nt] = ptx::lds128(xt + ((nt * 8 + g) * kSK * 128 + kx) * 2);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            tot[nt][0] = fmaf(acc[a][nt][0], sa, tot[nt][0]);
-            tot[nt][1] = fmaf(acc[a][nt][1], sa, tot[nt][1]);
-            tot[nt][2] = fmaf(acc[a][nt][2], sb, tot[nt][2]);
-            tot[nt][3] = fmaf(acc[a][nt][3], sb, tot[nt][3]);
+          for (int t = 0; t < kTiles; ++t) {
+            uint32_t pa[4], pb[4];
+            expand<TX>(wv[t][0][j], pa);
+            expand<TX>(wv[t][1][j], pb);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              Cvt<TX>::mma(acc[t][nt], pa[0], pb[0], pa[1], pb[1], xf[nt].x, xf[nt].y);
+              Cvt<TX>::mma(acc[t][nt], pa[2], pb[2], pa[3], pb[3], xf[nt].z, xf[nt].w);
+            }
+          }
+          if (last) {
+            int gi;
+            if (GPB == 1) gi = (bpg == 1) ? kb : kb / bpg;
+            else gi = kb * GPB + (GPB == 2 ? (j >> 1) : j);
+            const bool gok = gi < G;
+            const int gc = gok ? gi : 0;
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+              float sa = f16_bits_to_float(__ldg(sp[t][0] + gc));
+              float sb = f16_bits_to_float(__ldg(sp[t][1] + gc));
+              sa = gok ? sa : 0.0f;
+              sb = gok ? sb : 0.0f;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                tot[t][nt][0] = fmaf(acc[t][nt][0], sa, tot[t][nt][0]);
+                tot[t][nt][1] = fmaf(acc[t][nt][1], sa, tot[t][nt][1]);
+                tot[t][nt][2] = fmaf(acc[t][nt][2], sb, tot[t][nt][2]);
+                tot[t][nt][3] = fmaf(acc[t][nt][3], sb, tot[t][nt][3]);
+              }
+            }
           }
         }
       }
@@ -309,18 +344,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   }
 
   const bool ok = (*abort_flag == 0u);
-  // Output (m, row) of register i of n-tile nt: m = nt*8 + 2c + (i & 1),
-  // row = (i < 2) ? ra : rb.
+  // Output (m, row) of register i of tile t, n-tile nt: m = nt*8 + 2c + (i & 1),
+  // row = row0 + cw*32 + 16t + g + ((i < 2) ? 0 : 8).
   if (S == 1) {
     if (warp > 0 && ok) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = nt * 8 + 2 * c + (i & 1);
-          const int64_t row = (i < 2) ? ra : rb;
-          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = tot[nt][i];
-        }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int m = nt * 8 + 2 * c + (i & 1);
+            const int64_t row = row0 + cw * 16 * kTiles + 16 * t + g + ((i < 2) ? 0 : 8);
+            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = tot[t][nt][i];
+          }
     }
     return;
   }
@@ -328,25 +365,28 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   // Split-K: partials to shared memory, reduced across the cluster in rank order.
   if (warp > 0) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) red[((cw * NT + nt) * 4 + i) * 32 + lane] = tot[nt][i];
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          red[(((cw * kTiles + t) * NT + nt) * 4 + i) * 32 + lane] = tot[t][nt][i];
   }
   cg::cluster_group cluster = cg::this_cluster();
   cluster.sync();
-  const int total = kConsumers * NT * 4 * 32;
+  bool all_ok = true;
+  for (int r = 0; r < S; ++r)
+    all_ok = all_ok && (*cluster.map_shared_rank(const_cast<uint32_t*>(abort_flag), r) == 0u);
+  const int total = kConsumers * kTiles * NT * 4 * 32;
   for (int e = slice * blockDim.x + threadIdx.x; e < total; e += S * blockDim.x) {
     float sum = 0.0f;
-    bool all_ok = ok;
     for (int r = 0; r < S; ++r) sum += cluster.map_shared_rank(red, r)[e];
-    for (int r = 0; r < S; ++r)
-      all_ok = all_ok && (*cluster.map_shared_rank(const_cast<uint32_t*>(abort_flag), r) == 0u);
     const int ln = e & 31;
     const int i = (e >> 5) & 3;
     const int nt = (e >> 7) % NT;
-    const int wp = (e >> 7) / NT;
+    const int tw = (e >> 7) / NT;  // cw * kTiles + t
     const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
-    const int64_t row = row0 + wp * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
+    const int64_t row = row0 + tw * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
     if (all_ok && m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
   }
   cluster.sync();  // keep this CTA's partials alive until every rank has read them
@@ -381,8 +421,15 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
   const int G = static_cast<int>((K + group - 1) / group);
   const int64_t KB = (K + 127) / 128;
   const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
-  // One wave of CTAs (two per SM), at most 8 K slices per cluster.
-  const int64_t slots = 2LL * num_sms();
+  auto kern = decode_kernel<TX, NT, GPB>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  // One wave of CTAs at the occupancy limit, at most 8 K slices per cluster.
+  const int64_t slots = static_cast<int64_t>(occ) * num_sms();
   int64_t S = slots / R;
   if (S > kMaxCluster) S = kMaxCluster;
   if (S > KB) S = KB;
@@ -414,9 +461,6 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = decode_kernel<TX, NT, GPB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(R), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

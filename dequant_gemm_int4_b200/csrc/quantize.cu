@@ -24,20 +24,42 @@ namespace {
 struct ScaleInfo {
   uint32_t bits;  // fp16 bit pattern of the scale
   float sf;       // the scale widened to fp32
-  float r;        // fp32(1 / sf), or 0 when sf is 0 (or +inf)
+  float r;        // approximately 1 / sf (0 when sf is 0 or +inf)
 };
+
+// fp32(m / 7), correctly rounded, for finite m >= 0.  Division by a constant
+// with one residual correction (Markstein's method for a known divisor):
+// q0 = m * c with c = fp32(1/7), the residual e = m - 7 q0 is exact by FMA,
+// and q1 = q0 + e * c is the correctly rounded quotient.  The test suite
+// checks it against the IEEE division for every fp32 mantissa over the
+// normal exponents whose behaviour differs, and over the whole subnormal
+// range.
+__device__ __forceinline__ float div7_rn(float m) {
+  const float c = 0.142857149f;  // fp32 nearest to 1/7
+  const float q0 = __fmul_rn(m, c);
+  const float e = __fmaf_rn(-7.0f, q0, m);
+  return __fmaf_rn(e, c, q0);
+}
+
+// Hardware reciprocal approximation (relative error about 2^-23); only the
+// fast-path quotient uses it, which the certified check in code_fast covers.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 __device__ __forceinline__ ScaleInfo scale_from_bits(uint32_t bits) {
   ScaleInfo si;
   si.bits = bits;
   si.sf = f16_bits_to_float(bits);
-  si.r = (si.sf == 0.0f) ? 0.0f : __fdiv_rn(1.0f, si.sf);
+  si.r = (si.sf == 0.0f || bits == 0x7C00u) ? 0.0f : rcp_approx(si.sf);
   return si;
 }
 
-// s = fp16_RNE(fp32(m) / 7), with the IEEE-exact division.
+// s = fp16_RNE(fp32(m) / 7): the correctly rounded fp32 quotient, then RNE to fp16.
 __device__ __forceinline__ ScaleInfo scale_from_absmax(float m) {
-  const __half h = __float2half_rn(__fdiv_rn(m, 7.0f));
+  const __half h = __float2half_rn(div7_rn(m));
   return scale_from_bits(__half_as_ushort(h));
 }
 
@@ -51,26 +73,26 @@ __device__ __forceinline__ uint32_t code_exact(float v, const ScaleInfo& si) {
 }
 
 // Fast path of the same code.  The quotient is approximated as t = v * r
-// with r = fp32(1/sf).  With x the exact quotient, |t - x| <= |x| * 2^-23
-// (two roundings), and the correctly rounded fp32(x) lies within another half
-// ulp of x, so for |x| < 16 the two differ from t by less than 2^-19.
-// rint(fp32(x)) can only differ from rint(t) if a half-integer lies within
-// that distance of t; `near` is then set and the caller recomputes with the
-// IEEE division.  Clamping before rounding is the same as after (the bounds
-// are integers), and a clamped t is far from every half-integer that can
-// change the result (+-7.5 and beyond never do).  Rounding uses the exact
-// magic-number addition t + 1.5 * 2^23, whose fp32 result is rint(t) (ties to
-// even) in the low mantissa bits, so the nibble is read from its bit pattern
-// and no conversion instruction is needed.
+// with r within 2^-22 (relative) of 1/sf.  With x the exact quotient,
+// |t - x| <= |x| * 2^-21, and the correctly rounded fp32(x) lies within
+// another half ulp of x, so for |x| < 16 both differ from t by less than
+// 2^-16.  rint(fp32(x)) can only differ from rint(t) if a half-integer lies
+// within that distance of t; `near` is then set and the caller recomputes
+// with the IEEE division.  Clamping before rounding is the same as after
+// (the bounds are integers), and a clamped t is far from every half-integer
+// that can change the result (+-7.5 and beyond never do).  Rounding uses the
+// exact magic-number addition t + 1.5 * 2^23, whose fp32 result holds rint(t)
+// (ties to even) in its low mantissa bits, so the nibble is read from the bit
+// pattern and no conversion instruction is needed.
 __device__ __forceinline__ uint32_t code_fast(float v, float r, bool& near) {
-  const float t = fminf(fmaxf(v * r, -8.0f), 7.0f);
+  const float t = fminf(fmaxf(__fmul_rn(v, r), -8.0f), 7.0f);
   const float yv = __fadd_rn(t, 12582912.0f);
   const float d = __fsub_rn(t, __fsub_rn(yv, 12582912.0f));
-  near = near || (fabsf(d) >= 0.5f - 0x1p-18f);
+  near = near || (fabsf(d) >= 0.5f - 0x1p-15f);
   return __float_as_uint(yv) & 0xFu;
 }
 
-// Kept for the general kernels: the exact code via the fast path and its check.
+// The exact code, via the fast path and its check (general kernels).
 __device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
   bool near = false;
   const uint32_t q = code_fast(v, si.r, near);
@@ -118,32 +140,45 @@ constexpr int kUnroll = 4;  // windows in flight per warp
 
 // Fast path: K % 8 == 0, group = 8 * LPG with LPG a power of two <= 32,
 // w 16-byte aligned, packed 4-byte aligned.  One warp window = 32 chunks of 8
-// elements of one row; windows are numbered row-major over (row, window).
+// elements of one row.  Windows are numbered row-major over (row, window);
+// each warp takes a contiguous range of them, so the row and window of the
+// next one follow by increment (no division in the loop).
 template <typename T, int LPG>
 __global__ void __launch_bounds__(256) quantize_aligned_kernel(
     const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
     uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t chunks_per_row = K >> 3;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  int64_t wbeg = warp * per;
+  const int64_t wend = (wbeg + per < total_windows) ? wbeg + per : total_windows;
+  if (wbeg >= wend) return;
+  const int chunks_per_row = static_cast<int>(K >> 3);
   const int64_t Kp = K >> 1;
+  int64_t row = wbeg / windows_per_row;
+  int col = static_cast<int>(wbeg - row * windows_per_row);
+  const int wpr = static_cast<int>(windows_per_row);
 
-  for (int64_t base = warp0; base < total_windows; base += nwarps * kUnroll) {
+  for (; wbeg < wend; wbeg += kUnroll) {
     float v[kUnroll][8];
-    int64_t row[kUnroll], chunk[kUnroll];
+    int64_t rw[kUnroll];
+    int ch[kUnroll];
     bool valid[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t wi = base + u * nwarps;
-      row[u] = wi / windows_per_row;
-      chunk[u] = (wi - row[u] * windows_per_row) * 32 + lane;
-      valid[u] = (wi < total_windows) && (chunk[u] < chunks_per_row);
+      rw[u] = row;
+      ch[u] = col * 32 + lane;
+      valid[u] = (wbeg + u < wend) && (ch[u] < chunks_per_row);
       if (valid[u]) {
-        Load8<T>::run(w + row[u] * K + chunk[u] * 8, v[u]);
+        Load8<T>::run(w + row * K + static_cast<int64_t>(ch[u]) * 8, v[u]);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[u][i] = 0.0f;
+      }
+      if (++col == wpr) {
+        col = 0;
+        ++row;
       }
     }
 #pragma unroll
@@ -154,19 +189,20 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
 #pragma unroll
       for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       const ScaleInfo si = scale_from_absmax(m);
-      if (valid[u]) {
-        if ((lane & (LPG - 1)) == 0)
-          scales[row[u] * G + chunk[u] / LPG] = static_cast<uint16_t>(si.bits);
-        uint32_t word = 0;
-        bool near = false;
+      uint32_t word = 0;
+      bool near = false;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= code_fast(v[u][i], si.r, near) << (4 * i);
+      for (int i = 0; i < 8; ++i) word |= code_fast(v[u][i], si.r, near) << (4 * i);
+      if (__any_sync(0xffffffffu, near)) {
         if (near) {
           word = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) word |= code_exact(v[u][i], si) << (4 * i);
         }
-        *reinterpret_cast<uint32_t*>(packed + row[u] * Kp + chunk[u] * 4) = word;
+      }
+      if (valid[u]) {
+        if ((lane & (LPG - 1)) == 0) scales[rw[u] * G + ch[u] / LPG] = static_cast<uint16_t>(si.bits);
+        *reinterpret_cast<uint32_t*>(packed + rw[u] * Kp + static_cast<int64_t>(ch[u]) * 4) = word;
       }
     }
   }
@@ -228,7 +264,7 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
   if (aligned && pow2_group) {
     const int64_t wpr = (K / 8 + 31) / 32;
     const int64_t total = N * wpr;
-    const int grid = grid_for(total, 8 * kUnroll, 16);
+    const int grid = grid_for(total, 8 * kUnroll, 8);
     switch (lpg) {
 #define INT4_Q_CASE(L)                                                                       \
   case L:                                                                                    \

@@ -143,6 +143,30 @@ def test_quantize_bulk_full_size_sampled_rows(N, K, group):
     assert np.array_equal(q[torch.as_tensor(rows, device=DEV)].cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("exponents", [(0,), (-124, -125, -126), ("subnormal",), (15, 16)])
+def test_scale_division_exhaustive_over_mantissas(exponents):
+    """fp16(fp32(m / 7)) on every fp32 mantissa of the given binades (and on
+    every subnormal): the kernel's division by the constant 7 must equal the
+    IEEE division the oracle uses, bit for bit.  Group 1 makes every element
+    its own group, so each one yields a scale."""
+    mant = np.arange(1 << 23, dtype=np.uint32)
+    parts = []
+    for e in exponents:
+        if e == "subnormal":
+            parts.append(mant.view(np.float32))
+        else:
+            parts.append(((np.uint32(e + 127) << 23) | mant).view(np.float32))
+    m = np.concatenate(parts).reshape(1, -1)
+    w = torch.from_numpy(m).to(DEV)
+    packed, scales, K = q4.quantize_int4(w, 1)
+    got = scales.cpu().view(torch.int16).numpy().view(np.uint16)[0]
+    p_ref, s_ref, _ = oracle.quantize_int4(m, 1)
+    want = s_ref.view(np.uint16)[0]
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, f"{bad.size} scales differ, first m = {m[0, bad[0]]!r}"
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+
+
 def test_quantize_unaligned_pointers_take_the_general_path():
     base = make_weights(8, 1025, seed=3, device=DEV, dtype=torch.bfloat16).reshape(-1)
     w = base[1:1 + 8 * 1024].view(8, 1024)     # 2-byte aligned only
