@@ -47,14 +47,21 @@ namespace int4lib {
 
 namespace {
 
-constexpr int kConsumers = 4;               // consumer warps, 2 x 16 weight rows each
-constexpr int kTiles = 2;                   // 16-row tiles per consumer warp
-constexpr int kRowsPerCta = 16 * kTiles * kConsumers;
-constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kSK = 2;                      // 128-wide K blocks per stage
+constexpr int kRowGroups = 4;               // row groups per CTA
+constexpr int kConsumers = kRowGroups * kSK;  // one consumer warp per (row group, block of the stage)
+constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = 3;
 constexpr int kMaxCluster = 8;
-constexpr int kWBytes = kRowsPerCta * kSK * 64;  // 16 KB per stage
+
+// 16-row tiles per consumer warp: two for M <= 8 (NT = 1), one for M <= 16,
+// so that both fit two CTAs per SM without spilling.
+template <int NT>
+struct Tiles {
+  static constexpr int kTiles = NT == 1 ? 2 : 1;
+  static constexpr int kRowsPerCta = 16 * kTiles * kRowGroups;  // 128 or 64
+  static constexpr int kWBytes = kRowsPerCta * kSK * 64;          // 16 or 8 KB per stage
+};
 constexpr uint64_t kTimeoutNs = 250000000ull;
 
 template <typename TX>
@@ -127,8 +134,8 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t i = 1; i != 0; ++i) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((i & 127u) == 0u) {
+    if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 15u) == 0u) {
       if (*w.abort) return false;
       if (ptx::globaltimer() - t0 > kTimeoutNs) break;
     }
@@ -148,6 +155,8 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
 
 template <int NT>
 struct DLayout {
+  static constexpr int kTiles = Tiles<NT>::kTiles;
+  static constexpr int kWBytes = Tiles<NT>::kWBytes;
   // Per stage: W tile (1024-aligned for the swizzle), then the x tile with
   // NT * 8 rows (rows M.. stay zero).
   static constexpr int kXBytes = NT * 8 * kSK * 128 * 2;  // 4 KB per n-tile
@@ -161,11 +170,14 @@ struct DLayout {
 };
 
 template <typename TX, int NT, int GPB>
-__global__ void __launch_bounds__(kThreads, 3) decode_kernel(
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
     int64_t N, int kblocks_per_slice, int S, uint32_t* status) {
   using L = DLayout<NT>;
+  constexpr int kTiles = Tiles<NT>::kTiles;
+  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
+  constexpr int kWBytes = Tiles<NT>::kWBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -215,7 +227,9 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(
 
   const int c = lane & 3;
   const int g = lane >> 2;
-  const int cw = warp - 1;  // consumer index
+  const int cw = warp - 1;          // consumer index
+  const int rg = cw % kRowGroups;   // 32-row group of this consumer
+  const int bs = cw / kRowGroups;   // which K block of each stage it takes
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(
     for (int t = 0; t < kTiles; ++t)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        lr[t][h] = cw * 16 * kTiles + 16 * t + g + 8 * h;
+        lr[t][h] = rg * 16 * kTiles + 16 * t + g + 8 * h;
         int64_t r = row0 + lr[t][h];
         if (r >= N) r = N - 1;  // never written; keeps the scale load in bounds
         sp[t][h] = scales + r * G;
@@ -255,10 +269,10 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(
       if (!wait_bar(ptx::smem_u32(&full[s]), (it / kStages) & 1, wc)) break;
       const uint32_t wt = sbase + s * L::kStageBytes;
       const uint32_t xt = wt + kWBytes;
-#pragma unroll
-      for (int b = 0; b < kSK; ++b) {
+      {
+        const int b = bs;
         const int kb = kb0 + it * kSK + b;
-        if (kb >= kb1) break;
+        if (kb < kb1) {
         // This lane's four 8-k words of each of its rows in block b.
         uint32_t wv[kTiles][2][4];
 #pragma unroll
@@ -338,31 +352,14 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(
           }
         }
       }
+        }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
     }
   }
 
-  const bool ok = (*abort_flag == 0u);
-  // Output (m, row) of register i of tile t, n-tile nt: m = nt*8 + 2c + (i & 1),
-  // row = row0 + cw*32 + 16t + g + ((i < 2) ? 0 : 8).
-  if (S == 1) {
-    if (warp > 0 && ok) {
-#pragma unroll
-      for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int m = nt * 8 + 2 * c + (i & 1);
-            const int64_t row = row0 + cw * 16 * kTiles + 16 * t + g + ((i < 2) ? 0 : 8);
-            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = tot[t][nt][i];
-          }
-    }
-    return;
-  }
-
-  // Split-K: partials to shared memory, reduced across the cluster in rank order.
+  // Partials of every consumer to shared memory; each output is the sum over
+  // the CTA's two K-block slots (and over the cluster's ranks), in a fixed order.
   if (warp > 0) {
 #pragma unroll
     for (int t = 0; t < kTiles; ++t)
@@ -372,19 +369,41 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(
         for (int i = 0; i < 4; ++i)
           red[(((cw * kTiles + t) * NT + nt) * 4 + i) * 32 + lane] = tot[t][nt][i];
   }
+  constexpr int kPer = kRowGroups * kTiles * NT * 4 * 32;  // outputs per CTA
+  if (S == 1) {
+    __syncthreads();
+    if (*abort_flag == 0u) {
+      for (int e = threadIdx.x; e < kPer; e += blockDim.x) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kSK; ++q) sum += red[q * kPer + e];
+        const int ln = e & 31;
+        const int i = (e >> 5) & 3;
+        const int nt = (e >> 7) % NT;
+        const int tw = (e >> 7) / NT;  // rg * kTiles + t
+        const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
+        const int64_t row = row0 + tw * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
+        if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+      }
+    }
+    return;
+  }
   cg::cluster_group cluster = cg::this_cluster();
   cluster.sync();
   bool all_ok = true;
   for (int r = 0; r < S; ++r)
     all_ok = all_ok && (*cluster.map_shared_rank(const_cast<uint32_t*>(abort_flag), r) == 0u);
-  const int total = kConsumers * kTiles * NT * 4 * 32;
-  for (int e = slice * blockDim.x + threadIdx.x; e < total; e += S * blockDim.x) {
+  for (int e = slice * blockDim.x + threadIdx.x; e < kPer; e += S * blockDim.x) {
     float sum = 0.0f;
-    for (int r = 0; r < S; ++r) sum += cluster.map_shared_rank(red, r)[e];
+    for (int r = 0; r < S; ++r) {
+      const float* rr = cluster.map_shared_rank(red, r);
+#pragma unroll
+      for (int q = 0; q < kSK; ++q) sum += rr[q * kPer + e];
+    }
     const int ln = e & 31;
     const int i = (e >> 5) & 3;
     const int nt = (e >> 7) % NT;
-    const int tw = (e >> 7) / NT;  // cw * kTiles + t
+    const int tw = (e >> 7) / NT;
     const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
     const int64_t row = row0 + tw * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
     if (all_ok && m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
@@ -414,6 +433,7 @@ template <typename TX, int NT, int GPB>
 cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                            int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
   using L = DLayout<NT>;
+  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   uint32_t* status = status_word();
@@ -502,7 +522,7 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
   if (!(group == 32 || group == 64 || group % 128 == 0)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return false;
   if (reinterpret_cast<uintptr_t>(packed) % 16 != 0) return false;
-  if ((N + kRowsPerCta - 1) / kRowsPerCta > 65535) return false;
+  if ((N + 63) / 64 > 65535) return false;
   return true;
 }
 

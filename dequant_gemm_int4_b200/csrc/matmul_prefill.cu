@@ -124,8 +124,8 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Wa
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t i = 1; i != 0; ++i) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((i & 127u) == 0u) {
+    if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 15u) == 0u) {
       if (*w.abort) return false;
       if (ptx::globaltimer() - t0 > kTimeoutNs) break;
     }
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const WaitCtx wc{abort_flag, status};
 
   if (warp < 4) {
-    ptx::regs_dec<40>();
+    ptx::regs_dec<24>();
     if (warp == 0 && lane == 0) {
       // ---------------- TMA producer ----------------
       int it = 0;
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       }
     }
   } else if (warp < 8) {
-    ptx::regs_dec<88>();
+    ptx::regs_dec<72>();
     // ---------------- dequantizers: thread t owns weight row t ----------------
     const int t = threadIdx.x - 128;
     const int swz = t & 7;
@@ -259,21 +259,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
       if (!wait_bar(bar(&bars->full_tma[s]), ph, wc)) break;
-      const uint8_t* prow = smem + L::offP + s * L::kP + t * 32;
-      const uint4 va = *reinterpret_cast<const uint4*>(prow + 16 * first);
-      const uint4 vb = *reinterpret_cast<const uint4*>(prow + 16 * (first ^ 1));
+      const uint32_t prow = sP + s * L::kP + t * 32;
+      const uint4 va = ptx::lds128(prow + 16 * first);
+      const uint4 vb = ptx::lds128(prow + 16 * (first ^ 1));
       const uint4 lo = first ? vb : va;
       const uint4 hi = first ? va : vb;
       const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-      uint8_t* arow = smem + L::offA + s * L::kA + t * 128;
+      const uint32_t arow = sA + s * L::kA + t * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(arow + ((c ^ swz) << 4)) = expand8<TX>(wds[c]);
+      for (int c = 0; c < 8; ++c) ptx::sts128(arow + ((c ^ swz) << 4), expand8<TX>(wds[c]));
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(bar(&bars->full_a[s]));
     }
   } else {
-    ptx::regs_inc<192>();
+    ptx::regs_inc<208>();
     // ---------------- epilogue: lane quarter q, column half h ----------------
     const int q = warp & 3;
     const int h = (warp - 8) >> 2;

@@ -92,6 +92,34 @@ __device__ __forceinline__ uint32_t code_fast(float v, float r, bool& near) {
   return __float_as_uint(yv) & 0xFu;
 }
 
+// Eight codes of one lane for a normal fp16 scale (2^-14 <= s < +inf), packed
+// low nibble first.  Then |v / s| <= 7 / (1 - 2^-11) < 7.5, so no clamp is
+// needed, and t = v * r stays within 2^-16 of the exact quotient (see
+// code_fast).  Returns false if some quotient lies too close to a
+// half-integer, in which case the caller recomputes exactly.
+__device__ __forceinline__ bool codes8_normal(const float (&v)[8], float r, uint32_t& word) {
+  float dmax = 0.0f;
+  uint32_t nib[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float t = __fmul_rn(v[i], r);
+    const float yv = __fadd_rn(t, 12582912.0f);
+    const float d = __fsub_rn(t, __fsub_rn(yv, 12582912.0f));
+    dmax = fmaxf(dmax, fabsf(d));
+    nib[i] = __float_as_uint(yv);
+  }
+  // Two nibbles per byte, four bytes per word.
+  uint32_t b[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t o;
+    asm("lop3.b32 %0, %1, %2, %3, 0xb8;" : "=r"(o) : "r"(nib[2 * j + 1] << 4), "r"(0x0Fu), "r"(nib[2 * j]));
+    b[j] = o;  // (hi << 4 & ~0x0F) | (lo & 0x0F): byte 0 holds both nibbles
+  }
+  word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  return dmax < 0.5f - 0x1p-15f;
+}
+
 // The exact code, via the fast path and its check (general kernels).
 __device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
   bool near = false;
@@ -189,12 +217,15 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
 #pragma unroll
       for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       const ScaleInfo si = scale_from_absmax(m);
-      uint32_t word = 0;
-      bool near = false;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) word |= code_fast(v[u][i], si.r, near) << (4 * i);
-      if (__any_sync(0xffffffffu, near)) {
-        if (near) {
+      // Normal scale (exponent field neither 0 nor all ones) or zero scale
+      // (r == 0 makes every code 0) take the fast path; subnormal and
+      // infinite scales (rare) go to the exact path.
+      const uint32_t ex = si.bits & 0x7C00u;
+      const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
+      uint32_t word;
+      const bool ok = codes8_normal(v[u], si.r, word) && simple;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (!ok) {
           word = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) word |= code_exact(v[u][i], si) << (4 * i);
