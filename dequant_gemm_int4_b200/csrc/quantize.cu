@@ -16,6 +16,7 @@
 // group/8 lanes of each group, and stores 4 packed bytes per lane.
 #include "common.cuh"
 #include "internal.h"
+#include "realign.cuh"
 
 namespace int4lib {
 
@@ -239,6 +240,89 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
   }
 }
 
+// Rows at any alignment (odd K, unaligned pointers), same groups as the fast
+// path.  The weights are read as aligned 16-byte chunks of the byte range that
+// starts at `wbase` (16-byte aligned, w[0,0] at byte `wshift`): a lane loads
+// its chunk(s), takes the next lane's first chunk by shuffle and funnel-shifts
+// by the row's byte offset, which is the same for every lane of the window.
+// Packed bytes are written as aligned words with store_segment.
+template <typename T, int LPG>
+__global__ void __launch_bounds__(256) quantize_any_kernel(
+    const uint8_t* __restrict__ wbase, int64_t wshift, int64_t wbytes, int64_t K, int G,
+    int64_t windows_per_row, int64_t total_windows, uint8_t* __restrict__ pbase, int64_t pshift,
+    uint16_t* __restrict__ scales) {
+  constexpr int ELT = static_cast<int>(sizeof(T));
+  constexpr int NCH = ELT == 4 ? 2 : 1;  // 16-byte chunks per lane (8 elements)
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  int64_t wi = warp * per;
+  const int64_t wend = (wi + per < total_windows) ? wi + per : total_windows;
+  if (wi >= wend) return;
+  const int64_t Kp = (K + 1) >> 1;
+  int64_t row = wi / windows_per_row;
+  int64_t col = wi - row * windows_per_row;
+
+  for (; wi < wend; ++wi) {
+    const int64_t kl = col * 256 + lane * 8;  // first element of this lane in the row
+    const int64_t P = wshift + (row * K + kl) * ELT;
+    const int64_t c0 = P >> 4;
+    const int boff = static_cast<int>(P & 15);
+    uint32_t win[4 * (NCH + 1)];
+#pragma unroll
+    for (int q = 0; q < NCH; ++q) {
+      const uint4 v = load_chunk16(wbase, c0 + q, wbytes);
+      win[4 * q] = v.x; win[4 * q + 1] = v.y; win[4 * q + 2] = v.z; win[4 * q + 3] = v.w;
+    }
+    uint4 nx;
+    nx.x = __shfl_down_sync(0xffffffffu, win[0], 1);
+    nx.y = __shfl_down_sync(0xffffffffu, win[1], 1);
+    nx.z = __shfl_down_sync(0xffffffffu, win[2], 1);
+    nx.w = __shfl_down_sync(0xffffffffu, win[3], 1);
+    if (lane == 31) nx = load_chunk16(wbase, c0 + NCH, wbytes);
+    win[4 * NCH] = nx.x; win[4 * NCH + 1] = nx.y; win[4 * NCH + 2] = nx.z; win[4 * NCH + 3] = nx.w;
+    uint32_t e[4 * NCH];
+    byte_shift_words<4 * (NCH + 1), 4 * NCH>(win, boff, e);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float f;
+      if (ELT == 4) f = __uint_as_float(e[i]);
+      else if (std::is_same<T, __nv_bfloat16>::value) f = __uint_as_float((i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16));
+      else f = f16_bits_to_float((i & 1) ? (e[i >> 1] >> 16) : (e[i >> 1] & 0xFFFFu));
+      v[i] = (kl + i < K) ? f : 0.0f;
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+    for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const ScaleInfo si = scale_from_absmax(m);
+    const uint32_t ex = si.bits & 0x7C00u;
+    const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
+    uint32_t word;
+    const bool ok = codes8_normal(v, si.r, word) && simple;
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (!ok) {
+        word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= code_exact(v[i], si) << (4 * i);
+      }
+    }
+    if (kl < K && (lane & (LPG - 1)) == 0) scales[row * G + kl / (8 * LPG)] = static_cast<uint16_t>(si.bits);
+    const int64_t rowp = pshift + row * Kp;
+    const int64_t f0 = rowp + col * 128;
+    const int64_t hi = (f0 + 128 < rowp + Kp) ? f0 + 128 : rowp + Kp;
+    const uint32_t wd[1] = {word};
+    store_segment<1>(pbase, f0, f0, hi, wd, lane);
+    if (++col == windows_per_row) {
+      col = 0;
+      ++row;
+    }
+  }
+}
+
 // General path, step 1: one thread per (row, group) computes the scale.
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_scales_general_kernel(
@@ -308,6 +392,36 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
       INT4_Q_CASE(16)
       INT4_Q_CASE(32)
 #undef INT4_Q_CASE
+      default:
+        break;
+    }
+    return cudaGetLastError();
+  }
+  if (pow2_group) {
+    const uintptr_t wa = reinterpret_cast<uintptr_t>(w);
+    const uint8_t* wbase = reinterpret_cast<const uint8_t*>(wa & ~static_cast<uintptr_t>(15));
+    const int64_t wshift = static_cast<int64_t>(wa & 15);
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(packed);
+    uint8_t* pbase = reinterpret_cast<uint8_t*>(pa & ~static_cast<uintptr_t>(3));
+    const int64_t pshift = static_cast<int64_t>(pa & 3);
+    const int64_t wpr = (K + 255) / 256;
+    const int64_t total = N * wpr;
+    const int64_t wbytes = wshift + N * K * static_cast<int64_t>(sizeof(T));
+    const int grid = grid_for(total, 8 * 4, 8);
+    switch (lpg) {
+#define INT4_QA_CASE(L)                                                                        \
+  case L:                                                                                      \
+    quantize_any_kernel<T, L><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint8_t*>(wbase), \
+                                                        wshift, wbytes, K, G, wpr, total, pbase, \
+                                                        pshift, scales);                         \
+    break;
+      INT4_QA_CASE(1)
+      INT4_QA_CASE(2)
+      INT4_QA_CASE(4)
+      INT4_QA_CASE(8)
+      INT4_QA_CASE(16)
+      INT4_QA_CASE(32)
+#undef INT4_QA_CASE
       default:
         break;
     }

@@ -11,6 +11,7 @@
 // int8 outputs (one 16-byte store).
 #include "common.cuh"
 #include "internal.h"
+#include "realign.cuh"
 
 namespace int4lib {
 
@@ -55,19 +56,47 @@ __global__ void __launch_bounds__(256) unpack_flat_kernel(const uint8_t* __restr
   }
 }
 
-// General K and alignment: one thread per output element.
-__global__ void __launch_bounds__(256) unpack_general_kernel(const uint8_t* __restrict__ packed,
-                                                            int64_t N, int64_t K,
-                                                            int8_t* __restrict__ out) {
+// Any K and alignment: a warp window is 512 outputs (256 packed bytes) of one
+// row.  A lane takes its aligned 8-byte chunk of the packed byte range, the
+// next lane's chunk by shuffle, funnel-shifts by the row's byte offset, expands
+// 16 nibbles and writes them with aligned word stores (store_segment).
+__global__ void __launch_bounds__(256) unpack_any_kernel(const uint8_t* __restrict__ pbase,
+                                                        int64_t pshift, int64_t pbytes, int64_t K,
+                                                        int64_t windows_per_row, int64_t total_windows,
+                                                        uint8_t* __restrict__ obase, int64_t oshift) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  int64_t wi = warp * per;
+  const int64_t wend = (wi + per < total_windows) ? wi + per : total_windows;
+  if (wi >= wend) return;
   const int64_t Kp = (K + 1) >> 1;
-  const int64_t total = N * K;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += stride) {
-    const int64_t n = e / K;
-    const int64_t k = e - n * K;
-    const uint32_t byte = __ldg(packed + n * Kp + (k >> 1));
-    out[e] = sext4((k & 1) ? (byte >> 4) : (byte & 0xFu));
+  int64_t row = wi / windows_per_row;
+  int64_t col = wi - row * windows_per_row;
+  for (; wi < wend; ++wi) {
+    const int64_t P = pshift + row * Kp + col * 256 + lane * 8;
+    const int64_t c = P >> 3;
+    const int boff = static_cast<int>(P & 7);
+    const uint2 own = load_chunk8(pbase, c, pbytes);
+    uint2 nx;
+    nx.x = __shfl_down_sync(0xffffffffu, own.x, 1);
+    nx.y = __shfl_down_sync(0xffffffffu, own.y, 1);
+    if (lane == 31) nx = load_chunk8(pbase, c + 1, pbytes);
+    const uint32_t win[4] = {own.x, own.y, nx.x, nx.y};
+    uint32_t b8[2];
+    byte_shift_words<4, 2>(win, boff, b8);
+    const uint2 a = expand_word(b8[0]);
+    const uint2 b = expand_word(b8[1]);
+    const uint32_t o[4] = {a.x, a.y, b.x, b.y};
+    const int64_t rowo = oshift + row * K;
+    const int64_t f0 = rowo + col * 512;
+    const int64_t hi = (f0 + 512 < rowo + K) ? f0 + 512 : rowo + K;
+    store_segment<4>(obase, f0, f0, hi, o, lane);
+    if (++col == windows_per_row) {
+      col = 0;
+      ++row;
+    }
   }
 }
 
@@ -85,10 +114,19 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* o
     unpack_flat_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(packed, total, out);
     return cudaGetLastError();
   }
-  int64_t grid = (N * K + 255) / 256;
-  if (grid > cap) grid = cap;
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(packed);
+  const uint8_t* pbase = reinterpret_cast<const uint8_t*>(pa & ~static_cast<uintptr_t>(7));
+  const int64_t pshift = static_cast<int64_t>(pa & 7);
+  const uintptr_t oa = reinterpret_cast<uintptr_t>(out);
+  uint8_t* obase = reinterpret_cast<uint8_t*>(oa & ~static_cast<uintptr_t>(3));
+  const int64_t oshift = static_cast<int64_t>(oa & 3);
+  const int64_t wpr = (K + 511) / 512;
+  const int64_t total = N * wpr;
+  int64_t grid = (total + 31) / 32;
+  if (grid > static_cast<int64_t>(num_sms()) * 8) grid = static_cast<int64_t>(num_sms()) * 8;
   if (grid < 1) grid = 1;
-  unpack_general_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(packed, N, K, out);
+  unpack_any_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(
+      pbase, pshift, pshift + N * ((K + 1) / 2), K, wpr, total, obase, oshift);
   return cudaGetLastError();
 }
 

@@ -175,6 +175,55 @@ def test_quantize_unaligned_pointers_take_the_general_path():
     assert_quantize_exact(w, packed, scales, 128)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("K", [1024, 1031, 28673])
+@pytest.mark.parametrize("woff, poff", [(0, 0), (1, 3), (3, 1), (5, 2)])
+def test_quantize_any_alignment_through_the_abi(dtype, K, woff, poff):
+    """Weights and packed output at odd element / byte offsets (rows at any
+    alignment): bit-exact against the oracle, and nothing outside the output
+    range is written."""
+    import ctypes
+    N, group = 37, 64
+    wbuf = make_weights(N * K + woff, 1, seed=K + woff, device=DEV, dtype=dtype,
+                        dist="student_t3").reshape(-1)
+    w = wbuf[woff:woff + N * K].view(N, K)
+    Kp = (K + 1) // 2
+    pbuf = torch.full((N * Kp + poff + 8,), 0xA5, dtype=torch.uint8, device=DEV)
+    scales = torch.empty((N, -(-K // group)), dtype=torch.float16, device=DEV)
+    code = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}[dtype]
+    rc = q4.lib().int4_quantize(ctypes.c_void_p(w.data_ptr()), code, N, K, group,
+                                ctypes.c_void_p(pbuf.data_ptr() + poff),
+                                ctypes.c_void_p(scales.data_ptr()),
+                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    pb = pbuf.cpu().numpy()
+    assert (pb[:poff] == 0xA5).all() and (pb[poff + N * Kp:] == 0xA5).all()
+    packed = torch.from_numpy(pb[poff:poff + N * Kp].reshape(N, Kp).copy()).to(DEV)
+    assert_quantize_exact(w, packed, scales, group)
+
+
+@pytest.mark.parametrize("K", [2, 7, 1000, 1001, 28673])
+@pytest.mark.parametrize("poff, ooff", [(0, 0), (1, 0), (0, 3), (5, 7)])
+def test_unpack_any_alignment_through_the_abi(K, poff, ooff):
+    import ctypes
+    N = 23
+    Kp = (K + 1) // 2
+    g = torch.Generator(device=DEV)
+    g.manual_seed(K * 31 + poff)
+    pbuf = torch.randint(0, 256, (N * Kp + poff,), generator=g, device=DEV,
+                         dtype=torch.int32).to(torch.uint8)
+    packed = pbuf[poff:].view(N, Kp)
+    obuf = torch.full((N * K + ooff + 16,), 0x5A, dtype=torch.uint8, device=DEV)
+    rc = q4.lib().int4_unpack(ctypes.c_void_p(packed.data_ptr()), K, N,
+                              ctypes.c_void_p(obuf.data_ptr() + ooff),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    ob = obuf.cpu().numpy()
+    assert (ob[:ooff] == 0x5A).all() and (ob[ooff + N * K:] == 0x5A).all()
+    got = ob[ooff:ooff + N * K].view(np.int8).reshape(N, K)
+    assert np.array_equal(got, oracle.unpack_int4(packed.cpu().numpy(), K))
+
+
 def test_quantize_is_deterministic():
     w = make_weights(512, 2048, seed=4, device=DEV, dtype=torch.bfloat16, dist="student_t3")
     a = q4.quantize_int4(w, 64)
