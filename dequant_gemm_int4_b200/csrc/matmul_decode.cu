@@ -47,18 +47,36 @@ namespace int4lib {
 
 namespace {
 
-constexpr int kSK = 2;                      // 128-wide K blocks per stage
-constexpr int kRowGroups = 4;               // row groups per CTA
+// Shape of a CTA (compile-time; the defaults are the measured choice).
+#ifndef INT4_DECODE_SK
+#define INT4_DECODE_SK 2
+#endif
+#ifndef INT4_DECODE_ROW_GROUPS
+#define INT4_DECODE_ROW_GROUPS 4
+#endif
+#ifndef INT4_DECODE_STAGES
+#define INT4_DECODE_STAGES 3
+#endif
+#ifndef INT4_DECODE_TILES1
+#define INT4_DECODE_TILES1 2
+#endif
+#ifndef INT4_DECODE_MIN_BLOCKS
+#define INT4_DECODE_MIN_BLOCKS 2
+#endif
+constexpr int kSK = INT4_DECODE_SK;                // 128-wide K blocks per stage (even)
+constexpr int kSub = kSK / 2;                      // 256-k sub-tiles per stage (one copy each)
+static_assert(kSK % 2 == 0, "stages hold whole 256-k sub-tiles");
+constexpr int kRowGroups = INT4_DECODE_ROW_GROUPS;  // row groups per CTA
 constexpr int kConsumers = kRowGroups * kSK;  // one consumer warp per (row group, block of the stage)
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int kStages = 3;
+constexpr int kStages = INT4_DECODE_STAGES;
 constexpr int kMaxCluster = 8;
 
 // 16-row tiles per consumer warp: two for M <= 8 (NT = 1), one for M <= 16,
 // so that both fit two CTAs per SM without spilling.
 template <int NT>
 struct Tiles {
-  static constexpr int kTiles = NT == 1 ? 2 : 1;
+  static constexpr int kTiles = NT == 1 ? INT4_DECODE_TILES1 : 1;
   static constexpr int kRowsPerCta = 16 * kTiles * kRowGroups;  // 128 or 64
   static constexpr int kWBytes = kRowsPerCta * kSK * 64;          // 16 or 8 KB per stage
 };
@@ -159,7 +177,8 @@ struct DLayout {
   static constexpr int kWBytes = Tiles<NT>::kWBytes;
   // Per stage: W tile (1024-aligned for the swizzle), then the x tile with
   // NT * 8 rows (rows M.. stay zero).
-  static constexpr int kXBytes = NT * 8 * kSK * 128 * 2;  // 4 KB per n-tile
+  static constexpr int kXSub = NT * 8 * 256 * 2;          // x rows of one sub-tile
+  static constexpr int kXBytes = kSub * kXSub;
   static constexpr int kStageBytes = kWBytes + kXBytes;   // multiple of 1024
   static constexpr int offRed = kStages * kStageBytes;
   static constexpr int kRedBytes = kConsumers * kTiles * NT * 4 * 32 * 4;
@@ -170,7 +189,7 @@ struct DLayout {
 };
 
 template <typename TX, int NT, int GPB>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(
+__global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
     int64_t N, int kblocks_per_slice, int S, uint32_t* status) {
@@ -195,14 +214,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
   const int kb1 = (kb0 + kblocks_per_slice < KB) ? kb0 + kblocks_per_slice : KB;
   const int nst = (kb1 - kb0 + kSK - 1) / kSK;
   const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kRowsPerCta;
-  const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;
+  const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;  // all sub-tiles
   const WaitCtx wc{abort_flag, status};
 
-  // x rows M.. of every stage stay zero (the copies only write M rows).
+  // x rows M.. of every sub-tile stay zero (the copies only write M rows).
   for (int i = threadIdx.x; i < kStages * (L::kXBytes / 16); i += blockDim.x) {
     const int st = i / (L::kXBytes / 16);
     const int off = (i % (L::kXBytes / 16)) * 16;
-    if (off >= M * kSK * 128 * 2)
+    if (off % L::kXSub >= M * 256 * 2)
       ptx::sts128(sbase + st * L::kStageBytes + kWBytes + off, make_uint4(0u, 0u, 0u, 0u));
   }
   if (threadIdx.x == 0) {
@@ -241,8 +260,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
         const uint32_t st = sbase + s * L::kStageBytes;
         const int kb = kb0 + it * kSK;
         ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + xbytes);
-        ptx::tma_load_2d(st, &tm_w, kb * 64, static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
-        ptx::tma_load_2d(st + kWBytes, &tm_x, kb * 128, 0, ptx::smem_u32(&full[s]));
+#pragma unroll
+        for (int q = 0; q < kSub; ++q) {
+          ptx::tma_load_2d(st + q * (kWBytes / kSub), &tm_w, (kb + 2 * q) * 64,
+                           static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
+          ptx::tma_load_2d(st + kWBytes + q * L::kXSub, &tm_x, (kb + 2 * q) * 128, 0,
+                           ptx::smem_u32(&full[s]));
+        }
       }
       if (*abort_flag) {
         const int first = it - kStages > 0 ? it - kStages : 0;
@@ -280,22 +304,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int r = lr[t][h];
-            const uint32_t rb = wt + r * 128;
+            const uint32_t rb = wt + (b >> 1) * (kWBytes / kSub) + r * 128;
             const int sw = r & 7;
+            const int bl = b & 1;  // block within the 256-k sub-tile
             if (GPB == 1) {
-              const uint4 u = ptx::lds128(rb + ((((b * 64 + 16 * c) >> 4) ^ sw) << 4));
+              const uint4 u = ptx::lds128(rb + ((((bl * 64 + 16 * c) >> 4) ^ sw) << 4));
               wv[t][h][0] = u.x; wv[t][h][1] = u.y; wv[t][h][2] = u.z; wv[t][h][3] = u.w;
             } else if (GPB == 2) {
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
-                const int off = b * 64 + 32 * q + 8 * c;
+                const int off = bl * 64 + 32 * q + 8 * c;
                 const uint2 u = ptx::lds64(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
                 wv[t][h][2 * q] = u.x; wv[t][h][2 * q + 1] = u.y;
               }
             } else {
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                const int off = b * 64 + 16 * j + 4 * c;
+                const int off = bl * 64 + 16 * j + 4 * c;
                 wv[t][h][j] = ptx::lds32(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
               }
             }
@@ -314,10 +339,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[t][nt][i] = 0.0f;
           }
-          const int kx = b * 128 + 8 * word_index<GPB>(c, j);
+          const int kx = (b & 1) * 128 + 8 * word_index<GPB>(c, j);
+          const uint32_t xs = xt + (b >> 1) * L::kXSub;
           uint4 xf[NT];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) xf[nt] = ptx::lds128(xt + ((nt * 8 + g) * kSK * 128 + kx) * 2);
+          for (int nt = 0; nt < NT; ++nt) xf[nt] = ptx::lds128(xs + ((nt * 8 + g) * 256 + kx) * 2);
 #pragma unroll
           for (int t = 0; t < kTiles; ++t) {
             uint32_t pa[4], pb[4];
@@ -461,7 +487,7 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    const cuuint32_t box[2] = {kSK * 64, kRowsPerCta};
+    const cuuint32_t box[2] = {128, kRowsPerCta};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -471,7 +497,7 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {kSK * 128, static_cast<cuuint32_t>(M)};
+    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
                                        ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
