@@ -7,7 +7,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/int4.h"
+#include "int4.h"
 #include "common.cuh"
 #include "internal.h"
 

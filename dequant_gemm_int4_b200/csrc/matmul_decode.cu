@@ -15,14 +15,18 @@
 //     fragment feeds two independent MMA chains; per 128-wide K block a lane
 //     reads its 16 (or 2 x 8, 4 x 4 for group 64/32) bytes of four rows from
 //     shared memory and sign-extends nibble pairs to bf16/fp16 exactly in
-//     registers:
-//     byte j -> ((byte_j | byte_j >> 4 << 16) & 0x000F000F) ^ magic, then one
-//     packed subtract (magic = 128 + 8 (bf16) or 1024 + 8 (fp16) in each half,
-//     the XOR flips the nibble's sign bit so that the value is q + 136 or
-//     q + 1032 before the subtract);
+//     registers: for a 32-bit word of nibbles e0..e7, the pair (e_i, e_{i+4})
+//     is ((w >> 4i) & 0x000F000F) ^ magic, then one packed subtract (magic =
+//     128 + 8 (bf16) or 1024 + 8 (fp16) in each half; the XOR flips the
+//     nibble's sign bit so that the value is q + 136 or q + 1032 before the
+//     subtract).  The shifts are multiply-highs, which issue on the FMA pipe:
+//     the mask and permute instructions share a logic pipe that runs at half
+//     rate on this GPU and bounds the kernel;
 //   * the 16 x 8 x 16 warp MMA (mma.sync, fp32 accumulate) multiplies them by
-//     x straight from shared memory (natural k order, no permutation), so no
-//     multiply-add runs on the CUDA cores;
+//     x from shared memory; the MMA's k slots see the pairs (e_i, e_{i+4}), so
+//     x is paired the same way in registers (four byte permutes per 16 bytes,
+//     shared by the warp's two row tiles), and no multiply-add runs on the
+//     CUDA cores;
 //   * each K group gets its own fp32 accumulator, which is scaled by its
 //     group's scale and added into the fp32 running sum, per the page's order.
 // x rows M..15 of every stage are zeroed once, so lanes of padding batch rows
@@ -94,7 +98,7 @@ struct Cvt<__nv_bfloat16> {
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -111,7 +115,7 @@ struct Cvt<__half> {
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -119,18 +123,32 @@ struct Cvt<__half> {
   }
 };
 
-// Word w = 8 consecutive k (nibbles e0..e7).  p[i] = (e_{2i}, e_{2i+1}).
+// w >> n as a multiply-high, which issues on the FMA pipe; the logic pipe that
+// the masks and permutes need runs at half rate on this GPU.
+__device__ __forceinline__ uint32_t shr_mul(uint32_t w, uint32_t two_pow_32_minus_n) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(two_pow_32_minus_n));
+  return r;
+}
+
+// Word w = 8 consecutive k (nibbles e0..e7 at bits 4i).  p[i] = (e_i, e_{i+4})
+// as bf16x2 / f16x2: ((w >> 4i) & 0x000F000F) ^ magic, minus the bias.
 template <typename TX>
 __device__ __forceinline__ void expand(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t ws = w >> 4;
+  const uint32_t v[4] = {w, shr_mul(w, 1u << 28), shr_mul(w, 1u << 24), shr_mul(w, 1u << 20)};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t sel = static_cast<uint32_t>(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-    const uint32_t t = __byte_perm(w, ws, sel);
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(t), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(v[i]), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
     p[i] = Cvt<TX>::sub(r);
   }
+}
+
+// x fragments for the pairing above: from x[k0 .. k0+8) = (x0x1, x2x3, x4x5,
+// x6x7), MMA h = 0 takes (x0,x4), (x1,x5) and h = 1 takes (x2,x6), (x3,x7).
+__device__ __forceinline__ uint4 pair_x(uint4 n) {
+  return make_uint4(__byte_perm(n.x, n.z, 0x5410), __byte_perm(n.x, n.z, 0x7632),
+                    __byte_perm(n.y, n.w, 0x5410), __byte_perm(n.y, n.w, 0x7632));
 }
 
 // The 8-k word (0..15 of a 128-k block) that lane c of a quad uses as its
@@ -275,60 +293,71 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
     }
   } else {
     // ---------------- consumers ----------------
-    // Rows of this lane within the W tile: tile t covers rows cw*32 + 16t .. +15.
-    int lr[kTiles][2];
+    // Each consumer owns kTiles 16-row tiles of row group rg and K block `bs`
+    // of every stage.  Offsets within a stage are fixed per lane.
+    constexpr int kW = (GPB == 1) ? 1 : (GPB == 2 ? 2 : 4);  // shared loads per row
+    const int bl = bs & 1;                                   // block within its 256-k sub-tile
+    const uint32_t sub_w = static_cast<uint32_t>((bs >> 1) * (kWBytes / kSub));
+    uint32_t wofs[kTiles][2][kW];
     const uint16_t* sp[kTiles][2];
 #pragma unroll
     for (int t = 0; t < kTiles; ++t)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        lr[t][h] = rg * 16 * kTiles + 16 * t + g + 8 * h;
-        int64_t r = row0 + lr[t][h];
-        if (r >= N) r = N - 1;  // never written; keeps the scale load in bounds
-        sp[t][h] = scales + r * G;
+        const int r = rg * 16 * kTiles + 16 * t + g + 8 * h;  // row within the W tile
+        const int sw = r & 7;
+#pragma unroll
+        for (int q = 0; q < kW; ++q) {
+          const int off = (GPB == 1) ? bl * 64 + 16 * c
+                                     : (GPB == 2 ? bl * 64 + 32 * q + 8 * c : bl * 64 + 16 * q + 4 * c);
+          wofs[t][h][q] = sub_w + static_cast<uint32_t>(r * 128 + ((((off >> 4) ^ sw)) << 4) + (off & 15));
+        }
+        int64_t gr = row0 + r;
+        if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
+        sp[t][h] = scales + gr * G;
       }
+    uint32_t xofs[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      xofs[j] = static_cast<uint32_t>(kWBytes + (bs >> 1) * L::kXSub +
+                                      (g * 256 + bl * 128 + 8 * word_index<GPB>(c, j)) * 2);
     const int bpg = group / 128;  // K blocks per group when GPB == 1
     for (int it = 0; it < nst; ++it) {
       const int s = it % kStages;
       if (!wait_bar(ptx::smem_u32(&full[s]), (it / kStages) & 1, wc)) break;
-      const uint32_t wt = sbase + s * L::kStageBytes;
-      const uint32_t xt = wt + kWBytes;
-      {
-        const int b = bs;
-        const int kb = kb0 + it * kSK + b;
-        if (kb < kb1) {
-        // This lane's four 8-k words of each of its rows in block b.
+      const uint32_t st = sbase + s * L::kStageBytes;
+      const int kb = kb0 + it * kSK + bs;
+      if (kb < kb1) {
+        // This lane's four 8-k words of each of its rows.
         uint32_t wv[kTiles][2][4];
 #pragma unroll
         for (int t = 0; t < kTiles; ++t)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int r = lr[t][h];
-            const uint32_t rb = wt + (b >> 1) * (kWBytes / kSub) + r * 128;
-            const int sw = r & 7;
-            const int bl = b & 1;  // block within the 256-k sub-tile
             if (GPB == 1) {
-              const uint4 u = ptx::lds128(rb + ((((bl * 64 + 16 * c) >> 4) ^ sw) << 4));
+              const uint4 u = ptx::lds128(st + wofs[t][h][0]);
               wv[t][h][0] = u.x; wv[t][h][1] = u.y; wv[t][h][2] = u.z; wv[t][h][3] = u.w;
             } else if (GPB == 2) {
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
-                const int off = bl * 64 + 32 * q + 8 * c;
-                const uint2 u = ptx::lds64(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
+                const uint2 u = ptx::lds64(st + wofs[t][h][q]);
                 wv[t][h][2 * q] = u.x; wv[t][h][2 * q + 1] = u.y;
               }
             } else {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int off = bl * 64 + 16 * j + 4 * c;
-                wv[t][h][j] = ptx::lds32(rb + ((((off >> 4) ^ sw) << 4) | (off & 15)));
-              }
+              for (int q = 0; q < 4; ++q) wv[t][h][q] = ptx::lds32(st + wofs[t][h][q]);
             }
           }
+        // All x fragments of this block, paired for the MMA slots.
+        uint4 xf4[4][NT];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) xf4[j][nt] = ptx::lds128(st + xofs[j] + nt * 8 * 512);
         float acc[kTiles][NT][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          // Group a of word j; the accumulator restarts at the group's first word.
+          // The accumulator restarts at the first word of each group.
           const bool first = (GPB == 1) ? (j == 0) : (GPB == 2 ? (j % 2 == 0) : true);
           const bool last = (GPB == 1) ? (j == 3) : (GPB == 2 ? (j % 2 == 1) : true);
           if (first) {
@@ -339,11 +368,9 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[t][nt][i] = 0.0f;
           }
-          const int kx = (b & 1) * 128 + 8 * word_index<GPB>(c, j);
-          const uint32_t xs = xt + (b >> 1) * L::kXSub;
           uint4 xf[NT];
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) xf[nt] = ptx::lds128(xs + ((nt * 8 + g) * 256 + kx) * 2);
+          for (int nt = 0; nt < NT; ++nt) xf[nt] = pair_x(xf4[j][nt]);
 #pragma unroll
           for (int t = 0; t < kTiles; ++t) {
             uint32_t pa[4], pb[4];
@@ -378,7 +405,6 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           }
         }
       }
-        }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
     }

@@ -240,6 +240,86 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
   }
 }
 
+// Wide fast path: K % 16 == 0, group = 16 * LPG (LPG a power of two <= 32),
+// w 16-byte aligned, packed 8-byte aligned.  Each lane takes 16 consecutive
+// elements per window (two 16-byte loads for 16-bit weights) and stores 8
+// packed bytes, so the per-window work (scale, shuffles, addressing, stores)
+// is spread over twice as many elements as in quantize_aligned_kernel.
+template <typename T, int LPG>
+__global__ void __launch_bounds__(256) quantize_wide_kernel(
+    const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
+    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+  constexpr int kU = 2;  // windows in flight per warp
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  int64_t wbeg = warp * per;
+  const int64_t wend = (wbeg + per < total_windows) ? wbeg + per : total_windows;
+  if (wbeg >= wend) return;
+  const int chunks_per_row = static_cast<int>(K >> 4);
+  const int64_t Kp = K >> 1;
+  int64_t row = wbeg / windows_per_row;
+  int col = static_cast<int>(wbeg - row * windows_per_row);
+  const int wpr = static_cast<int>(windows_per_row);
+
+  for (; wbeg < wend; wbeg += kU) {
+    float v[kU][2][8];
+    int64_t rw[kU];
+    int ch[kU];
+    bool valid[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      rw[u] = row;
+      ch[u] = col * 32 + lane;
+      valid[u] = (wbeg + u < wend) && (ch[u] < chunks_per_row);
+      if (valid[u]) {
+        const T* p = w + row * K + static_cast<int64_t>(ch[u]) * 16;
+        Load8<T>::run(p, v[u][0]);
+        Load8<T>::run(p + 8, v[u][1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][0][i] = v[u][1][i] = 0.0f;
+      }
+      if (++col == wpr) {
+        col = 0;
+        ++row;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(v[u][0][i]), fabsf(v[u][1][i])));
+#pragma unroll
+      for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const ScaleInfo si = scale_from_absmax(m);
+      const uint32_t ex = si.bits & 0x7C00u;
+      const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
+      uint32_t w0, w1;
+      const bool ok0 = codes8_normal(v[u][0], si.r, w0);
+      const bool ok1 = codes8_normal(v[u][1], si.r, w1);
+      const bool ok = ok0 && ok1 && simple;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (!ok) {
+          w0 = 0;
+          w1 = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            w0 |= code_exact(v[u][0][i], si) << (4 * i);
+            w1 |= code_exact(v[u][1][i], si) << (4 * i);
+          }
+        }
+      }
+      if (valid[u]) {
+        if ((lane & (LPG - 1)) == 0) scales[rw[u] * G + ch[u] / LPG] = static_cast<uint16_t>(si.bits);
+        *reinterpret_cast<uint2*>(packed + rw[u] * Kp + static_cast<int64_t>(ch[u]) * 8) =
+            make_uint2(w0, w1);
+      }
+    }
+  }
+}
+
 // Rows at any alignment (odd K, unaligned pointers), same groups as the fast
 // path.  The weights are read as aligned 16-byte chunks of the byte range that
 // starts at `wbase` (16-byte aligned, w[0,0] at byte `wshift`): a lane loads
@@ -376,6 +456,31 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
                        (reinterpret_cast<uintptr_t>(packed) % 4 == 0);
   const int lpg = group / 8;
   const bool pow2_group = (group % 8 == 0) && lpg >= 1 && lpg <= 32 && (lpg & (lpg - 1)) == 0;
+  const int lpg16 = group / 16;
+  const bool wide = (K % 16 == 0) && (reinterpret_cast<uintptr_t>(w) % 16 == 0) &&
+                    (reinterpret_cast<uintptr_t>(packed) % 8 == 0) && (group % 16 == 0) &&
+                    lpg16 >= 1 && lpg16 <= 32 && (lpg16 & (lpg16 - 1)) == 0;
+  if (wide) {
+    const int64_t wpr = (K / 16 + 31) / 32;
+    const int64_t total = N * wpr;
+    const int grid = grid_for(total, 8 * 2, 8);
+    switch (lpg16) {
+#define INT4_QW_CASE(L)                                                                       \
+  case L:                                                                                     \
+    quantize_wide_kernel<T, L><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed, scales); \
+    break;
+      INT4_QW_CASE(1)
+      INT4_QW_CASE(2)
+      INT4_QW_CASE(4)
+      INT4_QW_CASE(8)
+      INT4_QW_CASE(16)
+      INT4_QW_CASE(32)
+#undef INT4_QW_CASE
+      default:
+        break;
+    }
+    return cudaGetLastError();
+  }
   if (aligned && pow2_group) {
     const int64_t wpr = (K / 8 + 31) / 32;
     const int64_t total = N * wpr;

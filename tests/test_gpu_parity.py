@@ -89,12 +89,13 @@ def test_quantize_special_values(K_pad):
     assert_quantize_exact(w, packed, scales, 8)
 
 
-def test_quantize_half_integer_quotients():
+@pytest.mark.parametrize("group", [8, 16, 32])
+def test_quantize_half_integer_quotients(group):
     """Weights placed exactly on and next to half-integer multiples of the
-    scale: the fast path must agree with the IEEE division on every tie."""
-    rng = np.random.default_rng(21)
+    scale: every fast path must agree with the IEEE division on every tie."""
+    rng = np.random.default_rng(21 + group)
     s = (rng.uniform(0.01, 2.0, size=(4096, 1))).astype(np.float16).astype(np.float32)
-    half = rng.integers(-7, 7, size=(4096, 7)) + 0.5     # -6.5 .. 6.5
+    half = rng.integers(-7, 7, size=(4096, group - 1)) + 0.5     # -6.5 .. 6.5
     w = (half * s).astype(np.float32)
     nudge = rng.integers(-2, 3, size=w.shape).astype(np.int32)
     w = (w.view(np.int32) + nudge).view(np.float32)
@@ -102,8 +103,8 @@ def test_quantize_half_integer_quotients():
     wt = torch.from_numpy(w.astype(np.float32)).to(DEV)
     for dtype in (torch.float32, torch.float16, torch.bfloat16):
         wd = wt.to(dtype)
-        packed, scales, K = q4.quantize_int4(wd, 8)
-        assert_quantize_exact(wd, packed, scales, 8)
+        packed, scales, K = q4.quantize_int4(wd, group)
+        assert_quantize_exact(wd, packed, scales, group)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
