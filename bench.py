@@ -145,7 +145,9 @@ def _max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    # NCCL reduces device tensors; the gloo backend (CPU tests) host tensors.
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -203,7 +205,7 @@ def run_reference(args):
     res = None
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        res = cpu_baseline(rows=4096)
+        res = cpu_baseline(rows=2048)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)

@@ -153,10 +153,14 @@ def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: 
         _need_cuda("out", out)
         if out.dtype != torch.float32 or tuple(out.shape) != (M, N):
             raise ValueError("out must be float32 [M, N]")
-    with torch.cuda.device(x.device):
-        _check(lib().int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
-                                      scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
-                                      int(path), _stream(x)))
+    L = _lib if _lib is not None else lib()
+    args = (x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(), scales.data_ptr(), K,
+            int(group), M, N, out.data_ptr(), int(path))
+    if x.device.index == torch.cuda.current_device():
+        _check(L.int4_matmul_path(*args, _stream(x)))
+    else:
+        with torch.cuda.device(x.device):
+            _check(L.int4_matmul_path(*args, _stream(x)))
     return out
 
 

@@ -44,4 +44,18 @@ cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Grid of at most one resident wave of `kern` (256-thread blocks, no dynamic
+// shared memory) for kernels whose blocks take equal contiguous shares of the
+// work, so no partial last wave trails the others.
+template <typename Kern>
+int resident_grid(Kern kern, int64_t want) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
+  const int64_t g = want < cap ? want : cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
 }  // namespace int4lib

@@ -7,14 +7,15 @@
 //
 // The kernel is bound by HBM: every packed weight byte is read once and at
 // M <= 16 feeds at most 32 multiply-adds.  Design:
-//   * a producer warp streams the CTA's 128 weight rows through a 4-stage
-//     shared-memory ring with TMA (each stage: 128 rows x 256 k = 16 KB of
-//     packed nibbles, 128-byte swizzle, plus x [M x 256] bf16/fp16), so about
-//     64 KB per CTA are in flight, with up to three CTAs per SM;
-//   * four consumer warps own 32 rows (two 16-row tiles) each, so every x
-//     fragment feeds two independent MMA chains; per 128-wide K block a lane
-//     reads its 16 (or 2 x 8, 4 x 4 for group 64/32) bytes of four rows from
-//     shared memory and sign-extends nibble pairs to bf16/fp16 exactly in
+//   * a producer warp streams 128 weight rows (64 for M > 8) through a
+//     3-stage shared-memory ring with TMA (each stage: the rows x 256 k of
+//     packed nibbles, 128-byte swizzle, plus x [M x 256] bf16/fp16), two CTAs
+//     per SM;
+//   * eight consumer warps, four row groups x two K-block slots per stage;
+//     a row group is 32 rows (two 16-row tiles) so every x fragment feeds two
+//     independent MMA chains; per 128-wide K block a lane reads its 16 (or
+//     2 x 8, 4 x 4 for group 64/32) bytes of four rows from shared memory and
+//     sign-extends nibble pairs to bf16/fp16 exactly in
 //     registers: for a 32-bit word of nibbles e0..e7, the pair (e_i, e_{i+4})
 //     is ((w >> 4i) & 0x000F000F) ^ magic, then one packed subtract (magic =
 //     128 + 8 (bf16) or 1024 + 8 (fp16) in each half; the XOR flips the
@@ -29,23 +30,29 @@
 //     CUDA cores;
 //   * each K group gets its own fp32 accumulator, which is scaled by its
 //     group's scale and added into the fp32 running sum, per the page's order.
-// x rows M..15 of every stage are zeroed once, so lanes of padding batch rows
-// need no predicate.  All four lanes of a quad read the same group for a given word, so each MMA
-// only sums k of one group.  Split-K: when N is small the K range is split
-// over the CTAs of a cluster (up to 8); partial sums are reduced in rank order
-// through distributed shared memory, so the result is deterministic.  Every
-// mbarrier wait is bounded in time; a wait that gives up aborts the CTA (the
-// status word records it), drains its copies and skips the output.
-#include <cooperative_groups.h>
+// Lanes of padding batch rows (n >= M) use zero x fragments and skip their
+// shared-memory loads.  All four lanes of a quad read the same group for a
+// given word, so each MMA only sums k of one group.  Weight rows are permuted
+// inside each 16-row tile so that the shared-memory loads are free of bank
+// conflicts.
+//
+// Work split (stream-K): the (row tile, 128-k block) units are dealt out in
+// row-major order as equal contiguous runs to one wave of CTAs (two per SM),
+// so every SM streams the same number of bytes whatever N and K are.  A tile
+// that a run covers whole is written to y by its CTA; the pieces of a tile
+// that straddles runs go to a partial buffer, and a small fix-up kernel,
+// launched behind the main one with programmatic dependent launch, adds them
+// in CTA order, so the result does not depend on timing.  Every mbarrier
+// wait is bounded in time; a wait that gives up aborts the CTA (the status
+// word records it), drains its copies and skips the output.
 #include <cuda.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace int4lib {
 
@@ -74,7 +81,6 @@ constexpr int kRowGroups = INT4_DECODE_ROW_GROUPS;  // row groups per CTA
 constexpr int kConsumers = kRowGroups * kSK;  // one consumer warp per (row group, block of the stage)
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = INT4_DECODE_STAGES;
-constexpr int kMaxCluster = 8;
 
 // 16-row tiles per consumer warp: two for M <= 8 (NT = 1), one for M <= 16,
 // so that both fit two CTAs per SM without spilling.
@@ -161,6 +167,19 @@ __device__ __forceinline__ int word_index(int c, int j) {
   return 4 * j + c;
 }
 
+// The W tile row that MMA row g (0..7, and g + 8) of a 16-row tile reads.
+// Rows are permuted inside the tile so that the lanes served by one shared-
+// memory wavefront hit distinct 16-byte bank groups under the 128-byte
+// swizzle (chunk c of row r sits at c ^ (r & 7)): 8 lanes per wavefront for
+// the 16-byte loads (group multiple of 128), 16 for the 8-byte loads (group
+// 64); 4-byte loads (group 32) are conflict-free in row order.
+template <int GPB>
+__device__ __forceinline__ int tile_row(int g) {
+  if (GPB == 1) return (g >> 1) | ((g & 1) << 2);
+  if (GPB == 2) return ((g & 3) << 1) | (g >> 2);
+  return g;
+}
+
 struct WaitCtx {
   volatile uint32_t* abort;
   uint32_t* status;
@@ -194,7 +213,7 @@ struct DLayout {
   static constexpr int kTiles = Tiles<NT>::kTiles;
   static constexpr int kWBytes = Tiles<NT>::kWBytes;
   // Per stage: W tile (1024-aligned for the swizzle), then the x tile with
-  // NT * 8 rows (rows M.. stay zero).
+  // room for NT * 8 rows (the copies write rows 0..M-1).
   static constexpr int kXSub = NT * 8 * 256 * 2;          // x rows of one sub-tile
   static constexpr int kXBytes = kSub * kXSub;
   static constexpr int kStageBytes = kWBytes + kXBytes;   // multiple of 1024
@@ -210,7 +229,7 @@ template <typename TX, int NT, int GPB>
 __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
-    int64_t N, int kblocks_per_slice, int S, uint32_t* status) {
+    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* status) {
   using L = DLayout<NT>;
   constexpr int kTiles = Tiles<NT>::kTiles;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
@@ -226,22 +245,16 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int slice = blockIdx.x;  // rank in the cluster when S > 1
-  const int KB = static_cast<int>((K + 127) / 128);
-  const int kb0 = slice * kblocks_per_slice;
-  const int kb1 = (kb0 + kblocks_per_slice < KB) ? kb0 + kblocks_per_slice : KB;
-  const int nst = (kb1 - kb0 + kSK - 1) / kSK;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kRowsPerCta;
+  // Stream-K split: the units are (row tile, 128-k block) pairs in row-major
+  // order, and CTA p takes units [p U / P, (p + 1) U / P).  The run crosses
+  // at most two tile boundaries; a tile it covers whole goes straight to y,
+  // a partial tile to its partial slot (2p for the run's first segment when
+  // that starts inside a tile, else 2p + 1), which the fix-up kernel sums.
+  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * U / P;
+  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * U / P;
   const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;  // all sub-tiles
   const WaitCtx wc{abort_flag, status};
 
-  // x rows M.. of every sub-tile stay zero (the copies only write M rows).
-  for (int i = threadIdx.x; i < kStages * (L::kXBytes / 16); i += blockDim.x) {
-    const int st = i / (L::kXBytes / 16);
-    const int off = (i % (L::kXBytes / 16)) * 16;
-    if (off % L::kXSub >= M * 256 * 2)
-      ptx::sts128(sbase + st * L::kStageBytes + kWBytes + off, make_uint4(0u, 0u, 0u, 0u));
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
@@ -253,42 +266,47 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
     ptx::prefetch_tmap(&tm_x);
   }
   __syncthreads();
-
-  float tot[kTiles][NT][4];
-#pragma unroll
-  for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tot[t][nt][i] = 0.0f;
+  // The fix-up grid may be scheduled now; it waits for this grid to finish.
+  ptx::launch_dependents();
 
   const int c = lane & 3;
   const int g = lane >> 2;
   const int cw = warp - 1;          // consumer index
-  const int rg = cw % kRowGroups;   // 32-row group of this consumer
+  const int rg = cw % kRowGroups;   // row group of this consumer
   const int bs = cw / kRowGroups;   // which K block of each stage it takes
 
   if (warp == 0) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      int it = 0;
-      for (; it < nst; ++it) {
-        const int s = it % kStages;
-        if (!wait_bar(ptx::smem_u32(&empty[s]), ((it / kStages) & 1) ^ 1u, wc)) break;
-        const uint32_t st = sbase + s * L::kStageBytes;
-        const int kb = kb0 + it * kSK;
-        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + xbytes);
+      int gs = 0;  // stages issued so far (ring slot and phase)
+      bool ok = true;
+      for (int64_t u = u_begin; ok && u < u_end;) {
+        const int64_t r = u / KB;
+        const int blo = static_cast<int>(u - r * KB);
+        const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+        const int32_t row0 = static_cast<int32_t>(r * kRowsPerCta);
+        for (int kb = blo; kb < bhi; kb += kSK, ++gs) {
+          const int s = gs % kStages;
+          if (!wait_bar(ptx::smem_u32(&empty[s]), ((gs / kStages) & 1) ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sbase + s * L::kStageBytes;
+          ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + xbytes);
 #pragma unroll
-        for (int q = 0; q < kSub; ++q) {
-          ptx::tma_load_2d(st + q * (kWBytes / kSub), &tm_w, (kb + 2 * q) * 64,
-                           static_cast<int32_t>(row0), ptx::smem_u32(&full[s]));
-          ptx::tma_load_2d(st + kWBytes + q * L::kXSub, &tm_x, (kb + 2 * q) * 128, 0,
-                           ptx::smem_u32(&full[s]));
+          for (int q = 0; q < kSub; ++q) {
+            ptx::tma_load_2d(st + q * (kWBytes / kSub), &tm_w, (kb + 2 * q) * 64, row0,
+                             ptx::smem_u32(&full[s]));
+            ptx::tma_load_2d(st + kWBytes + q * L::kXSub, &tm_x, (kb + 2 * q) * 128, 0,
+                             ptx::smem_u32(&full[s]));
+          }
         }
+        u = r * KB + bhi;
       }
       if (*abort_flag) {
-        const int first = it - kStages > 0 ? it - kStages : 0;
-        for (int j = first; j < it; ++j) drain_bar(ptx::smem_u32(&full[j % kStages]), (j / kStages) & 1);
+        // Wait (bounded) for the copies that may still be in flight.
+        const int first = gs - kStages > 0 ? gs - kStages : 0;
+        for (int j = first; j < gs; ++j) drain_bar(ptx::smem_u32(&full[j % kStages]), (j / kStages) & 1);
       }
     }
   } else {
@@ -299,12 +317,11 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
     const int bl = bs & 1;                                   // block within its 256-k sub-tile
     const uint32_t sub_w = static_cast<uint32_t>((bs >> 1) * (kWBytes / kSub));
     uint32_t wofs[kTiles][2][kW];
-    const uint16_t* sp[kTiles][2];
 #pragma unroll
     for (int t = 0; t < kTiles; ++t)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = rg * 16 * kTiles + 16 * t + g + 8 * h;  // row within the W tile
+        const int r = rg * 16 * kTiles + 16 * t + tile_row<GPB>(g) + 8 * h;  // row within the W tile
         const int sw = r & 7;
 #pragma unroll
         for (int q = 0; q < kW; ++q) {
@@ -312,9 +329,6 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
                                      : (GPB == 2 ? bl * 64 + 32 * q + 8 * c : bl * 64 + 16 * q + 4 * c);
           wofs[t][h][q] = sub_w + static_cast<uint32_t>(r * 128 + ((((off >> 4) ^ sw)) << 4) + (off & 15));
         }
-        int64_t gr = row0 + r;
-        if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
-        sp[t][h] = scales + gr * G;
       }
     uint32_t xofs[4];
 #pragma unroll
@@ -322,12 +336,40 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
       xofs[j] = static_cast<uint32_t>(kWBytes + (bs >> 1) * L::kXSub +
                                       (g * 256 + bl * 128 + 8 * word_index<GPB>(c, j)) * 2);
     const int bpg = group / 128;  // K blocks per group when GPB == 1
-    for (int it = 0; it < nst; ++it) {
-      const int s = it % kStages;
-      if (!wait_bar(ptx::smem_u32(&full[s]), (it / kStages) & 1, wc)) break;
-      const uint32_t st = sbase + s * L::kStageBytes;
-      const int kb = kb0 + it * kSK + bs;
-      if (kb < kb1) {
+    constexpr int kPer = kRowGroups * kTiles * NT * 4 * 32;  // outputs of a tile
+    int gs = 0;
+    for (int64_t u = u_begin; u < u_end;) {
+      const int64_t r = u / KB;
+      const int blo = static_cast<int>(u - r * KB);
+      const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+      const int64_t row0 = r * kRowsPerCta;
+      const uint16_t* sp[kTiles][2];
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          int64_t gr = row0 + rg * 16 * kTiles + 16 * t + tile_row<GPB>(g) + 8 * h;
+          if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
+          sp[t][h] = scales + gr * G;
+        }
+      float tot[kTiles][NT][4];
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tot[t][nt][i] = 0.0f;
+      bool ok = true;
+      for (int kb_stage = blo; kb_stage < bhi; kb_stage += kSK, ++gs) {
+        const int s = gs % kStages;
+        // Every lane polls the barrier (its completion makes the copied bytes
+        // visible to the lane); the vote keeps the warp together if a bounded
+        // wait gave up in some lanes only.
+        ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&full[s]), (gs / kStages) & 1, wc));
+        if (!ok) break;
+        const uint32_t st = sbase + s * L::kStageBytes;
+        const int kb = kb_stage + bs;
+        if (kb < bhi) {
         // This lane's four 8-k words of each of its rows.
         uint32_t wv[kTiles][2][4];
 #pragma unroll
@@ -348,12 +390,30 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
               for (int q = 0; q < 4; ++q) wv[t][h][q] = ptx::lds32(st + wofs[t][h][q]);
             }
           }
-        // All x fragments of this block, paired for the MMA slots.
+        // All x fragments of this block.  Lanes of padding batch rows (n >= M)
+        // take zeros without touching shared memory, which at small M saves
+        // most of the x wavefronts (the rows share bank groups).
         uint4 xf4[4][NT];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) xf4[j][nt] = ptx::lds128(st + xofs[j] + nt * 8 * 512);
+          for (int nt = 0; nt < NT; ++nt)
+            xf4[j][nt] = (g + 8 * nt < M) ? ptx::lds128(st + xofs[j] + nt * 8 * 512) : make_uint4(0u, 0u, 0u, 0u);
+        // The block's scales (one per row and group) are loaded before they
+        // are needed, as raw fp16 bits (two per register for group 64); group
+        // 32 loads them at use, to stay within registers.
+        uint32_t sraw[kTiles][2];
+        if (GPB <= 2) {
+          const int gi0 = (GPB == 1) ? ((bpg == 1) ? kb : kb / bpg) : kb * 2;
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t r = (gi0 < G) ? __ldg(sp[t][h] + gi0) : 0u;
+              if (GPB == 2) r |= (gi0 + 1 < G) ? static_cast<uint32_t>(__ldg(sp[t][h] + gi0 + 1)) << 16 : 0u;
+              sraw[t][h] = r;
+            }
+        }
         float acc[kTiles][NT][4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -383,17 +443,20 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
             }
           }
           if (last) {
-            int gi;
-            if (GPB == 1) gi = (bpg == 1) ? kb : kb / bpg;
-            else gi = kb * GPB + (GPB == 2 ? (j >> 1) : j);
-            const bool gok = gi < G;
-            const int gc = gok ? gi : 0;
+            const int a = (GPB == 1) ? 0 : (GPB == 2 ? (j >> 1) : j);
 #pragma unroll
             for (int t = 0; t < kTiles; ++t) {
-              float sa = f16_bits_to_float(__ldg(sp[t][0] + gc));
-              float sb = f16_bits_to_float(__ldg(sp[t][1] + gc));
-              sa = gok ? sa : 0.0f;
-              sb = gok ? sb : 0.0f;
+              float sa, sb;
+              if (GPB <= 2) {
+                sa = f16_bits_to_float((sraw[t][0] >> (16 * a)) & 0xFFFFu);
+                sb = f16_bits_to_float((sraw[t][1] >> (16 * a)) & 0xFFFFu);
+              } else {
+                const int gi = kb * GPB + a;
+                const bool gok = gi < G;
+                const int gc = gok ? gi : 0;
+                sa = gok ? f16_bits_to_float(__ldg(sp[t][0] + gc)) : 0.0f;
+                sb = gok ? f16_bits_to_float(__ldg(sp[t][1] + gc)) : 0.0f;
+              }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 tot[t][nt][0] = fmaf(acc[t][nt][0], sa, tot[t][nt][0]);
@@ -405,62 +468,86 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
-    }
-  }
-
-  // Partials of every consumer to shared memory; each output is the sum over
-  // the CTA's two K-block slots (and over the cluster's ranks), in a fixed order.
-  if (warp > 0) {
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          red[(((cw * kTiles + t) * NT + nt) * 4 + i) * 32 + lane] = tot[t][nt][i];
-  }
-  constexpr int kPer = kRowGroups * kTiles * NT * 4 * 32;  // outputs per CTA
-  if (S == 1) {
-    __syncthreads();
-    if (*abort_flag == 0u) {
-      for (int e = threadIdx.x; e < kPer; e += blockDim.x) {
-        float sum = 0.0f;
-#pragma unroll
-        for (int q = 0; q < kSK; ++q) sum += red[q * kPer + e];
-        const int ln = e & 31;
-        const int i = (e >> 5) & 3;
-        const int nt = (e >> 7) % NT;
-        const int tw = (e >> 7) / NT;  // rg * kTiles + t
-        const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
-        const int64_t row = row0 + tw * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
-        if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
       }
-    }
-    return;
-  }
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  bool all_ok = true;
-  for (int r = 0; r < S; ++r)
-    all_ok = all_ok && (*cluster.map_shared_rank(const_cast<uint32_t*>(abort_flag), r) == 0u);
-  for (int e = slice * blockDim.x + threadIdx.x; e < kPer; e += S * blockDim.x) {
-    float sum = 0.0f;
-    for (int r = 0; r < S; ++r) {
-      const float* rr = cluster.map_shared_rank(red, r);
+      // Segment end: the two K-block slots of each row group are summed in a
+      // fixed order.  The first barrier also agrees on whether any wait gave
+      // up, so that every consumer leaves the loop at the same segment.
 #pragma unroll
-      for (int q = 0; q < kSK; ++q) sum += rr[q * kPer + e];
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            red[(((cw * kTiles + t) * NT + nt) * 4 + i) * 32 + lane] = tot[t][nt][i];
+      const bool stop = ptx::bar_red_or(1, kConsumers * 32, !ok || *abort_flag != 0u);
+      if (!stop) {
+        const bool whole = (blo == 0 && bhi == KB);
+        float* dst = whole ? nullptr
+                           : partials + (2 * static_cast<int64_t>(blockIdx.x) + (blo == 0 ? 1 : 0)) * kPer;
+        for (int e = threadIdx.x - 32; e < kPer; e += kConsumers * 32) {
+          float sum = 0.0f;
+#pragma unroll
+          for (int q = 0; q < kSK; ++q) sum += red[q * kPer + e];
+          if (!whole) {
+            dst[e] = sum;
+            continue;
+          }
+          const int ln = e & 31;
+          const int i = (e >> 5) & 3;
+          const int nt = (e >> 7) % NT;
+          const int tw = (e >> 7) / NT;  // rg * kTiles + t
+          const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
+          const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
+          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+        }
+      }
+      ptx::bar_sync(1, kConsumers * 32);  // red is rewritten by the next segment
+      if (stop) break;
+      u = r * KB + bhi;
     }
+  }
+}
+
+// Sums the partial tiles of the stream-K split in CTA order and writes y.
+// Block b handles the tile that holds the start of decode CTA b + 1's run,
+// if that start lies inside a tile and is the first such start in it.
+template <int NT, int GPB>
+__global__ void __launch_bounds__(256) decode_fixup_kernel(const float* __restrict__ partials,
+                                                           float* __restrict__ y, int M, int64_t N,
+                                                           int KB, int64_t U, int P) {
+  constexpr int kTiles = Tiles<NT>::kTiles;
+  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
+  constexpr int kPer = kRowGroups * kTiles * NT * 4 * 32;
+  const int64_t start = static_cast<int64_t>(blockIdx.x + 1) * U / P;
+  const int64_t r = start / KB;
+  if (start % KB == 0) return;
+  // CTAs whose runs meet tile r: p_first is the last CTA starting at or
+  // before the tile start, p_last the last starting before the tile end.
+  const int64_t t0 = r * KB, t1 = (r + 1) * KB;
+  const int p_first = static_cast<int>(((t0 + 1) * P + U - 1) / U - 1);
+  const int p_last = static_cast<int>((t1 * P + U - 1) / U - 1);
+  if (p_first != static_cast<int>(blockIdx.x)) return;  // another block owns this tile
+  ptx::grid_dependency_wait();
+  const int64_t row0 = r * kRowsPerCta;
+  // p_first starts at or before the tile start, so its piece is its run's
+  // last segment (slot 2p + 1); every later contributor starts inside the
+  // tile, so its piece is its run's first segment (slot 2p).
+  const float* first = partials + (2 * static_cast<int64_t>(p_first) + 1) * kPer;
+  const float* rest = partials + 2 * static_cast<int64_t>(p_first + 1) * kPer;
+  const int n_rest = p_last - p_first;
+  for (int e = threadIdx.x; e < kPer; e += blockDim.x) {
+    float sum = first[e];
+    for (int q = 0; q < n_rest; ++q) sum += rest[static_cast<int64_t>(2 * q) * kPer + e];
     const int ln = e & 31;
     const int i = (e >> 5) & 3;
     const int nt = (e >> 7) % NT;
     const int tw = (e >> 7) / NT;
     const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
-    const int64_t row = row0 + tw * 16 + (ln >> 2) + ((i < 2) ? 0 : 8);
-    if (all_ok && m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+    const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
+    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
   }
-  cluster.sync();  // keep this CTA's partials alive until every rank has read them
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -481,33 +568,86 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Pool for the partial tiles of the stream-K split, one per device, owned by
+// the library.  Blocks are taken and returned in stream order, so calls on
+// different streams never share one; freed blocks stay in the pool for reuse.
+cudaError_t partials_pool(cudaMemPool_t* out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (pools[dev] == nullptr) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
 template <typename TX, int NT, int GPB>
 cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                            int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
   using L = DLayout<NT>;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
+  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   uint32_t* status = status_word();
   if (status == nullptr) return cudaErrorInvalidSymbol;
   const int G = static_cast<int>((K + group - 1) / group);
-  const int64_t KB = (K + 127) / 128;
+  const int KB = static_cast<int>((K + 127) / 128);
   const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t U = R * KB;  // (row tile, K block) units
   auto kern = decode_kernel<TX, NT, GPB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  // Shared-memory opt-in and occupancy, once per device for this kernel.
+  constexpr int kMaxDevices = 64;
+  static std::atomic<int> occ_cache[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
-  if (e != cudaSuccess) return e;
-  if (occ < 1) occ = 1;
-  // One wave of CTAs at the occupancy limit, at most 8 K slices per cluster.
-  const int64_t slots = static_cast<int64_t>(occ) * num_sms();
-  int64_t S = slots / R;
-  if (S > kMaxCluster) S = kMaxCluster;
-  if (S > KB) S = KB;
-  if (S < 1) S = 1;
-  const int kbps = static_cast<int>((KB + S - 1) / S);
-  S = (KB + kbps - 1) / kbps;  // no empty slices
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int occ = occ_cache[dev].load(std::memory_order_relaxed);
+  if (occ == 0) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    occ_cache[dev].store(occ, std::memory_order_relaxed);
+  }
+  // One wave of CTAs at the occupancy limit, each with an equal run of units.
+  int64_t P = static_cast<int64_t>(occ) * num_sms();
+  if (P > U) P = U;
+  // Does any run start inside a tile?  (Remembered for the last shape seen by
+  // this thread: the scan costs a division per CTA.)
+  thread_local int64_t last_U = -1, last_P = -1, last_KB = -1;
+  thread_local bool last_split = false;
+  if (U != last_U || P != last_P || KB != last_KB) {
+    bool sp = false;
+    for (int64_t p = 1; p < P && !sp; ++p) sp = (p * U / P) % KB != 0;
+    last_U = U;
+    last_P = P;
+    last_KB = KB;
+    last_split = sp;
+  }
+  const bool split = last_split;
 
   CUtensorMap tw, tx;
   {
@@ -533,20 +673,38 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(S), static_cast<unsigned>(R), 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = L::kAlloc;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tw, tx, scales, y, K, group, G, static_cast<int>(M), N, kbps,
-                            static_cast<int>(S), status);
+  float* partials = nullptr;
+  if (split) {
+    cudaMemPool_t pool = nullptr;
+    e = partials_pool(&pool);
+    if (e != cudaSuccess) return e;
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&partials),
+                                static_cast<size_t>(2 * P) * kPer * sizeof(float), pool, stream);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<static_cast<unsigned>(P), kThreads, L::kAlloc, stream>>>(
+      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, KB, U, static_cast<int>(P), partials,
+      status);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && split) {
+    // The fix-up grid is launched early and waits in the kernel for this one.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P - 1), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_fixup_kernel<NT, GPB>, static_cast<const float*>(partials), y,
+                           static_cast<int>(M), N, KB, U, static_cast<int>(P));
+  }
+  if (partials != nullptr) {
+    const cudaError_t f = cudaFreeAsync(partials, stream);
+    if (e == cudaSuccess) e = f;
+  }
+  return e;
 }
 
 template <typename TX, int NT>
@@ -574,7 +732,7 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
   if (!(group == 32 || group == 64 || group % 128 == 0)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return false;
   if (reinterpret_cast<uintptr_t>(packed) % 16 != 0) return false;
-  if ((N + 63) / 64 > 65535) return false;
+  if (N > 0x7FFFFFFFLL) return false;
   return true;
 }
 

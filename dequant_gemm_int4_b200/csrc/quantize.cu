@@ -121,6 +121,45 @@ __device__ __forceinline__ bool codes8_normal(const float (&v)[8], float r, uint
   return dmax < 0.5f - 0x1p-15f;
 }
 
+// Eight codes of one lane for 16-bit weights (bf16 or fp16) and a normal
+// fp16 scale, packed low nibble first; exact with no check.  For such inputs
+// a quotient v / s that is not itself a half-integer lies at least 2^-14
+// away from every half-integer: 2v - (2k + 1)s is a multiple of the smaller
+// of the two unit steps (of 2v and of s), and dividing that step by 2s leaves
+// at least 2^-14 when |v / s| >= 1/8 (smaller quotients round to 0 anyway).
+// fma(v, r, 192) rounds v * r (within 2^-19.5 of the quotient) to the 2^-16
+// grid of [128, 256), which puts an exact tie exactly on k + 1/2 and leaves
+// every other quotient on its own side of the nearest half-integer; adding
+// 1.5 * 2^23 - 192 then rounds that grid value to an integer, ties to even,
+// as rint does on the IEEE quotient.
+__device__ __forceinline__ void codes8_snap(const float (&v)[8], float r, uint32_t& word) {
+  uint32_t nib[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float y1 = __fmaf_rn(v[i], r, 192.0f);
+    nib[i] = __float_as_uint(__fadd_rn(y1, 12582720.0f));
+  }
+  uint32_t b[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t o;
+    asm("lop3.b32 %0, %1, %2, %3, 0xb8;" : "=r"(o) : "r"(nib[2 * j + 1] << 4), "r"(0x0Fu), "r"(nib[2 * j]));
+    b[j] = o;
+  }
+  word = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+}
+
+// Codes of eight weights of type T under a normal (or zero) scale: the
+// checked fast path for fp32 weights, the snapped one for 16-bit weights.
+template <typename T>
+__device__ __forceinline__ bool codes8(const float (&v)[8], float r, uint32_t& word) {
+  if (sizeof(T) == 2) {
+    codes8_snap(v, r, word);
+    return true;
+  }
+  return codes8_normal(v, r, word);
+}
+
 // The exact code, via the fast path and its check (general kernels).
 __device__ __forceinline__ uint32_t code_of(float v, const ScaleInfo& si) {
   bool near = false;
@@ -224,7 +263,7 @@ __global__ void __launch_bounds__(256) quantize_aligned_kernel(
       const uint32_t ex = si.bits & 0x7C00u;
       const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
       uint32_t word;
-      const bool ok = codes8_normal(v[u], si.r, word) && simple;
+      const bool ok = codes8<T>(v[u], si.r, word) && simple;
       if (!__all_sync(0xffffffffu, ok)) {
         if (!ok) {
           word = 0;
@@ -249,7 +288,8 @@ template <typename T, int LPG>
 __global__ void __launch_bounds__(256) quantize_wide_kernel(
     const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
     uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
-  constexpr int kU = 2;  // windows in flight per warp
+  constexpr int kU = 2;                                       // windows per step
+  constexpr int kV = sizeof(T) == 4 ? 4 : 2;                  // 16-byte loads per lane per window
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -263,42 +303,74 @@ __global__ void __launch_bounds__(256) quantize_wide_kernel(
   int col = static_cast<int>(wbeg - row * windows_per_row);
   const int wpr = static_cast<int>(windows_per_row);
 
-  for (; wbeg < wend; wbeg += kU) {
-    float v[kU][2][8];
-    int64_t rw[kU];
-    int ch[kU];
-    bool valid[kU];
+  // Raw 16-byte words of the next step are loaded while the current one is
+  // quantized, so every warp keeps its next loads in flight.
+  uint4 raw[kU][kV], nraw[kU][kV];
+  int64_t rw[kU], nrw[kU];
+  int ch[kU], nch[kU];
+  bool valid[kU], nvalid[kU];
+  auto fetch = [&](int64_t wb, uint4 (&r)[kU][kV], int64_t (&rr)[kU], int (&cc)[kU], bool (&vv)[kU]) {
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      rw[u] = row;
-      ch[u] = col * 32 + lane;
-      valid[u] = (wbeg + u < wend) && (ch[u] < chunks_per_row);
-      if (valid[u]) {
-        const T* p = w + row * K + static_cast<int64_t>(ch[u]) * 16;
-        Load8<T>::run(p, v[u][0]);
-        Load8<T>::run(p + 8, v[u][1]);
-      } else {
+      rr[u] = row;
+      cc[u] = col * 32 + lane;
+      vv[u] = (wb + u < wend) && (cc[u] < chunks_per_row);
+      const uint4* p = reinterpret_cast<const uint4*>(w + row * K + static_cast<int64_t>(cc[u]) * 16);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[u][0][i] = v[u][1][i] = 0.0f;
-      }
+      for (int q = 0; q < kV; ++q) r[u][q] = vv[u] ? __ldg(p + q) : make_uint4(0u, 0u, 0u, 0u);
       if (++col == wpr) {
         col = 0;
         ++row;
       }
     }
+  };
+  fetch(wbeg, nraw, nrw, nch, nvalid);
+  for (; wbeg < wend; wbeg += kU) {
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
+      rw[u] = nrw[u];
+      ch[u] = nch[u];
+      valid[u] = nvalid[u];
+#pragma unroll
+      for (int q = 0; q < kV; ++q) raw[u][q] = nraw[u][q];
+    }
+    if (wbeg + kU < wend) fetch(wbeg + kU, nraw, nrw, nch, nvalid);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      float v[2][8];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        if (sizeof(T) == 4) {
+          const uint4 a = raw[u][2 * hh], bq = raw[u][2 * hh + 1];
+          const uint32_t ws[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[hh][i] = __uint_as_float(ws[i]);
+        } else {
+          const uint4 a = raw[u][hh];
+          const uint32_t ws[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (std::is_same<T, __nv_bfloat16>::value) {
+              v[hh][2 * i] = __uint_as_float(ws[i] << 16);
+              v[hh][2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+            } else {
+              v[hh][2 * i] = f16_bits_to_float(ws[i] & 0xFFFFu);
+              v[hh][2 * i + 1] = f16_bits_to_float(ws[i] >> 16);
+            }
+          }
+        }
+      }
       float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(v[u][0][i]), fabsf(v[u][1][i])));
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fabsf(v[0][i]), fabsf(v[1][i])));
 #pragma unroll
       for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       const ScaleInfo si = scale_from_absmax(m);
       const uint32_t ex = si.bits & 0x7C00u;
       const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
       uint32_t w0, w1;
-      const bool ok0 = codes8_normal(v[u][0], si.r, w0);
-      const bool ok1 = codes8_normal(v[u][1], si.r, w1);
+      const bool ok0 = codes8<T>(v[0], si.r, w0);
+      const bool ok1 = codes8<T>(v[1], si.r, w1);
       const bool ok = ok0 && ok1 && simple;
       if (!__all_sync(0xffffffffu, ok)) {
         if (!ok) {
@@ -306,8 +378,8 @@ __global__ void __launch_bounds__(256) quantize_wide_kernel(
           w1 = 0;
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            w0 |= code_exact(v[u][0][i], si) << (4 * i);
-            w1 |= code_exact(v[u][1][i], si) << (4 * i);
+            w0 |= code_exact(v[0][i], si) << (4 * i);
+            w1 |= code_exact(v[1][i], si) << (4 * i);
           }
         }
       }
@@ -344,23 +416,40 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
   int64_t row = wi / windows_per_row;
   int64_t col = wi - row * windows_per_row;
 
-  for (; wi < wend; ++wi) {
+  // The next window's chunks are loaded while the current one is quantized.
+  auto fetch = [&](int64_t r, int64_t cl, uint4 (&own)[NCH], uint4& extra) {
+    const int64_t c0 = (wshift + (r * K + cl * 256 + lane * 8) * ELT) >> 4;
+#pragma unroll
+    for (int q = 0; q < NCH; ++q) own[q] = load_chunk16(wbase, c0 + q, wbytes);
+    extra = (lane == 31) ? load_chunk16(wbase, c0 + NCH, wbytes) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 own[NCH], extra;
+  fetch(row, col, own, extra);
+  for (; wi < wend;) {
+    uint4 cur[NCH];
+#pragma unroll
+    for (int q = 0; q < NCH; ++q) cur[q] = own[q];
+    const uint4 cur_extra = extra;
     const int64_t kl = col * 256 + lane * 8;  // first element of this lane in the row
     const int64_t P = wshift + (row * K + kl) * ELT;
-    const int64_t c0 = P >> 4;
     const int boff = static_cast<int>(P & 15);
+    const int64_t crow = row, ccol = col;
+    if (++col == windows_per_row) {
+      col = 0;
+      ++row;
+    }
+    if (++wi < wend) fetch(row, col, own, extra);
     uint32_t win[4 * (NCH + 1)];
 #pragma unroll
     for (int q = 0; q < NCH; ++q) {
-      const uint4 v = load_chunk16(wbase, c0 + q, wbytes);
-      win[4 * q] = v.x; win[4 * q + 1] = v.y; win[4 * q + 2] = v.z; win[4 * q + 3] = v.w;
+      win[4 * q] = cur[q].x; win[4 * q + 1] = cur[q].y; win[4 * q + 2] = cur[q].z; win[4 * q + 3] = cur[q].w;
     }
     uint4 nx;
     nx.x = __shfl_down_sync(0xffffffffu, win[0], 1);
     nx.y = __shfl_down_sync(0xffffffffu, win[1], 1);
     nx.z = __shfl_down_sync(0xffffffffu, win[2], 1);
     nx.w = __shfl_down_sync(0xffffffffu, win[3], 1);
-    if (lane == 31) nx = load_chunk16(wbase, c0 + NCH, wbytes);
+    if (lane == 31) nx = cur_extra;
     win[4 * NCH] = nx.x; win[4 * NCH + 1] = nx.y; win[4 * NCH + 2] = nx.z; win[4 * NCH + 3] = nx.w;
     uint32_t e[4 * NCH];
     byte_shift_words<4 * (NCH + 1), 4 * NCH>(win, boff, e);
@@ -382,7 +471,7 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
     const uint32_t ex = si.bits & 0x7C00u;
     const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
     uint32_t word;
-    const bool ok = codes8_normal(v, si.r, word) && simple;
+    const bool ok = codes8<T>(v, si.r, word) && simple;
     if (!__all_sync(0xffffffffu, ok)) {
       if (!ok) {
         word = 0;
@@ -390,16 +479,12 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
         for (int i = 0; i < 8; ++i) word |= code_exact(v[i], si) << (4 * i);
       }
     }
-    if (kl < K && (lane & (LPG - 1)) == 0) scales[row * G + kl / (8 * LPG)] = static_cast<uint16_t>(si.bits);
-    const int64_t rowp = pshift + row * Kp;
-    const int64_t f0 = rowp + col * 128;
+    if (kl < K && (lane & (LPG - 1)) == 0) scales[crow * G + kl / (8 * LPG)] = static_cast<uint16_t>(si.bits);
+    const int64_t rowp = pshift + crow * Kp;
+    const int64_t f0 = rowp + ccol * 128;
     const int64_t hi = (f0 + 128 < rowp + Kp) ? f0 + 128 : rowp + Kp;
     const uint32_t wd[1] = {word};
     store_segment<1>(pbase, f0, f0, hi, wd, lane);
-    if (++col == windows_per_row) {
-      col = 0;
-      ++row;
-    }
   }
 }
 
@@ -463,11 +548,12 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
   if (wide) {
     const int64_t wpr = (K / 16 + 31) / 32;
     const int64_t total = N * wpr;
-    const int grid = grid_for(total, 8 * 2, 8);
+    const int64_t want = (total + 15) / 16;  // two windows per warp at least
     switch (lpg16) {
-#define INT4_QW_CASE(L)                                                                       \
-  case L:                                                                                     \
-    quantize_wide_kernel<T, L><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed, scales); \
+#define INT4_QW_CASE(L)                                                                     \
+  case L:                                                                                   \
+    quantize_wide_kernel<T, L><<<resident_grid(quantize_wide_kernel<T, L>, want), 256, 0,   \
+                                 stream>>>(w, K, G, wpr, total, packed, scales);            \
     break;
       INT4_QW_CASE(1)
       INT4_QW_CASE(2)
@@ -484,11 +570,12 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
   if (aligned && pow2_group) {
     const int64_t wpr = (K / 8 + 31) / 32;
     const int64_t total = N * wpr;
-    const int grid = grid_for(total, 8 * kUnroll, 8);
+    const int64_t want = (total + 8 * kUnroll - 1) / (8 * kUnroll);
     switch (lpg) {
 #define INT4_Q_CASE(L)                                                                       \
   case L:                                                                                    \
-    quantize_aligned_kernel<T, L><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed, scales); \
+    quantize_aligned_kernel<T, L><<<resident_grid(quantize_aligned_kernel<T, L>, want), 256, \
+                                    0, stream>>>(w, K, G, wpr, total, packed, scales);       \
     break;
       INT4_Q_CASE(1)
       INT4_Q_CASE(2)
@@ -512,11 +599,12 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
     const int64_t wpr = (K + 255) / 256;
     const int64_t total = N * wpr;
     const int64_t wbytes = wshift + N * K * static_cast<int64_t>(sizeof(T));
-    const int grid = grid_for(total, 8 * 4, 8);
+    const int64_t want = (total + 31) / 32;
     switch (lpg) {
 #define INT4_QA_CASE(L)                                                                        \
   case L:                                                                                      \
-    quantize_any_kernel<T, L><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint8_t*>(wbase), \
+    quantize_any_kernel<T, L><<<resident_grid(quantize_any_kernel<T, L>, want), 256, 0,        \
+                                stream>>>(reinterpret_cast<const uint8_t*>(wbase),             \
                                                         wshift, wbytes, K, G, wpr, total, pbase, \
                                                         pshift, scales);                         \
     break;

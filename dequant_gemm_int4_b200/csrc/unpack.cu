@@ -74,29 +74,37 @@ __global__ void __launch_bounds__(256) unpack_any_kernel(const uint8_t* __restri
   const int64_t Kp = (K + 1) >> 1;
   int64_t row = wi / windows_per_row;
   int64_t col = wi - row * windows_per_row;
-  for (; wi < wend; ++wi) {
-    const int64_t P = pshift + row * Kp + col * 256 + lane * 8;
-    const int64_t c = P >> 3;
-    const int boff = static_cast<int>(P & 7);
-    const uint2 own = load_chunk8(pbase, c, pbytes);
+  // The next window's chunk is loaded while the current one is expanded.
+  auto fetch = [&](int64_t r, int64_t cl, uint2& own, uint2& extra) {
+    const int64_t c = (pshift + r * Kp + cl * 256 + lane * 8) >> 3;
+    own = load_chunk8(pbase, c, pbytes);
+    extra = (lane == 31) ? load_chunk8(pbase, c + 1, pbytes) : make_uint2(0u, 0u);
+  };
+  uint2 own, extra;
+  fetch(row, col, own, extra);
+  for (; wi < wend;) {
+    const uint2 cur = own, cur_extra = extra;
+    const int boff = static_cast<int>((pshift + row * Kp + col * 256 + lane * 8) & 7);
+    const int64_t crow = row, ccol = col;
+    if (++col == windows_per_row) {
+      col = 0;
+      ++row;
+    }
+    if (++wi < wend) fetch(row, col, own, extra);
     uint2 nx;
-    nx.x = __shfl_down_sync(0xffffffffu, own.x, 1);
-    nx.y = __shfl_down_sync(0xffffffffu, own.y, 1);
-    if (lane == 31) nx = load_chunk8(pbase, c + 1, pbytes);
-    const uint32_t win[4] = {own.x, own.y, nx.x, nx.y};
+    nx.x = __shfl_down_sync(0xffffffffu, cur.x, 1);
+    nx.y = __shfl_down_sync(0xffffffffu, cur.y, 1);
+    if (lane == 31) nx = cur_extra;
+    const uint32_t win[4] = {cur.x, cur.y, nx.x, nx.y};
     uint32_t b8[2];
     byte_shift_words<4, 2>(win, boff, b8);
     const uint2 a = expand_word(b8[0]);
     const uint2 b = expand_word(b8[1]);
     const uint32_t o[4] = {a.x, a.y, b.x, b.y};
-    const int64_t rowo = oshift + row * K;
-    const int64_t f0 = rowo + col * 512;
+    const int64_t rowo = oshift + crow * K;
+    const int64_t f0 = rowo + ccol * 512;
     const int64_t hi = (f0 + 512 < rowo + K) ? f0 + 512 : rowo + K;
     store_segment<4>(obase, f0, f0, hi, o, lane);
-    if (++col == windows_per_row) {
-      col = 0;
-      ++row;
-    }
   }
 }
 
@@ -122,10 +130,8 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* o
   const int64_t oshift = static_cast<int64_t>(oa & 3);
   const int64_t wpr = (K + 511) / 512;
   const int64_t total = N * wpr;
-  int64_t grid = (total + 31) / 32;
-  if (grid > static_cast<int64_t>(num_sms()) * 8) grid = static_cast<int64_t>(num_sms()) * 8;
-  if (grid < 1) grid = 1;
-  unpack_any_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(
+  const int grid = resident_grid(unpack_any_kernel, (total + 31) / 32);
+  unpack_any_kernel<<<grid, 256, 0, stream>>>(
       pbase, pshift, pshift + N * ((K + 1) / 2), K, wpr, total, obase, oshift);
   return cudaGetLastError();
 }

@@ -107,6 +107,44 @@ def test_quantize_half_integer_quotients(group):
         assert_quantize_exact(wd, packed, scales, group)
 
 
+def _every_16bit_weight_under_anchors(dtype, n_anchors, seed):
+    """Groups of 16: an anchor a (the group's absmax, so the scale is
+    fp16(a / 7)) followed by 15 weights taken from every finite value of the
+    16-bit type with |v| <= |a|, both signs.  Anchors span the normal fp16
+    scale range with random significands."""
+    rng = np.random.default_rng(seed)
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    if dtype == torch.bfloat16:
+        vals = (allbits.astype(np.uint32) << 16).view(np.float32)
+    else:
+        vals = allbits.view(np.float16).astype(np.float32)
+    vals = vals[np.isfinite(vals)]
+    rows = []
+    for _ in range(n_anchors):
+        e = rng.integers(-14, 13)
+        a = np.float32(7.0 * (1.0 + rng.random()) * 2.0 ** e)
+        a = np.float32(torch.tensor(a).to(dtype).float().item())   # representable anchor
+        v = vals[np.abs(vals) <= a]
+        v = rng.permutation(v)
+        pad = (-len(v)) % 15
+        v = np.concatenate([v, np.zeros(pad, np.float32)]).reshape(-1, 15)
+        rows.append(np.concatenate([np.full((len(v), 1), a, np.float32), v], axis=1))
+    g = np.concatenate(rows, axis=0)                      # [groups, 16]
+    g = np.concatenate([g, np.zeros(((-len(g)) % 16, 16), np.float32)])
+    w = g.reshape(-1, 256)                                # 16 groups per row
+    return torch.from_numpy(w).to(DEV).to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_every_16bit_weight(dtype):
+    """Every finite bf16 / fp16 weight value, under scales from all normal
+    fp16 binades, quantized by the 16-bit fast path (no tie check): codes and
+    scales bit-exact against the oracle's IEEE division and rint."""
+    w = _every_16bit_weight_under_anchors(dtype, n_anchors=24, seed=5 if dtype == torch.bfloat16 else 6)
+    packed, scales, K = q4.quantize_int4(w, 16)
+    assert_quantize_exact(w, packed, scales, 16)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("N, K, group", [
     (1, 8, 8), (3, 256, 32), (17, 1024, 128), (5, 1000, 64), (64, 4096, 256),
@@ -351,6 +389,28 @@ def test_matmul_decode_is_deterministic_and_matches_simt():
     assert torch.equal(a, b)
     rel = ((a - c).abs().max() / c.abs().max()).item()
     assert rel < 1e-4
+
+
+@pytest.mark.parametrize("M, N, K, group", [
+    (1, 128, 8192, 128),     # one row tile over up to 64 CTAs: every run is a partial tile
+    (3, 256, 16384, 64),     # two tiles, many runs inside each
+    (16, 64, 4096, 32),      # 64-row tiles, one tile
+    (8, 1000, 12288, 128),   # ragged last tile, runs cross tile boundaries
+    (2, 37, 4096, 256),      # a single short tile, group spanning two blocks
+    (5, 6000, 1024, 128),    # many tiles, runs of whole tiles plus boundary pieces
+])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_matmul_decode_split_tiles(M, N, K, group, dtype):
+    """Decode work split into equal runs of (row tile, K block) units, with the
+    partial tiles summed afterwards: shapes whose runs start and end inside
+    tiles, many runs per tile, and ragged tiles."""
+    packed, scales, _ = _quantized(N, K, group, seed=N + K, dist="student_t3", zero_group_frac=0.02)
+    x = make_activations(M, K, seed=M + K, device=DEV, dtype=dtype)
+    a = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
+    b = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert_matmul_close(a, x, packed, scales, K, group, _tol(dtype))
 
 
 @pytest.mark.parametrize("layer", LLAMA7B_DECODE_LINEARS, ids=lambda l: l.name)
