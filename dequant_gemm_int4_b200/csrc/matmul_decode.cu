@@ -20,9 +20,7 @@
 //     is ((w >> 4i) & 0x000F000F) ^ magic, then one packed subtract (magic =
 //     128 + 8 (bf16) or 1024 + 8 (fp16) in each half; the XOR flips the
 //     nibble's sign bit so that the value is q + 136 or q + 1032 before the
-//     subtract).  The shifts are multiply-highs, which issue on the FMA pipe:
-//     the mask and permute instructions share a logic pipe that runs at half
-//     rate on this GPU and bounds the kernel;
+//     subtract);
 //   * the 16 x 8 x 16 warp MMA (mma.sync, fp32 accumulate) multiplies them by
 //     x from shared memory; the MMA's k slots see the pairs (e_i, e_{i+4}), so
 //     x is paired the same way in registers (four byte permutes per 16 bytes,
@@ -129,19 +127,11 @@ struct Cvt<__half> {
   }
 };
 
-// w >> n as a multiply-high, which issues on the FMA pipe; the logic pipe that
-// the masks and permutes need runs at half rate on this GPU.
-__device__ __forceinline__ uint32_t shr_mul(uint32_t w, uint32_t two_pow_32_minus_n) {
-  uint32_t r;
-  asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(two_pow_32_minus_n));
-  return r;
-}
-
 // Word w = 8 consecutive k (nibbles e0..e7 at bits 4i).  p[i] = (e_i, e_{i+4})
 // as bf16x2 / f16x2: ((w >> 4i) & 0x000F000F) ^ magic, minus the bias.
 template <typename TX>
 __device__ __forceinline__ void expand(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t v[4] = {w, shr_mul(w, 1u << 28), shr_mul(w, 1u << 24), shr_mul(w, 1u << 20)};
+  const uint32_t v[4] = {w, w >> 4, w >> 8, w >> 12};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t r;
