@@ -71,12 +71,14 @@ def lib() -> ctypes.CDLL:
         L.int4_matmul.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
         L.int4_matmul_path.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, i32, vp]
         L.int4_matmul_select.argtypes = [i32, i64, i32, i64, i64]
+        L.int4_matmul_decode_noalloc.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
         L.int4_device_status.argtypes = [vp]
         L.int4_selftest_wait_timeout.argtypes = [u32, vp]
         L.int4_last_error.restype = ctypes.c_char_p
         L.int4_last_error.argtypes = []
         L.int4_version.argtypes = []
         for name in ("int4_quantize", "int4_unpack", "int4_matmul", "int4_matmul_path",
+                     "int4_matmul_decode_noalloc",
                      "int4_matmul_select", "int4_device_status", "int4_selftest_wait_timeout",
                      "int4_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -161,6 +163,27 @@ def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: 
     else:
         with torch.cuda.device(x.device):
             _check(L.int4_matmul_path(*args, _stream(x)))
+    return out
+
+
+def int4_matmul_decode_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                               K: int, group: int, out: torch.Tensor) -> torch.Tensor:
+    """The decode matmul into a caller-provided `out` [M, N] float32, with no
+    device allocation in the call (the library's fixed scratch holds the
+    partial tiles).  Calls that may overlap in time race on that scratch."""
+    _need_cuda("x", x)
+    _need_cuda("packed", packed)
+    _need_cuda("scales", scales)
+    _need_cuda("out", out)
+    M, N = x.shape[0], packed.shape[0]
+    if x.dim() != 2 or x.shape[1] != K or x.dtype not in _DTYPE_CODE:
+        raise ValueError("x must be [M, K] float32, bfloat16 or float16")
+    if out.dtype != torch.float32 or tuple(out.shape) != (M, N):
+        raise ValueError("out must be float32 [M, N]")
+    with torch.cuda.device(x.device):
+        _check(lib().int4_matmul_decode_noalloc(x.data_ptr(), _DTYPE_CODE[x.dtype],
+                                                packed.data_ptr(), scales.data_ptr(), K,
+                                                int(group), M, N, out.data_ptr(), _stream(x)))
     return out
 
 

@@ -203,6 +203,31 @@ int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uin
   return int4_matmul_path(x, x_dtype, packed, scales, K, group, M, N, y, INT4_PATH_AUTO, stream);
 }
 
+int int4_matmul_decode_noalloc(const void* x, int32_t x_dtype, const uint8_t* packed,
+                               const uint16_t* scales, int64_t K, int32_t group, int64_t M,
+                               int64_t N, float* y, void* stream) {
+  const int rc = matmul_check(x, x_dtype, packed, scales, K, group, M, N, y);
+  if (rc != INT4_OK || M == 0 || N == 0) return rc;
+  const DType t = static_cast<DType>(x_dtype);
+  if (!int4lib::decode_supported(t, K, group, M, N, x, packed))
+    return int4lib::fail(INT4_ERR_UNSUPPORTED,
+                         "int4_matmul_decode_noalloc: the decode kernel cannot run this shape "
+                         "(needs bf16/fp16 x, M <= 16, K % 32 == 0, group 32, 64 or a multiple of "
+                         "128, 16-byte aligned x and packed)");
+  size_t need = 0;
+  const cudaError_t e = int4lib::launch_matmul_decode_noalloc(
+      x, t, packed, scales, K, group, M, N, y, static_cast<cudaStream_t>(stream), &need);
+  if (e == cudaErrorInvalidValue && need > 0) {
+    char msg[200];
+    std::snprintf(msg, sizeof msg,
+                  "int4_matmul_decode_noalloc: this split needs %zu bytes of scratch, the static "
+                  "scratch holds %zu",
+                  need, int4lib::decode_noalloc_scratch_bytes());
+    return int4lib::fail(INT4_ERR_ARG, msg);
+  }
+  return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_matmul_decode_noalloc");
+}
+
 int int4_matmul_select(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N) {
   if (!int4lib::dtype_ok(x_dtype)) return -INT4_ERR_DTYPE;
   if (M < 0 || N < 0 || K < 1 || group < 1) return -INT4_ERR_ARG;

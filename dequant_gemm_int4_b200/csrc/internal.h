@@ -35,6 +35,12 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
 cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
                                  const uint16_t* scales, int64_t K, int group, int64_t M,
                                  int64_t N, float* y, cudaStream_t stream);
+// The same decode matmul with its partial tiles in a fixed static scratch
+// (no allocation).  cudaErrorInvalidValue with *need set: scratch too small.
+cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t* packed,
+                                         const uint16_t* scales, int64_t K, int group, int64_t M,
+                                         int64_t N, float* y, cudaStream_t stream, size_t* need);
+size_t decode_noalloc_scratch_bytes();
 // matmul_prefill.cu
 bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                        const uint8_t* packed);

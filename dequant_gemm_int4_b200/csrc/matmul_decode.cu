@@ -697,6 +697,137 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
   return e;
 }
 
+// Scratch of int4_matmul_decode_noalloc: the partial tiles of the stream-K
+// split live in this fixed device array instead of pool memory.  2 slots of
+// 1024 floats per CTA, so 4 MiB holds one wave of up to 512 CTAs (B200 runs
+// 296: 2 per SM).
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the scratch on the current device, resolved once per
+// device with cudaGetSymbolAddress (no allocation).
+cudaError_t noalloc_scratch(float** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static float* cache[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess) return e;
+    cache[dev] = static_cast<float*>(p);
+  }
+  *out = cache[dev];
+  return cudaSuccess;
+}
+
+// The decode launch of launch_variant with the partial tiles in the static
+// scratch.  Returns cudaErrorInvalidValue with *need set when the split needs
+// more scratch than the array holds (more than 512 CTAs in one wave).
+template <typename TX, int NT, int GPB>
+cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                                   int64_t K, int group, int64_t M, int64_t N, float* y,
+                                   cudaStream_t stream, size_t* need) {
+  using L = DLayout<NT>;
+  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
+  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
+  float* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  const int G = static_cast<int>((K + group - 1) / group);
+  const int KB = static_cast<int>((K + 127) / 128);
+  const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t U = R * KB;
+  auto kern = decode_kernel<TX, NT, GPB>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) occ = 1;
+  int64_t P = static_cast<int64_t>(occ) * num_sms();
+  if (P > U) P = U;
+  bool split = false;
+  for (int64_t p = 1; p < P && !split; ++p) split = (p * U / P) % KB != 0;
+  if (split) {
+    const size_t bytes = static_cast<size_t>(2 * P) * kPer * sizeof(float);
+    if (bytes > kNoAllocScratchBytes) {
+      *need = bytes;
+      return cudaErrorInvalidValue;
+    }
+  }
+  CUtensorMap tw, tx;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {128, kRowsPerCta};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
+                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  float* partials = split ? scratch : nullptr;
+  kern<<<static_cast<unsigned>(P), kThreads, L::kAlloc, stream>>>(
+      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, KB, U, static_cast<int>(P), partials,
+      status);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && split) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(P - 1), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_fixup_kernel<NT, GPB>, static_cast<const float*>(partials), y,
+                           static_cast<int>(M), N, KB, U, static_cast<int>(P));
+  }
+  return e;
+}
+
+template <typename TX, int NT>
+cudaError_t launch_nt_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
+                              size_t* need) {
+  if (group % 128 == 0)
+    return launch_variant_noalloc<TX, NT, 1>(x, packed, scales, K, group, M, N, y, stream, need);
+  if (group == 64)
+    return launch_variant_noalloc<TX, NT, 2>(x, packed, scales, K, group, M, N, y, stream, need);
+  return launch_variant_noalloc<TX, NT, 4>(x, packed, scales, K, group, M, N, y, stream, need);
+}
+
+template <typename TX>
+cudaError_t launch_tx_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
+                              size_t* need) {
+  if (M <= 8) return launch_nt_noalloc<TX, 1>(x, packed, scales, K, group, M, N, y, stream, need);
+  return launch_nt_noalloc<TX, 2>(x, packed, scales, K, group, M, N, y, stream, need);
+}
+
 template <typename TX, int NT>
 cudaError_t launch_nt(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                       int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
@@ -713,6 +844,18 @@ cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales
 }
 
 }  // namespace
+
+size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t* packed,
+                                         const uint16_t* scales, int64_t K, int group, int64_t M,
+                                         int64_t N, float* y, cudaStream_t stream, size_t* need) {
+  if (xt == DType::BF16)
+    return launch_tx_noalloc(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N,
+                             y, stream, need);
+  return launch_tx_noalloc(static_cast<const __half*>(x), packed, scales, K, group, M, N, y, stream,
+                           need);
+}
 
 bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                       const uint8_t* packed) {

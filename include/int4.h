@@ -152,6 +152,34 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
  * (one of INT4_PATH_SIMT / _DECODE / _PREFILL), or a negative status if the
  * arguments are invalid.  Host-only; launches nothing.
  */
+/* Allocation-free decode matmul.  The pages have no counterpart: this entry
+ * exists for callers that must not allocate device memory during the call,
+ * such as a serving loop that runs inside a fixed memory budget, or a
+ * latency-critical path that must not enter an allocator (whose calls can
+ * block, synchronize or fail under memory pressure).
+ *
+ * Computes what int4_matmul computes on its decode path (same kernels, same
+ * result bits), with the partial tiles of the split kept in a fixed
+ * library-owned device array of 4 MiB (one wave of up to 512 CTAs) instead of
+ * pool memory.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ * Nothing in the array needs to start at zero: every partial is written before
+ * it is read in the same call.
+ *
+ * Arguments and layouts are those of int4_matmul.  Returns
+ * INT4_ERR_UNSUPPORTED when the decode kernel cannot run the shape (x must be
+ * bf16 or fp16, M <= 16, K % 32 == 0, group 32, 64 or a multiple of 128, x and
+ * packed 16-byte aligned), and INT4_ERR_ARG with a message naming both sizes
+ * when the split needs more scratch than the array holds.
+ *
+ * The first call on each device resolves the array's address with
+ * cudaGetSymbolAddress (that device current); make that first call before any
+ * stream capture.  The array is shared by all calls on a device: calls that
+ * can overlap in time (different streams, or host threads) race on it and
+ * must be serialized by the caller. */
+int int4_matmul_decode_noalloc(const void* x, int32_t x_dtype, const uint8_t* packed,
+                               const uint16_t* scales, int64_t K, int32_t group, int64_t M,
+                               int64_t N, float* y, void* stream);
+
 int int4_matmul_select(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N);
 
 /*

@@ -1,0 +1,50 @@
+"""The allocation-free decode entry point against the regular one.
+
+Collected last (file name), so it also runs after every other GPU test has
+used the regular path on the same device."""
+
+import numpy as np
+import pytest
+import torch
+
+import dequant_gemm_int4_b200 as q4
+from gpu_util import TOL_HALF, assert_matmul_close
+from workloads import make_activations, make_weights
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.mark.parametrize("M, N, K, group, dtype", [
+    (1, 28672, 8192, 128, torch.bfloat16),   # partial tiles at most run ends
+    (4, 4096, 4096, 128, torch.bfloat16),    # many runs per tile
+    (16, 1000, 12288, 64, torch.float16),    # 64-row tiles, ragged last tile
+    (3, 37, 4096, 32, torch.bfloat16),       # a single short tile
+])
+def test_noalloc_matches_regular_entry(M, N, K, group, dtype):
+    w = make_weights(N, K, seed=N + K, device=DEV, dtype=torch.float32, dist="student_t3",
+                     zero_group_frac=0.01, group=group)
+    packed, scales, _ = q4.quantize_int4(w, group)
+    del w
+    x = make_activations(M, K, seed=M + 3, device=DEV, dtype=dtype)
+    ref = [q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE) for _ in range(2)]
+    outs = [torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV) for _ in range(2)]
+    for o in outs:                         # two calls in a row
+        q4.int4_matmul_decode_noalloc(x, packed, scales, K, group, o)
+    torch.cuda.synchronize()
+    assert q4.device_status() == q4.OK
+    for r, o in zip(ref, outs):
+        assert torch.equal(r, o)           # same kernels, same split, same bits
+    cols = np.unique(np.random.default_rng(N).integers(0, N, 512))
+    assert_matmul_close(outs[1], x, packed, scales, K, group, TOL_HALF, cols=cols)
+
+
+def test_noalloc_rejects_shapes_the_decode_kernel_cannot_run():
+    K, group, N = 4096, 128, 256
+    w = make_weights(N, K, seed=1, device=DEV, dtype=torch.float32)
+    packed, scales, _ = q4.quantize_int4(w, group)
+    x = make_activations(17, K, seed=1, device=DEV, dtype=torch.bfloat16)   # M > 16
+    out = torch.empty((17, N), dtype=torch.float32, device=DEV)
+    with pytest.raises(q4.Int4Error) as ei:
+        q4.int4_matmul_decode_noalloc(x, packed, scales, K, group, out)
+    assert ei.value.code == q4.ERR_UNSUPPORTED
