@@ -100,7 +100,10 @@ cudaError_t read_and_clear_status(uint32_t* out, cudaStream_t stream) {
   e = cudaMemcpyFromSymbol(out, g_int4_status, sizeof(uint32_t));
   if (e != cudaSuccess) return e;
   const uint32_t zero = 0;
-  return cudaMemcpyToSymbol(g_int4_status, &zero, sizeof(uint32_t));
+  e = cudaMemcpyToSymbol(g_int4_status, &zero, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  if (*out & kStatusTimeout) return reset_split_counters();
+  return cudaSuccess;
 }
 
 cudaError_t launch_wait_timeout_selftest(uint32_t spins, cudaStream_t stream) {

@@ -41,6 +41,9 @@ cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t*
                                          const uint16_t* scales, int64_t K, int group, int64_t M,
                                          int64_t N, float* y, cudaStream_t stream, size_t* need);
 size_t decode_noalloc_scratch_bytes();
+// Zeroes the arrival counters of every split-tile scratch on the current
+// device (after a device-side wait gave up); synchronizes the device.
+cudaError_t reset_split_counters();
 // matmul_prefill.cu
 bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                        const uint8_t* packed);

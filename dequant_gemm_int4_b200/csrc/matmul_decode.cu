@@ -37,16 +37,18 @@
 // Work split (stream-K): the (row tile, 128-k block) units are dealt out in
 // row-major order as equal contiguous runs to one wave of CTAs (two per SM),
 // so every SM streams the same number of bytes whatever N and K are.  A tile
-// that a run covers whole is written to y by its CTA; the pieces of a tile
-// that straddles runs go to a partial buffer, and a small fix-up kernel,
-// launched behind the main one with programmatic dependent launch, adds them
-// in CTA order, so the result does not depend on timing.  Every mbarrier
+// that a run covers whole is written to y by its CTA; each piece of a tile
+// that straddles runs goes to a partial slot, its CTA counts its arrival, and
+// the last contributor to arrive adds the pieces in CTA order (so the result
+// does not depend on timing), writes y and resets the count.  Every mbarrier
 // wait is bounded in time; a wait that gives up aborts the CTA (the status
 // word records it), drains its copies and skips the output.
 #include <cuda.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -219,7 +221,8 @@ template <typename TX, int NT, int GPB>
 __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
-    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* status) {
+    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* __restrict__ counters,
+    uint32_t* status) {
   using L = DLayout<NT>;
   constexpr int kTiles = Tiles<NT>::kTiles;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::offBar);
   uint64_t* empty = full + kStages;
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + L::offMisc);
+  volatile uint32_t* last_flag = abort_flag + 1;
   float* red = reinterpret_cast<float*>(smem + L::offRed);
 
   const int warp = threadIdx.x >> 5;
@@ -239,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
   // order, and CTA p takes units [p U / P, (p + 1) U / P).  The run crosses
   // at most two tile boundaries; a tile it covers whole goes straight to y,
   // a partial tile to its partial slot (2p for the run's first segment when
-  // that starts inside a tile, else 2p + 1), which the fix-up kernel sums.
+  // that starts inside a tile, else 2p + 1), summed by the tile's last
+  // contributor to finish.
   const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * U / P;
   const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * U / P;
   const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;  // all sub-tiles
@@ -256,8 +261,6 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
     ptx::prefetch_tmap(&tm_x);
   }
   __syncthreads();
-  // The fix-up grid may be scheduled now; it waits for this grid to finish.
-  ptx::launch_dependents();
 
   const int c = lane & 3;
   const int g = lane >> 2;
@@ -472,8 +475,8 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           for (int i = 0; i < 4; ++i)
             red[(((cw * kTiles + t) * NT + nt) * 4 + i) * 32 + lane] = tot[t][nt][i];
       const bool stop = ptx::bar_red_or(1, kConsumers * 32, !ok || *abort_flag != 0u);
+      const bool whole = (blo == 0 && bhi == KB);
       if (!stop) {
-        const bool whole = (blo == 0 && bhi == KB);
         float* dst = whole ? nullptr
                            : partials + (2 * static_cast<int64_t>(blockIdx.x) + (blo == 0 ? 1 : 0)) * kPer;
         for (int e = threadIdx.x - 32; e < kPer; e += kConsumers * 32) {
@@ -492,51 +495,46 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
           if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
         }
+        if (!whole) __threadfence();  // this CTA's piece is visible before its arrival counts
       }
       ptx::bar_sync(1, kConsumers * 32);  // red is rewritten by the next segment
       if (stop) break;
+      if (!whole) {
+        // Tile r straddles runs.  Its contributors are CTAs p_first..p_last
+        // (p_first: the last run starting at or before the tile start); each
+        // counts its arrival, and the last to arrive adds the pieces in CTA
+        // order (p_first's is its run's last segment, slot 2p + 1; every later
+        // one starts inside the tile, slot 2p), writes y and resets the count.
+        const int64_t t0 = r * KB, t1 = (r + 1) * KB;
+        const int p_first = static_cast<int>(((t0 + 1) * P + U - 1) / U - 1);
+        const int p_last = static_cast<int>((t1 * P + U - 1) / U - 1);
+        if (cw == 0 && lane == 0) {
+          const uint32_t before = atomicAdd(&counters[p_first], 1u);
+          const bool last = before == static_cast<uint32_t>(p_last - p_first);
+          if (last) __threadfence();
+          *last_flag = last ? 1u : 0u;
+        }
+        ptx::bar_sync(1, kConsumers * 32);
+        if (*last_flag) {
+          const float* first = partials + (2 * static_cast<int64_t>(p_first) + 1) * kPer;
+          const float* rest = partials + 2 * static_cast<int64_t>(p_first + 1) * kPer;
+          const int n_rest = p_last - p_first;
+          for (int e = threadIdx.x - 32; e < kPer; e += kConsumers * 32) {
+            float sum = __ldcg(first + e);
+            for (int q = 0; q < n_rest; ++q) sum += __ldcg(rest + static_cast<int64_t>(2 * q) * kPer + e);
+            const int ln = e & 31;
+            const int i = (e >> 5) & 3;
+            const int nt = (e >> 7) % NT;
+            const int tw = (e >> 7) / NT;
+            const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
+            const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
+            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+          }
+          if (cw == 0 && lane == 0) counters[p_first] = 0u;
+        }
+      }
       u = r * KB + bhi;
     }
-  }
-}
-
-// Sums the partial tiles of the stream-K split in CTA order and writes y.
-// Block b handles the tile that holds the start of decode CTA b + 1's run,
-// if that start lies inside a tile and is the first such start in it.
-template <int NT, int GPB>
-__global__ void __launch_bounds__(256) decode_fixup_kernel(const float* __restrict__ partials,
-                                                           float* __restrict__ y, int M, int64_t N,
-                                                           int KB, int64_t U, int P) {
-  constexpr int kTiles = Tiles<NT>::kTiles;
-  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
-  constexpr int kPer = kRowGroups * kTiles * NT * 4 * 32;
-  const int64_t start = static_cast<int64_t>(blockIdx.x + 1) * U / P;
-  const int64_t r = start / KB;
-  if (start % KB == 0) return;
-  // CTAs whose runs meet tile r: p_first is the last CTA starting at or
-  // before the tile start, p_last the last starting before the tile end.
-  const int64_t t0 = r * KB, t1 = (r + 1) * KB;
-  const int p_first = static_cast<int>(((t0 + 1) * P + U - 1) / U - 1);
-  const int p_last = static_cast<int>((t1 * P + U - 1) / U - 1);
-  if (p_first != static_cast<int>(blockIdx.x)) return;  // another block owns this tile
-  ptx::grid_dependency_wait();
-  const int64_t row0 = r * kRowsPerCta;
-  // p_first starts at or before the tile start, so its piece is its run's
-  // last segment (slot 2p + 1); every later contributor starts inside the
-  // tile, so its piece is its run's first segment (slot 2p).
-  const float* first = partials + (2 * static_cast<int64_t>(p_first) + 1) * kPer;
-  const float* rest = partials + 2 * static_cast<int64_t>(p_first + 1) * kPer;
-  const int n_rest = p_last - p_first;
-  for (int e = threadIdx.x; e < kPer; e += blockDim.x) {
-    float sum = first[e];
-    for (int q = 0; q < n_rest; ++q) sum += rest[static_cast<int64_t>(2 * q) * kPer + e];
-    const int ln = e & 31;
-    const int i = (e >> 5) & 3;
-    const int nt = (e >> 7) % NT;
-    const int tw = (e >> 7) / NT;
-    const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
-    const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
-    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
   }
 }
 
@@ -558,53 +556,101 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Pool for the partial tiles of the stream-K split, one per device, owned by
-// the library.  Blocks are taken and returned in stream order, so calls on
-// different streams never share one; freed blocks stay in the pool for reuse.
-cudaError_t partials_pool(cudaMemPool_t* out) {
+// Scratch of split tiles for one (device, stream): 2 partial slots of kPer
+// floats per CTA and one arrival counter per CTA.  The counters are zeroed
+// when the scratch is made and every call leaves them zero, so calls on one
+// stream (ordered) can share it; calls on different streams use different
+// scratch.  It grows (after the stream drains) when a call needs more.
+struct SplitScratch {
+  float* partials = nullptr;
+  uint32_t* counters = nullptr;
+  size_t partial_floats = 0;
+  size_t counter_count = 0;
+};
+
+std::mutex g_scratch_mu;
+std::map<std::pair<int, cudaStream_t>, SplitScratch>& scratch_map() {
+  static std::map<std::pair<int, cudaStream_t>, SplitScratch> m;
+  return m;
+}
+
+cudaError_t stream_scratch(cudaStream_t stream, size_t partial_floats, size_t counters,
+                           float** p_out, uint32_t** c_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  SplitScratch& sc = scratch_map()[{dev, stream}];
+  if (sc.partial_floats < partial_floats || sc.counter_count < counters) {
+    if (sc.partials != nullptr) {
+      e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return e;
+      cudaFree(sc.partials);
+      sc = SplitScratch{};
+    }
+    const size_t pbytes = (partial_floats * sizeof(float) + 255) & ~static_cast<size_t>(255);
+    void* base = nullptr;
+    e = cudaMalloc(&base, pbytes + counters * sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + pbytes);
+    e = cudaMemsetAsync(cnt, 0, counters * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) {
+      cudaFree(base);
+      return e;
+    }
+    sc.partials = static_cast<float*>(base);
+    sc.counters = cnt;
+    sc.partial_floats = partial_floats;
+    sc.counter_count = counters;
+  }
+  *p_out = sc.partials;
+  *c_out = sc.counters;
+  return cudaSuccess;
+}
+
+// Scratch of int4_matmul_decode_noalloc: partial slots and arrival counters
+// in one fixed device array (zero at load; every call leaves the counters
+// zero).  4 MiB of partials hold one wave of up to 512 CTAs (B200 runs 296:
+// 2 per SM).
+constexpr int kNoAllocMaxCtas = 512;
+constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;
+constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocMaxCtas * sizeof(uint32_t);
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the array on the current device, resolved once per
+// device with cudaGetSymbolAddress (no allocation).
+cudaError_t noalloc_scratch(float** out) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
-  static cudaMemPool_t pools[kMaxDevices] = {};
+  static float* cache[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (pools[dev] == nullptr) {
-    cudaMemPoolProps props = {};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.handleTypes = cudaMemHandleTypeNone;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t pool = nullptr;
-    e = cudaMemPoolCreate(&pool, &props);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    uint64_t keep = ~0ull;
-    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    if (e != cudaSuccess) {
-      cudaMemPoolDestroy(pool);
-      return e;
-    }
-    pools[dev] = pool;
+    cache[dev] = static_cast<float*>(p);
   }
-  *out = pools[dev];
+  *out = cache[dev];
   return cudaSuccess;
 }
 
+// Grid and split of one decode call: one wave of CTAs at the occupancy
+// limit, each with an equal run of (row tile, K block) units.
+struct DecodePlan {
+  int KB = 0;
+  int64_t U = 0;
+  int64_t P = 0;
+  bool split = false;  // does some run start inside a tile?
+};
+
 template <typename TX, int NT, int GPB>
-cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                           int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+cudaError_t plan_decode(int64_t K, int64_t N, DecodePlan* pl) {
   using L = DLayout<NT>;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
-  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return cudaErrorNotSupported;
-  uint32_t* status = status_word();
-  if (status == nullptr) return cudaErrorInvalidSymbol;
-  const int G = static_cast<int>((K + group - 1) / group);
-  const int KB = static_cast<int>((K + 127) / 128);
-  const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
-  const int64_t U = R * KB;  // (row tile, K block) units
   auto kern = decode_kernel<TX, NT, GPB>;
   // Shared-memory opt-in and occupancy, once per device for this kernel.
   constexpr int kMaxDevices = 64;
@@ -622,148 +668,37 @@ cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* s
     if (occ < 1) occ = 1;
     occ_cache[dev].store(occ, std::memory_order_relaxed);
   }
-  // One wave of CTAs at the occupancy limit, each with an equal run of units.
-  int64_t P = static_cast<int64_t>(occ) * num_sms();
-  if (P > U) P = U;
-  // Does any run start inside a tile?  (Remembered for the last shape seen by
-  // this thread: the scan costs a division per CTA.)
+  pl->KB = static_cast<int>((K + 127) / 128);
+  pl->U = ((N + kRowsPerCta - 1) / kRowsPerCta) * pl->KB;
+  pl->P = static_cast<int64_t>(occ) * num_sms();
+  if (pl->P > pl->U) pl->P = pl->U;
+  // Remembered for the last shape seen by this thread: the scan costs a
+  // division per CTA.
   thread_local int64_t last_U = -1, last_P = -1, last_KB = -1;
   thread_local bool last_split = false;
-  if (U != last_U || P != last_P || KB != last_KB) {
+  if (pl->U != last_U || pl->P != last_P || pl->KB != last_KB) {
     bool sp = false;
-    for (int64_t p = 1; p < P && !sp; ++p) sp = (p * U / P) % KB != 0;
-    last_U = U;
-    last_P = P;
-    last_KB = KB;
+    for (int64_t p = 1; p < pl->P && !sp; ++p) sp = (p * pl->U / pl->P) % pl->KB != 0;
+    last_U = pl->U;
+    last_P = pl->P;
+    last_KB = pl->KB;
     last_split = sp;
   }
-  const bool split = last_split;
-
-  CUtensorMap tw, tx;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    const cuuint32_t box[2] = {128, kRowsPerCta};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
-                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  float* partials = nullptr;
-  if (split) {
-    cudaMemPool_t pool = nullptr;
-    e = partials_pool(&pool);
-    if (e != cudaSuccess) return e;
-    e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&partials),
-                                static_cast<size_t>(2 * P) * kPer * sizeof(float), pool, stream);
-    if (e != cudaSuccess) return e;
-  }
-  kern<<<static_cast<unsigned>(P), kThreads, L::kAlloc, stream>>>(
-      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, KB, U, static_cast<int>(P), partials,
-      status);
-  e = cudaGetLastError();
-  if (e == cudaSuccess && split) {
-    // The fix-up grid is launched early and waits in the kernel for this one.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(P - 1), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_fixup_kernel<NT, GPB>, static_cast<const float*>(partials), y,
-                           static_cast<int>(M), N, KB, U, static_cast<int>(P));
-  }
-  if (partials != nullptr) {
-    const cudaError_t f = cudaFreeAsync(partials, stream);
-    if (e == cudaSuccess) e = f;
-  }
-  return e;
-}
-
-// Scratch of int4_matmul_decode_noalloc: the partial tiles of the stream-K
-// split live in this fixed device array instead of pool memory.  2 slots of
-// 1024 floats per CTA, so 4 MiB holds one wave of up to 512 CTAs (B200 runs
-// 296: 2 per SM).
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
-static __device__ __align__(256) float g_noalloc_partials[kNoAllocScratchBytes / sizeof(float)];
-
-// Device address of the scratch on the current device, resolved once per
-// device with cudaGetSymbolAddress (no allocation).
-cudaError_t noalloc_scratch(float** out) {
-  constexpr int kMaxDevices = 64;
-  static std::mutex mu;
-  static float* cache[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-    if (e != cudaSuccess) return e;
-    cache[dev] = static_cast<float*>(p);
-  }
-  *out = cache[dev];
+  pl->split = last_split;
   return cudaSuccess;
 }
 
-// The decode launch of launch_variant with the partial tiles in the static
-// scratch.  Returns cudaErrorInvalidValue with *need set when the split needs
-// more scratch than the array holds (more than 512 CTAs in one wave).
 template <typename TX, int NT, int GPB>
-cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                                   int64_t K, int group, int64_t M, int64_t N, float* y,
-                                   cudaStream_t stream, size_t* need) {
+cudaError_t launch_decode(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                          int group, int64_t M, int64_t N, float* y, const DecodePlan& pl,
+                          float* partials, uint32_t* counters, cudaStream_t stream) {
   using L = DLayout<NT>;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
-  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   uint32_t* status = status_word();
   if (status == nullptr) return cudaErrorInvalidSymbol;
-  float* scratch = nullptr;
-  cudaError_t e = noalloc_scratch(&scratch);
-  if (e != cudaSuccess) return e;
   const int G = static_cast<int>((K + group - 1) / group);
-  const int KB = static_cast<int>((K + 127) / 128);
-  const int64_t R = (N + kRowsPerCta - 1) / kRowsPerCta;
-  const int64_t U = R * KB;
-  auto kern = decode_kernel<TX, NT, GPB>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-  if (e != cudaSuccess) return e;
-  int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
-  if (e != cudaSuccess) return e;
-  if (occ < 1) occ = 1;
-  int64_t P = static_cast<int64_t>(occ) * num_sms();
-  if (P > U) P = U;
-  bool split = false;
-  for (int64_t p = 1; p < P && !split; ++p) split = (p * U / P) % KB != 0;
-  if (split) {
-    const size_t bytes = static_cast<size_t>(2 * P) * kPer * sizeof(float);
-    if (bytes > kNoAllocScratchBytes) {
-      *need = bytes;
-      return cudaErrorInvalidValue;
-    }
-  }
   CUtensorMap tw, tx;
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
@@ -788,25 +723,57 @@ cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  float* partials = split ? scratch : nullptr;
-  kern<<<static_cast<unsigned>(P), kThreads, L::kAlloc, stream>>>(
-      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, KB, U, static_cast<int>(P), partials,
-      status);
-  e = cudaGetLastError();
-  if (e == cudaSuccess && split) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(P - 1), 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_fixup_kernel<NT, GPB>, static_cast<const float*>(partials), y,
-                           static_cast<int>(M), N, KB, U, static_cast<int>(P));
+  decode_kernel<TX, NT, GPB><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, stream>>>(
+      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, pl.KB, pl.U, static_cast<int>(pl.P),
+      partials, counters, status);
+  return cudaGetLastError();
+}
+
+template <typename TX, int NT, int GPB>
+cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                           int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
+  DecodePlan pl;
+  cudaError_t e = plan_decode<TX, NT, GPB>(K, N, &pl);
+  if (e != cudaSuccess) return e;
+  float* partials = nullptr;
+  uint32_t* counters = nullptr;
+  if (pl.split) {
+    e = stream_scratch(stream, static_cast<size_t>(2 * pl.P) * kPer, static_cast<size_t>(pl.P),
+                       &partials, &counters);
+    if (e != cudaSuccess) return e;
   }
-  return e;
+  return launch_decode<TX, NT, GPB>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
+                                    stream);
+}
+
+// launch_variant with the split's scratch in the static array.  Returns
+// cudaErrorInvalidValue with *need set when the split needs more scratch
+// than the array holds (more than 512 CTAs in one wave).
+template <typename TX, int NT, int GPB>
+cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                                   int64_t K, int group, int64_t M, int64_t N, float* y,
+                                   cudaStream_t stream, size_t* need) {
+  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;
+  float* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  DecodePlan pl;
+  e = plan_decode<TX, NT, GPB>(K, N, &pl);
+  if (e != cudaSuccess) return e;
+  float* partials = nullptr;
+  uint32_t* counters = nullptr;
+  if (pl.split) {
+    const size_t bytes = static_cast<size_t>(2 * pl.P) * kPer * sizeof(float);
+    if (bytes > kNoAllocPartialBytes || pl.P > kNoAllocMaxCtas) {
+      *need = bytes + static_cast<size_t>(pl.P) * sizeof(uint32_t);
+      return cudaErrorInvalidValue;
+    }
+    partials = scratch;
+    counters = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(scratch) + kNoAllocPartialBytes);
+  }
+  return launch_decode<TX, NT, GPB>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
+                                    stream);
 }
 
 template <typename TX, int NT>
@@ -844,6 +811,28 @@ cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales
 }
 
 }  // namespace
+
+cudaError_t reset_split_counters() {
+  // After a bounded wait gave up, a CTA may have left an arrival counted.
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    for (auto& kv : scratch_map())
+      if (kv.first.first == dev && kv.second.counters != nullptr) {
+        e = cudaMemset(kv.second.counters, 0, kv.second.counter_count * sizeof(uint32_t));
+        if (e != cudaSuccess) return e;
+      }
+  }
+  float* scratch = nullptr;
+  e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  return cudaMemset(reinterpret_cast<char*>(scratch) + kNoAllocPartialBytes, 0,
+                    kNoAllocMaxCtas * sizeof(uint32_t));
+}
 
 size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 

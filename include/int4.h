@@ -160,10 +160,11 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
  *
  * Computes what int4_matmul computes on its decode path (same kernels, same
  * result bits), with the partial tiles of the split kept in a fixed
- * library-owned device array of 4 MiB (one wave of up to 512 CTAs) instead of
- * pool memory.  It calls no cudaMalloc, cudaFree or other allocating routine.
- * Nothing in the array needs to start at zero: every partial is written before
- * it is read in the same call.
+ * library-owned device array of 4 MiB plus 2 KiB (one wave of up to 512 CTAs)
+ * instead of per-stream scratch.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.  The array's arrival counters must start at zero: they
+ * are zero when the library loads and every call leaves them zero (after a
+ * device-side wait gave up, int4_device_status zeroes them again).
  *
  * Arguments and layouts are those of int4_matmul.  Returns
  * INT4_ERR_UNSUPPORTED when the decode kernel cannot run the shape (x must be
