@@ -133,11 +133,18 @@ __device__ __forceinline__ bool codes8_normal(const float (&v)[8], float r, uint
 // 1.5 * 2^23 - 192 then rounds that grid value to an integer, ties to even,
 // as rint does on the IEEE quotient.
 __device__ __forceinline__ void codes8_snap(const float (&v)[8], float r, uint32_t& word) {
+  // Two weights per instruction (packed fp32 FMA and add, each lane rounded
+  // exactly as its scalar form).
   uint32_t nib[8];
+  const float2 rr = make_float2(r, r);
+  const float2 c192 = make_float2(192.0f, 192.0f);
+  const float2 cmag = make_float2(12582720.0f, 12582720.0f);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float y1 = __fmaf_rn(v[i], r, 192.0f);
-    nib[i] = __float_as_uint(__fadd_rn(y1, 12582720.0f));
+  for (int i = 0; i < 8; i += 2) {
+    const float2 y1 = __ffma2_rn(make_float2(v[i], v[i + 1]), rr, c192);
+    const float2 yv = __fadd2_rn(y1, cmag);
+    nib[i] = __float_as_uint(yv.x);
+    nib[i + 1] = __float_as_uint(yv.y);
   }
   uint32_t b[4];
 #pragma unroll

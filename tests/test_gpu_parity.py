@@ -455,3 +455,45 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     x = make_activations(2, 256, seed=1, device=DEV, dtype=torch.bfloat16)
     y = q4.int4_matmul(x, packed, scales, 256, 64)
     assert_matmul_close(y, x, packed, scales, 256, 64, TOL_HALF)
+
+
+def test_decode_split_scratch_on_concurrent_streams():
+    """Split-tile decode on two streams at once: each stream has its own
+    partial slots and arrival counters, so both results match the oracle
+    bound and equal a serial run bit for bit."""
+    N, K, group = 1000, 12288, 128
+    packed, scales, _ = _quantized(N, K, group, seed=77, dist="student_t3", zero_group_frac=0.02)
+    xa = make_activations(3, K, seed=1, device=DEV, dtype=torch.bfloat16)
+    xb = make_activations(5, K, seed=2, device=DEV, dtype=torch.bfloat16)
+    ref_a = q4.int4_matmul(xa, packed, scales, K, group, path=q4.PATH_DECODE)
+    ref_b = q4.int4_matmul(xb, packed, scales, K, group, path=q4.PATH_DECODE)
+    torch.cuda.synchronize()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    outs_a, outs_b = [], []
+    for _ in range(8):
+        with torch.cuda.stream(sa):
+            outs_a.append(q4.int4_matmul(xa, packed, scales, K, group, path=q4.PATH_DECODE))
+        with torch.cuda.stream(sb):
+            outs_b.append(q4.int4_matmul(xb, packed, scales, K, group, path=q4.PATH_DECODE))
+    torch.cuda.synchronize()
+    assert q4.device_status() == q4.OK
+    for o in outs_a:
+        assert torch.equal(o, ref_a)
+    for o in outs_b:
+        assert torch.equal(o, ref_b)
+    assert_matmul_close(ref_a, xa, packed, scales, K, group, TOL_HALF)
+
+
+def test_decode_split_scratch_grows_between_shapes():
+    """A small split first, then a larger one on the same stream: the stream's
+    scratch grows and the counters stay consistent for both."""
+    for N, K in [(128, 4096), (28672, 8192), (300, 8192)]:
+        packed, scales, _ = _quantized(N, K, 128, seed=N, dist="normal")
+        x = make_activations(1, K, seed=3, device=DEV, dtype=torch.bfloat16)
+        y1 = q4.int4_matmul(x, packed, scales, K, 128, path=q4.PATH_DECODE)
+        y2 = q4.int4_matmul(x, packed, scales, K, 128, path=q4.PATH_DECODE)
+        torch.cuda.synchronize()
+        assert torch.equal(y1, y2)
+        cols = np.unique(np.random.default_rng(N).integers(0, N, 256))
+        assert_matmul_close(y1, x, packed, scales, K, 128, TOL_HALF, cols=cols)
+    assert q4.device_status() == q4.OK
