@@ -810,6 +810,147 @@ cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales
   return launch_nt<TX, 2>(x, packed, scales, K, group, M, N, y, stream);
 }
 
+// ---------------- small matrices ----------------
+// Decode for matrices whose 16-row tiles fit one wave: one CTA per tile,
+// kSmallWarps warps splitting K (warp w takes 128-k blocks w, w + 8, ...,
+// two at a time for M <= 8).  A lane loads its weight words and x fragments straight
+// from global memory with 128-bit loads, expands and multiplies them exactly
+// as the pipelined kernel does, and scales each block by its group's scale;
+// the warps' partial sums are added in warp order through shared memory.  No
+// copy engine, barrier ring or scratch: the pipelined kernel's fixed latency
+// dominates at these sizes.
+constexpr int kSmallWarps = 8;
+constexpr int kSmallCtasPerSm = 3;
+
+template <typename TX, int NT>
+__global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_small_kernel(
+    const TX* __restrict__ x, const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
+    float* __restrict__ y, int64_t K, int group, int G, int M, int64_t N, int KB) {
+  __shared__ float red[kSmallWarps * NT * 4 * 32];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 16;
+  const int64_t ra = (row0 + g < N) ? row0 + g : N - 1;          // loads stay in bounds
+  const int64_t rb = (row0 + g + 8 < N) ? row0 + g + 8 : N - 1;
+  const int64_t Kp = K / 2;
+  const uint8_t* wa = packed + ra * Kp + 16 * c;
+  const uint8_t* wb = packed + rb * Kp + 16 * c;
+  const uint16_t* sa_row = scales + ra * G;
+  const uint16_t* sb_row = scales + rb * G;
+  float tot[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tot[nt][i] = 0.0f;
+  constexpr int kStep = NT == 1 ? 2 : 1;  // blocks per step (x fragments of M > 8 take twice the registers)
+  for (int kb0 = warp; kb0 < KB; kb0 += kStep * kSmallWarps) {
+    // kStep blocks per step, all loads issued before any use.
+    uint4 ua[kStep], ub[kStep], xf4[kStep][4][NT];
+    uint32_t sraw[kStep][2];
+#pragma unroll
+    for (int q = 0; q < kStep; ++q) {
+      const int kb = kb0 + kSmallWarps * q;
+      const bool ok = kb < KB;
+      const int kc = ok ? kb : kb0;
+      ua[q] = __ldg(reinterpret_cast<const uint4*>(wa + static_cast<int64_t>(kc) * 64));
+      ub[q] = __ldg(reinterpret_cast<const uint4*>(wb + static_cast<int64_t>(kc) * 64));
+      const int gi = static_cast<int>(static_cast<int64_t>(kc) * 128 / group);
+      sraw[q][0] = __ldg(sa_row + gi);
+      sraw[q][1] = __ldg(sb_row + gi);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = g + 8 * nt;
+        const TX* xp = x + static_cast<int64_t>(n < M ? n : 0) * K + static_cast<int64_t>(kc) * 128 + 32 * c;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          xf4[q][j][nt] = (n < M) ? __ldg(reinterpret_cast<const uint4*>(xp + 8 * j)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kStep; ++q) {
+      if (kb0 + kSmallWarps * q >= KB) break;
+      const uint32_t wva[4] = {ua[q].x, ua[q].y, ua[q].z, ua[q].w};
+      const uint32_t wvb[4] = {ub[q].x, ub[q].y, ub[q].z, ub[q].w};
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t pa[4], pb[4];
+        expand<TX>(wva[j], pa);
+        expand<TX>(wvb[j], pb);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4 xf = pair_x(xf4[q][j][nt]);
+          Cvt<TX>::mma(acc[nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
+          Cvt<TX>::mma(acc[nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
+        }
+      }
+      const float sa = f16_bits_to_float(sraw[q][0]);
+      const float sb = f16_bits_to_float(sraw[q][1]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        tot[nt][0] = fmaf(acc[nt][0], sa, tot[nt][0]);
+        tot[nt][1] = fmaf(acc[nt][1], sa, tot[nt][1]);
+        tot[nt][2] = fmaf(acc[nt][2], sb, tot[nt][2]);
+        tot[nt][3] = fmaf(acc[nt][3], sb, tot[nt][3]);
+      }
+    }
+  }
+  // Warps' partials summed in warp order.
+  constexpr int kPerWarp = NT * 4 * 32;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) red[warp * kPerWarp + (nt * 4 + i) * 32 + lane] = tot[nt][i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < kPerWarp; e += blockDim.x) {
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kSmallWarps; ++w) sum += red[w * kPerWarp + e];
+    const int ln = e & 31;
+    const int i = (e >> 5) & 3;
+    const int nt = e >> 7;
+    const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
+    const int64_t row = row0 + (ln >> 2) + ((i < 2) ? 0 : 8);
+    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+  }
+}
+
+template <typename TX>
+cudaError_t launch_small(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                         int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  const int G = static_cast<int>((K + group - 1) / group);
+  const int KB = static_cast<int>((K + 127) / 128);
+  const unsigned grid = static_cast<unsigned>((N + 15) / 16);
+  if (M <= 8)
+    decode_small_kernel<TX, 1><<<grid, kSmallWarps * 32, 0, stream>>>(x, packed, scales, y, K, group, G,
+                                                                       static_cast<int>(M), N, KB);
+  else
+    decode_small_kernel<TX, 2><<<grid, kSmallWarps * 32, 0, stream>>>(x, packed, scales, y, K, group, G,
+                                                                       static_cast<int>(M), N, KB);
+  return cudaGetLastError();
+}
+
+// Small matrices: 16-row tiles that fit one wave, K a multiple of 128 (so
+// every block is whole) and groups of whole blocks.
+bool small_applies(int64_t K, int group, int64_t N) {
+  if (group % 128 != 0 || K % 128 != 0) return false;
+  return (N + 15) / 16 <= static_cast<int64_t>(kSmallCtasPerSm) * num_sms();
+}
+
+cudaError_t launch_small_any(const void* x, DType xt, const uint8_t* packed, const uint16_t* scales,
+                             int64_t K, int group, int64_t M, int64_t N, float* y,
+                             cudaStream_t stream) {
+  if (xt == DType::BF16)
+    return launch_small(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N, y,
+                        stream);
+  return launch_small(static_cast<const __half*>(x), packed, scales, K, group, M, N, y, stream);
+}
+
 }  // namespace
 
 cudaError_t reset_split_counters() {
@@ -839,6 +980,8 @@ size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t* packed,
                                          const uint16_t* scales, int64_t K, int group, int64_t M,
                                          int64_t N, float* y, cudaStream_t stream, size_t* need) {
+  if (small_applies(K, group, N))
+    return launch_small_any(x, xt, packed, scales, K, group, M, N, y, stream);
   if (xt == DType::BF16)
     return launch_tx_noalloc(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N,
                              y, stream, need);
@@ -861,6 +1004,8 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
 cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
                                  const uint16_t* scales, int64_t K, int group, int64_t M,
                                  int64_t N, float* y, cudaStream_t stream) {
+  if (small_applies(K, group, N))
+    return launch_small_any(x, xt, packed, scales, K, group, M, N, y, stream);
   if (xt == DType::BF16)
     return launch_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N, y,
                      stream);
