@@ -314,10 +314,11 @@ def run_ours(args):
         kernels["quantize"]()
         torch.cuda.synchronize()
         w = None
-    # Kernels of this library per call: the decode matmul at this shape splits
-    # tiles across CTAs, so it launches its fix-up kernel after the main one.
+    # Kernels of this library per call: one each.  At M <= 2 the decode
+    # matmul converts x inside its own launch and reduces the tiles it splits
+    # across CTAs there too.
     launches_per_step = {
-        "quantize": 1, "unpack": 1, "decode": 2,
+        "quantize": 1, "unpack": 1, "decode": 1,
         "prefill": 1,
     }
 

@@ -223,7 +223,7 @@ int int4_matmul_decode_noalloc(const void* x, int32_t x_dtype, const uint8_t* pa
   if (e == cudaErrorInvalidValue && need > 0) {
     char msg[200];
     std::snprintf(msg, sizeof msg,
-                  "int4_matmul_decode_noalloc: this split needs %zu bytes of scratch, the static "
+                  "int4_matmul_decode_noalloc: this call needs %zu bytes of scratch, the static "
                   "scratch holds %zu",
                   need, int4lib::decode_noalloc_scratch_bytes());
     return int4lib::fail(INT4_ERR_ARG, msg);

@@ -5,6 +5,12 @@
 // and a dequantizing matmul" (problem statement), integer weights times x
 // first, then the group's scale per output column.
 //
+// Two kernels share the CTA structure below.  For a group that is a multiple
+// of 128 (the common case) decode_i8_kernel runs the products on the int8
+// warp MMA, with x split into base-256 digits (its comment block gives the
+// arithmetic); for groups of 32 and 64, decode_kernel expands nibbles to
+// bf16/fp16 and runs the 16-bit warp MMA, as described here.
+//
 // The kernel is bound by HBM: every packed weight byte is read once and at
 // M <= 16 feeds at most 32 multiply-adds.  Design:
 //   * a producer warp streams 128 weight rows (64 for M > 8) through a
@@ -46,8 +52,10 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <cstring>
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "common.cuh"
@@ -74,7 +82,17 @@ namespace {
 #ifndef INT4_DECODE_MIN_BLOCKS
 #define INT4_DECODE_MIN_BLOCKS 2
 #endif
+#ifndef INT4_DECODE_I8_MINB1
+#define INT4_DECODE_I8_MINB1 2
+#endif
+#ifndef INT4_DECODE_I8_FUSE_MAX_M
+#define INT4_DECODE_I8_FUSE_MAX_M 2
+#endif
+#ifndef INT4_DECODE_I8_SCALE_AHEAD
+#define INT4_DECODE_I8_SCALE_AHEAD 1
+#endif
 constexpr int kSK = INT4_DECODE_SK;                // 128-wide K blocks per stage (even)
+constexpr int kFuseMaxM = INT4_DECODE_I8_FUSE_MAX_M;  // batch rows the in-kernel x conversion serves
 constexpr int kSub = kSK / 2;                      // 256-k sub-tiles per stage (one copy each)
 static_assert(kSK % 2 == 0, "stages hold whole 256-k sub-tiles");
 constexpr int kRowGroups = INT4_DECODE_ROW_GROUPS;  // row groups per CTA
@@ -495,7 +513,6 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
           if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
         }
-        if (!whole) __threadfence();  // this CTA's piece is visible before its arrival counts
       }
       ptx::bar_sync(1, kConsumers * 32);  // red is rewritten by the next segment
       if (stop) break;
@@ -509,6 +526,9 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
         const int p_first = static_cast<int>(((t0 + 1) * P + U - 1) / U - 1);
         const int p_last = static_cast<int>((t1 * P + U - 1) / U - 1);
         if (cw == 0 && lane == 0) {
+          // The barrier above orders the CTA's partial stores before this
+          // fence; fence and count release them to the last contributor.
+          __threadfence();
           const uint32_t before = atomicAdd(&counters[p_first], 1u);
           const bool last = before == static_cast<uint32_t>(p_last - p_first);
           if (last) __threadfence();
@@ -528,6 +548,551 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
             const int tw = (e >> 7) / NT;
             const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
             const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
+            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+          }
+          if (cw == 0 && lane == 0) counters[p_first] = 0u;
+        }
+      }
+      u = r * KB + bhi;
+    }
+  }
+}
+
+// ---------------- integer-MMA decode (group a multiple of 128) ----------------
+// The weights enter the int8 warp MMA as they are stored: the high nibble of
+// a byte, masked in place, is the int8 value 16 q, and the low nibble is the
+// same after a 4-bit left shift; two logic operations and a shift per 8
+// weights, against eleven for the bf16 expansion.  x is split once per call
+// (x_digits_kernel) into base-256 digits: for batch row m and 128-k block b,
+// with e the binary exponent of the block's largest |x| (2^e <= max < 2^(e+1)),
+//   v = rint(x 2^(29-e)),  |v| < 2^30,  v = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3,
+// with signed digits d_i (d0..d2 in [-128, 127], d3 in [-64, 64]).  v is x
+// exactly for every bf16 x within 2^22 of the block's largest magnitude (fp16:
+// 2^19); below that the rounding error is at most 2^-30 of the largest.  The
+// MMA sums S_i = sum_k (16 q) d_i over the block exactly in int32 (|S_i| <=
+// 2^21), and the block's x.q is
+//   sum_k x q = 2^(e-33) (P01 + 2^16 P23),  P01 = S0 + 2^8 S1,  P23 = S2 + 2^8 S3,
+// both P below 2^30, so the block needs two int-to-float conversions per
+// output; the group's scale multiplies the block sum before the fp32 running
+// sum, as on the page.  The four digits of row m sit in four MMA columns, so
+// one n = 8 MMA serves two batch rows: lane c of a quad holds columns 2c and
+// 2c + 1, i.e. P01 (c even) or P23 (c odd) of row 2nt + c / 2, and the two
+// halves are added when the tile is written.
+//
+// Digit record of one 128-k block: NP n-tiles of 1 KB (8 columns x 128 k, one
+// byte each, in MMA fragment order), then 32 fp32 factors 2^(e-33) and
+// 2^(e-17) for the 16 rows.  Column col of an n-tile holds digit col % 4 of row
+// 2nt + col / 4; inside a column, the 16-byte chunk ((2c + j / 2) ^ (col & 1))
+// holds, at byte 8 (j % 2), the B fragment of lane c for the MMA over words
+// 4c + j of the block's 16 words: 4 digits of the word's even k, then 4 of its
+// odd k.  The XOR spreads the 16-byte loads of a quarter warp over all banks.
+constexpr int kDigitTile = 1024;
+
+__device__ __forceinline__ void transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                             uint32_t (&o)[4]) {
+  const uint32_t ab_lo = __byte_perm(a, b, 0x5140);  // a0 b0 a1 b1
+  const uint32_t ab_hi = __byte_perm(a, b, 0x7362);  // a2 b2 a3 b3
+  const uint32_t cd_lo = __byte_perm(c, d, 0x5140);
+  const uint32_t cd_hi = __byte_perm(c, d, 0x7362);
+  o[0] = __byte_perm(ab_lo, cd_lo, 0x5410);  // a0 b0 c0 d0
+  o[1] = __byte_perm(ab_lo, cd_lo, 0x7632);  // a1 b1 c1 d1
+  o[2] = __byte_perm(ab_hi, cd_hi, 0x5410);  // a2 b2 c2 d2
+  o[3] = __byte_perm(ab_hi, cd_hi, 0x7632);  // a3 b3 c3 d3
+}
+
+// 8 x values (one 8-k word) from 16 bytes of bf16 or fp16, exactly.
+template <typename TX>
+__device__ __forceinline__ void word_as_float(uint4 u, float (&v)[8]);
+template <>
+__device__ __forceinline__ void word_as_float<__nv_bfloat16>(uint4 u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void word_as_float<__half>(uint4 u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+// Bits of the largest |x| of a 128-k block (8 values per lane, 16 lanes: a
+// half warp), as an unsigned max over the magnitude bits, which orders every
+// finite value below infinity and infinity below NaN.  All 32 lanes must call
+// it together.
+__device__ __forceinline__ uint32_t block_absmax_bits(const float (&v)[8]) {
+  uint32_t mb = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mb = max(mb, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+  return mb;
+}
+
+// The digits of one word of a block: ev[i] / od[i] hold digit i of the
+// word's even / odd k (one byte each, k order), f the block's factor
+// 2^(e-33).  A block of zeros gives zero digits and factor; a block holding a
+// NaN or an infinity gives a NaN factor, so the rows it feeds come out NaN.
+// Blocks whose largest |x| is below 2^-93 are scaled as if it were 2^-93,
+// which keeps the factors normal floats (and loses digits of x below about
+// 2^-122).
+__device__ __forceinline__ void word_digits(const float (&v)[8], uint32_t amax_bits,
+                                            uint32_t (&ev)[4], uint32_t (&od)[4], float& f) {
+  uint32_t dd[8];
+  f = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dd[i] = 0u;
+  if (amax_bits >= 0x7F800000u) {
+    f = __uint_as_float(0x7FC00000u);
+  } else if (amax_bits != 0u) {
+    // The exponent field (subnormals read as -127, below the clamp).
+    int e = static_cast<int>(amax_bits >> 23) - 127;
+    if (e < -93) e = -93;
+    const int p = 29 - e;  // in [-98, 122]: two normal power-of-two factors
+    const int p1 = p >> 1, p2 = p - p1;
+    const float s1 = __uint_as_float(static_cast<uint32_t>(p1 + 127) << 23);
+    const float s2 = __uint_as_float(static_cast<uint32_t>(p2 + 127) << 23);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int vi = __float2int_rn((v[i] * s1) * s2);
+      // Balanced base-256 digits: the bytes of v + 0x808080 with the low three
+      // flipped back by 128.
+      dd[i] = (static_cast<uint32_t>(vi) + 0x808080u) ^ 0x808080u;
+    }
+    f = __uint_as_float(static_cast<uint32_t>(e - 33 + 127) << 23);
+  }
+  transpose4x4(dd[0], dd[2], dd[4], dd[6], ev);
+  transpose4x4(dd[1], dd[3], dd[5], dd[7], od);
+}
+
+// Byte offset, inside a record, of the fragment pair (digit i of row m, word h).
+__device__ __forceinline__ int digit_offset(int m, int i, int h) {
+  const int col = 4 * (m & 1) + i;
+  const int c = h >> 2, j = h & 3;
+  return (m >> 1) * kDigitTile + col * 128 + (((2 * c + (j >> 1)) ^ (col & 1)) << 4) + (j & 1) * 8;
+}
+
+// Digit records of rows 0 .. R-1 of one block from its x rows in shared
+// memory (row pitch 512 bytes): xs addresses this lane's word h of row 0, rb
+// the block's record.  All 32 lanes call it together (one block per half
+// warp).
+template <typename TX, int R, int NP>
+__device__ __forceinline__ void convert_rows(uint32_t xs, uint32_t rb, int h) {
+  float v[R][8];
+  uint32_t mb[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) word_as_float<TX>(ptx::lds128(xs + r * 512), v[r]);
+#pragma unroll
+  for (int r = 0; r < R; ++r) mb[r] = block_absmax_bits(v[r]);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    uint32_t ev[4], od[4];
+    float f;
+    word_digits(v[r], mb[r], ev, od, f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ptx::sts64(rb + digit_offset(r, i, h), ev[i], od[i]);
+    if (h == 0) {
+      ptx::sts32(rb + NP * kDigitTile + 8 * r, __float_as_uint(f));
+      ptx::sts32(rb + NP * kDigitTile + 8 * r + 4, __float_as_uint(f * 65536.0f));
+    }
+  }
+}
+
+// One half warp per (batch row m < MP, record b < nrec); lane h takes the
+// 8-k word h of the block.  Rows m >= M and k >= K are zero.
+template <typename TX>
+__global__ void __launch_bounds__(256) x_digits_kernel(const TX* __restrict__ x, int64_t K, int M,
+                                                      int MP, int NP, int64_t nrec,
+                                                      uint8_t* __restrict__ rec) {
+  // Launched as a programmatic dependent: the matmul grid may start its
+  // set-up now; this grid waits for the kernel before it (which may write x,
+  // or still read the records) to complete.
+  ptx::launch_dependents();
+  ptx::grid_dependency_wait();
+  const int64_t hw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  const int h = threadIdx.x & 15;
+  const bool live = hw < static_cast<int64_t>(MP) * nrec;
+  const int m = live ? static_cast<int>(hw % MP) : 0;
+  const int64_t b = live ? hw / MP : 0;
+  const int64_t k0 = b * 128 + 8 * h;
+  float v[8];
+  if (live && m < M && k0 < K) {
+    word_as_float<TX>(__ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0)), v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+  }
+  const uint32_t amax_bits = block_absmax_bits(v);
+  if (!live) return;
+  uint32_t ev[4], od[4];
+  float f;
+  word_digits(v, amax_bits, ev, od, f);
+  uint8_t* r = rec + b * (static_cast<int64_t>(NP) * kDigitTile + 128);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint2*>(r + digit_offset(m, i, h)) = make_uint2(ev[i], od[i]);
+  if (h == 0) {
+    float* fr = reinterpret_cast<float*>(r + NP * kDigitTile);
+    fr[2 * m] = f;
+    fr[2 * m + 1] = f * 65536.0f;
+  }
+}
+
+// Shape of the integer-MMA decode for NP n-tiles (batch rows up to 2 NP).
+// FUSE (M <= 2): the kernel converts x itself; a converter warp turns each
+// stage's x tile (copied on its own barrier, ahead of the weights) into the
+// stage's digit records, so one launch does the whole call.  For larger M
+// that per-CTA conversion would cost more than the matmul, and
+// x_digits_kernel writes the records once per call.
+template <int NP, bool FUSE>
+struct I8Shape {
+  static constexpr bool kFuse = FUSE;                                // converter warp in the CTA
+  static_assert(!FUSE || NP == 1, "the converter warp serves up to two batch rows");
+  static constexpr int kTiles = NP <= 2 ? 2 : 1;                    // 16-row tiles per consumer
+  static constexpr int kRowsPerCta = 16 * kTiles * kRowGroups;       // 128 or 64
+  static constexpr int kWBytes = kRowsPerCta * kSK * 64;             // packed W of a stage
+  static constexpr int kRec = NP * kDigitTile + 128;                 // digit record of a block
+  static constexpr int kXBytes = kFuse ? 2 * NP * 256 * 2 : 0;       // x rows of the stage (fused)
+  static constexpr int offX = kWBytes + kSK * kRec;                  // within a stage
+  static constexpr int kStageBytes = (offX + kXBytes + 1023) / 1024 * 1024;
+  static constexpr int kRedPer = kRowGroups * kTiles * NP * 2 * 32;  // lane sums of one K slot
+  static constexpr int kOut = kRowGroups * kTiles * NP * 2 * 16;     // (row, batch row) outputs of a tile
+  static constexpr int kThreads = 32 * (kConsumers + 1 + (kFuse ? 1 : 0));
+  static constexpr int offRed = kStages * kStageBytes;
+  static constexpr int offBar = offRed + kSK * kRedPer * 4;
+  static constexpr int offMisc = offBar + 4 * kStages * 8;
+  static constexpr int kAlloc = offMisc + 16 + 1024;
+  static constexpr int kMinBlocks = NP == 1 ? INT4_DECODE_I8_MINB1 : 2;  // CTAs per SM
+  static_assert(kSK == 2, "a stage is one 256-k copy of W: K slot bs reads its 64-byte half");
+  static_assert(offX % 128 == 0, "x tile copies need 128-byte aligned destinations");
+};
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Same CTA roles, ring, stream-K split and last-contributor reduction as
+// decode_kernel.  Each stage carries the digit records of its two blocks:
+// converted in the CTA from the stage's x tile (FUSE), or one bulk copy of
+// the records x_digits_kernel wrote.
+template <typename TX, int NP, bool FUSE>
+__global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>::kMinBlocks) decode_i8_kernel(
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+    const uint8_t* __restrict__ rec,
+    const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
+    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* __restrict__ counters,
+    uint32_t* status) {
+  using S = I8Shape<NP, FUSE>;
+  constexpr int kTiles = S::kTiles;
+  constexpr int kRowsPerCta = S::kRowsPerCta;
+  constexpr int kWBytes = S::kWBytes;
+  constexpr int kRec = S::kRec;
+  constexpr int kOut = S::kOut;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = ptx::smem_u32(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::offBar);
+  uint64_t* empty = full + kStages;
+  uint64_t* ready = empty + kStages;  // records of the stage written (fused)
+  uint64_t* xfull = ready + kStages;  // x tile of the stage landed (fused)
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::offMisc);
+  volatile uint32_t* last_flag = abort_flag + 1;
+  float* red = reinterpret_cast<float*>(smem + S::offRed);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * U / P;
+  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * U / P;
+  const WaitCtx wc{abort_flag, status};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&empty[s]), kConsumers);
+      ptx::mbar_init(ptx::smem_u32(&ready[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&xfull[s]), 1);
+    }
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_w);
+    if (S::kFuse) ptx::prefetch_tmap(&tm_x);
+  }
+  __syncthreads();
+  // Launched as a programmatic dependent of what precedes it on the stream
+  // (the digits grid, or any kernel): the set-up above overlaps that grid's
+  // tail, and every thread waits for it to complete (its writes visible)
+  // before reading an input or writing an output.  The next kernel may
+  // likewise start its set-up early.
+  ptx::launch_dependents();
+  ptx::grid_dependency_wait();
+
+  const int c = lane & 3;
+  const int g = lane >> 2;
+  const int cw = warp - 1;
+  const int rg = cw % kRowGroups;
+  const int bs = cw / kRowGroups;
+
+  if (S::kFuse && warp == kConsumers + 1) {
+    // ---------------- converter (NP <= 2) ----------------
+    // Rows M .. 2NP - 1 of every record stay zero: cleared once here, before
+    // the first stage is declared ready.
+    for (int o = lane * 16; o < kStages * S::kStageBytes; o += 32 * 16) {
+      const int ws = o % S::kStageBytes;
+      if (ws >= kWBytes && ws < S::offX) ptx::sts128(sbase + o, make_uint4(0u, 0u, 0u, 0u));
+    }
+    int nst = 0;  // stages of this CTA, counted as the producer issues them
+    for (int64_t u = u_begin; u < u_end;) {
+      const int64_t r = u / KB;
+      const int blo = static_cast<int>(u - r * KB);
+      const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+      nst += (bhi - blo + kSK - 1) / kSK;
+      u = r * KB + bhi;
+    }
+    for (int gs = 0; gs < nst; ++gs) {
+      const int s = gs % kStages;
+      if (!__all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&xfull[s]), (gs / kStages) & 1, wc))) break;
+      const uint32_t st = sbase + s * S::kStageBytes;
+      // Half warp bl takes block bl of the stage, lane h its word h, for
+      // every batch row (both rows' chains interleaved when M = 2).
+      const int bl = lane >> 4, h = lane & 15;
+      const uint32_t xs = st + S::offX + bl * 256 + 16 * h;
+      const uint32_t rb = st + kWBytes + bl * kRec;
+      if (M == 2)
+        convert_rows<TX, 2, NP>(xs, rb, h);
+      else
+        convert_rows<TX, 1, NP>(xs, rb, h);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ready[s]));
+    }
+  } else if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int gs = 0;
+      bool ok = true;
+      for (int64_t u = u_begin; ok && u < u_end;) {
+        const int64_t r = u / KB;
+        const int blo = static_cast<int>(u - r * KB);
+        const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+        const int32_t row0 = static_cast<int32_t>(r * kRowsPerCta);
+        for (int kb = blo; kb < bhi; kb += kSK, ++gs) {
+          const int s = gs % kStages;
+          if (!wait_bar(ptx::smem_u32(&empty[s]), ((gs / kStages) & 1) ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = sbase + s * S::kStageBytes;
+          if (S::kFuse) {
+            // The stage's x rows (256 k; past K the copy fills zeros) on their
+            // own barrier, so the converter starts while W is in flight.
+            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&xfull[s]), static_cast<uint32_t>(M) * 512);
+            ptx::tma_load_2d(st + S::offX, &tm_x, kb * 128, 0, ptx::smem_u32(&xfull[s]));
+            ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes);
+            ptx::tma_load_2d(st, &tm_w, kb * 64, row0, ptx::smem_u32(&full[s]));
+            continue;
+          }
+          ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), kWBytes + kSK * kRec);
+          ptx::tma_load_2d(st, &tm_w, kb * 64, row0, ptx::smem_u32(&full[s]));
+          ptx::bulk_load(st + kWBytes, rec + static_cast<int64_t>(kb) * kRec, kSK * kRec,
+                         ptx::smem_u32(&full[s]));
+        }
+        u = r * KB + bhi;
+      }
+      if (*abort_flag) {
+        const int first = gs - kStages > 0 ? gs - kStages : 0;
+        for (int j = first; j < gs; ++j) {
+          drain_bar(ptx::smem_u32(&full[j % kStages]), (j / kStages) & 1);
+          if (S::kFuse) drain_bar(ptx::smem_u32(&xfull[j % kStages]), (j / kStages) & 1);
+        }
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    // Consumer (rg, bs) takes kTiles 16-row tiles of row group rg and K block
+    // bs of every stage: per tile, lane (g, c) reads the 16 bytes (words
+    // 4c .. 4c + 3) of rows g and g + 8 (permuted as in decode_kernel), one
+    // word per MMA.
+    uint32_t wofs[kTiles][2];
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = rg * 16 * kTiles + 16 * t + tile_row<1>(g) + 8 * h;
+        const int off = bs * 64 + 16 * c;
+        wofs[t][h] = static_cast<uint32_t>(r * 128 + (((off >> 4) ^ (r & 7)) << 4));
+      }
+    const uint32_t xrec = static_cast<uint32_t>(kWBytes + bs * kRec);
+    uint32_t bofs[2];
+#pragma unroll
+    for (int jp = 0; jp < 2; ++jp)
+      bofs[jp] = xrec + static_cast<uint32_t>(g * 128 + (((2 * c + jp) ^ (g & 1)) << 4));
+    const uint32_t fofs = xrec + static_cast<uint32_t>(NP * kDigitTile + 4 * c);
+    const int bpg = group / 128;
+    int gs = 0;
+    for (int64_t u = u_begin; u < u_end;) {
+      const int64_t r = u / KB;
+      const int blo = static_cast<int>(u - r * KB);
+      const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+      const int64_t row0 = r * kRowsPerCta;
+      const uint16_t* sp[kTiles][2];
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          int64_t gr = row0 + rg * 16 * kTiles + 16 * t + tile_row<1>(g) + 8 * h;
+          if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
+          sp[t][h] = scales + gr * G;
+        }
+      float tot[kTiles][NP][2];
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int nt = 0; nt < NP; ++nt) tot[t][nt][0] = tot[t][nt][1] = 0.0f;
+      // The scales of a block are loaded kAhead blocks ahead (a register
+      // queue): a block's work is shorter than a load's latency.
+      constexpr int kAhead = INT4_DECODE_I8_SCALE_AHEAD;
+      uint16_t sraw[kAhead][kTiles][2];
+      auto load_scales = [&](int kb, uint16_t (&dst)[kTiles][2]) {
+        const int gi = (bpg == 1) ? kb : kb / bpg;
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+          dst[t][0] = __ldg(sp[t][0] + gi);
+          dst[t][1] = __ldg(sp[t][1] + gi);
+        }
+      };
+#pragma unroll
+      for (int q = 0; q < kAhead; ++q)
+        if (blo + bs + q * kSK < bhi) load_scales(blo + bs + q * kSK, sraw[q]);
+      bool ok = true;
+      for (int kb_stage = blo; kb_stage < bhi; kb_stage += kSK, ++gs) {
+        const int s = gs % kStages;
+        const int kb = kb_stage + bs;
+        float sa[kTiles], sb[kTiles];
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+          sa[t] = f16_bits_to_float(sraw[0][t][0]);
+          sb[t] = f16_bits_to_float(sraw[0][t][1]);
+        }
+#pragma unroll
+        for (int q = 0; q + 1 < kAhead; ++q)
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t) {
+            sraw[q][t][0] = sraw[q + 1][t][0];
+            sraw[q][t][1] = sraw[q + 1][t][1];
+          }
+        if (kb + kAhead * kSK < bhi) load_scales(kb + kAhead * kSK, sraw[kAhead - 1]);
+        ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&full[s]), (gs / kStages) & 1, wc));
+        if (ok && S::kFuse)
+          ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&ready[s]), (gs / kStages) & 1, wc));
+        if (!ok) break;
+        const uint32_t st = sbase + s * S::kStageBytes;
+        if (kb < bhi) {
+          // A fragments of the block's four MMAs (k32 each): rows g and g + 8,
+          // low nibbles (shifted) in k slots 0..15, high nibbles in 16..31.
+          uint32_t a[kTiles][4][4];
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t) {
+            const uint4 u0 = ptx::lds128(st + wofs[t][0]);
+            const uint4 u1 = ptx::lds128(st + wofs[t][1]);
+            const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w};
+            const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              a[t][j][0] = (w0[j] << 4) & 0xF0F0F0F0u;
+              a[t][j][1] = (w1[j] << 4) & 0xF0F0F0F0u;
+              a[t][j][2] = w0[j] & 0xF0F0F0F0u;
+              a[t][j][3] = w1[j] & 0xF0F0F0F0u;
+            }
+          }
+#pragma unroll
+          for (int nt = 0; nt < NP; ++nt) {
+            const uint4 b01 = ptx::lds128(st + bofs[0] + nt * kDigitTile);
+            const uint4 b23 = ptx::lds128(st + bofs[1] + nt * kDigitTile);
+            const float fct = __uint_as_float(ptx::lds32(st + fofs + nt * 16));
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+              int acc[4] = {0, 0, 0, 0};
+              mma_s8(acc, a[t][0], b01.x, b01.y);
+              mma_s8(acc, a[t][1], b01.z, b01.w);
+              mma_s8(acc, a[t][2], b23.x, b23.y);
+              mma_s8(acc, a[t][3], b23.z, b23.w);
+              const float p0 = static_cast<float>(acc[0] + 256 * acc[1]);
+              const float p1 = static_cast<float>(acc[2] + 256 * acc[3]);
+              tot[t][nt][0] = fmaf(p0 * fct, sa[t], tot[t][nt][0]);
+              tot[t][nt][1] = fmaf(p1 * fct, sb[t], tot[t][nt][1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&empty[s]));
+      }
+      // Segment end: lane sums of both K slots, each output the sum of its
+      // even (P01) and odd (P23) lane, in a fixed order.
+#pragma unroll
+      for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+        for (int nt = 0; nt < NP; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            red[(((cw * kTiles + t) * NP + nt) * 2 + h) * 32 + lane] = tot[t][nt][h];
+      const bool stop = ptx::bar_red_or(1, kConsumers * 32, !ok || *abort_flag != 0u);
+      const bool whole = (blo == 0 && bhi == KB);
+      if (!stop) {
+        float* dst = whole ? nullptr
+                           : partials + (2 * static_cast<int64_t>(blockIdx.x) + (blo == 0 ? 1 : 0)) * kOut;
+        for (int e = threadIdx.x - 32; e < kOut; e += kConsumers * 32) {
+          const int mp = e & 1, gq = (e >> 1) & 7, hh = (e >> 4) & 1, rest = e >> 5;
+          const int nt = rest % NP, tw = rest / NP;
+          const int base = ((tw * NP + nt) * 2 + hh) * 32 + 4 * gq + 2 * mp;
+          float sum = 0.0f;
+#pragma unroll
+          for (int q = 0; q < kSK; ++q) sum += red[q * S::kRedPer + base] + red[q * S::kRedPer + base + 1];
+          if (!whole) {
+            dst[e] = sum;
+            continue;
+          }
+          const int m = 2 * nt + mp;
+          const int64_t row = row0 + tw * 16 + tile_row<1>(gq) + 8 * hh;
+          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+        }
+      }
+      ptx::bar_sync(1, kConsumers * 32);
+      if (stop) break;
+      if (!whole) {
+        const int64_t t0 = r * KB, t1 = (r + 1) * KB;
+        const int p_first = static_cast<int>(((t0 + 1) * P + U - 1) / U - 1);
+        const int p_last = static_cast<int>((t1 * P + U - 1) / U - 1);
+        if (cw == 0 && lane == 0) {
+          // The barrier above orders the CTA's partial stores before this
+          // fence; fence and count release them to the last contributor.
+          __threadfence();
+          const uint32_t before = atomicAdd(&counters[p_first], 1u);
+          const bool last = before == static_cast<uint32_t>(p_last - p_first);
+          if (last) __threadfence();
+          *last_flag = last ? 1u : 0u;
+        }
+        ptx::bar_sync(1, kConsumers * 32);
+        if (*last_flag) {
+          const float* first = partials + (2 * static_cast<int64_t>(p_first) + 1) * kOut;
+          const float* rest = partials + 2 * static_cast<int64_t>(p_first + 1) * kOut;
+          const int n_rest = p_last - p_first;
+          for (int e = threadIdx.x - 32; e < kOut; e += kConsumers * 32) {
+            float sum = __ldcg(first + e);
+            for (int q = 0; q < n_rest; ++q) sum += __ldcg(rest + static_cast<int64_t>(2 * q) * kOut + e);
+            const int mp = e & 1, gq = (e >> 1) & 7, hh = (e >> 4) & 1, rest_i = e >> 5;
+            const int m = 2 * (rest_i % NP) + mp;
+            const int tw = rest_i / NP;
+            const int64_t row = row0 + tw * 16 + tile_row<1>(gq) + 8 * hh;
             if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
           }
           if (cw == 0 && lane == 0) counters[p_first] = 0u;
@@ -566,6 +1131,8 @@ struct SplitScratch {
   uint32_t* counters = nullptr;
   size_t partial_floats = 0;
   size_t counter_count = 0;
+  uint8_t* records = nullptr;  // digit records of x (integer-MMA decode)
+  size_t record_bytes = 0;
 };
 
 std::mutex g_scratch_mu;
@@ -586,7 +1153,10 @@ cudaError_t stream_scratch(cudaStream_t stream, size_t partial_floats, size_t co
       e = cudaStreamSynchronize(stream);
       if (e != cudaSuccess) return e;
       cudaFree(sc.partials);
-      sc = SplitScratch{};
+      sc.partials = nullptr;
+      sc.counters = nullptr;
+      sc.partial_floats = 0;
+      sc.counter_count = 0;
     }
     const size_t pbytes = (partial_floats * sizeof(float) + 255) & ~static_cast<size_t>(255);
     void* base = nullptr;
@@ -608,13 +1178,41 @@ cudaError_t stream_scratch(cudaStream_t stream, size_t partial_floats, size_t co
   return cudaSuccess;
 }
 
-// Scratch of int4_matmul_decode_noalloc: partial slots and arrival counters
-// in one fixed device array (zero at load; every call leaves the counters
-// zero).  4 MiB of partials hold one wave of up to 512 CTAs (B200 runs 296:
-// 2 per SM).
+// Digit records of x for one (device, stream), grown like the split scratch.
+cudaError_t stream_records(cudaStream_t stream, size_t bytes, uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  SplitScratch& sc = scratch_map()[{dev, stream}];
+  if (sc.record_bytes < bytes) {
+    if (sc.records != nullptr) {
+      e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return e;
+      cudaFree(sc.records);
+      sc.records = nullptr;
+      sc.record_bytes = 0;
+    }
+    void* p = nullptr;
+    e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return e;
+    sc.records = static_cast<uint8_t*>(p);
+    sc.record_bytes = bytes;
+  }
+  *out = sc.records;
+  return cudaSuccess;
+}
+
+// Scratch of int4_matmul_decode_noalloc: partial slots, arrival counters and
+// the x digit records in one fixed device array (zero at load; every call
+// leaves the counters zero).  4 MiB of partials hold one wave of up to 512
+// CTAs (B200 runs 296: 2 per SM); 4 MiB of records hold K up to 64384 at
+// M = 16 (246528 at M <= 4; M <= 2 converts x in the matmul and needs none).
 constexpr int kNoAllocMaxCtas = 512;
 constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;
-constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocMaxCtas * sizeof(uint32_t);
+constexpr size_t kNoAllocCounterBytes = kNoAllocMaxCtas * sizeof(uint32_t);
+constexpr size_t kNoAllocRecordBytes = size_t(4) << 20;  // x digit records
+constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocCounterBytes + kNoAllocRecordBytes;
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 // Device address of the array on the current device, resolved once per
@@ -647,29 +1245,31 @@ struct DecodePlan {
   bool split = false;  // does some run start inside a tile?
 };
 
-template <typename TX, int NT, int GPB>
-cudaError_t plan_decode(int64_t K, int64_t N, DecodePlan* pl) {
-  using L = DLayout<NT>;
-  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
-  auto kern = decode_kernel<TX, NT, GPB>;
-  // Shared-memory opt-in and occupancy, once per device for this kernel.
+// Shared-memory opt-in and occupancy of a decode kernel, once per device.
+cudaError_t kernel_occupancy(const void* fn, int threads, int alloc, std::atomic<int>* cache,
+                             int* occ_out) {
   constexpr int kMaxDevices = 64;
-  static std::atomic<int> occ_cache[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  int occ = occ_cache[dev].load(std::memory_order_relaxed);
+  int occ = cache[dev].load(std::memory_order_relaxed);
   if (occ == 0) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::kAlloc);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, alloc);
     if (e != cudaSuccess) return e;
     if (occ < 1) occ = 1;
-    occ_cache[dev].store(occ, std::memory_order_relaxed);
+    cache[dev].store(occ, std::memory_order_relaxed);
   }
+  *occ_out = occ;
+  return cudaSuccess;
+}
+
+// The split for `occ` CTAs per SM over row tiles of `rows` rows.
+void plan_split(int occ, int rows, int64_t K, int64_t N, DecodePlan* pl) {
   pl->KB = static_cast<int>((K + 127) / 128);
-  pl->U = ((N + kRowsPerCta - 1) / kRowsPerCta) * pl->KB;
+  pl->U = ((N + rows - 1) / rows) * pl->KB;
   pl->P = static_cast<int64_t>(occ) * num_sms();
   if (pl->P > pl->U) pl->P = pl->U;
   // Remembered for the last shape seen by this thread: the scan costs a
@@ -685,6 +1285,28 @@ cudaError_t plan_decode(int64_t K, int64_t N, DecodePlan* pl) {
     last_split = sp;
   }
   pl->split = last_split;
+}
+
+template <typename TX, int NT, int GPB>
+cudaError_t plan_decode(int64_t K, int64_t N, DecodePlan* pl) {
+  static std::atomic<int> occ_cache[64];
+  int occ = 0;
+  const cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_kernel<TX, NT, GPB>),
+                                         kThreads, DLayout<NT>::kAlloc, occ_cache, &occ);
+  if (e != cudaSuccess) return e;
+  plan_split(occ, Tiles<NT>::kRowsPerCta, K, N, pl);
+  return cudaSuccess;
+}
+
+template <typename TX, int NP, bool FUSE>
+cudaError_t plan_decode_i8(int64_t K, int64_t N, DecodePlan* pl) {
+  using S = I8Shape<NP, FUSE>;
+  static std::atomic<int> occ_cache[64];
+  int occ = 0;
+  const cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_i8_kernel<TX, NP, FUSE>),
+                                         S::kThreads, S::kAlloc, occ_cache, &occ);
+  if (e != cudaSuccess) return e;
+  plan_split(occ, S::kRowsPerCta, K, N, pl);
   return cudaSuccess;
 }
 
@@ -776,12 +1398,163 @@ cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uin
                                     stream);
 }
 
+template <typename TX, int NP, bool FUSE>
+cudaError_t launch_decode_i8(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                             int group, int64_t M, int64_t N, float* y, const DecodePlan& pl,
+                             float* partials, uint32_t* counters, uint8_t* records,
+                             cudaStream_t stream) {
+  using S = I8Shape<NP, FUSE>;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
+  const int G = static_cast<int>((K + group - 1) / group);
+  CUtensorMap tw, tx;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    const cuuint32_t box[2] = {128, S::kRowsPerCta};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  std::memset(&tx, 0, sizeof tx);
+  if (S::kFuse) {
+    // x [M, K]: boxes of 256 k by all M rows.
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
+                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
+    cfg.blockDim = dim3(S::kThreads);
+    cfg.dynamicSmemBytes = S::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx, static_cast<const uint8_t*>(nullptr),
+                              scales, y, K, group, G, static_cast<int>(M), N, pl.KB, pl.U,
+                              static_cast<int>(pl.P), partials, counters, status);
+  }
+  // Records 0 .. KB: a stage whose second block is past the last reads the
+  // zero record KB.
+  const int64_t nrec = static_cast<int64_t>(pl.KB) + 1;
+  const int MP = 2 * NP;
+  const int64_t threads = 16 * MP * nrec;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  {
+    cudaLaunchConfig_t dcfg = {};
+    dcfg.gridDim = dim3(static_cast<unsigned>((threads + 255) / 256));
+    dcfg.blockDim = dim3(256);
+    dcfg.stream = stream;
+    dcfg.attrs = attr;
+    dcfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&dcfg, x_digits_kernel<TX>, x, K, static_cast<int>(M),
+                                             MP, NP, nrec, records);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
+  cfg.blockDim = dim3(S::kThreads);
+  cfg.dynamicSmemBytes = S::kAlloc;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx,
+                            static_cast<const uint8_t*>(records), scales, y, K, group, G,
+                            static_cast<int>(M), N, pl.KB, pl.U, static_cast<int>(pl.P), partials,
+                            counters, status);
+}
+
+template <typename TX, int NP, bool FUSE>
+cudaError_t launch_i8_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  using S = I8Shape<NP, FUSE>;
+  DecodePlan pl;
+  cudaError_t e = plan_decode_i8<TX, NP, FUSE>(K, N, &pl);
+  if (e != cudaSuccess) return e;
+  float* partials = nullptr;
+  uint32_t* counters = nullptr;
+  if (pl.split) {
+    e = stream_scratch(stream, static_cast<size_t>(2 * pl.P) * S::kOut, static_cast<size_t>(pl.P),
+                       &partials, &counters);
+    if (e != cudaSuccess) return e;
+  }
+  uint8_t* records = nullptr;
+  if (!S::kFuse) {
+    e = stream_records(stream, static_cast<size_t>(pl.KB + 1) * S::kRec, &records);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_decode_i8<TX, NP, FUSE>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
+                                  records, stream);
+}
+
+template <typename TX, int NP, bool FUSE>
+cudaError_t launch_i8_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                                      int64_t K, int group, int64_t M, int64_t N, float* y,
+                                      cudaStream_t stream, size_t* need) {
+  using S = I8Shape<NP, FUSE>;
+  float* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  DecodePlan pl;
+  e = plan_decode_i8<TX, NP, FUSE>(K, N, &pl);
+  if (e != cudaSuccess) return e;
+  const size_t pbytes = pl.split ? static_cast<size_t>(2 * pl.P) * S::kOut * sizeof(float) : 0;
+  const size_t rbytes = S::kFuse ? 0 : static_cast<size_t>(pl.KB + 1) * S::kRec;
+  if (pbytes > kNoAllocPartialBytes || pl.P > kNoAllocMaxCtas || rbytes > kNoAllocRecordBytes) {
+    *need = pbytes + static_cast<size_t>(pl.P) * sizeof(uint32_t) + rbytes;
+    return cudaErrorInvalidValue;
+  }
+  char* base = reinterpret_cast<char*>(scratch);
+  float* partials = pl.split ? scratch : nullptr;
+  uint32_t* counters = pl.split ? reinterpret_cast<uint32_t*>(base + kNoAllocPartialBytes) : nullptr;
+  uint8_t* records =
+      S::kFuse ? nullptr : reinterpret_cast<uint8_t*>(base + kNoAllocPartialBytes + kNoAllocCounterBytes);
+  return launch_decode_i8<TX, NP, FUSE>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
+                                  records, stream);
+}
+
+template <typename TX>
+cudaError_t launch_i8_any(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
+                          int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  if (M <= kFuseMaxM) return launch_i8_variant<TX, 1, true>(x, packed, scales, K, group, M, N, y, stream);
+  if (M <= 2) return launch_i8_variant<TX, 1, false>(x, packed, scales, K, group, M, N, y, stream);
+  if (M <= 4) return launch_i8_variant<TX, 2, false>(x, packed, scales, K, group, M, N, y, stream);
+  if (M <= 8) return launch_i8_variant<TX, 4, false>(x, packed, scales, K, group, M, N, y, stream);
+  return launch_i8_variant<TX, 8, false>(x, packed, scales, K, group, M, N, y, stream);
+}
+
+template <typename TX>
+cudaError_t launch_i8_any_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                                  int64_t K, int group, int64_t M, int64_t N, float* y,
+                                  cudaStream_t stream, size_t* need) {
+  if (M <= kFuseMaxM)
+    return launch_i8_variant_noalloc<TX, 1, true>(x, packed, scales, K, group, M, N, y, stream, need);
+  if (M <= 2) return launch_i8_variant_noalloc<TX, 1, false>(x, packed, scales, K, group, M, N, y, stream, need);
+  if (M <= 4) return launch_i8_variant_noalloc<TX, 2, false>(x, packed, scales, K, group, M, N, y, stream, need);
+  if (M <= 8) return launch_i8_variant_noalloc<TX, 4, false>(x, packed, scales, K, group, M, N, y, stream, need);
+  return launch_i8_variant_noalloc<TX, 8, false>(x, packed, scales, K, group, M, N, y, stream, need);
+}
+
 template <typename TX, int NT>
 cudaError_t launch_nt_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                               int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
                               size_t* need) {
-  if (group % 128 == 0)
-    return launch_variant_noalloc<TX, NT, 1>(x, packed, scales, K, group, M, N, y, stream, need);
   if (group == 64)
     return launch_variant_noalloc<TX, NT, 2>(x, packed, scales, K, group, M, N, y, stream, need);
   return launch_variant_noalloc<TX, NT, 4>(x, packed, scales, K, group, M, N, y, stream, need);
@@ -791,6 +1564,7 @@ template <typename TX>
 cudaError_t launch_tx_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                               int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
                               size_t* need) {
+  if (group % 128 == 0) return launch_i8_any_noalloc(x, packed, scales, K, group, M, N, y, stream, need);
   if (M <= 8) return launch_nt_noalloc<TX, 1>(x, packed, scales, K, group, M, N, y, stream, need);
   return launch_nt_noalloc<TX, 2>(x, packed, scales, K, group, M, N, y, stream, need);
 }
@@ -798,7 +1572,6 @@ cudaError_t launch_tx_noalloc(const TX* x, const uint8_t* packed, const uint16_t
 template <typename TX, int NT>
 cudaError_t launch_nt(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                       int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  if (group % 128 == 0) return launch_variant<TX, NT, 1>(x, packed, scales, K, group, M, N, y, stream);
   if (group == 64) return launch_variant<TX, NT, 2>(x, packed, scales, K, group, M, N, y, stream);
   return launch_variant<TX, NT, 4>(x, packed, scales, K, group, M, N, y, stream);
 }
@@ -806,6 +1579,7 @@ cudaError_t launch_nt(const TX* x, const uint8_t* packed, const uint16_t* scales
 template <typename TX>
 cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
                       int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  if (group % 128 == 0) return launch_i8_any(x, packed, scales, K, group, M, N, y, stream);
   if (M <= 8) return launch_nt<TX, 1>(x, packed, scales, K, group, M, N, y, stream);
   return launch_nt<TX, 2>(x, packed, scales, K, group, M, N, y, stream);
 }

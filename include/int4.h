@@ -112,7 +112,13 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
  * Integer weights enter the arithmetic exactly (-8..7 is exact in bf16, fp16
  * and fp32); group partial sums are accumulated in fp32 (fp64 across groups
  * for fp32 x); the group's scale is applied to each partial before it joins
- * the running sum.  Accuracy: |y - y_exact| <= c * sum_k |x[m,k]| |w_hat[n,k]|
+ * the running sum.  The decode kernel for groups that are a multiple of 128
+ * forms each 128-k block's sum x.q exactly in integers: x is written per
+ * block as a 30-bit integer times a power of two (exact for every bf16 x
+ * within 2^22 of the block's largest |x|, fp16 within 2^19; otherwise off by
+ * at most 2^-30 of that largest), a NaN or infinity in a block makes the
+ * row's outputs NaN, and blocks whose largest |x| is below 2^-93 keep fewer
+ * low digits.  Accuracy: |y - y_exact| <= c * sum_k |x[m,k]| |w_hat[n,k]|
  * with c = 1e-5 for fp32 x and c = 4e-3 for bf16 / fp16 x.  Summation order
  * differs between kernels; results are deterministic for a given shape,
  * dtype and device.
@@ -147,11 +153,6 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
                      int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
                      void* stream);
 
-/*
- * int4_matmul_select - the path int4_matmul would take for this problem
- * (one of INT4_PATH_SIMT / _DECODE / _PREFILL), or a negative status if the
- * arguments are invalid.  Host-only; launches nothing.
- */
 /* Allocation-free decode matmul.  The pages have no counterpart: this entry
  * exists for callers that must not allocate device memory during the call,
  * such as a serving loop that runs inside a fixed memory budget, or a
@@ -159,9 +160,10 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
  * block, synchronize or fail under memory pressure).
  *
  * Computes what int4_matmul computes on its decode path (same kernels, same
- * result bits), with the partial tiles of the split kept in a fixed
- * library-owned device array of 4 MiB plus 2 KiB (one wave of up to 512 CTAs)
- * instead of per-stream scratch.  It calls no cudaMalloc, cudaFree or other
+ * result bits), with the partial tiles of the split (4 MiB: one wave of up to
+ * 512 CTAs), their arrival counters (2 KiB) and the integer digits of x
+ * (4 MiB: K up to 64384 at M = 16, 246528 at M <= 4; not used at M <= 2) kept
+ * in a fixed library-owned device array instead of per-stream scratch.  It calls no cudaMalloc, cudaFree or other
  * allocating routine.  The array's arrival counters must start at zero: they
  * are zero when the library loads and every call leaves them zero (after a
  * device-side wait gave up, int4_device_status zeroes them again).
@@ -170,7 +172,7 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
  * INT4_ERR_UNSUPPORTED when the decode kernel cannot run the shape (x must be
  * bf16 or fp16, M <= 16, K % 32 == 0, group 32, 64 or a multiple of 128, x and
  * packed 16-byte aligned), and INT4_ERR_ARG with a message naming both sizes
- * when the split needs more scratch than the array holds.
+ * when the call needs more scratch than the array holds.
  *
  * The first call on each device resolves the array's address with
  * cudaGetSymbolAddress (that device current); make that first call before any
@@ -181,6 +183,11 @@ int int4_matmul_decode_noalloc(const void* x, int32_t x_dtype, const uint8_t* pa
                                const uint16_t* scales, int64_t K, int32_t group, int64_t M,
                                int64_t N, float* y, void* stream);
 
+/*
+ * int4_matmul_select - the path int4_matmul would take for this problem
+ * (one of INT4_PATH_SIMT / _DECODE / _PREFILL), or a negative status if the
+ * arguments are invalid.  Host-only; launches nothing.
+ */
 int int4_matmul_select(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N);
 
 /*

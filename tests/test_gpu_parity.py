@@ -413,6 +413,50 @@ def test_matmul_decode_split_tiles(M, N, K, group, dtype):
     assert_matmul_close(a, x, packed, scales, K, group, _tol(dtype))
 
 
+def _wide_range_x(M, K, dtype, seed, outlier=2.0 ** 12, tiny=2.0 ** -14):
+    """N(0, 1) activations with outlier columns (x outlier) and tiny ones (x tiny)."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, K, generator=g)
+    x[:, torch.randint(0, K, (max(K // 64, 1),), generator=g)] *= outlier
+    x[:, torch.randint(0, K, (max(K // 16, 1),), generator=g)] *= tiny
+    return x.to(dtype).to(DEV)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
+def test_matmul_decode_x_dynamic_range(dtype, M):
+    """The decode kernel represents each 128-k block of a batch row as
+    integers relative to the block's largest |x|: blocks holding outlier
+    features 2^12 above the typical value, and values 2^14 below it, must
+    still meet the bound."""
+    N, K, group = 512, 2048, 128
+    packed, scales, _ = _quantized(N, K, group, seed=7, dist="student_t3", zero_group_frac=0.05)
+    x = _wide_range_x(M, K, dtype, seed=M)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF)
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -90, 2.0 ** -60, 2.0 ** 60, 2.0 ** 100])
+def test_matmul_decode_extreme_magnitudes_bf16(scale):
+    """bf16 activations far from 1 in both directions (whole rows scaled)."""
+    N, K, group = 256, 1024, 256
+    packed, scales, _ = _quantized(N, K, group, seed=11)
+    x = (make_activations(4, K, seed=5, device=DEV, dtype=torch.float32) * scale).to(torch.bfloat16)
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF)
+
+
+@pytest.mark.parametrize("N", [300, 20000])   # the small-matrix and the streaming kernel
+def test_matmul_decode_nonfinite_x_poisons_only_its_row(N):
+    K, group = 1024, 128
+    packed, scales, _ = _quantized(N, K, group, seed=4)
+    x = make_activations(3, K, seed=6, device=DEV, dtype=torch.bfloat16)
+    x[1, 200] = float("inf")
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
+    assert not torch.isfinite(y[1]).any()
+    assert_matmul_close(y[[0, 2]], x[[0, 2]], packed, scales, K, group, TOL_HALF)
+
+
 @pytest.mark.parametrize("layer", LLAMA7B_DECODE_LINEARS, ids=lambda l: l.name)
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_matmul_llama7b_decode_full_size(layer, M):

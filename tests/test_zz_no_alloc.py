@@ -18,6 +18,8 @@ DEV = "cuda"
 @pytest.mark.parametrize("M, N, K, group, dtype", [
     (1, 28672, 8192, 128, torch.bfloat16),   # partial tiles at most run ends
     (4, 4096, 4096, 128, torch.bfloat16),    # many runs per tile
+    (16, 20000, 4096, 128, torch.bfloat16),  # x digits in the static array
+    (2, 11008, 4096, 256, torch.float16),    # x converted inside the matmul
     (16, 1000, 12288, 64, torch.float16),    # 64-row tiles, ragged last tile
     (3, 37, 4096, 32, torch.bfloat16),       # a single short tile
 ])
@@ -48,3 +50,20 @@ def test_noalloc_rejects_shapes_the_decode_kernel_cannot_run():
     with pytest.raises(q4.Int4Error) as ei:
         q4.int4_matmul_decode_noalloc(x, packed, scales, K, group, out)
     assert ei.value.code == q4.ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_x_digits_beyond_the_static_array():
+    """At M = 16 the x digit records of K = 65536 (513 blocks of 8320 bytes)
+    exceed the 4 MiB the array keeps for them: the call is refused on the
+    host before anything launches."""
+    M, N, K, group = 16, 7200, 65536, 128
+    packed = torch.zeros((N, K // 2), dtype=torch.uint8, device=DEV)
+    scales = torch.zeros((N, K // group), dtype=torch.float16, device=DEV)
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device=DEV)
+    out = torch.full((M, N), 7.0, dtype=torch.float32, device=DEV)
+    with pytest.raises(q4.Int4Error) as ei:
+        q4.int4_matmul_decode_noalloc(x, packed, scales, K, group, out)
+    assert ei.value.code == q4.ERR_ARG
+    assert "scratch" in str(ei.value)
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())        # nothing ran
