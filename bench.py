@@ -51,10 +51,10 @@ KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
     "prefill": (3_925_588_000 + 920_221_696, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
                 "009294f3ae9d1c445ad32b0380ace3d8f9cb911804642ade540a76cdcf693f64"),
-    "decode": (125_215_744 + 4_575_744, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
-               "12264ac9d2ce5c656a6178dccd451f1274c47f2a8046a32456cbbc2c87b4babd"),
-    "quantize": (469_871_872 + 105_121_024, "dequant_gemm_int4_b200/csrc/quantize.cu",
-                 "e481dd90e6bf89151b943029f526998eb4bc27e2c9e269c7822f18745f40de65"),
+    "decode": (125_660_928 + 3_920_896, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
+               "d0ae35aa9c1a6fc5949a408f3e689c6f55df617ca49d0068f1fa22a230ef7c37"),
+    "quantize": (469_870_592 + 105_440_512, "dequant_gemm_int4_b200/csrc/quantize.cu",
+                 "b1d0625c98d5c79ff67cce0033f11115c392cbd51898b59e617efd38a73f960a"),
     "unpack": (117_453_568 + 180_738_816, "dequant_gemm_int4_b200/csrc/unpack.cu",
                "5d7f0c52a24a85e10103ad6ca335aa3e8ec965bd076335ea69f00af1073f2e82"),
 }
