@@ -88,6 +88,15 @@ namespace {
 #ifndef INT4_DECODE_I8_FUSE_MAX_M
 #define INT4_DECODE_I8_FUSE_MAX_M 2
 #endif
+#ifndef INT4_DECODE_WAIT_MODE
+#define INT4_DECODE_WAIT_MODE 0  // 0: try_wait, then 20 us suspend hints; 1: test_wait polling; 2: 500 ns hints
+#endif
+#ifndef INT4_DECODE_SMALL
+#define INT4_DECODE_SMALL 1
+#endif
+#ifndef INT4_DECODE_I8_TILES
+#define INT4_DECODE_I8_TILES 2
+#endif
 #ifndef INT4_DECODE_I8_SCALE_AHEAD
 #define INT4_DECODE_I8_SCALE_AHEAD 1
 #endif
@@ -196,10 +205,20 @@ struct WaitCtx {
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+#if INT4_DECODE_WAIT_MODE == 1
+  if (ptx::mbar_test_wait(bar, parity)) return true;
+#else
   if (ptx::mbar_try_wait(bar, parity)) return true;
+#endif
   const uint64_t t0 = ptx::globaltimer();
   for (uint32_t i = 1; i != 0; ++i) {
+#if INT4_DECODE_WAIT_MODE == 1
+    if (ptx::mbar_test_wait(bar, parity)) return true;
+#elif INT4_DECODE_WAIT_MODE == 2
+    if (ptx::mbar_try_wait_sleep(bar, parity, 500u)) return true;
+#else
     if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+#endif
     if ((i & 15u) == 0u) {
       if (*w.abort) return false;
       if (ptx::globaltimer() - t0 > kTimeoutNs) break;
@@ -755,7 +774,7 @@ template <int NP, bool FUSE>
 struct I8Shape {
   static constexpr bool kFuse = FUSE;                                // converter warp in the CTA
   static_assert(!FUSE || NP == 1, "the converter warp serves up to two batch rows");
-  static constexpr int kTiles = NP <= 2 ? 2 : 1;                    // 16-row tiles per consumer
+  static constexpr int kTiles = NP <= 2 ? INT4_DECODE_I8_TILES : 1;  // 16-row tiles per consumer
   static constexpr int kRowsPerCta = 16 * kTiles * kRowGroups;       // 128 or 64
   static constexpr int kWBytes = kRowsPerCta * kSK * 64;             // packed W of a stage
   static constexpr int kRec = NP * kDigitTile + 128;                 // digit record of a block
@@ -832,8 +851,21 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
   // Launched as a programmatic dependent of what precedes it on the stream
   // (the digits grid, or any kernel): the set-up above overlaps that grid's
   // tail, and every thread waits for it to complete (its writes visible)
-  // before reading an input or writing an output.  The next kernel may
-  // likewise start its set-up early.
+  // before reading an input or writing an output.  Before that wait the
+  // producer only asks L2 to prefetch the weight tiles of its first stages
+  // (L2 is coherent, so a tile the earlier kernel still writes is read
+  // fresh after the wait).  The next kernel may likewise start early.
+  if (warp == 0 && lane == 0) {
+    int pf = 0;
+    for (int64_t u = u_begin; pf < kStages && u < u_end;) {
+      const int64_t r = u / KB;
+      const int blo = static_cast<int>(u - r * KB);
+      const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
+      for (int kb = blo; pf < kStages && kb < bhi; kb += kSK, ++pf)
+        ptx::tma_prefetch_2d(&tm_w, kb * 64, static_cast<int32_t>(r * kRowsPerCta));
+      u = r * KB + bhi;
+    }
+  }
   ptx::launch_dependents();
   ptx::grid_dependency_wait();
 
@@ -1712,7 +1744,7 @@ cudaError_t launch_small(const TX* x, const uint8_t* packed, const uint16_t* sca
 // Small matrices: 16-row tiles that fit one wave, K a multiple of 128 (so
 // every block is whole) and groups of whole blocks.
 bool small_applies(int64_t K, int group, int64_t N) {
-  if (group % 128 != 0 || K % 128 != 0) return false;
+  if (!INT4_DECODE_SMALL || group % 128 != 0 || K % 128 != 0) return false;
   return (N + 15) / 16 <= static_cast<int64_t>(kSmallCtasPerSm) * num_sms();
 }
 

@@ -400,18 +400,23 @@ __global__ void __launch_bounds__(256) quantize_wide_kernel(
 }
 
 // Rows at any alignment (odd K, unaligned pointers), same groups as the fast
-// path.  The weights are read as aligned 16-byte chunks of the byte range that
-// starts at `wbase` (16-byte aligned, w[0,0] at byte `wshift`): a lane loads
-// its chunk(s), takes the next lane's first chunk by shuffle and funnel-shifts
-// by the row's byte offset, which is the same for every lane of the window.
-// Packed bytes are written as aligned words with store_segment.
-template <typename T, int LPG>
+// path.  A lane takes EPL consecutive elements (NCH 16-byte chunks: 16 for
+// 16-bit weights with NCH = 2, else 8), a warp a window of 32 EPL elements
+// of one row.  The weights are read as aligned 16-byte chunks of the byte
+// range that starts at `wbase` (16-byte aligned, w[0,0] at byte `wshift`): a
+// lane loads its chunks, takes the next lane's first chunk by shuffle and
+// funnel-shifts by the row's byte offset, which is the same for every lane of
+// the window.  Packed bytes are written as aligned words with store_segment.
+template <typename T, int LPG, int NCH>
 __global__ void __launch_bounds__(256) quantize_any_kernel(
     const uint8_t* __restrict__ wbase, int64_t wshift, int64_t wbytes, int64_t K, int G,
     int64_t windows_per_row, int64_t total_windows, uint8_t* __restrict__ pbase, int64_t pshift,
     uint16_t* __restrict__ scales) {
   constexpr int ELT = static_cast<int>(sizeof(T));
-  constexpr int NCH = ELT == 4 ? 2 : 1;  // 16-byte chunks per lane (8 elements)
+  constexpr int EPL = NCH * 16 / ELT;  // elements per lane
+  constexpr int WIN = 32 * EPL;        // elements per window
+  constexpr int PW = EPL / 8;          // packed words per lane
+  static_assert(EPL % 8 == 0, "whole 8-element code words per lane");
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -425,7 +430,7 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
 
   // The next window's chunks are loaded while the current one is quantized.
   auto fetch = [&](int64_t r, int64_t cl, uint4 (&own)[NCH], uint4& extra) {
-    const int64_t c0 = (wshift + (r * K + cl * 256 + lane * 8) * ELT) >> 4;
+    const int64_t c0 = (wshift + (r * K + cl * WIN + lane * EPL) * ELT) >> 4;
 #pragma unroll
     for (int q = 0; q < NCH; ++q) own[q] = load_chunk16(wbase, c0 + q, wbytes);
     extra = (lane == 31) ? load_chunk16(wbase, c0 + NCH, wbytes) : make_uint4(0u, 0u, 0u, 0u);
@@ -437,7 +442,7 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
 #pragma unroll
     for (int q = 0; q < NCH; ++q) cur[q] = own[q];
     const uint4 cur_extra = extra;
-    const int64_t kl = col * 256 + lane * 8;  // first element of this lane in the row
+    const int64_t kl = col * WIN + lane * EPL;  // first element of this lane in the row
     const int64_t P = wshift + (row * K + kl) * ELT;
     const int boff = static_cast<int>(P & 15);
     const int64_t crow = row, ccol = col;
@@ -460,9 +465,9 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
     win[4 * NCH] = nx.x; win[4 * NCH + 1] = nx.y; win[4 * NCH + 2] = nx.z; win[4 * NCH + 3] = nx.w;
     uint32_t e[4 * NCH];
     byte_shift_words<4 * (NCH + 1), 4 * NCH>(win, boff, e);
-    float v[8];
+    float v[EPL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < EPL; ++i) {
       float f;
       if (ELT == 4) f = __uint_as_float(e[i]);
       else if (std::is_same<T, __nv_bfloat16>::value) f = __uint_as_float((i & 1) ? (e[i >> 1] & 0xFFFF0000u) : (e[i >> 1] << 16));
@@ -471,27 +476,36 @@ __global__ void __launch_bounds__(256) quantize_any_kernel(
     }
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+    for (int i = 0; i < EPL; ++i) m = fmaxf(m, fabsf(v[i]));
 #pragma unroll
     for (int off = 1; off < LPG; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     const ScaleInfo si = scale_from_absmax(m);
     const uint32_t ex = si.bits & 0x7C00u;
     const bool simple = (ex != 0u && ex != 0x7C00u) || si.bits == 0u;
-    uint32_t word;
-    const bool ok = codes8<T>(v, si.r, word) && simple;
+    uint32_t words[PW];
+    bool ok = simple;
+#pragma unroll
+    for (int p = 0; p < PW; ++p) {
+      float v8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v8[i] = v[8 * p + i];
+      ok = codes8<T>(v8, si.r, words[p]) && ok;
+    }
     if (!__all_sync(0xffffffffu, ok)) {
       if (!ok) {
-        word = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) word |= code_exact(v[i], si) << (4 * i);
+        for (int p = 0; p < PW; ++p) {
+          words[p] = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) words[p] |= code_exact(v[8 * p + i], si) << (4 * i);
+        }
       }
     }
-    if (kl < K && (lane & (LPG - 1)) == 0) scales[crow * G + kl / (8 * LPG)] = static_cast<uint16_t>(si.bits);
+    if (kl < K && (lane & (LPG - 1)) == 0) scales[crow * G + kl / (EPL * LPG)] = static_cast<uint16_t>(si.bits);
     const int64_t rowp = pshift + crow * Kp;
-    const int64_t f0 = rowp + ccol * 128;
-    const int64_t hi = (f0 + 128 < rowp + Kp) ? f0 + 128 : rowp + Kp;
-    const uint32_t wd[1] = {word};
-    store_segment<1>(pbase, f0, f0, hi, wd, lane);
+    const int64_t f0 = rowp + ccol * (WIN / 2);
+    const int64_t hi = (f0 + WIN / 2 < rowp + Kp) ? f0 + WIN / 2 : rowp + Kp;
+    store_segment<PW>(pbase, f0, f0, hi, words, lane);
   }
 }
 
@@ -603,28 +617,45 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
     const uintptr_t pa = reinterpret_cast<uintptr_t>(packed);
     uint8_t* pbase = reinterpret_cast<uint8_t*>(pa & ~static_cast<uintptr_t>(3));
     const int64_t pshift = static_cast<int64_t>(pa & 3);
-    const int64_t wpr = (K + 255) / 256;
-    const int64_t total = N * wpr;
     const int64_t wbytes = wshift + N * K * static_cast<int64_t>(sizeof(T));
+    // 16 elements per lane for 16-bit weights when a group spans whole lanes.
+    const bool two = sizeof(T) == 2 && group % 16 == 0 && group / 16 <= 32;
+    const int epl = two ? 16 : 8;
+    const int lanes = group / epl;
+    const int64_t wpr = (K + 32 * epl - 1) / (32 * epl);
+    const int64_t total = N * wpr;
     const int64_t want = (total + 31) / 32;
-    switch (lpg) {
-#define INT4_QA_CASE(L)                                                                        \
+#define INT4_QA_CASE(L, C)                                                                     \
   case L:                                                                                      \
-    quantize_any_kernel<T, L><<<resident_grid(quantize_any_kernel<T, L>, want), 256, 0,        \
-                                stream>>>(reinterpret_cast<const uint8_t*>(wbase),             \
-                                                        wshift, wbytes, K, G, wpr, total, pbase, \
-                                                        pshift, scales);                         \
+    quantize_any_kernel<T, L, C><<<resident_grid(quantize_any_kernel<T, L, C>, want), 256, 0,  \
+                                   stream>>>(reinterpret_cast<const uint8_t*>(wbase), wshift,  \
+                                             wbytes, K, G, wpr, total, pbase, pshift, scales); \
     break;
-      INT4_QA_CASE(1)
-      INT4_QA_CASE(2)
-      INT4_QA_CASE(4)
-      INT4_QA_CASE(8)
-      INT4_QA_CASE(16)
-      INT4_QA_CASE(32)
-#undef INT4_QA_CASE
-      default:
-        break;
+    if (two) {
+      switch (lanes) {
+        INT4_QA_CASE(1, 2)
+        INT4_QA_CASE(2, 2)
+        INT4_QA_CASE(4, 2)
+        INT4_QA_CASE(8, 2)
+        INT4_QA_CASE(16, 2)
+        INT4_QA_CASE(32, 2)
+        default:
+          break;
+      }
+    } else {
+      constexpr int kC = sizeof(T) == 4 ? 2 : 1;  // 8 elements per lane
+      switch (lanes) {
+        INT4_QA_CASE(1, kC)
+        INT4_QA_CASE(2, kC)
+        INT4_QA_CASE(4, kC)
+        INT4_QA_CASE(8, kC)
+        INT4_QA_CASE(16, kC)
+        INT4_QA_CASE(32, kC)
+        default:
+          break;
+      }
     }
+#undef INT4_QA_CASE
     return cudaGetLastError();
   }
   quantize_scales_general_kernel<T><<<grid_for(N * G, 256, 16), 256, 0, stream>>>(w, N, K, group, G,
