@@ -399,9 +399,14 @@ __global__ void __launch_bounds__(256) quantize_wide_kernel(
   }
 }
 
+#ifndef INT4_QUANT_ANY_CHUNKS
+#define INT4_QUANT_ANY_CHUNKS 4
+#endif
+constexpr int kAnyChunks16 = INT4_QUANT_ANY_CHUNKS;  // 16-byte chunks per lane, 16-bit weights
+
 // Rows at any alignment (odd K, unaligned pointers), same groups as the fast
-// path.  A lane takes EPL consecutive elements (NCH 16-byte chunks: 16 for
-// 16-bit weights with NCH = 2, else 8), a warp a window of 32 EPL elements
+// path.  A lane takes EPL consecutive elements (NCH 16-byte chunks: 8 NCH for
+// 16-bit weights, 8 for fp32), a warp a window of 32 EPL elements
 // of one row.  The weights are read as aligned 16-byte chunks of the byte
 // range that starts at `wbase` (16-byte aligned, w[0,0] at byte `wshift`): a
 // lane loads its chunks, takes the next lane's first chunk by shuffle and
@@ -618,9 +623,11 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
     uint8_t* pbase = reinterpret_cast<uint8_t*>(pa & ~static_cast<uintptr_t>(3));
     const int64_t pshift = static_cast<int64_t>(pa & 3);
     const int64_t wbytes = wshift + N * K * static_cast<int64_t>(sizeof(T));
-    // 16 elements per lane for 16-bit weights when a group spans whole lanes.
-    const bool two = sizeof(T) == 2 && group % 16 == 0 && group / 16 <= 32;
-    const int epl = two ? 16 : 8;
+    // kAnyChunks16 16-byte chunks per lane for 16-bit weights when a group
+    // spans whole lanes.
+    constexpr int kWideEpl = 8 * kAnyChunks16;
+    const bool two = sizeof(T) == 2 && group % kWideEpl == 0 && group / kWideEpl <= 32;
+    const int epl = two ? kWideEpl : 8;
     const int lanes = group / epl;
     const int64_t wpr = (K + 32 * epl - 1) / (32 * epl);
     const int64_t total = N * wpr;
@@ -633,12 +640,12 @@ cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* p
     break;
     if (two) {
       switch (lanes) {
-        INT4_QA_CASE(1, 2)
-        INT4_QA_CASE(2, 2)
-        INT4_QA_CASE(4, 2)
-        INT4_QA_CASE(8, 2)
-        INT4_QA_CASE(16, 2)
-        INT4_QA_CASE(32, 2)
+        INT4_QA_CASE(1, kAnyChunks16)
+        INT4_QA_CASE(2, kAnyChunks16)
+        INT4_QA_CASE(4, kAnyChunks16)
+        INT4_QA_CASE(8, kAnyChunks16)
+        INT4_QA_CASE(16, kAnyChunks16)
+        INT4_QA_CASE(32, kAnyChunks16)
         default:
           break;
       }

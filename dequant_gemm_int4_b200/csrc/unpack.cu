@@ -56,14 +56,43 @@ __global__ void __launch_bounds__(256) unpack_flat_kernel(const uint8_t* __restr
   }
 }
 
-// Any K and alignment: a warp window is 512 outputs (256 packed bytes) of one
-// row.  A lane takes its aligned 8-byte chunk of the packed byte range, the
-// next lane's chunk by shuffle, funnel-shifts by the row's byte offset, expands
-// 16 nibbles and writes them with aligned word stores (store_segment).
+// Any K and alignment: a lane takes NB packed bytes (2 NB outputs), a warp a
+// window of 64 NB outputs of one row.  A lane takes its aligned NB-byte
+// chunk of the packed byte range, the next lane's chunk by shuffle,
+// funnel-shifts by the row's byte offset, expands the nibbles and writes
+// them with aligned word stores (store_segment).
+#ifndef INT4_UNPACK_ANY_BYTES
+#define INT4_UNPACK_ANY_BYTES 8
+#endif
+// packed bytes per lane: 8 measured faster than 16 (2.1 against 1.2 TB/s on
+// W [8192, 28673]), whose eight clipped word stores per lane cost more than
+// the halved window count saves.
+constexpr int kUnpackAnyBytes = INT4_UNPACK_ANY_BYTES;
+
+template <int NB>
+__device__ __forceinline__ void load_packed_chunk(const uint8_t* base, int64_t c, int64_t nbytes,
+                                                  uint32_t (&w)[NB / 4]) {
+  if (NB == 8) {
+    const uint2 v = load_chunk8(base, c, nbytes);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+    const uint4 v = load_chunk16(base, c, nbytes);
+    w[0] = v.x;
+    w[1] = v.y;
+    w[NB / 4 > 2 ? 2 : 0] = v.z;
+    w[NB / 4 > 3 ? 3 : 0] = v.w;
+  }
+}
+
+template <int NB>
 __global__ void __launch_bounds__(256) unpack_any_kernel(const uint8_t* __restrict__ pbase,
                                                         int64_t pshift, int64_t pbytes, int64_t K,
                                                         int64_t windows_per_row, int64_t total_windows,
                                                         uint8_t* __restrict__ obase, int64_t oshift) {
+  static_assert(NB == 8 || NB == 16, "8- or 16-byte chunks");
+  constexpr int NW = NB / 4;     // packed words per lane
+  constexpr int WOUT = 64 * NB;  // outputs per window
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -74,37 +103,52 @@ __global__ void __launch_bounds__(256) unpack_any_kernel(const uint8_t* __restri
   const int64_t Kp = (K + 1) >> 1;
   int64_t row = wi / windows_per_row;
   int64_t col = wi - row * windows_per_row;
+
   // The next window's chunk is loaded while the current one is expanded.
-  auto fetch = [&](int64_t r, int64_t cl, uint2& own, uint2& extra) {
-    const int64_t c = (pshift + r * Kp + cl * 256 + lane * 8) >> 3;
-    own = load_chunk8(pbase, c, pbytes);
-    extra = (lane == 31) ? load_chunk8(pbase, c + 1, pbytes) : make_uint2(0u, 0u);
+  auto fetch = [&](int64_t r, int64_t cl, uint32_t (&own)[NW], uint32_t (&extra)[NW]) {
+    const int64_t c = (pshift + r * Kp + cl * (32 * NB) + lane * NB) / NB;
+    load_packed_chunk<NB>(pbase, c, pbytes, own);
+    if (lane == 31) {
+      load_packed_chunk<NB>(pbase, c + 1, pbytes, extra);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NW; ++j) extra[j] = 0u;
+    }
   };
-  uint2 own, extra;
+  uint32_t own[NW], extra[NW];
   fetch(row, col, own, extra);
   for (; wi < wend;) {
-    const uint2 cur = own, cur_extra = extra;
-    const int boff = static_cast<int>((pshift + row * Kp + col * 256 + lane * 8) & 7);
+    uint32_t win[2 * NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) win[j] = own[j];
+    uint32_t cur_extra[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) cur_extra[j] = extra[j];
+    const int boff = static_cast<int>((pshift + row * Kp + col * (32 * NB) + lane * NB) & (NB - 1));
     const int64_t crow = row, ccol = col;
     if (++col == windows_per_row) {
       col = 0;
       ++row;
     }
     if (++wi < wend) fetch(row, col, own, extra);
-    uint2 nx;
-    nx.x = __shfl_down_sync(0xffffffffu, cur.x, 1);
-    nx.y = __shfl_down_sync(0xffffffffu, cur.y, 1);
-    if (lane == 31) nx = cur_extra;
-    const uint32_t win[4] = {cur.x, cur.y, nx.x, nx.y};
-    uint32_t b8[2];
-    byte_shift_words<4, 2>(win, boff, b8);
-    const uint2 a = expand_word(b8[0]);
-    const uint2 b = expand_word(b8[1]);
-    const uint32_t o[4] = {a.x, a.y, b.x, b.y};
+#pragma unroll
+    for (int j = 0; j < NW; ++j) {
+      const uint32_t nx = __shfl_down_sync(0xffffffffu, win[j], 1);
+      win[NW + j] = (lane == 31) ? cur_extra[j] : nx;
+    }
+    uint32_t bw[NW];
+    byte_shift_words<2 * NW, NW>(win, boff, bw);
+    uint32_t o[2 * NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) {
+      const uint2 e = expand_word(bw[j]);
+      o[2 * j] = e.x;
+      o[2 * j + 1] = e.y;
+    }
     const int64_t rowo = oshift + crow * K;
-    const int64_t f0 = rowo + ccol * 512;
-    const int64_t hi = (f0 + 512 < rowo + K) ? f0 + 512 : rowo + K;
-    store_segment<4>(obase, f0, f0, hi, o, lane);
+    const int64_t f0 = rowo + ccol * WOUT;
+    const int64_t hi = (f0 + WOUT < rowo + K) ? f0 + WOUT : rowo + K;
+    store_segment<2 * NW>(obase, f0, f0, hi, o, lane);
   }
 }
 
@@ -122,16 +166,17 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* o
     unpack_flat_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(packed, total, out);
     return cudaGetLastError();
   }
+  constexpr int NB = kUnpackAnyBytes;
   const uintptr_t pa = reinterpret_cast<uintptr_t>(packed);
-  const uint8_t* pbase = reinterpret_cast<const uint8_t*>(pa & ~static_cast<uintptr_t>(7));
-  const int64_t pshift = static_cast<int64_t>(pa & 7);
+  const uint8_t* pbase = reinterpret_cast<const uint8_t*>(pa & ~static_cast<uintptr_t>(NB - 1));
+  const int64_t pshift = static_cast<int64_t>(pa & (NB - 1));
   const uintptr_t oa = reinterpret_cast<uintptr_t>(out);
   uint8_t* obase = reinterpret_cast<uint8_t*>(oa & ~static_cast<uintptr_t>(3));
   const int64_t oshift = static_cast<int64_t>(oa & 3);
-  const int64_t wpr = (K + 511) / 512;
+  const int64_t wpr = (K + 64 * NB - 1) / (64 * NB);
   const int64_t total = N * wpr;
-  const int grid = resident_grid(unpack_any_kernel, (total + 31) / 32);
-  unpack_any_kernel<<<grid, 256, 0, stream>>>(
+  const int grid = resident_grid(unpack_any_kernel<NB>, (total + 31) / 32);
+  unpack_any_kernel<NB><<<grid, 256, 0, stream>>>(
       pbase, pshift, pshift + N * ((K + 1) / 2), K, wpr, total, obase, oshift);
   return cudaGetLastError();
 }
