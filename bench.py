@@ -51,12 +51,12 @@ KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
     "prefill": (3_925_588_000 + 920_221_696, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
                 "009294f3ae9d1c445ad32b0380ace3d8f9cb911804642ade540a76cdcf693f64"),
-    "decode": (125_660_928 + 3_920_896, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
-               "d0ae35aa9c1a6fc5949a408f3e689c6f55df617ca49d0068f1fa22a230ef7c37"),
-    "quantize": (469_870_592 + 105_440_512, "dequant_gemm_int4_b200/csrc/quantize.cu",
-                 "b1d0625c98d5c79ff67cce0033f11115c392cbd51898b59e617efd38a73f960a"),
-    "unpack": (117_453_568 + 180_738_816, "dequant_gemm_int4_b200/csrc/unpack.cu",
-               "5d7f0c52a24a85e10103ad6ca335aa3e8ec965bd076335ea69f00af1073f2e82"),
+    "decode": (125_485_312 + 3_899_904, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
+               "f3ac46c0847c0e41bb556fe66ffc7f43a78eba80f11968fcbb4f105fd034a952"),
+    "quantize": (469_856_256 + 104_254_208, "dequant_gemm_int4_b200/csrc/quantize.cu",
+                 "24a51fde9c6ea1afd8a159345f565f16441d8a085e241e8e6d8d123c71573f57"),
+    "unpack": (117_453_056 + 182_672_128, "dequant_gemm_int4_b200/csrc/unpack.cu",
+               "044a340e737101c2f50713e331878458fb60661e3db5fb9b849e7f5a7588956a"),
 }
 
 
