@@ -132,6 +132,13 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
  * decode kernel; bf16/fp16 x with larger M takes the tcgen05 tensor-core
  * kernel; fp32 x, and shapes the fast kernels do not cover (K or group not a
  * multiple of 32, unaligned rows), take the general CUDA-core kernel.
+ *
+ * Stream ordering: the decode kernels for groups that are a multiple of 128
+ * launch with programmatic stream serialization and wait for the preceding
+ * work on `stream` before touching memory, so ordinary stream order holds.
+ * They also signal dependents early: a kernel that the caller launches after
+ * them with programmatic stream serialization must execute
+ * griddepcontrol.wait (cudaGridDependencySynchronize) before it reads y.
  */
 int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                 int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* stream);
