@@ -103,8 +103,11 @@ def _need_cuda(name: str, t: torch.Tensor) -> None:
         raise ValueError(f"{name} must be contiguous (row-major, no padding)")
 
 
-def quantize_int4(w: torch.Tensor, group: int = 128):
-    """Quantize w [N, K] (fp32/bf16/fp16) -> (packed uint8 [N, ceil(K/2)], scales fp16 [N, G], K)."""
+def quantize_int4(w: torch.Tensor, group: int = 128, *, packed: torch.Tensor | None = None,
+                  scales: torch.Tensor | None = None):
+    """Quantize w [N, K] (fp32/bf16/fp16) -> (packed uint8 [N, ceil(K/2)], scales fp16 [N, G], K).
+
+    `packed` and `scales`, if given, are written in place (same shapes and dtypes)."""
     _need_cuda("w", w)
     if w.dim() != 2:
         raise ValueError("w must be [N, K]")
@@ -112,8 +115,16 @@ def quantize_int4(w: torch.Tensor, group: int = 128):
         raise TypeError("w must be float32, bfloat16 or float16")
     N, K = w.shape
     G = -(-K // group) if group >= 1 else 0
-    packed = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=w.device)
-    scales = torch.empty((N, max(G, 0)), dtype=torch.float16, device=w.device)
+    if packed is None:
+        packed = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=w.device)
+    elif (packed.dtype != torch.uint8 or tuple(packed.shape) != (N, (K + 1) // 2)
+          or not packed.is_contiguous() or packed.device != w.device):
+        raise ValueError("packed must be contiguous uint8 [N, ceil(K/2)] on w's device")
+    if scales is None:
+        scales = torch.empty((N, max(G, 0)), dtype=torch.float16, device=w.device)
+    elif (scales.dtype != torch.float16 or tuple(scales.shape) != (N, max(G, 0))
+          or not scales.is_contiguous() or scales.device != w.device):
+        raise ValueError("scales must be contiguous float16 [N, ceil(K/group)] on w's device")
     with torch.cuda.device(w.device):
         _check(lib().int4_quantize(w.data_ptr(), _DTYPE_CODE[w.dtype], N, K, int(group),
                                    packed.data_ptr(), scales.data_ptr(), _stream(w)))

@@ -413,6 +413,28 @@ def test_matmul_decode_split_tiles(M, N, K, group, dtype):
     assert_matmul_close(a, x, packed, scales, K, group, _tol(dtype))
 
 
+@pytest.mark.parametrize("M", [1, 5])   # x converted in the matmul; x digits from their own kernel
+def test_decode_sees_weights_rewritten_just_before(M):
+    """The decode kernels launch as programmatic dependents of the preceding
+    kernel and ask L2 to prefetch their first weight tiles before waiting for
+    it: a quantize that rewrites the same buffers right before each call,
+    with no synchronization, must still be what the matmul reads."""
+    N, K, group = 20000, 4096, 128
+    ws = [make_weights(N, K, seed=s, device=DEV, dtype=torch.bfloat16) for s in (21, 22)]
+    packed, scales, _ = q4.quantize_int4(ws[0], group)
+    x = make_activations(M, K, seed=9, device=DEV, dtype=torch.bfloat16)
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(M).integers(0, N, 400)]))
+    ys = []
+    for i in range(4):
+        q4.quantize_int4(ws[(i + 1) % 2], group, packed=packed, scales=scales)
+        ys.append((q4.int4_matmul(x, packed, scales, K, group), (i + 1) % 2))
+    torch.cuda.synchronize()
+    for y, j in ys[-2:]:
+        p_j, s_j, _ = q4.quantize_int4(ws[j], group)
+        assert_matmul_close(y, x, p_j, s_j, K, group, TOL_HALF, cols=cols)
+    assert not torch.equal(ys[-1][0], ys[-2][0])
+
+
 def _wide_range_x(M, K, dtype, seed, outlier=2.0 ** 12, tiny=2.0 ** -14):
     """N(0, 1) activations with outlier columns (x outlier) and tiny ones (x tiny)."""
     g = torch.Generator().manual_seed(seed)
