@@ -444,28 +444,65 @@ def _wide_range_x(M, K, dtype, seed, outlier=2.0 ** 12, tiny=2.0 ** -14):
     return x.to(dtype).to(DEV)
 
 
+# Decode kernels by matrix height: N = 512 fits one wave of 16-row tiles and
+# takes the small-matrix kernel (bf16 expansion); N = 8192 takes the integer
+# tensor-core kernel (x as digits: converted in the CTA at M <= 2, by the
+# digits kernel above).
+DECODE_KERNEL_N = [512, 8192]
+
+
+def _cols(N, seed):
+    if N <= 2048:
+        return None
+    return np.unique(np.concatenate([[0, N - 1], np.random.default_rng(seed).integers(0, N, 600)]))
+
+
+@pytest.mark.parametrize("N", DECODE_KERNEL_N)
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16])
-def test_matmul_decode_x_dynamic_range(dtype, M):
-    """The decode kernel represents each 128-k block of a batch row as
+def test_matmul_decode_x_dynamic_range(N, dtype, M):
+    """The integer decode kernel represents each 128-k block of a batch row as
     integers relative to the block's largest |x|: blocks holding outlier
     features 2^12 above the typical value, and values 2^14 below it, must
-    still meet the bound."""
-    N, K, group = 512, 2048, 128
+    still meet the bound (on both decode kernels)."""
+    K, group = 2048, 128
     packed, scales, _ = _quantized(N, K, group, seed=7, dist="student_t3", zero_group_frac=0.05)
     x = _wide_range_x(M, K, dtype, seed=M)
     y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
-    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF, cols=_cols(N, M))
 
 
+@pytest.mark.parametrize("N", DECODE_KERNEL_N)
+@pytest.mark.parametrize("M", [1, 4])
 @pytest.mark.parametrize("scale", [2.0 ** -90, 2.0 ** -60, 2.0 ** 60, 2.0 ** 100])
-def test_matmul_decode_extreme_magnitudes_bf16(scale):
+def test_matmul_decode_extreme_magnitudes_bf16(N, M, scale):
     """bf16 activations far from 1 in both directions (whole rows scaled)."""
-    N, K, group = 256, 1024, 256
+    K, group = 1024, 256
     packed, scales, _ = _quantized(N, K, group, seed=11)
-    x = (make_activations(4, K, seed=5, device=DEV, dtype=torch.float32) * scale).to(torch.bfloat16)
+    x = (make_activations(M, K, seed=5, device=DEV, dtype=torch.float32) * scale).to(torch.bfloat16)
     y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_DECODE)
-    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF, cols=_cols(N, M))
+
+
+@pytest.mark.parametrize("M, N, K, group", [
+    (1, 20000, 8224, 128),   # last 128-k block holds 32 k; 65 blocks (odd): a stage past the end
+    (2, 9000, 8352, 256),    # groups of two blocks, the last one partial
+    (3, 8000, 4128, 128),    # digits kernel, ragged last block
+    (16, 8000, 1056, 384),   # groups of three blocks, 9 blocks in all
+    (1, 7200, 384, 128),     # three blocks: a run of one and a half stages
+])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_matmul_decode_integer_kernel_ragged_k(M, N, K, group, dtype):
+    """The integer decode kernel on K that is not a multiple of 128 or of the
+    256-k stage, and on groups spanning several 128-k blocks."""
+    assert q4.matmul_select(dtype, K, group, M, N) == q4.PATH_DECODE
+    packed, scales, _ = _quantized(N, K, group, seed=K + M, dist="student_t3", zero_group_frac=0.02)
+    x = make_activations(M, K, seed=K, device=DEV, dtype=dtype)
+    y = q4.int4_matmul(x, packed, scales, K, group)
+    a = q4.int4_matmul(x, packed, scales, K, group)
+    torch.cuda.synchronize()
+    assert torch.equal(y, a)
+    assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF, cols=_cols(N, K))
 
 
 @pytest.mark.parametrize("N", [300, 20000])   # the small-matrix and the streaming kernel
