@@ -560,14 +560,19 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert_matmul_close(y, x, packed, scales, 256, 64, TOL_HALF)
 
 
-def test_decode_split_scratch_on_concurrent_streams():
+@pytest.mark.parametrize("N, Ma, Mb", [
+    (1000, 3, 5),   # the small-matrix kernel
+    (9000, 3, 5),   # the integer kernel, x digits in per-stream records
+    (9000, 1, 2),   # the integer kernel, x converted in the CTA
+])
+def test_decode_split_scratch_on_concurrent_streams(N, Ma, Mb):
     """Split-tile decode on two streams at once: each stream has its own
-    partial slots and arrival counters, so both results match the oracle
-    bound and equal a serial run bit for bit."""
-    N, K, group = 1000, 12288, 128
+    partial slots, arrival counters and x digit records, so both results
+    match the oracle bound and equal a serial run bit for bit."""
+    K, group = 12288, 128
     packed, scales, _ = _quantized(N, K, group, seed=77, dist="student_t3", zero_group_frac=0.02)
-    xa = make_activations(3, K, seed=1, device=DEV, dtype=torch.bfloat16)
-    xb = make_activations(5, K, seed=2, device=DEV, dtype=torch.bfloat16)
+    xa = make_activations(Ma, K, seed=1, device=DEV, dtype=torch.bfloat16)
+    xb = make_activations(Mb, K, seed=2, device=DEV, dtype=torch.bfloat16)
     ref_a = q4.int4_matmul(xa, packed, scales, K, group, path=q4.PATH_DECODE)
     ref_b = q4.int4_matmul(xb, packed, scales, K, group, path=q4.PATH_DECODE)
     torch.cuda.synchronize()
@@ -584,15 +589,18 @@ def test_decode_split_scratch_on_concurrent_streams():
         assert torch.equal(o, ref_a)
     for o in outs_b:
         assert torch.equal(o, ref_b)
-    assert_matmul_close(ref_a, xa, packed, scales, K, group, TOL_HALF)
+    assert_matmul_close(ref_a, xa, packed, scales, K, group, TOL_HALF, cols=_cols(N, 5))
+    assert_matmul_close(ref_b, xb, packed, scales, K, group, TOL_HALF, cols=_cols(N, 6))
 
 
-def test_decode_split_scratch_grows_between_shapes():
+@pytest.mark.parametrize("M", [1, 5])
+def test_decode_split_scratch_grows_between_shapes(M):
     """A small split first, then a larger one on the same stream: the stream's
-    scratch grows and the counters stay consistent for both."""
-    for N, K in [(128, 4096), (28672, 8192), (300, 8192)]:
+    scratch (and, at M = 5, its x digit records) grows and the counters stay
+    consistent for both."""
+    for N, K in [(128, 4096), (9000, 2048), (28672, 8192), (300, 8192), (9000, 4096)]:
         packed, scales, _ = _quantized(N, K, 128, seed=N, dist="normal")
-        x = make_activations(1, K, seed=3, device=DEV, dtype=torch.bfloat16)
+        x = make_activations(M, K, seed=3, device=DEV, dtype=torch.bfloat16)
         y1 = q4.int4_matmul(x, packed, scales, K, 128, path=q4.PATH_DECODE)
         y2 = q4.int4_matmul(x, packed, scales, K, 128, path=q4.PATH_DECODE)
         torch.cuda.synchronize()
