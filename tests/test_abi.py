@@ -93,6 +93,23 @@ def test_matmul_rejects_bad_arguments(L):
     assert rc == q4.ERR_ARG
 
 
+def test_noalloc_rejects_what_the_decode_kernels_cannot_run(L):
+    """The allocation-free entry validates and refuses on the host, before any
+    CUDA call: shapes outside the decode kernels, and bad arguments."""
+    fake = ctypes.c_void_p(256)
+    f = L.int4_matmul_decode_noalloc
+    assert f(fake, 1, fake, fake, 4096, 128, 17, 64, fake, None) == q4.ERR_UNSUPPORTED  # M > 16
+    assert b"decode" in L.int4_last_error()
+    assert f(fake, 0, fake, fake, 4096, 128, 2, 64, fake, None) == q4.ERR_UNSUPPORTED   # fp32 x
+    assert f(fake, 1, fake, fake, 4112, 128, 2, 64, fake, None) == q4.ERR_UNSUPPORTED   # K % 32
+    assert f(fake, 1, fake, fake, 4096, 96, 2, 64, fake, None) == q4.ERR_UNSUPPORTED    # group 96
+    assert f(ctypes.c_void_p(264), 1, fake, fake, 4096, 128, 2, 64, fake, None) == q4.ERR_UNSUPPORTED
+    assert f(None, 1, fake, fake, 4096, 128, 2, 64, fake, None) == q4.ERR_ARG
+    assert f(fake, 1, fake, fake, 4096, 128, 2, 64, None, None) == q4.ERR_ARG
+    assert f(fake, 9, fake, fake, 4096, 128, 2, 64, fake, None) == q4.ERR_DTYPE
+    assert f(fake, 1, fake, fake, 4096, 128, 0, 64, fake, None) == q4.OK                # no work
+
+
 def test_error_message_is_set(L):
     fake = ctypes.c_void_p(256)
     assert L.int4_unpack(fake, 0, 4, fake, None) == q4.ERR_ARG
