@@ -262,6 +262,81 @@ def run_reference(args):
     return 0
 
 
+# Decode at the Llama-7B-shaped linears (group 128, bf16 x, M = 1, 4, 16): per
+# shape and batch, calls back to back over rotating copies of the packed
+# weights whose total exceeds 3x L2, so every call streams its weights from
+# HBM.  The loop is timed twice: replayed from a CUDA graph (the kernels' own
+# rate; launch gaps only) and launched call by call from the host.
+DECODE_SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]
+DECODE_MS = (1, 4, 16)
+
+
+def decode_shape_rows(dev, peaks, reps: int = 10):
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+    from workloads import make_activations, make_weights
+
+    L = q4.lib()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    rows = {}
+    for N, K in DECODE_SHAPES:
+        w = make_weights(N, K, seed=3, device=dev, dtype=torch.float32)
+        packed, scales, _ = q4.quantize_int4(w, GROUP)
+        del w
+        per_copy = packed.numel() + 2 * scales.numel()
+        ncopy = max(2, -(-3 * l2 // per_copy))
+        copies = [(packed.clone(), scales.clone()) for _ in range(ncopy)]
+        for M in DECODE_MS:
+            x = make_activations(M, K, seed=M, device=dev, dtype=torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            nb = q4.matmul_workspace_size(torch.bfloat16, K, GROUP, M, N, dev)
+            ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=dev)
+
+            def run():
+                sp = torch.cuda.current_stream(dev).cuda_stream
+                for pk, sc in copies:
+                    rc = L.int4_matmul_ws(x.data_ptr(), 1, pk.data_ptr(), sc.data_ptr(), K, GROUP,
+                                          M, N, y.data_ptr(), ws.data_ptr(), ws.numel(), sp)
+                    if rc != 0:
+                        raise RuntimeError(f"INT4 library error {rc}: {L.int4_last_error()}")
+
+            def timed(fn):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                fn()
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(reps):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                return e0.elapsed_time(e1) * 1e3 / (reps * ncopy)
+
+            for _ in range(3):
+                run()
+            torch.cuda.synchronize()
+            host_us = timed(run)
+            graph_us = None
+            try:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    run()
+                graph_us = timed(g.replay)
+                del g
+            except RuntimeError:
+                graph_us = None
+            us = graph_us if graph_us is not None else host_us
+            gbs = N * (K // 2) / (us * 1e-6) / 1e9
+            rows[f"{N}x{K}_m{M}"] = {
+                "us_per_call": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                "timing": "cuda graph replay" if graph_us is not None else "host launched",
+                "us_per_call_host_launched": host_us,
+                "path": q4.matmul_select(torch.bfloat16, K, GROUP, M, N), "copies": ncopy}
+        del copies
+    return rows
+
+
 def run_ours(args):
     import torch
 
@@ -297,6 +372,9 @@ def run_ours(args):
         yp = torch.empty((M_PREFILL, N_W), dtype=torch.float32, device=dev)
     if "unpack" in order:
         unpacked = torch.empty((N_W, K_W), dtype=torch.int8, device=dev)
+    # The decode matmul's workspace (zero-filled once; every call leaves it so).
+    ws_bytes = q4.matmul_workspace_size(torch.bfloat16, K_W, GROUP, M_DECODE, N_W, dev)
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
@@ -317,12 +395,13 @@ def run_ours(args):
         "quantize": lambda: call(L.int4_quantize(w.data_ptr(), 1, N_W, K_W, GROUP, packed.data_ptr(),
                                                  scales.data_ptr(), sp())),
         "unpack": lambda: call(L.int4_unpack(packed.data_ptr(), K_W, N_W, unpacked.data_ptr(), sp())),
-        "decode": lambda: [call(L.int4_matmul(xd.data_ptr(), 1, pk.data_ptr(), sc.data_ptr(), K_W,
-                                               GROUP, M_DECODE, N_W, yd.data_ptr(), sp()))
+        "decode": lambda: [call(L.int4_matmul_ws(xd.data_ptr(), 1, pk.data_ptr(), sc.data_ptr(), K_W,
+                                                  GROUP, M_DECODE, N_W, yd.data_ptr(), ws.data_ptr(),
+                                                  ws.numel(), sp()))
                            for pk, sc in [(packed, scales)] + dcopies],
-        "decode_single": lambda: call(L.int4_matmul(xd.data_ptr(), 1, packed.data_ptr(),
-                                                    scales.data_ptr(), K_W, GROUP, M_DECODE, N_W,
-                                                    yd.data_ptr(), sp())),
+        "decode_single": lambda: call(L.int4_matmul_ws(xd.data_ptr(), 1, packed.data_ptr(),
+                                                       scales.data_ptr(), K_W, GROUP, M_DECODE, N_W,
+                                                       yd.data_ptr(), ws.data_ptr(), ws.numel(), sp())),
         "prefill": lambda: call(L.int4_matmul(xp.data_ptr(), 1, packed.data_ptr(), scales.data_ptr(),
                                               K_W, GROUP, M_PREFILL, N_W, yp.data_ptr(), sp())),
     }
@@ -413,6 +492,10 @@ def run_ours(args):
     roof["peak_source"] = peaks["source"] + (" bf16 burst" if roof["bound"] == "tensor" else " copy")
     roof["traffic"] = _traffic(dom)
 
+    shape_rows = None
+    if not args.no_shapes and not args.only:
+        shape_rows = decode_shape_rows(dev, peaks)
+
     # End to end through the public Python API: pinned host x in, y out.
     e2e = None
     if not args.no_e2e and not args.only:
@@ -460,7 +543,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "flushed before every row (256 MiB write, then 256 MiB read of another buffer); the decode row's back-to-back calls read distinct weight copies (940 MB > L2)",
                    "parallelism": f"replicas x{world}"},
-        "rows": rows, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "rows": rows, "decode_llama7b": shape_rows, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * sum(launches_per_step[n] for n in order),
         "wall_ms_timed_region": wall_ms,
     }
@@ -479,6 +562,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="skip the decode rows at the Llama-7B-shaped linears")
     ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,
                     help="run one kernel of the step only (for profiling); no e2e or CPU baseline")
     args = ap.parse_args()

@@ -25,7 +25,8 @@ import threading
 import torch
 
 __all__ = [
-    "quantize_int4", "unpack_int4", "int4_matmul", "matmul_select", "device_status",
+    "quantize_int4", "unpack_int4", "int4_matmul", "int4_matmul_decode_noalloc",
+    "matmul_workspace_size", "matmul_select", "device_status",
     "selftest_wait_timeout", "lib", "library_path", "Int4Error",
     "PATH_AUTO", "PATH_SIMT", "PATH_DECODE", "PATH_PREFILL",
 ]
@@ -68,8 +69,11 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64, u32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
         L.int4_quantize.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp]
         L.int4_unpack.argtypes = [vp, i64, i64, vp, vp]
+        sz = ctypes.c_size_t
         L.int4_matmul.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
-        L.int4_matmul_path.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, i32, vp]
+        L.int4_matmul_ws.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp, sz, vp]
+        L.int4_matmul_path.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, i32, vp, sz, vp]
+        L.int4_matmul_workspace_size.argtypes = [i32, i64, i32, i64, i64, ctypes.POINTER(sz)]
         L.int4_matmul_select.argtypes = [i32, i64, i32, i64, i64]
         L.int4_matmul_decode_noalloc.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
         L.int4_device_status.argtypes = [vp]
@@ -78,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.int4_last_error.argtypes = []
         L.int4_version.argtypes = []
         for name in ("int4_quantize", "int4_unpack", "int4_matmul", "int4_matmul_path",
-                     "int4_matmul_decode_noalloc",
+                     "int4_matmul_ws", "int4_matmul_workspace_size", "int4_matmul_decode_noalloc",
                      "int4_matmul_select", "int4_device_status", "int4_selftest_wait_timeout",
                      "int4_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -143,38 +147,110 @@ def unpack_int4(packed: torch.Tensor, K: int) -> torch.Tensor:
     return out
 
 
-def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: int,
-                group: int = 128, *, path: int = PATH_AUTO, out: torch.Tensor | None = None):
-    """y = x @ dequantize(W).T as float32 [M, N]; x is [M, K] fp32/bf16/fp16."""
-    _need_cuda("x", x)
-    _need_cuda("packed", packed)
-    _need_cuda("scales", scales)
+def _matmul_operands(x, packed, scales, K: int, group: int, out=None):
+    """Checks the matmul's operands (shapes and dtypes first, then that every
+    tensor is a contiguous CUDA tensor on x's device) and returns (M, N)."""
+    for name, t in (("x", x), ("packed", packed), ("scales", scales)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
     if x.dim() != 2 or x.shape[1] != K:
         raise ValueError("x must be [M, K]")
     if x.dtype not in _DTYPE_CODE:
         raise TypeError("x must be float32, bfloat16 or float16")
-    N = packed.shape[0]
-    G = -(-K // group)
+    if group < 1:
+        raise ValueError("group must be >= 1")
+    if packed.dim() != 2:
+        raise ValueError("packed must be uint8 [N, ceil(K/2)]")
+    M, N = x.shape[0], packed.shape[0]
     if packed.dtype != torch.uint8 or tuple(packed.shape) != (N, (K + 1) // 2):
         raise ValueError("packed must be uint8 [N, ceil(K/2)]")
-    if scales.dtype != torch.float16 or tuple(scales.shape) != (N, G):
+    if scales.dtype != torch.float16 or tuple(scales.shape) != (N, -(-K // group)):
         raise ValueError("scales must be float16 [N, ceil(K/group)]")
-    M = x.shape[0]
+    if out is not None and (not isinstance(out, torch.Tensor) or out.dtype != torch.float32
+                            or tuple(out.shape) != (M, N)):
+        raise ValueError("out must be float32 [M, N]")
+    for name, t in (("x", x), ("packed", packed), ("scales", scales), ("out", out)):
+        if t is None:
+            continue
+        _need_cuda(name, t)
+        if t.device != x.device:
+            raise ValueError(f"{name} must be on x's device")
+    return M, N
+
+
+def matmul_workspace_size(x_dtype: torch.dtype, K: int, group: int, M: int, N: int,
+                          device=None) -> int:
+    """Bytes of workspace the matmul needs for this problem on `device` (0: none)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(),
+           x_dtype, int(K), int(group), int(M), int(N))
+    n = _ws_size_cache.get(key)
+    if n is None:
+        out = ctypes.c_size_t(0)
+        with torch.cuda.device(key[0]):
+            _check(lib().int4_matmul_workspace_size(_DTYPE_CODE[x_dtype], K, int(group), M, N,
+                                                    ctypes.byref(out)))
+        n = _ws_size_cache[key] = int(out.value)
+    return n
+
+
+# Workspaces the binding keeps for the matmul, one per (device, stream):
+# allocated zero-filled with torch on the stream that uses them (the kernels
+# leave them zeroed after every call), grown when a call needs more.
+_ws_size_cache: dict = {}
+_ws_cache: dict = {}
+
+
+def _workspace_for(x: torch.Tensor, nbytes: int) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    stream = torch.cuda.current_stream(x.device)
+    key = (x.device.index, stream.cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        # torch.zeros runs on the current stream, before the call that uses it.
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=x.device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: int,
+                group: int = 128, *, path: int = PATH_AUTO, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | bool | None = None):
+    """y = x @ dequantize(W).T as float32 [M, N]; x is [M, K] fp32/bf16/fp16.
+
+    `workspace`: None uses a zero-filled workspace the binding keeps per device
+    and stream; a uint8 CUDA tensor (zero-filled before its first use, at
+    least matmul_workspace_size bytes) is used as given; False runs the
+    schedule that needs no workspace (the C entry int4_matmul)."""
+    M, N = _matmul_operands(x, packed, scales, K, group, out)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    else:
-        _need_cuda("out", out)
-        if out.dtype != torch.float32 or tuple(out.shape) != (M, N):
-            raise ValueError("out must be float32 [M, N]")
     L = _lib if _lib is not None else lib()
-    args = (x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(), scales.data_ptr(), K,
-            int(group), M, N, out.data_ptr(), int(path))
-    if x.device.index == torch.cuda.current_device():
-        _check(L.int4_matmul_path(*args, _stream(x)))
-    else:
-        with torch.cuda.device(x.device):
-            _check(L.int4_matmul_path(*args, _stream(x)))
+    same_dev = x.device.index == torch.cuda.current_device()
+    with (_nullctx() if same_dev else torch.cuda.device(x.device)):
+        if workspace is False:
+            ws_ptr, ws_bytes = None, 0
+        elif workspace is None:
+            ws = _workspace_for(x, matmul_workspace_size(x.dtype, K, group, M, N, x.device))
+            ws_ptr, ws_bytes = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
+        else:
+            _need_cuda("workspace", workspace)
+            if workspace.dtype != torch.uint8 or workspace.device != x.device:
+                raise ValueError("workspace must be a uint8 tensor on x's device")
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        _check(L.int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
+                                  scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
+                                  int(path), ws_ptr, ws_bytes, _stream(x)))
     return out
+
+
+class _nullctx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
 
 
 def int4_matmul_decode_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
@@ -182,15 +258,9 @@ def int4_matmul_decode_noalloc(x: torch.Tensor, packed: torch.Tensor, scales: to
     """The decode matmul into a caller-provided `out` [M, N] float32, with no
     device allocation in the call (the library's fixed scratch holds the
     partial tiles).  Calls that may overlap in time race on that scratch."""
-    _need_cuda("x", x)
-    _need_cuda("packed", packed)
-    _need_cuda("scales", scales)
-    _need_cuda("out", out)
-    M, N = x.shape[0], packed.shape[0]
-    if x.dim() != 2 or x.shape[1] != K or x.dtype not in _DTYPE_CODE:
-        raise ValueError("x must be [M, K] float32, bfloat16 or float16")
-    if out.dtype != torch.float32 or tuple(out.shape) != (M, N):
+    if out is None:
         raise ValueError("out must be float32 [M, N]")
+    M, N = _matmul_operands(x, packed, scales, K, group, out)
     with torch.cuda.device(x.device):
         _check(lib().int4_matmul_decode_noalloc(x.data_ptr(), _DTYPE_CODE[x.dtype],
                                                 packed.data_ptr(), scales.data_ptr(), K,
@@ -215,6 +285,12 @@ def device_status(device=None) -> int:
         rc = lib().int4_device_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
     if rc not in (OK, ERR_TIMEOUT):
         _check(rc)
+    if rc == ERR_TIMEOUT:
+        # A CTA that gave up may have left an arrival counted in a workspace:
+        # start over with zero-filled ones on this device.
+        idx = dev.index if dev.index is not None else torch.cuda.current_device()
+        for key in [k for k in _ws_cache if k[0] == idx]:
+            del _ws_cache[key]
     return rc
 
 

@@ -174,9 +174,13 @@ static int matmul_choose(DType t, int64_t K, int32_t group, int64_t M, int64_t N
 
 int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                      int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
-                     void* stream) {
+                     void* workspace, size_t workspace_bytes, void* stream) {
   const int rc = matmul_check(x, x_dtype, packed, scales, K, group, M, N, y);
   if (rc != INT4_OK || M == 0 || N == 0) return rc;
+  if (workspace == nullptr && workspace_bytes != 0)
+    return int4lib::fail(INT4_ERR_ARG, "int4_matmul: null workspace with a non-zero size");
+  if (!int4lib::aligned(workspace, 256))
+    return int4lib::fail(INT4_ERR_ALIGN, "int4_matmul: workspace not 256-byte aligned");
   const DType t = static_cast<DType>(x_dtype);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (path == INT4_PATH_AUTO) path = matmul_choose(t, K, group, M, N, x, packed);
@@ -185,11 +189,22 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
     case INT4_PATH_SIMT:
       e = int4lib::launch_matmul_simt(x, t, packed, scales, K, group, M, N, y, s);
       break;
-    case INT4_PATH_DECODE:
+    case INT4_PATH_DECODE: {
       if (!int4lib::decode_supported(t, K, group, M, N, x, packed))
         return int4lib::fail(INT4_ERR_UNSUPPORTED, "int4_matmul: decode kernel cannot run this shape");
-      e = int4lib::launch_matmul_decode(x, t, packed, scales, K, group, M, N, y, s);
+      size_t need = 0;
+      e = int4lib::launch_matmul_decode(x, t, packed, scales, K, group, M, N, y, workspace,
+                                        workspace_bytes, s, &need);
+      if (e == cudaErrorInvalidValue && need > 0) {
+        char msg[200];
+        std::snprintf(msg, sizeof msg,
+                      "int4_matmul: this call needs a workspace of %zu bytes, %zu given "
+                      "(int4_matmul_workspace_size)",
+                      need, workspace_bytes);
+        return int4lib::fail(INT4_ERR_ARG, msg);
+      }
       break;
+    }
     case INT4_PATH_PREFILL:
       if (!int4lib::prefill_supported(t, K, group, M, N, x, packed))
         return int4lib::fail(INT4_ERR_UNSUPPORTED, "int4_matmul: tensor-core kernel cannot run this shape");
@@ -203,7 +218,33 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
 
 int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                 int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* stream) {
-  return int4_matmul_path(x, x_dtype, packed, scales, K, group, M, N, y, INT4_PATH_AUTO, stream);
+  return int4_matmul_path(x, x_dtype, packed, scales, K, group, M, N, y, INT4_PATH_AUTO, nullptr, 0,
+                          stream);
+}
+
+int int4_matmul_ws(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                   int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  return int4_matmul_path(x, x_dtype, packed, scales, K, group, M, N, y, INT4_PATH_AUTO, workspace,
+                          workspace_bytes, stream);
+}
+
+int int4_matmul_workspace_size(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N,
+                               size_t* bytes) {
+  if (bytes == nullptr) return int4lib::fail(INT4_ERR_ARG, "int4_matmul_workspace_size: null output");
+  *bytes = 0;
+  if (!int4lib::dtype_ok(x_dtype))
+    return int4lib::fail(INT4_ERR_DTYPE, "int4_matmul_workspace_size: unknown x_dtype");
+  if (M < 0 || N < 0 || K < 1 || group < 1)
+    return int4lib::fail(INT4_ERR_ARG, "int4_matmul_workspace_size: need M, N >= 0, K >= 1, group >= 1");
+  if (!int4lib::mul_ok(M, K) || !int4lib::mul_ok(N, K) || !int4lib::mul_ok(M, N))
+    return int4lib::fail(INT4_ERR_ARG, "int4_matmul_workspace_size: sizes too large");
+  if (M == 0 || N == 0) return INT4_OK;
+  const DType t = static_cast<DType>(x_dtype);
+  static const uint8_t* const kAligned = reinterpret_cast<const uint8_t*>(static_cast<uintptr_t>(256));
+  if (matmul_choose(t, K, group, M, N, kAligned, kAligned) != INT4_PATH_DECODE) return INT4_OK;
+  const cudaError_t e = int4lib::decode_workspace_size(t, K, group, M, N, bytes);
+  return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_matmul_workspace_size");
 }
 
 int int4_matmul_decode_noalloc(const void* x, int32_t x_dtype, const uint8_t* packed,

@@ -32,17 +32,27 @@ cudaError_t launch_matmul_simt(const void* x, DType xt, const uint8_t* packed,
 // matmul_decode.cu
 bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                       const uint8_t* packed);
+// Bytes of caller workspace the decode path needs for this problem on the
+// current device (0: none); the schedule int4_matmul_ws runs with it.
+cudaError_t decode_workspace_size(DType xt, int64_t K, int group, int64_t M, int64_t N,
+                                  size_t* bytes);
+// The decode matmul.  workspace == nullptr with workspace_bytes == 0: the
+// schedule that needs no scratch.  Otherwise the workspace (zero-filled
+// before its first use, 256-byte aligned) must hold decode_workspace_size
+// bytes, else cudaErrorInvalidValue with *need set.
 cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
                                  const uint16_t* scales, int64_t K, int group, int64_t M,
-                                 int64_t N, float* y, cudaStream_t stream);
-// The same decode matmul with its partial tiles in a fixed static scratch
-// (no allocation).  cudaErrorInvalidValue with *need set: scratch too small.
+                                 int64_t N, float* y, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream, size_t* need);
+// The same decode matmul with its scratch in the library's fixed device
+// array (no allocation).  cudaErrorInvalidValue with *need set: the array is
+// too small for this call.
 cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t* packed,
                                          const uint16_t* scales, int64_t K, int group, int64_t M,
                                          int64_t N, float* y, cudaStream_t stream, size_t* need);
 size_t decode_noalloc_scratch_bytes();
-// Zeroes the arrival counters of every split-tile scratch on the current
-// device (after a device-side wait gave up); synchronizes the device.
+// Zeroes the arrival counters of the fixed array on the current device
+// (after a device-side wait gave up); synchronizes the device.
 cudaError_t reset_split_counters();
 // matmul_prefill.cu
 bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,

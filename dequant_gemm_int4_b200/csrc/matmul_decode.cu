@@ -258,8 +258,8 @@ template <typename TX, int NT, int GPB>
 __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
-    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* __restrict__ counters,
-    uint32_t* status) {
+    int64_t N, int KB, int64_t U, int P, int64_t gran, float* __restrict__ partials,
+    uint32_t* __restrict__ counters, uint32_t* status) {
   using L = DLayout<NT>;
   constexpr int kTiles = Tiles<NT>::kTiles;
   constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
@@ -277,13 +277,16 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // Stream-K split: the units are (row tile, 128-k block) pairs in row-major
-  // order, and CTA p takes units [p U / P, (p + 1) U / P).  The run crosses
-  // at most two tile boundaries; a tile it covers whole goes straight to y,
-  // a partial tile to its partial slot (2p for the run's first segment when
-  // that starts inside a tile, else 2p + 1), summed by the tile's last
-  // contributor to finish.
-  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * U / P;
-  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * U / P;
+  // order, and CTA p takes units [p U / P, (p + 1) U / P).  Only the first
+  // and the last segment of a run can be a partial tile; a tile the run
+  // covers whole goes straight to y, a partial tile to its partial slot (2p
+  // for the run's first segment when that starts inside a tile, else 2p + 1),
+  // summed by the tile's last contributor to finish.
+  // Runs start and end on multiples of `gran` units: 1 (any block, the
+  // split) or KB (whole tiles, no partial tile: the schedule without scratch).
+  const int64_t runs = U / gran;
+  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * runs / P * gran;
+  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * runs / P * gran;
   const uint32_t xbytes = static_cast<uint32_t>(M) * kSK * 128 * 2;  // all sub-tiles
   const WaitCtx wc{abort_flag, status};
 
@@ -586,26 +589,37 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
 // with e the binary exponent of the block's largest |x| (2^e <= max < 2^(e+1)),
 //   v = rint(x 2^(29-e)),  |v| < 2^30,  v = d0 + 2^8 d1 + 2^16 d2 + 2^24 d3,
 // with signed digits d_i (d0..d2 in [-128, 127], d3 in [-64, 64]).  v is x
-// exactly for every bf16 x within 2^22 of the block's largest magnitude (fp16:
-// 2^19); below that the rounding error is at most 2^-30 of the largest.  The
-// MMA sums S_i = sum_k (16 q) d_i over the block exactly in int32 (|S_i| <=
-// 2^21), and the block's x.q is
+// exactly whenever x 2^(29-e) is an integer: for every bf16 x within 2^22 of
+// the block's largest magnitude (fp16: 2^19), zeros, and smaller values whose
+// low significand bits are zero.  The MMA sums S_i = sum_k (16 q) d_i over the
+// block exactly in int32 (|S_i| <= 2^21), and the block's x.q is
 //   sum_k x q = 2^(e-33) (P01 + 2^16 P23),  P01 = S0 + 2^8 S1,  P23 = S2 + 2^8 S3,
 // both P below 2^30, so the block needs two int-to-float conversions per
 // output; the group's scale multiplies the block sum before the fp32 running
 // sum, as on the page.  The four digits of row m sit in four MMA columns, so
 // one n = 8 MMA serves two batch rows: lane c of a quad holds columns 2c and
 // 2c + 1, i.e. P01 (c even) or P23 (c odd) of row 2nt + c / 2, and the two
-// halves are added when the tile is written.
+// halves are added when the tile is written (the odd lanes' 2^16 rides on the
+// scale they multiply by, which is exact).
+//
+// A block row that some value does not fit exactly (a block spanning more
+// than that range, values below 2^-93 times a power of two, NaN or infinity)
+// is flagged in its record, and the consumers compute that block on the
+// 16-bit MMA with x as stored instead (the bf16/fp16 products are exact, as in
+// decode_kernel).  So the integer form never rounds x, and the result meets
+// the accuracy of the floating-point path on every input.
 //
 // Digit record of one 128-k block: NP n-tiles of 1 KB (8 columns x 128 k, one
-// byte each, in MMA fragment order), then 32 fp32 factors 2^(e-33) and
-// 2^(e-17) for the 16 rows.  Column col of an n-tile holds digit col % 4 of row
-// 2nt + col / 4; inside a column, the 16-byte chunk ((2c + j / 2) ^ (col & 1))
-// holds, at byte 8 (j % 2), the B fragment of lane c for the MMA over words
-// 4c + j of the block's 16 words: 4 digits of the word's even k, then 4 of its
-// odd k.  The XOR spreads the 16-byte loads of a quarter warp over all banks.
+// byte each, in MMA fragment order), then 16 fp32 factors 2^(e-33) (one per
+// batch row), then 16 flag bytes (non-zero: the row's block takes the 16-bit
+// path), then padding to 128 bytes.  Column col of an n-tile holds digit
+// col % 4 of row 2nt + col / 4; inside a column, the 16-byte chunk
+// ((2c + j / 2) ^ (col & 1)) holds, at byte 8 (j % 2), the B fragment of lane c
+// for the MMA over words 4c + j of the block's 16 words: 4 digits of the
+// word's even k, then 4 of its odd k.  The XOR spreads the 16-byte loads of a
+// quarter warp over all banks.
 constexpr int kDigitTile = 1024;
+constexpr int kRecFlags = 64;  // flag bytes of a record, after its factors
 
 __device__ __forceinline__ void transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d,
                                              uint32_t (&o)[4]) {
@@ -655,21 +669,34 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const float (&v)[8]) {
   return mb;
 }
 
+// Whether x 2^p is an integer, i.e. whether the lowest set bit of x's
+// significand sits at or above 2^-p (x finite).
+__device__ __forceinline__ bool digits_exact(float xv, int p) {
+  const uint32_t b = __float_as_uint(xv) & 0x7FFFFFFFu;
+  if (b == 0u) return true;
+  const int E = static_cast<int>(b >> 23);
+  const uint32_t sig = E != 0 ? ((b & 0x7FFFFFu) | 0x800000u) : b;
+  const int lsb = (E != 0 ? E : 1) - 150 + (__ffs(static_cast<int>(sig)) - 1);  // x = sig 2^(..)
+  return lsb + p >= 0;
+}
+
 // The digits of one word of a block: ev[i] / od[i] hold digit i of the
 // word's even / odd k (one byte each, k order), f the block's factor
-// 2^(e-33).  A block of zeros gives zero digits and factor; a block holding a
-// NaN or an infinity gives a NaN factor, so the rows it feeds come out NaN.
-// Blocks whose largest |x| is below 2^-93 are scaled as if it were 2^-93,
-// which keeps the factors normal floats (and loses digits of x below about
-// 2^-122).
+// 2^(e-33), and `inexact` whether some value of the word is not an integer
+// multiple of 2^(e-29) (or the block holds a NaN or an infinity): the block
+// row is then flagged for the 16-bit path.  A block of zeros gives zero
+// digits and factor.  Blocks whose largest |x| is below 2^-93 are scaled as if
+// it were 2^-93, which keeps the factors normal floats.
 __device__ __forceinline__ void word_digits(const float (&v)[8], uint32_t amax_bits,
-                                            uint32_t (&ev)[4], uint32_t (&od)[4], float& f) {
+                                            uint32_t (&ev)[4], uint32_t (&od)[4], float& f,
+                                            bool& inexact) {
   uint32_t dd[8];
   f = 0.0f;
+  inexact = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) dd[i] = 0u;
   if (amax_bits >= 0x7F800000u) {
-    f = __uint_as_float(0x7FC00000u);
+    inexact = true;
   } else if (amax_bits != 0u) {
     // The exponent field (subnormals read as -127, below the clamp).
     int e = static_cast<int>(amax_bits >> 23) - 127;
@@ -684,11 +711,19 @@ __device__ __forceinline__ void word_digits(const float (&v)[8], uint32_t amax_b
       // Balanced base-256 digits: the bytes of v + 0x808080 with the low three
       // flipped back by 128.
       dd[i] = (static_cast<uint32_t>(vi) + 0x808080u) ^ 0x808080u;
+      inexact |= !digits_exact(v[i], p);
     }
     f = __uint_as_float(static_cast<uint32_t>(e - 33 + 127) << 23);
   }
   transpose4x4(dd[0], dd[2], dd[4], dd[6], ev);
   transpose4x4(dd[1], dd[3], dd[5], dd[7], od);
+}
+
+// Whether any lane of this lane's half warp (one block) set `pred`.  All 32
+// lanes must call it together.
+__device__ __forceinline__ bool half_warp_any(bool pred) {
+  const uint32_t bal = __ballot_sync(0xffffffffu, pred);
+  return ((bal >> (threadIdx.x & 16u)) & 0xFFFFu) != 0u;
 }
 
 // Byte offset, inside a record, of the fragment pair (digit i of row m, word h).
@@ -704,24 +739,27 @@ __device__ __forceinline__ int digit_offset(int m, int i, int h) {
 // warp).
 template <typename TX, int R, int NP>
 __device__ __forceinline__ void convert_rows(uint32_t xs, uint32_t rb, int h) {
+  static_assert(R <= 4, "the flag bytes of the converted rows share one word");
   float v[R][8];
   uint32_t mb[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) word_as_float<TX>(ptx::lds128(xs + r * 512), v[r]);
 #pragma unroll
   for (int r = 0; r < R; ++r) mb[r] = block_absmax_bits(v[r]);
+  uint32_t flags = 0u;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     uint32_t ev[4], od[4];
     float f;
-    word_digits(v[r], mb[r], ev, od, f);
+    bool inexact;
+    word_digits(v[r], mb[r], ev, od, f, inexact);
+    if (half_warp_any(inexact)) flags |= 1u << (8 * r);
 #pragma unroll
     for (int i = 0; i < 4; ++i) ptx::sts64(rb + digit_offset(r, i, h), ev[i], od[i]);
-    if (h == 0) {
-      ptx::sts32(rb + NP * kDigitTile + 8 * r, __float_as_uint(f));
-      ptx::sts32(rb + NP * kDigitTile + 8 * r + 4, __float_as_uint(f * 65536.0f));
-    }
+    if (h == 0) ptx::sts32(rb + NP * kDigitTile + 4 * r, __float_as_uint(f));
   }
+  // Rows R .. 3 of the word stay zero (rows past M are never written).
+  if (h == 0) ptx::sts32(rb + NP * kDigitTile + kRecFlags, flags);
 }
 
 // One half warp per (batch row m < MP, record b < nrec); lane h takes the
@@ -749,18 +787,19 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const TX* __restrict__ x,
     for (int i = 0; i < 8; ++i) v[i] = 0.0f;
   }
   const uint32_t amax_bits = block_absmax_bits(v);
-  if (!live) return;
   uint32_t ev[4], od[4];
   float f;
-  word_digits(v, amax_bits, ev, od, f);
+  bool inexact;
+  word_digits(v, amax_bits, ev, od, f, inexact);
+  const bool flag = half_warp_any(inexact);  // every lane votes, live or not
+  if (!live) return;
   uint8_t* r = rec + b * (static_cast<int64_t>(NP) * kDigitTile + 128);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     *reinterpret_cast<uint2*>(r + digit_offset(m, i, h)) = make_uint2(ev[i], od[i]);
   if (h == 0) {
-    float* fr = reinterpret_cast<float*>(r + NP * kDigitTile);
-    fr[2 * m] = f;
-    fr[2 * m + 1] = f * 65536.0f;
+    reinterpret_cast<float*>(r + NP * kDigitTile)[m] = f;
+    r[NP * kDigitTile + kRecFlags + m] = flag ? 1u : 0u;
   }
 }
 
@@ -800,6 +839,87 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Whether any of the 2 NP batch rows of a record is flagged (its flag bytes
+// start at `a`, 16-byte aligned; bytes of rows past 2 NP are not read).
+template <int NP>
+__device__ __forceinline__ bool record_flagged(uint32_t a) {
+  if (NP == 1) return (ptx::lds32(a) & 0xFFFFu) != 0u;
+  if (NP == 2) return ptx::lds32(a) != 0u;
+  if (NP == 4) {
+    const uint2 f = ptx::lds64(a);
+    return (f.x | f.y) != 0u;
+  }
+  const uint4 f = ptx::lds128(a);
+  return (f.x | f.y | f.z | f.w) != 0u;
+}
+
+// One 128-k block (kb) of a flagged record, on the 16-bit warp MMA with x as
+// stored, read from global memory (L2 holds it): the nibbles are expanded to
+// bf16/fp16 and paired with x as in decode_kernel, so every product is exact
+// and the block sums in fp32.  The MMA's columns are batch rows here (8 per
+// n-tile), so each lane then fetches, for n-tile nt of the integer layout,
+// the sums of its batch row 2nt + c / 2 from lane (g, nt % 4) of the quad
+// row, and the even lanes add them (times the scale) to their totals.  wr
+// holds words 4c .. 4c + 3 of rows g and g + 8 of each tile.  All 32 lanes
+// call it together.
+template <typename TX, int NP, int kTiles>
+__device__ __forceinline__ void block_fallback(const TX* __restrict__ x, int64_t K, int M, int kb,
+                                               int g, int c, const uint4 (&wr)[kTiles][2],
+                                               const float (&sa)[kTiles], const float (&sb)[kTiles],
+                                               float (&tot)[kTiles][NP][2]) {
+  constexpr int NTB = (2 * NP + 7) / 8;  // 16-bit MMA n-tiles (8 batch rows each)
+  float acc[kTiles][NTB][4];
+#pragma unroll
+  for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+    for (int nb = 0; nb < NTB; ++nb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[t][nb][i] = 0.0f;
+  const int64_t k0 = static_cast<int64_t>(kb) * 128 + 32 * c;  // this lane's 32 k (K % 32 == 0)
+  const bool kin = k0 < K;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 xf[NTB];
+#pragma unroll
+    for (int nb = 0; nb < NTB; ++nb) {
+      const int m = 8 * nb + g;
+      xf[nb] = (kin && m < M)
+                   ? pair_x(__ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0 + 8 * j)))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+      const uint32_t w0[4] = {wr[t][0].x, wr[t][0].y, wr[t][0].z, wr[t][0].w};
+      const uint32_t w1[4] = {wr[t][1].x, wr[t][1].y, wr[t][1].z, wr[t][1].w};
+      uint32_t pa[4], pb[4];
+      expand<TX>(w0[j], pa);
+      expand<TX>(w1[j], pb);
+#pragma unroll
+      for (int nb = 0; nb < NTB; ++nb) {
+        Cvt<TX>::mma(acc[t][nb], pa[0], pb[0], pa[1], pb[1], xf[nb].x, xf[nb].y);
+        Cvt<TX>::mma(acc[t][nb], pa[2], pb[2], pa[3], pb[3], xf[nb].z, xf[nb].w);
+      }
+    }
+  }
+  const int lane_base = g << 2;
+  const bool odd_row = (c >> 1) != 0;  // batch row 2nt + 1
+#pragma unroll
+  for (int nt = 0; nt < NP; ++nt) {
+    const int src = lane_base | (nt & 3);
+#pragma unroll
+    for (int t = 0; t < kTiles; ++t) {
+      const float r0 = __shfl_sync(0xffffffffu, acc[t][nt >> 2][0], src);
+      const float r1 = __shfl_sync(0xffffffffu, acc[t][nt >> 2][1], src);
+      const float r2 = __shfl_sync(0xffffffffu, acc[t][nt >> 2][2], src);
+      const float r3 = __shfl_sync(0xffffffffu, acc[t][nt >> 2][3], src);
+      if ((c & 1) == 0) {
+        tot[t][nt][0] = fmaf(odd_row ? r1 : r0, sa[t], tot[t][nt][0]);
+        tot[t][nt][1] = fmaf(odd_row ? r3 : r2, sb[t], tot[t][nt][1]);
+      }
+    }
+  }
+}
+
 // Same CTA roles, ring, stream-K split and last-contributor reduction as
 // decode_kernel.  Each stage carries the digit records of its two blocks:
 // converted in the CTA from the stage's x tile (FUSE), or one bulk copy of
@@ -807,10 +927,10 @@ __device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint
 template <typename TX, int NP, bool FUSE>
 __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>::kMinBlocks) decode_i8_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-    const uint8_t* __restrict__ rec,
+    const TX* __restrict__ x, const uint8_t* __restrict__ rec,
     const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
-    int64_t N, int KB, int64_t U, int P, float* __restrict__ partials, uint32_t* __restrict__ counters,
-    uint32_t* status) {
+    int64_t N, int KB, int64_t U, int P, int64_t gran, float* __restrict__ partials,
+    uint32_t* __restrict__ counters, uint32_t* status) {
   using S = I8Shape<NP, FUSE>;
   constexpr int kTiles = S::kTiles;
   constexpr int kRowsPerCta = S::kRowsPerCta;
@@ -831,8 +951,11 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * U / P;
-  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * U / P;
+  // Runs start and end on multiples of `gran` units: 1 (any block, the
+  // split) or KB (whole tiles, no partial tile: the schedule without scratch).
+  const int64_t runs = U / gran;
+  const int64_t u_begin = static_cast<int64_t>(blockIdx.x) * runs / P * gran;
+  const int64_t u_end = static_cast<int64_t>(blockIdx.x + 1) * runs / P * gran;
   const WaitCtx wc{abort_flag, status};
 
   if (threadIdx.x == 0) {
@@ -968,7 +1091,11 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
 #pragma unroll
     for (int jp = 0; jp < 2; ++jp)
       bofs[jp] = xrec + static_cast<uint32_t>(g * 128 + (((2 * c + jp) ^ (g & 1)) << 4));
-    const uint32_t fofs = xrec + static_cast<uint32_t>(NP * kDigitTile + 4 * c);
+    // Factor of batch row 2nt + c / 2 (plus 8 nt bytes); the odd lanes' P23
+    // weighs 2^16 more, which they fold into their scale.
+    const uint32_t fofs = xrec + static_cast<uint32_t>(NP * kDigitTile + 4 * (c >> 1));
+    const uint32_t flagofs = xrec + static_cast<uint32_t>(NP * kDigitTile + kRecFlags);
+    const float lane_mul = (c & 1) ? 65536.0f : 1.0f;
     const int bpg = group / 128;
     int gs = 0;
     for (int64_t u = u_begin; u < u_end;) {
@@ -1029,39 +1156,57 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
         if (!ok) break;
         const uint32_t st = sbase + s * S::kStageBytes;
         if (kb < bhi) {
-          // A fragments of the block's four MMAs (k32 each): rows g and g + 8,
-          // low nibbles (shifted) in k slots 0..15, high nibbles in 16..31.
-          uint32_t a[kTiles][4][4];
+          // The words of rows g and g + 8 of each tile (words 4c .. 4c + 3).
+          uint4 wr[kTiles][2];
 #pragma unroll
           for (int t = 0; t < kTiles; ++t) {
-            const uint4 u0 = ptx::lds128(st + wofs[t][0]);
-            const uint4 u1 = ptx::lds128(st + wofs[t][1]);
-            const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w};
-            const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              a[t][j][0] = (w0[j] << 4) & 0xF0F0F0F0u;
-              a[t][j][1] = (w1[j] << 4) & 0xF0F0F0F0u;
-              a[t][j][2] = w0[j] & 0xF0F0F0F0u;
-              a[t][j][3] = w1[j] & 0xF0F0F0F0u;
-            }
+            wr[t][0] = ptx::lds128(st + wofs[t][0]);
+            wr[t][1] = ptx::lds128(st + wofs[t][1]);
           }
-#pragma unroll
-          for (int nt = 0; nt < NP; ++nt) {
-            const uint4 b01 = ptx::lds128(st + bofs[0] + nt * kDigitTile);
-            const uint4 b23 = ptx::lds128(st + bofs[1] + nt * kDigitTile);
-            const float fct = __uint_as_float(ptx::lds32(st + fofs + nt * 16));
+          if (__builtin_expect(record_flagged<NP>(st + flagofs), 0)) {
+            // Some batch row's x does not fit its digits exactly: the whole
+            // block runs on the 16-bit MMA with x as stored.
+            block_fallback<TX, NP, kTiles>(x, K, M, kb, g, c, wr, sa, sb, tot);
+          } else {
+            // A fragments of the block's four MMAs (k32 each): rows g and
+            // g + 8, low nibbles (shifted) in k slots 0..15, high nibbles in
+            // 16..31.
+            uint32_t a[kTiles][4][4];
 #pragma unroll
             for (int t = 0; t < kTiles; ++t) {
-              int acc[4] = {0, 0, 0, 0};
-              mma_s8(acc, a[t][0], b01.x, b01.y);
-              mma_s8(acc, a[t][1], b01.z, b01.w);
-              mma_s8(acc, a[t][2], b23.x, b23.y);
-              mma_s8(acc, a[t][3], b23.z, b23.w);
-              const float p0 = static_cast<float>(acc[0] + 256 * acc[1]);
-              const float p1 = static_cast<float>(acc[2] + 256 * acc[3]);
-              tot[t][nt][0] = fmaf(p0 * fct, sa[t], tot[t][nt][0]);
-              tot[t][nt][1] = fmaf(p1 * fct, sb[t], tot[t][nt][1]);
+              const uint32_t w0[4] = {wr[t][0].x, wr[t][0].y, wr[t][0].z, wr[t][0].w};
+              const uint32_t w1[4] = {wr[t][1].x, wr[t][1].y, wr[t][1].z, wr[t][1].w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                a[t][j][0] = (w0[j] << 4) & 0xF0F0F0F0u;
+                a[t][j][1] = (w1[j] << 4) & 0xF0F0F0F0u;
+                a[t][j][2] = w0[j] & 0xF0F0F0F0u;
+                a[t][j][3] = w1[j] & 0xF0F0F0F0u;
+              }
+            }
+            float sal[kTiles], sbl[kTiles];
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+              sal[t] = sa[t] * lane_mul;  // exact: a power of two
+              sbl[t] = sb[t] * lane_mul;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NP; ++nt) {
+              const uint4 b01 = ptx::lds128(st + bofs[0] + nt * kDigitTile);
+              const uint4 b23 = ptx::lds128(st + bofs[1] + nt * kDigitTile);
+              const float fct = __uint_as_float(ptx::lds32(st + fofs + nt * 8));
+#pragma unroll
+              for (int t = 0; t < kTiles; ++t) {
+                int acc[4] = {0, 0, 0, 0};
+                mma_s8(acc, a[t][0], b01.x, b01.y);
+                mma_s8(acc, a[t][1], b01.z, b01.w);
+                mma_s8(acc, a[t][2], b23.x, b23.y);
+                mma_s8(acc, a[t][3], b23.z, b23.w);
+                const float p0 = static_cast<float>(acc[0] + 256 * acc[1]);
+                const float p1 = static_cast<float>(acc[2] + 256 * acc[3]);
+                tot[t][nt][0] = fmaf(p0 * fct, sal[t], tot[t][nt][0]);
+                tot[t][nt][1] = fmaf(p1 * fct, sbl[t], tot[t][nt][1]);
+              }
             }
           }
         }
@@ -1151,469 +1296,6 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
   return fn;
-}
-
-// Scratch of split tiles for one (device, stream): 2 partial slots of kPer
-// floats per CTA and one arrival counter per CTA.  The counters are zeroed
-// when the scratch is made and every call leaves them zero, so calls on one
-// stream (ordered) can share it; calls on different streams use different
-// scratch.  It grows (after the stream drains) when a call needs more.
-struct SplitScratch {
-  float* partials = nullptr;
-  uint32_t* counters = nullptr;
-  size_t partial_floats = 0;
-  size_t counter_count = 0;
-  uint8_t* records = nullptr;  // digit records of x (integer-MMA decode)
-  size_t record_bytes = 0;
-};
-
-std::mutex g_scratch_mu;
-std::map<std::pair<int, cudaStream_t>, SplitScratch>& scratch_map() {
-  static std::map<std::pair<int, cudaStream_t>, SplitScratch> m;
-  return m;
-}
-
-cudaError_t stream_scratch(cudaStream_t stream, size_t partial_floats, size_t counters,
-                           float** p_out, uint32_t** c_out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  SplitScratch& sc = scratch_map()[{dev, stream}];
-  if (sc.partial_floats < partial_floats || sc.counter_count < counters) {
-    if (sc.partials != nullptr) {
-      e = cudaStreamSynchronize(stream);
-      if (e != cudaSuccess) return e;
-      cudaFree(sc.partials);
-      sc.partials = nullptr;
-      sc.counters = nullptr;
-      sc.partial_floats = 0;
-      sc.counter_count = 0;
-    }
-    const size_t pbytes = (partial_floats * sizeof(float) + 255) & ~static_cast<size_t>(255);
-    void* base = nullptr;
-    e = cudaMalloc(&base, pbytes + counters * sizeof(uint32_t));
-    if (e != cudaSuccess) return e;
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(base) + pbytes);
-    e = cudaMemsetAsync(cnt, 0, counters * sizeof(uint32_t), stream);
-    if (e != cudaSuccess) {
-      cudaFree(base);
-      return e;
-    }
-    sc.partials = static_cast<float*>(base);
-    sc.counters = cnt;
-    sc.partial_floats = partial_floats;
-    sc.counter_count = counters;
-  }
-  *p_out = sc.partials;
-  *c_out = sc.counters;
-  return cudaSuccess;
-}
-
-// Digit records of x for one (device, stream), grown like the split scratch.
-cudaError_t stream_records(cudaStream_t stream, size_t bytes, uint8_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  SplitScratch& sc = scratch_map()[{dev, stream}];
-  if (sc.record_bytes < bytes) {
-    if (sc.records != nullptr) {
-      e = cudaStreamSynchronize(stream);
-      if (e != cudaSuccess) return e;
-      cudaFree(sc.records);
-      sc.records = nullptr;
-      sc.record_bytes = 0;
-    }
-    void* p = nullptr;
-    e = cudaMalloc(&p, bytes);
-    if (e != cudaSuccess) return e;
-    sc.records = static_cast<uint8_t*>(p);
-    sc.record_bytes = bytes;
-  }
-  *out = sc.records;
-  return cudaSuccess;
-}
-
-// Scratch of int4_matmul_decode_noalloc: partial slots, arrival counters and
-// the x digit records in one fixed device array (zero at load; every call
-// leaves the counters zero).  4 MiB of partials hold one wave of up to 512
-// CTAs (B200 runs 296: 2 per SM); 4 MiB of records hold K up to 64384 at
-// M = 16 (246528 at M <= 4; M <= 2 converts x in the matmul and needs none).
-constexpr int kNoAllocMaxCtas = 512;
-constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;
-constexpr size_t kNoAllocCounterBytes = kNoAllocMaxCtas * sizeof(uint32_t);
-constexpr size_t kNoAllocRecordBytes = size_t(4) << 20;  // x digit records
-constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocCounterBytes + kNoAllocRecordBytes;
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
-
-// Device address of the array on the current device, resolved once per
-// device with cudaGetSymbolAddress (no allocation).
-cudaError_t noalloc_scratch(float** out) {
-  constexpr int kMaxDevices = 64;
-  static std::mutex mu;
-  static float* cache[kMaxDevices] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    cache[dev] = static_cast<float*>(p);
-  }
-  *out = cache[dev];
-  return cudaSuccess;
-}
-
-// Grid and split of one decode call: one wave of CTAs at the occupancy
-// limit, each with an equal run of (row tile, K block) units.
-struct DecodePlan {
-  int KB = 0;
-  int64_t U = 0;
-  int64_t P = 0;
-  bool split = false;  // does some run start inside a tile?
-};
-
-// Shared-memory opt-in and occupancy of a decode kernel, once per device.
-cudaError_t kernel_occupancy(const void* fn, int threads, int alloc, std::atomic<int>* cache,
-                             int* occ_out) {
-  constexpr int kMaxDevices = 64;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  int occ = cache[dev].load(std::memory_order_relaxed);
-  if (occ == 0) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, alloc);
-    if (e != cudaSuccess) return e;
-    if (occ < 1) occ = 1;
-    cache[dev].store(occ, std::memory_order_relaxed);
-  }
-  *occ_out = occ;
-  return cudaSuccess;
-}
-
-// The split for `occ` CTAs per SM over row tiles of `rows` rows.
-void plan_split(int occ, int rows, int64_t K, int64_t N, DecodePlan* pl) {
-  pl->KB = static_cast<int>((K + 127) / 128);
-  pl->U = ((N + rows - 1) / rows) * pl->KB;
-  pl->P = static_cast<int64_t>(occ) * num_sms();
-  if (pl->P > pl->U) pl->P = pl->U;
-  // Remembered for the last shape seen by this thread: the scan costs a
-  // division per CTA.
-  thread_local int64_t last_U = -1, last_P = -1, last_KB = -1;
-  thread_local bool last_split = false;
-  if (pl->U != last_U || pl->P != last_P || pl->KB != last_KB) {
-    bool sp = false;
-    for (int64_t p = 1; p < pl->P && !sp; ++p) sp = (p * pl->U / pl->P) % pl->KB != 0;
-    last_U = pl->U;
-    last_P = pl->P;
-    last_KB = pl->KB;
-    last_split = sp;
-  }
-  pl->split = last_split;
-}
-
-template <typename TX, int NT, int GPB>
-cudaError_t plan_decode(int64_t K, int64_t N, DecodePlan* pl) {
-  static std::atomic<int> occ_cache[64];
-  int occ = 0;
-  const cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_kernel<TX, NT, GPB>),
-                                         kThreads, DLayout<NT>::kAlloc, occ_cache, &occ);
-  if (e != cudaSuccess) return e;
-  plan_split(occ, Tiles<NT>::kRowsPerCta, K, N, pl);
-  return cudaSuccess;
-}
-
-template <typename TX, int NP, bool FUSE>
-cudaError_t plan_decode_i8(int64_t K, int64_t N, DecodePlan* pl) {
-  using S = I8Shape<NP, FUSE>;
-  static std::atomic<int> occ_cache[64];
-  int occ = 0;
-  const cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_i8_kernel<TX, NP, FUSE>),
-                                         S::kThreads, S::kAlloc, occ_cache, &occ);
-  if (e != cudaSuccess) return e;
-  plan_split(occ, S::kRowsPerCta, K, N, pl);
-  return cudaSuccess;
-}
-
-template <typename TX, int NT, int GPB>
-cudaError_t launch_decode(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                          int group, int64_t M, int64_t N, float* y, const DecodePlan& pl,
-                          float* partials, uint32_t* counters, cudaStream_t stream) {
-  using L = DLayout<NT>;
-  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return cudaErrorNotSupported;
-  uint32_t* status = status_word();
-  if (status == nullptr) return cudaErrorInvalidSymbol;
-  const int G = static_cast<int>((K + group - 1) / group);
-  CUtensorMap tw, tx;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    const cuuint32_t box[2] = {128, kRowsPerCta};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
-                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  decode_kernel<TX, NT, GPB><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, stream>>>(
-      tw, tx, scales, y, K, group, G, static_cast<int>(M), N, pl.KB, pl.U, static_cast<int>(pl.P),
-      partials, counters, status);
-  return cudaGetLastError();
-}
-
-template <typename TX, int NT, int GPB>
-cudaError_t launch_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                           int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
-  DecodePlan pl;
-  cudaError_t e = plan_decode<TX, NT, GPB>(K, N, &pl);
-  if (e != cudaSuccess) return e;
-  float* partials = nullptr;
-  uint32_t* counters = nullptr;
-  if (pl.split) {
-    e = stream_scratch(stream, static_cast<size_t>(2 * pl.P) * kPer, static_cast<size_t>(pl.P),
-                       &partials, &counters);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_decode<TX, NT, GPB>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
-                                    stream);
-}
-
-// launch_variant with the split's scratch in the static array.  Returns
-// cudaErrorInvalidValue with *need set when the split needs more scratch
-// than the array holds (more than 512 CTAs in one wave).
-template <typename TX, int NT, int GPB>
-cudaError_t launch_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                                   int64_t K, int group, int64_t M, int64_t N, float* y,
-                                   cudaStream_t stream, size_t* need) {
-  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;
-  float* scratch = nullptr;
-  cudaError_t e = noalloc_scratch(&scratch);
-  if (e != cudaSuccess) return e;
-  DecodePlan pl;
-  e = plan_decode<TX, NT, GPB>(K, N, &pl);
-  if (e != cudaSuccess) return e;
-  float* partials = nullptr;
-  uint32_t* counters = nullptr;
-  if (pl.split) {
-    const size_t bytes = static_cast<size_t>(2 * pl.P) * kPer * sizeof(float);
-    if (bytes > kNoAllocPartialBytes || pl.P > kNoAllocMaxCtas) {
-      *need = bytes + static_cast<size_t>(pl.P) * sizeof(uint32_t);
-      return cudaErrorInvalidValue;
-    }
-    partials = scratch;
-    counters = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(scratch) + kNoAllocPartialBytes);
-  }
-  return launch_decode<TX, NT, GPB>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
-                                    stream);
-}
-
-template <typename TX, int NP, bool FUSE>
-cudaError_t launch_decode_i8(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                             int group, int64_t M, int64_t N, float* y, const DecodePlan& pl,
-                             float* partials, uint32_t* counters, uint8_t* records,
-                             cudaStream_t stream) {
-  using S = I8Shape<NP, FUSE>;
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return cudaErrorNotSupported;
-  uint32_t* status = status_word();
-  if (status == nullptr) return cudaErrorInvalidSymbol;
-  const int G = static_cast<int>((K + group - 1) / group);
-  CUtensorMap tw, tx;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-    const cuuint32_t box[2] = {128, S::kRowsPerCta};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
-  std::memset(&tx, 0, sizeof tx);
-  if (S::kFuse) {
-    // x [M, K]: boxes of 256 k by all M rows.
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(M)};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
-                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
-    cfg.blockDim = dim3(S::kThreads);
-    cfg.dynamicSmemBytes = S::kAlloc;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx, static_cast<const uint8_t*>(nullptr),
-                              scales, y, K, group, G, static_cast<int>(M), N, pl.KB, pl.U,
-                              static_cast<int>(pl.P), partials, counters, status);
-  }
-  // Records 0 .. KB: a stage whose second block is past the last reads the
-  // zero record KB.
-  const int64_t nrec = static_cast<int64_t>(pl.KB) + 1;
-  const int MP = 2 * NP;
-  const int64_t threads = 16 * MP * nrec;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  {
-    cudaLaunchConfig_t dcfg = {};
-    dcfg.gridDim = dim3(static_cast<unsigned>((threads + 255) / 256));
-    dcfg.blockDim = dim3(256);
-    dcfg.stream = stream;
-    dcfg.attrs = attr;
-    dcfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&dcfg, x_digits_kernel<TX>, x, K, static_cast<int>(M),
-                                             MP, NP, nrec, records);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
-  cfg.blockDim = dim3(S::kThreads);
-  cfg.dynamicSmemBytes = S::kAlloc;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx,
-                            static_cast<const uint8_t*>(records), scales, y, K, group, G,
-                            static_cast<int>(M), N, pl.KB, pl.U, static_cast<int>(pl.P), partials,
-                            counters, status);
-}
-
-template <typename TX, int NP, bool FUSE>
-cudaError_t launch_i8_variant(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  using S = I8Shape<NP, FUSE>;
-  DecodePlan pl;
-  cudaError_t e = plan_decode_i8<TX, NP, FUSE>(K, N, &pl);
-  if (e != cudaSuccess) return e;
-  float* partials = nullptr;
-  uint32_t* counters = nullptr;
-  if (pl.split) {
-    e = stream_scratch(stream, static_cast<size_t>(2 * pl.P) * S::kOut, static_cast<size_t>(pl.P),
-                       &partials, &counters);
-    if (e != cudaSuccess) return e;
-  }
-  uint8_t* records = nullptr;
-  if (!S::kFuse) {
-    e = stream_records(stream, static_cast<size_t>(pl.KB + 1) * S::kRec, &records);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_decode_i8<TX, NP, FUSE>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
-                                  records, stream);
-}
-
-template <typename TX, int NP, bool FUSE>
-cudaError_t launch_i8_variant_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                                      int64_t K, int group, int64_t M, int64_t N, float* y,
-                                      cudaStream_t stream, size_t* need) {
-  using S = I8Shape<NP, FUSE>;
-  float* scratch = nullptr;
-  cudaError_t e = noalloc_scratch(&scratch);
-  if (e != cudaSuccess) return e;
-  DecodePlan pl;
-  e = plan_decode_i8<TX, NP, FUSE>(K, N, &pl);
-  if (e != cudaSuccess) return e;
-  const size_t pbytes = pl.split ? static_cast<size_t>(2 * pl.P) * S::kOut * sizeof(float) : 0;
-  const size_t rbytes = S::kFuse ? 0 : static_cast<size_t>(pl.KB + 1) * S::kRec;
-  if (pbytes > kNoAllocPartialBytes || pl.P > kNoAllocMaxCtas || rbytes > kNoAllocRecordBytes) {
-    *need = pbytes + static_cast<size_t>(pl.P) * sizeof(uint32_t) + rbytes;
-    return cudaErrorInvalidValue;
-  }
-  char* base = reinterpret_cast<char*>(scratch);
-  float* partials = pl.split ? scratch : nullptr;
-  uint32_t* counters = pl.split ? reinterpret_cast<uint32_t*>(base + kNoAllocPartialBytes) : nullptr;
-  uint8_t* records =
-      S::kFuse ? nullptr : reinterpret_cast<uint8_t*>(base + kNoAllocPartialBytes + kNoAllocCounterBytes);
-  return launch_decode_i8<TX, NP, FUSE>(x, packed, scales, K, group, M, N, y, pl, partials, counters,
-                                  records, stream);
-}
-
-template <typename TX>
-cudaError_t launch_i8_any(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                          int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  if (M <= kFuseMaxM) return launch_i8_variant<TX, 1, true>(x, packed, scales, K, group, M, N, y, stream);
-  if (M <= 2) return launch_i8_variant<TX, 1, false>(x, packed, scales, K, group, M, N, y, stream);
-  if (M <= 4) return launch_i8_variant<TX, 2, false>(x, packed, scales, K, group, M, N, y, stream);
-  if (M <= 8) return launch_i8_variant<TX, 4, false>(x, packed, scales, K, group, M, N, y, stream);
-  return launch_i8_variant<TX, 8, false>(x, packed, scales, K, group, M, N, y, stream);
-}
-
-template <typename TX>
-cudaError_t launch_i8_any_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                                  int64_t K, int group, int64_t M, int64_t N, float* y,
-                                  cudaStream_t stream, size_t* need) {
-  if (M <= kFuseMaxM)
-    return launch_i8_variant_noalloc<TX, 1, true>(x, packed, scales, K, group, M, N, y, stream, need);
-  if (M <= 2) return launch_i8_variant_noalloc<TX, 1, false>(x, packed, scales, K, group, M, N, y, stream, need);
-  if (M <= 4) return launch_i8_variant_noalloc<TX, 2, false>(x, packed, scales, K, group, M, N, y, stream, need);
-  if (M <= 8) return launch_i8_variant_noalloc<TX, 4, false>(x, packed, scales, K, group, M, N, y, stream, need);
-  return launch_i8_variant_noalloc<TX, 8, false>(x, packed, scales, K, group, M, N, y, stream, need);
-}
-
-template <typename TX, int NT>
-cudaError_t launch_nt_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
-                              size_t* need) {
-  if (group == 64)
-    return launch_variant_noalloc<TX, NT, 2>(x, packed, scales, K, group, M, N, y, stream, need);
-  return launch_variant_noalloc<TX, NT, 4>(x, packed, scales, K, group, M, N, y, stream, need);
-}
-
-template <typename TX>
-cudaError_t launch_tx_noalloc(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                              int group, int64_t M, int64_t N, float* y, cudaStream_t stream,
-                              size_t* need) {
-  if (group % 128 == 0) return launch_i8_any_noalloc(x, packed, scales, K, group, M, N, y, stream, need);
-  if (M <= 8) return launch_nt_noalloc<TX, 1>(x, packed, scales, K, group, M, N, y, stream, need);
-  return launch_nt_noalloc<TX, 2>(x, packed, scales, K, group, M, N, y, stream, need);
-}
-
-template <typename TX, int NT>
-cudaError_t launch_nt(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                      int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  if (group == 64) return launch_variant<TX, NT, 2>(x, packed, scales, K, group, M, N, y, stream);
-  return launch_variant<TX, NT, 4>(x, packed, scales, K, group, M, N, y, stream);
-}
-
-template <typename TX>
-cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                      int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  if (group % 128 == 0) return launch_i8_any(x, packed, scales, K, group, M, N, y, stream);
-  if (M <= 8) return launch_nt<TX, 1>(x, packed, scales, K, group, M, N, y, stream);
-  return launch_nt<TX, 2>(x, packed, scales, K, group, M, N, y, stream);
 }
 
 // ---------------- small matrices ----------------
@@ -1748,32 +1430,389 @@ bool small_applies(int64_t K, int group, int64_t N) {
   return (N + 15) / 16 <= static_cast<int64_t>(kSmallCtasPerSm) * num_sms();
 }
 
-cudaError_t launch_small_any(const void* x, DType xt, const uint8_t* packed, const uint16_t* scales,
-                             int64_t K, int group, int64_t M, int64_t N, float* y,
-                             cudaStream_t stream) {
-  if (xt == DType::BF16)
-    return launch_small(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N, y,
-                        stream);
-  return launch_small(static_cast<const __half*>(x), packed, scales, K, group, M, N, y, stream);
+// ---------------- host side: scratch, schedule, launch ----------------
+// A decode call may need device scratch: one arrival counter per CTA (zero
+// when the call starts; every call leaves its counters zero), two partial-
+// tile slots per CTA for the split, and the x digit records of the integer
+// kernel at M > 2.  The caller provides it (int4_matmul_ws), or it is the
+// library's fixed array (int4_matmul_decode_noalloc).  Without any
+// (int4_matmul), the runs cover whole row tiles, so no tile is split, and
+// batches that would need digit records take the 16-bit kernel.
+struct DecodeScratch {
+  uint32_t* counters = nullptr;
+  size_t counter_cap = 0;  // entries
+  float* partials = nullptr;
+  size_t partial_cap = 0;  // floats
+  uint8_t* records = nullptr;
+  size_t record_cap = 0;   // bytes
+};
+
+struct DecodeNeed {
+  size_t counters = 0;  // entries
+  size_t partials = 0;  // floats
+  size_t records = 0;   // bytes
+};
+
+// A caller's workspace: the counters in a fixed first region (so that calls
+// of any shape sharing the workspace find zeros there), then the partial
+// tiles, then the records, each region 256-byte aligned.
+constexpr size_t kWsCounterCap = 1024;
+constexpr size_t kWsCounterBytes = kWsCounterCap * sizeof(uint32_t);
+
+size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+size_t workspace_bytes(const DecodeNeed& n) {
+  if (n.counters == 0 && n.partials == 0 && n.records == 0) return 0;
+  return kWsCounterBytes + round256(n.partials * sizeof(float)) + n.records;
+}
+
+DecodeScratch carve_workspace(void* ws, const DecodeNeed& n) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  DecodeScratch s;
+  s.counters = reinterpret_cast<uint32_t*>(b);
+  s.counter_cap = kWsCounterCap;
+  s.partials = reinterpret_cast<float*>(b + kWsCounterBytes);
+  s.partial_cap = n.partials;
+  s.records = b + kWsCounterBytes + round256(n.partials * sizeof(float));
+  s.record_cap = n.records;
+  return s;
+}
+
+// Scratch of int4_matmul_decode_noalloc: partial slots, arrival counters and
+// the x digit records in one fixed device array (zero at load; every call
+// leaves the counters zero).  4 MiB of partials hold one wave of up to 512
+// CTAs (B200 runs 296: 2 per SM); 4 MiB of records hold K up to 64384 at
+// M = 16 (246528 at M <= 4; M <= 2 converts x in the matmul and needs none).
+constexpr int kNoAllocMaxCtas = 512;
+constexpr size_t kNoAllocPartialBytes = size_t(4) << 20;
+constexpr size_t kNoAllocCounterBytes = kNoAllocMaxCtas * sizeof(uint32_t);
+constexpr size_t kNoAllocRecordBytes = size_t(4) << 20;  // x digit records
+constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocCounterBytes + kNoAllocRecordBytes;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the array on the current device, resolved once per
+// device with cudaGetSymbolAddress (no allocation).
+cudaError_t noalloc_scratch(float** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static float* cache[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    cache[dev] = static_cast<float*>(p);
+  }
+  *out = cache[dev];
+  return cudaSuccess;
+}
+
+// The array's regions as a scratch descriptor.
+DecodeScratch noalloc_regions(float* base) {
+  char* b = reinterpret_cast<char*>(base);
+  DecodeScratch s;
+  s.partials = base;
+  s.partial_cap = kNoAllocPartialBytes / sizeof(float);
+  s.counters = reinterpret_cast<uint32_t*>(b + kNoAllocPartialBytes);
+  s.counter_cap = kNoAllocMaxCtas;
+  s.records = reinterpret_cast<uint8_t*>(b + kNoAllocPartialBytes + kNoAllocCounterBytes);
+  s.record_cap = kNoAllocRecordBytes;
+  return s;
+}
+
+// Grid and runs of one decode call: P CTAs (one wave at the occupancy limit,
+// at most one per counter of the workspace layout), each with an equal run
+// of (row tile, K block) units whose ends fall on multiples of `gran`.
+struct DecodePlan {
+  int KB = 0;
+  int64_t U = 0;
+  int64_t P = 0;
+  int64_t gran = 1;
+  bool split = false;  // does some run start or end inside a tile?
+};
+
+// Shared-memory opt-in and occupancy of a decode kernel, once per device.
+cudaError_t kernel_occupancy(const void* fn, int threads, int alloc, std::atomic<int>* cache,
+                             int* occ_out) {
+  constexpr int kMaxDevices = 64;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int occ = cache[dev].load(std::memory_order_relaxed);
+  if (occ == 0) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, alloc);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    cache[dev].store(occ, std::memory_order_relaxed);
+  }
+  *occ_out = occ;
+  return cudaSuccess;
+}
+
+// The runs for `occ` CTAs per SM over row tiles of `rows` rows: equal runs
+// of blocks (the split) when scratch holds the partial tiles, else runs of
+// whole tiles.
+void plan_runs(int occ, int rows, int64_t K, int64_t N, bool may_split, DecodePlan* pl) {
+  pl->KB = static_cast<int>((K + 127) / 128);
+  const int64_t tiles = (N + rows - 1) / rows;
+  pl->U = tiles * pl->KB;
+  int64_t slots = static_cast<int64_t>(occ) * num_sms();
+  if (slots > static_cast<int64_t>(kWsCounterCap)) slots = kWsCounterCap;
+  if (!may_split) {
+    pl->gran = pl->KB;
+    pl->P = slots < tiles ? slots : tiles;
+    pl->split = false;
+    return;
+  }
+  pl->gran = 1;
+  pl->P = slots < pl->U ? slots : pl->U;
+  // Remembered for the last shape seen by this thread: the scan costs a
+  // division per CTA.
+  thread_local int64_t last_U = -1, last_P = -1, last_KB = -1;
+  thread_local bool last_split = false;
+  if (pl->U != last_U || pl->P != last_P || pl->KB != last_KB) {
+    bool sp = false;
+    for (int64_t p = 1; p < pl->P && !sp; ++p) sp = (p * pl->U / pl->P) % pl->KB != 0;
+    last_U = pl->U;
+    last_P = pl->P;
+    last_KB = pl->KB;
+    last_split = sp;
+  }
+  pl->split = last_split;
+}
+
+// Arguments of one decode call.
+struct DecodeArgs {
+  const void* x;
+  const uint8_t* packed;
+  const uint16_t* scales;
+  int64_t K;
+  int group;
+  int64_t M;
+  int64_t N;
+  float* y;
+  cudaStream_t stream;
+};
+
+bool fits(const DecodeNeed& n, const DecodeScratch* sc) {
+  if (n.counters == 0 && n.partials == 0 && n.records == 0) return true;
+  return sc != nullptr && n.counters <= sc->counter_cap && n.partials <= sc->partial_cap &&
+         n.records <= sc->record_cap;
+}
+
+template <typename TX, int NT, int GPB>
+cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& pl, float* partials,
+                          uint32_t* counters) {
+  using L = DLayout<NT>;
+  constexpr int kRowsPerCta = Tiles<NT>::kRowsPerCta;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
+  const int G = static_cast<int>((a.K + a.group - 1) / a.group);
+  CUtensorMap tw, tx;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
+    const cuuint32_t box[2] = {128, kRowsPerCta};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
+    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(a.M)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
+                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (enc(&tx, dt, 2, const_cast<void*>(a.x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  decode_kernel<TX, NT, GPB><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, a.stream>>>(
+      tw, tx, a.scales, a.y, a.K, a.group, G, static_cast<int>(a.M), a.N, pl.KB, pl.U,
+      static_cast<int>(pl.P), pl.gran, partials, counters, status);
+  return cudaGetLastError();
+}
+
+// The 16-bit decode kernel: plan, scratch need and (if `launch`) the launch.
+template <typename TX, int NT, int GPB>
+cudaError_t run_bf(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
+                   bool launch) {
+  constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
+  static std::atomic<int> occ_cache[64];
+  int occ = 0;
+  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_kernel<TX, NT, GPB>),
+                                   kThreads, DLayout<NT>::kAlloc, occ_cache, &occ);
+  if (e != cudaSuccess) return e;
+  DecodePlan pl;
+  plan_runs(occ, Tiles<NT>::kRowsPerCta, a.K, a.N, scratch, &pl);
+  DecodeNeed n;
+  if (pl.split) {
+    n.counters = static_cast<size_t>(pl.P);
+    n.partials = static_cast<size_t>(2 * pl.P) * kPer;
+  }
+  *need = n;
+  if (!launch) return cudaSuccess;
+  if (!fits(n, sc)) return cudaErrorInvalidValue;
+  return launch_decode<TX, NT, GPB>(a, pl, pl.split ? sc->partials : nullptr,
+                                    pl.split ? sc->counters : nullptr);
+}
+
+template <typename TX, int NP, bool FUSE>
+cudaError_t launch_decode_i8(const DecodeArgs& a, const DecodePlan& pl, float* partials,
+                             uint32_t* counters, uint8_t* records) {
+  using S = I8Shape<NP, FUSE>;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
+  const TX* x = static_cast<const TX*>(a.x);
+  const int G = static_cast<int>((a.K + a.group - 1) / a.group);
+  CUtensorMap tw, tx;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K / 2), static_cast<cuuint64_t>(a.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K / 2)};
+    const cuuint32_t box[2] = {128, S::kRowsPerCta};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.packed), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  std::memset(&tx, 0, sizeof tx);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (S::kFuse) {
+    // x [M, K]: boxes of 256 k by all M rows.
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.K) * 2};
+    const cuuint32_t box[2] = {256, static_cast<cuuint32_t>(a.M)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
+                                       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (enc(&tx, dt, 2, const_cast<TX*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    // Records 0 .. KB: a stage whose second block is past the last reads the
+    // zero record KB.
+    const int64_t nrec = static_cast<int64_t>(pl.KB) + 1;
+    const int MP = 2 * NP;
+    const int64_t threads = 16 * MP * nrec;
+    cudaLaunchConfig_t dcfg = {};
+    dcfg.gridDim = dim3(static_cast<unsigned>((threads + 255) / 256));
+    dcfg.blockDim = dim3(256);
+    dcfg.stream = a.stream;
+    dcfg.attrs = attr;
+    dcfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&dcfg, x_digits_kernel<TX>, x, a.K,
+                                             static_cast<int>(a.M), MP, NP, nrec, records);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
+  cfg.blockDim = dim3(S::kThreads);
+  cfg.dynamicSmemBytes = S::kAlloc;
+  cfg.stream = a.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx, x,
+                            static_cast<const uint8_t*>(records), a.scales, a.y, a.K, a.group, G,
+                            static_cast<int>(a.M), a.N, pl.KB, pl.U, static_cast<int>(pl.P),
+                            pl.gran, partials, counters, status);
+}
+
+// The integer decode kernel: plan, scratch need and (if `launch`) the launch.
+template <typename TX, int NP, bool FUSE>
+cudaError_t run_i8(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
+                   bool launch) {
+  using S = I8Shape<NP, FUSE>;
+  static std::atomic<int> occ_cache[64];
+  int occ = 0;
+  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_i8_kernel<TX, NP, FUSE>),
+                                   S::kThreads, S::kAlloc, occ_cache, &occ);
+  if (e != cudaSuccess) return e;
+  DecodePlan pl;
+  plan_runs(occ, S::kRowsPerCta, a.K, a.N, scratch, &pl);
+  DecodeNeed n;
+  if (pl.split) {
+    n.counters = static_cast<size_t>(pl.P);
+    n.partials = static_cast<size_t>(2 * pl.P) * S::kOut;
+  }
+  if (!S::kFuse) n.records = static_cast<size_t>(pl.KB + 1) * S::kRec;
+  *need = n;
+  if (!launch) return cudaSuccess;
+  if (!fits(n, sc)) return cudaErrorInvalidValue;
+  return launch_decode_i8<TX, NP, FUSE>(a, pl, pl.split ? sc->partials : nullptr,
+                                        pl.split ? sc->counters : nullptr,
+                                        S::kFuse ? nullptr : sc->records);
+}
+
+// Kernel choice of a decode call.  `scratch`: whether scratch will be there
+// (the split schedule and, at M > 2 with groups of whole 128-k blocks, the
+// integer kernel with digit records); without it the runs cover whole tiles
+// and such batches take the 16-bit kernel.
+template <typename TX>
+cudaError_t run_decode(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
+                       bool launch) {
+  if (small_applies(a.K, a.group, a.N)) {
+    *need = DecodeNeed{};
+    if (!launch) return cudaSuccess;
+    return launch_small(static_cast<const TX*>(a.x), a.packed, a.scales, a.K, a.group, a.M, a.N,
+                        a.y, a.stream);
+  }
+  if (a.group % 128 == 0) {
+    if (a.M <= kFuseMaxM) return run_i8<TX, 1, true>(a, scratch, sc, need, launch);
+    if (!scratch) {
+      if (a.M <= 8) return run_bf<TX, 1, 1>(a, scratch, sc, need, launch);
+      return run_bf<TX, 2, 1>(a, scratch, sc, need, launch);
+    }
+    if (a.M <= 2) return run_i8<TX, 1, false>(a, scratch, sc, need, launch);
+    if (a.M <= 4) return run_i8<TX, 2, false>(a, scratch, sc, need, launch);
+    if (a.M <= 8) return run_i8<TX, 4, false>(a, scratch, sc, need, launch);
+    return run_i8<TX, 8, false>(a, scratch, sc, need, launch);
+  }
+  if (a.M <= 8) {
+    if (a.group == 64) return run_bf<TX, 1, 2>(a, scratch, sc, need, launch);
+    return run_bf<TX, 1, 4>(a, scratch, sc, need, launch);
+  }
+  if (a.group == 64) return run_bf<TX, 2, 2>(a, scratch, sc, need, launch);
+  return run_bf<TX, 2, 4>(a, scratch, sc, need, launch);
+}
+
+cudaError_t run_decode_any(DType xt, const DecodeArgs& a, bool scratch, const DecodeScratch* sc,
+                           DecodeNeed* need, bool launch) {
+  if (xt == DType::BF16) return run_decode<__nv_bfloat16>(a, scratch, sc, need, launch);
+  return run_decode<__half>(a, scratch, sc, need, launch);
+}
+
+size_t need_total_bytes(const DecodeNeed& n) {
+  return n.counters * sizeof(uint32_t) + n.partials * sizeof(float) + n.records;
 }
 
 }  // namespace
 
 cudaError_t reset_split_counters() {
-  // After a bounded wait gave up, a CTA may have left an arrival counted.
+  // After a bounded wait gave up, a CTA may have left an arrival counted in
+  // the library's fixed array (callers' workspaces are theirs to clear).
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;
-  {
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    for (auto& kv : scratch_map())
-      if (kv.first.first == dev && kv.second.counters != nullptr) {
-        e = cudaMemset(kv.second.counters, 0, kv.second.counter_count * sizeof(uint32_t));
-        if (e != cudaSuccess) return e;
-      }
-  }
   float* scratch = nullptr;
   e = noalloc_scratch(&scratch);
   if (e != cudaSuccess) return e;
@@ -1783,16 +1822,49 @@ cudaError_t reset_split_counters() {
 
 size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
+cudaError_t decode_workspace_size(DType xt, int64_t K, int group, int64_t M, int64_t N,
+                                  size_t* bytes) {
+  const DecodeArgs a{nullptr, nullptr, nullptr, K, group, M, N, nullptr, nullptr};
+  DecodeNeed n;
+  const cudaError_t e = run_decode_any(xt, a, true, nullptr, &n, false);
+  if (e != cudaSuccess) return e;
+  *bytes = workspace_bytes(n);
+  return cudaSuccess;
+}
+
+cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
+                                 const uint16_t* scales, int64_t K, int group, int64_t M,
+                                 int64_t N, float* y, void* workspace, size_t workspace_bytes_given,
+                                 cudaStream_t stream, size_t* need) {
+  const DecodeArgs a{x, packed, scales, K, group, M, N, y, stream};
+  if (workspace == nullptr && workspace_bytes_given == 0) {
+    DecodeNeed n;
+    return run_decode_any(xt, a, false, nullptr, &n, true);
+  }
+  DecodeNeed n;
+  cudaError_t e = run_decode_any(xt, a, true, nullptr, &n, false);
+  if (e != cudaSuccess) return e;
+  const size_t bytes = workspace_bytes(n);
+  if (bytes > workspace_bytes_given || (bytes > 0 && workspace == nullptr)) {
+    *need = bytes;
+    return cudaErrorInvalidValue;
+  }
+  const DecodeScratch sc = carve_workspace(workspace, n);
+  return run_decode_any(xt, a, true, &sc, &n, true);
+}
+
 cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t* packed,
                                          const uint16_t* scales, int64_t K, int group, int64_t M,
                                          int64_t N, float* y, cudaStream_t stream, size_t* need) {
-  if (small_applies(K, group, N))
-    return launch_small_any(x, xt, packed, scales, K, group, M, N, y, stream);
-  if (xt == DType::BF16)
-    return launch_tx_noalloc(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N,
-                             y, stream, need);
-  return launch_tx_noalloc(static_cast<const __half*>(x), packed, scales, K, group, M, N, y, stream,
-                           need);
+  float* base = nullptr;
+  cudaError_t e = noalloc_scratch(&base);
+  if (e != cudaSuccess) return e;
+  const DecodeArgs a{x, packed, scales, K, group, M, N, y, stream};
+  const DecodeScratch sc = noalloc_regions(base);
+  DecodeNeed n;
+  e = run_decode_any(xt, a, true, &sc, &n, true);
+  if (e == cudaErrorInvalidValue && !fits(n, &sc)) *need = need_total_bytes(n);
+  return e;
 }
 
 bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
@@ -1805,17 +1877,6 @@ bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, cons
   if (reinterpret_cast<uintptr_t>(packed) % 16 != 0) return false;
   if (N > 0x7FFFFFFFLL) return false;
   return true;
-}
-
-cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
-                                 const uint16_t* scales, int64_t K, int group, int64_t M,
-                                 int64_t N, float* y, cudaStream_t stream) {
-  if (small_applies(K, group, N))
-    return launch_small_any(x, xt, packed, scales, K, group, M, N, y, stream);
-  if (xt == DType::BF16)
-    return launch_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, M, N, y,
-                     stream);
-  return launch_tx(static_cast<const __half*>(x), packed, scales, K, group, M, N, y, stream);
 }
 
 }  // namespace int4lib

@@ -113,15 +113,17 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
  * and fp32); group partial sums are accumulated in fp32 (fp64 across groups
  * for fp32 x); the group's scale is applied to each partial before it joins
  * the running sum.  The decode kernel for groups that are a multiple of 128
- * forms each 128-k block's sum x.q exactly in integers: x is written per
- * block as a 30-bit integer times a power of two (exact for every bf16 x
- * within 2^22 of the block's largest |x|, fp16 within 2^19; otherwise off by
- * at most 2^-30 of that largest), a NaN or infinity in a block makes the
- * row's outputs NaN, and blocks whose largest |x| is below 2^-93 keep fewer
- * low digits.  Accuracy: |y - y_exact| <= c * sum_k |x[m,k]| |w_hat[n,k]|
- * with c = 1e-5 for fp32 x and c = 4e-3 for bf16 / fp16 x.  Summation order
- * differs between kernels; results are deterministic for a given shape,
- * dtype and device.
+ * forms each 128-k block's sum x.q exactly in integers wherever x is an
+ * integer multiple of 2^-29 times the block's largest power of two (every
+ * bf16 x within 2^22 of the block's largest |x|, fp16 within 2^19); a block
+ * of a batch row where that does not hold (a wider span, values below about
+ * 2^-93, NaN or infinity) is computed with bf16/fp16 products and fp32 sums
+ * instead, so x is never rounded.
+ * Accuracy, for every finite input: |y - y_exact| <= c * sum_k |x[m,k]| |w_hat[n,k]|
+ * with c = 1e-5 for fp32 x and c = 4e-3 for bf16 / fp16 x.  NaN or infinity
+ * in x propagates as in IEEE arithmetic.  Summation order differs between
+ * kernels; results are deterministic for a given shape, dtype, schedule
+ * (with or without a workspace) and device.
  *
  * x       [M, K] device input of x_dtype; alignment: its element size.
  * packed  [N, ceil(K/2)] device input; any alignment.
@@ -133,6 +135,12 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
  * kernel; fp32 x, and shapes the fast kernels do not cover (K or group not a
  * multiple of 32, unaligned rows), take the general CUDA-core kernel.
  *
+ * int4_matmul needs no workspace.  Its decode schedule gives each CTA whole
+ * row tiles, and batches of 3..16 rows take the bf16/fp16 decode kernel; with
+ * a workspace (int4_matmul_ws) the decode splits tiles evenly over one wave
+ * of CTAs and runs the integer kernel at every M, which is faster when the
+ * row tiles do not fill the GPU evenly.
+ *
  * Stream ordering: the decode kernels for groups that are a multiple of 128
  * launch with programmatic stream serialization and wait for the preceding
  * work on `stream` before touching memory, so ordinary stream order holds.
@@ -143,6 +151,37 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
 int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                 int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* stream);
 
+/*
+ * int4_matmul_workspace_size - bytes of device workspace int4_matmul_ws
+ * needs for this problem on the current device (written to *bytes; 0 when
+ * the chosen kernel needs none).  Host-only; launches nothing.  The size
+ * depends on the device (its SM count), so query it on the device that runs
+ * the call.
+ */
+int int4_matmul_workspace_size(int32_t x_dtype, int64_t K, int32_t group, int64_t M, int64_t N,
+                               size_t* bytes);
+
+/*
+ * int4_matmul_ws - int4_matmul with a caller-owned device workspace.
+ *
+ * Same contract and result bounds as int4_matmul.  The library allocates
+ * nothing: `workspace` holds the decode kernels' scratch (arrival counters,
+ * partial tiles of the split, and the integer digits of x at M > 2).
+ *   - workspace_bytes must be at least int4_matmul_workspace_size(...) for
+ *     this problem, else INT4_ERR_ARG (nothing launched).  workspace == NULL
+ *     with workspace_bytes == 0 selects the schedule of int4_matmul.
+ *   - workspace must be 256-byte aligned (INT4_ERR_ALIGN) and zero-filled
+ *     before its first use; every call leaves its counters zero again, so a
+ *     workspace can serve any number of calls, of any shape, that are
+ *     ordered on one stream.  Calls that may overlap in time (different
+ *     streams) need different workspaces.
+ *   - After int4_device_status reports INT4_ERR_TIMEOUT, zero-fill the
+ *     workspaces that were in use before reusing them.
+ */
+int int4_matmul_ws(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                   int64_t K, int32_t group, int64_t M, int64_t N, float* y, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
 /* Kernel selectors for int4_matmul_path. */
 #define INT4_PATH_AUTO     0
 #define INT4_PATH_SIMT     1  /* general CUDA-core kernel (any shape, any dtype) */
@@ -150,15 +189,16 @@ int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uin
 #define INT4_PATH_PREFILL  3  /* tcgen05 tensor-core kernel (bf16/fp16 x) */
 
 /*
- * int4_matmul_path - int4_matmul with the kernel chosen by the caller.
+ * int4_matmul_path - int4_matmul_ws with the kernel chosen by the caller.
  *
- * Same contract as int4_matmul; `path` is one of INT4_PATH_*.  A forced path
- * that cannot run the given shape or dtype returns INT4_ERR_UNSUPPORTED and
- * launches nothing.  Used to test every kernel on every shape it accepts.
+ * Same contract as int4_matmul_ws (workspace == NULL with workspace_bytes ==
+ * 0: no workspace); `path` is one of INT4_PATH_*.  A forced path that cannot
+ * run the given shape or dtype returns INT4_ERR_UNSUPPORTED and launches
+ * nothing.  Used to test every kernel on every shape it accepts.
  */
 int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                      int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
-                     void* stream);
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Allocation-free decode matmul.  The pages have no counterpart: this entry
  * exists for callers that must not allocate device memory during the call,

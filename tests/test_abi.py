@@ -89,8 +89,43 @@ def test_matmul_rejects_bad_arguments(L):
     assert call(N=0) == q4.OK
     msg = L.int4_last_error()
     assert isinstance(msg, bytes)
-    rc = L.int4_matmul_path(fake, 1, fake, fake, 64, 32, 2, 3, fake, 42, None)
+    rc = L.int4_matmul_path(fake, 1, fake, fake, 64, 32, 2, 3, fake, 42, None, 0, None)
     assert rc == q4.ERR_ARG
+
+
+def test_matmul_ws_rejects_bad_workspaces_before_launching(L):
+    """The workspace entry checks its workspace on the host: a null workspace
+    with a non-zero size, and one that is not 256-byte aligned."""
+    fake = ctypes.c_void_p(256)
+    f = L.int4_matmul_ws
+    assert f(fake, 1, fake, fake, 4096, 128, 1, 8192, fake, None, 4096, None) == q4.ERR_ARG
+    assert b"workspace" in L.int4_last_error()
+    assert f(fake, 1, fake, fake, 4096, 128, 1, 8192, fake, ctypes.c_void_p(256 + 16), 4096,
+             None) == q4.ERR_ALIGN
+    assert b"256" in L.int4_last_error()
+    # Argument checks come first, as for int4_matmul.
+    assert f(None, 1, fake, fake, 4096, 128, 1, 8192, fake, fake, 4096, None) == q4.ERR_ARG
+    assert f(fake, 5, fake, fake, 4096, 128, 1, 8192, fake, fake, 4096, None) == q4.ERR_DTYPE
+    assert f(fake, 1, fake, fake, 4096, 128, 0, 8192, fake, None, 0, None) == q4.OK   # no work
+
+
+def test_workspace_size_rejects_bad_arguments(L):
+    out = ctypes.c_size_t(123)
+    q = L.int4_matmul_workspace_size
+    assert q(1, 4096, 128, 1, 8192, None) == q4.ERR_ARG
+    assert q(7, 4096, 128, 1, 8192, ctypes.byref(out)) == q4.ERR_DTYPE
+    assert q(1, 0, 128, 1, 8192, ctypes.byref(out)) == q4.ERR_ARG
+    assert q(1, 4096, 0, 1, 8192, ctypes.byref(out)) == q4.ERR_ARG
+    assert q(1, 4096, 128, -1, 8192, ctypes.byref(out)) == q4.ERR_ARG
+    assert q(1, 1 << 40, 128, 1 << 30, 8192, ctypes.byref(out)) == q4.ERR_ARG
+    # Paths that use no scratch need no workspace, and need no GPU to say so.
+    for args in [(0, 4096, 128, 1, 8192),        # fp32 x: the CUDA-core kernel
+                 (1, 4096, 128, 64, 8192),       # M > 16: the tensor-core kernel
+                 (1, 4100, 128, 1, 8192),        # K % 32 != 0
+                 (1, 4096, 128, 0, 8192)]:       # empty
+        out.value = 123
+        assert q(*args, ctypes.byref(out)) == q4.OK
+        assert out.value == 0
 
 
 def test_noalloc_rejects_what_the_decode_kernels_cannot_run(L):
@@ -135,3 +170,38 @@ def test_python_binding_refuses_cpu_tensors():
         q4.quantize_int4(torch.zeros(4, 8), 4)
     with pytest.raises(TypeError):
         q4.unpack_int4(torch.zeros(4, 4, dtype=torch.uint8), 8)
+
+
+@pytest.mark.parametrize("fn", ["int4_matmul", "int4_matmul_decode_noalloc"])
+def test_matmul_bindings_check_operand_shapes_before_anything_runs(fn):
+    """Both matmul wrappers refuse wrong-shaped or wrong-typed operands before
+    reaching the library (the C side sees only pointers), and refuse CPU
+    tensors of the right shapes: there is no CPU path."""
+    import torch
+    K, group, N, M = 256, 128, 8, 2
+    x = torch.zeros(M, K, dtype=torch.bfloat16)
+    packed = torch.zeros(N, K // 2, dtype=torch.uint8)
+    scales = torch.zeros(N, 2, dtype=torch.float16)
+    out = torch.zeros(M, N)
+    f = getattr(q4, fn)
+
+    def call(**kw):
+        a = dict(dict(x=x, packed=packed, scales=scales, out=out), **kw)
+        if fn == "int4_matmul":
+            return f(a["x"], a["packed"], a["scales"], K, group, out=a["out"])
+        return f(a["x"], a["packed"], a["scales"], K, group, a["out"])
+
+    for bad in (torch.zeros(N, 1, dtype=torch.float16), torch.zeros(N - 1, 2, dtype=torch.float16),
+                torch.zeros(N, 2, dtype=torch.float32), torch.zeros(N * 2, dtype=torch.float16)):
+        with pytest.raises(ValueError, match="scales"):
+            call(scales=bad)
+    for bad in (torch.zeros(N, K // 2 - 1, dtype=torch.uint8), torch.zeros(N, K // 2, dtype=torch.int8),
+                torch.zeros(N * K // 2, dtype=torch.uint8)):
+        with pytest.raises(ValueError, match="packed"):
+            call(packed=bad)
+    with pytest.raises(ValueError, match="x must"):
+        call(x=torch.zeros(M, K + 2, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out"):
+        call(out=torch.zeros(M, N + 1))
+    with pytest.raises(TypeError, match="CUDA"):
+        call()

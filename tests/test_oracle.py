@@ -398,6 +398,50 @@ def test_error_bound_is_zero_only_where_it_must_be():
     assert np.array_equal(b[0] == 0.0, w_hat[:, 130] == 0.0)
 
 
+def test_error_bound_by_hand_mixed_signs():
+    """sum_k |x||w_hat| worked by hand on hand-made bytes with mixed signs.
+
+    Row 0: q = [-8, 5, 3, -2] with scale 0.5 (bytes 0x58, 0xE3), so w_hat =
+    [-4, 2.5, 1.5, -1].  x = [-2, 3, -1, 4]:
+      sum |x||w_hat| = 8 + 7.5 + 1.5 + 4 = 21
+    whereas x.w_hat = 10, |x|.w_hat = -3 and x.|w_hat| = 2, so a dropped
+    abs() on either side (or both) gives another number.  Row 1 holds the same
+    bytes with two groups of two, scales 0.5 and 2: w_hat = [-4, 2.5, 6, -4],
+    sum = 8 + 7.5 + 6 + 16 = 37.5 (one scale for the whole row gives 21 or
+    84).  The second batch row is -x: the bound is even in x."""
+    packed = np.array([[0x58, 0xE3]], dtype=np.uint8)
+    x = np.array([[-2.0, 3.0, -1.0, 4.0], [2.0, -3.0, 1.0, -4.0]], dtype=np.float32)
+    for c in (4e-3, 1e-5, 1.0):
+        b4 = oracle.matmul_error_bound(x, packed, np.array([[0.5]], np.float16), 4, 4, c)
+        assert b4.shape == (2, 1)
+        assert b4[0, 0] == c * 21.0 and b4[1, 0] == c * 21.0
+        b2 = oracle.matmul_error_bound(x, packed, np.array([[0.5, 2.0]], np.float16), 4, 2, c)
+        assert b2[0, 0] == c * 37.5 and b2[1, 0] == c * 37.5
+
+
+def test_error_bound_uses_the_dequantized_weights_not_w():
+    """The bound is over w_hat = q s, not over the weights before rounding.
+
+    w = [1, 0.3, -0.55, 0.9] in one group of 4: s = fp16(1/7) = 0.1428...,
+    codes rint(w/s) = [7, 2, -4, 6] (0.3/s = 2.1005, 0.55/s = 3.8509, 0.9/s =
+    6.3015), so sum |x||w_hat| with x = [1, 10, 100, 1000] is
+    s (7 + 20 + 400 + 6000) = 6427 s = 917.9, against sum |x||w| = 959.  The
+    codes and s are taken here from the drill's definition by exact
+    arithmetic."""
+    w = np.array([[1.0, 0.3, -0.55, 0.9]], dtype=np.float32)
+    x = np.array([[1.0, 10.0, 100.0, 1000.0]], dtype=np.float32)
+    packed, scales, K = oracle.quantize_int4(w, 4)
+    s = exact_scale(1.0)
+    q = [exact_code(float(v), s) for v in w[0]]
+    assert q == [7, 2, -4, 6]
+    want = Fraction(s) * sum(abs(Fraction(float(a))) * abs(qq) for a, qq in zip(x[0], q))
+    assert want == Fraction(s) * 6427
+    b = oracle.matmul_error_bound(x, packed, scales, K, 4, 1.0)
+    assert Fraction(float(b[0, 0])) == want          # exact: every term is exact in fp64
+    unquantized = float(np.abs(x[0].astype(np.float64)) @ np.abs(w[0].astype(np.float64)))
+    assert abs(float(b[0, 0]) - unquantized) > 1.0
+
+
 def test_tiny_case_golden():
     """Regression against the committed expected values of the tiny case
     (written by tests/golden/make_golden.py, which calls only the oracle)."""
