@@ -337,6 +337,54 @@ def decode_shape_rows(dev, peaks, reps: int = 10):
     return rows
 
 
+def unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks, reps: int = 5):
+    """The unfused design the fused matmul replaces, as context: the library's
+    int4_dequantize to a bf16 w_hat [N, K], then a cuBLAS bf16 GEMM (torch)
+    x @ w_hat^T with fp32 accumulation and bf16 output.  Timed per call with
+    CUDA events after an L2 flush, the dequantization included."""
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+
+    rows = {}
+    for name, x in (("decode", xd), ("prefill", xp)):
+        if x is None:
+            continue
+        M = x.shape[0]
+
+        def once():
+            w_hat = q4.dequantize_int4(packed, scales, K_W, GROUP, dtype=torch.bfloat16)
+            return torch.matmul(x, w_hat.t())
+
+        for _ in range(2):
+            once()
+        tot_ms, deq_ms = 0.0, 0.0
+        for _ in range(reps):
+            flush_l2()
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record()
+            w_hat = q4.dequantize_int4(packed, scales, K_W, GROUP, dtype=torch.bfloat16)
+            e1.record()
+            torch.matmul(x, w_hat.t())
+            e2.record()
+            torch.cuda.synchronize()
+            tot_ms += e0.elapsed_time(e2)
+            deq_ms += e0.elapsed_time(e1)
+            del w_hat
+        tot_ms /= reps
+        deq_ms /= reps
+        row = {"ms": tot_ms, "dequantize_ms": deq_ms, "gemm_ms": tot_ms - deq_ms,
+               "what": "int4_dequantize to bf16, then torch.matmul (cuBLAS) bf16 out"}
+        if name == "decode":
+            row["GB/s_on_packed_bytes"] = N_W * (K_W // 2) / (tot_ms * 1e-3) / 1e9
+        else:
+            row["TFLOP/s"] = 2 * M * N_W * K_W / (tot_ms * 1e-3) / 1e12
+        deq_bytes = N_W * (K_W // 2) + 2 * N_W * (K_W // GROUP) + 2 * N_W * K_W
+        row["dequantize_GB/s"] = deq_bytes / (deq_ms * 1e-3) / 1e9
+        rows[name] = row
+    return rows
+
+
 def run_ours(args):
     import torch
 
@@ -495,6 +543,9 @@ def run_ours(args):
     shape_rows = None
     if not args.no_shapes and not args.only:
         shape_rows = decode_shape_rows(dev, peaks)
+    unfused = None
+    if not args.no_unfused and not args.only:
+        unfused = unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks)
 
     # End to end through the public Python API: pinned host x in, y out.
     e2e = None
@@ -543,7 +594,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "flushed before every row (256 MiB write, then 256 MiB read of another buffer); the decode row's back-to-back calls read distinct weight copies (940 MB > L2)",
                    "parallelism": f"replicas x{world}"},
-        "rows": rows, "decode_llama7b": shape_rows, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "rows": rows, "decode_llama7b": shape_rows, "unfused": unfused, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * sum(launches_per_step[n] for n in order),
         "wall_ms_timed_region": wall_ms,
     }
@@ -562,6 +613,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-unfused", action="store_true",
+                    help="skip the dequantize-then-GEMM comparison rows")
     ap.add_argument("--no-shapes", action="store_true",
                     help="skip the decode rows at the Llama-7B-shaped linears")
     ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,

@@ -25,7 +25,8 @@ import threading
 import torch
 
 __all__ = [
-    "quantize_int4", "unpack_int4", "int4_matmul", "int4_matmul_decode_noalloc",
+    "quantize_int4", "unpack_int4", "dequantize_int4", "int4_matmul", "int4_matmul_decode_noalloc",
+    "quantize_int4_affine", "EPI_RELU",
     "matmul_workspace_size", "matmul_select", "device_status",
     "selftest_wait_timeout", "lib", "library_path", "Int4Error",
     "PATH_AUTO", "PATH_SIMT", "PATH_DECODE", "PATH_PREFILL",
@@ -37,6 +38,7 @@ _LIB_PATH = os.path.join(_HERE, "libint4.so")
 OK, ERR_ARG, ERR_DTYPE, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = range(7)
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 PATH_AUTO, PATH_SIMT, PATH_DECODE, PATH_PREFILL = 0, 1, 2, 3
+EPI_RELU = 1
 
 _DTYPE_CODE = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
 
@@ -69,10 +71,15 @@ def lib() -> ctypes.CDLL:
         vp, i32, i64, u32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
         L.int4_quantize.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp]
         L.int4_unpack.argtypes = [vp, i64, i64, vp, vp]
+        L.int4_dequantize.argtypes = [vp, vp, i64, i32, i64, vp, i32, vp]
+        L.int4_quantize_affine.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp, vp]
+        L.int4_dequantize_affine.argtypes = [vp, vp, vp, i64, i32, i64, vp, i32, vp]
         sz = ctypes.c_size_t
         L.int4_matmul.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
         L.int4_matmul_ws.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp, sz, vp]
         L.int4_matmul_path.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, i32, vp, sz, vp]
+        L.int4_matmul_ex.argtypes = [vp, i32, vp, vp, vp, i64, i32, i64, i64, vp, i32, vp, i32, vp,
+                                     sz, vp]
         L.int4_matmul_workspace_size.argtypes = [i32, i64, i32, i64, i64, ctypes.POINTER(sz)]
         L.int4_matmul_select.argtypes = [i32, i64, i32, i64, i64]
         L.int4_matmul_decode_noalloc.argtypes = [vp, i32, vp, vp, i64, i32, i64, i64, vp, vp]
@@ -81,7 +88,9 @@ def lib() -> ctypes.CDLL:
         L.int4_last_error.restype = ctypes.c_char_p
         L.int4_last_error.argtypes = []
         L.int4_version.argtypes = []
-        for name in ("int4_quantize", "int4_unpack", "int4_matmul", "int4_matmul_path",
+        for name in ("int4_quantize", "int4_unpack", "int4_dequantize", "int4_matmul",
+                     "int4_matmul_path", "int4_matmul_ex", "int4_quantize_affine",
+                     "int4_dequantize_affine",
                      "int4_matmul_ws", "int4_matmul_workspace_size", "int4_matmul_decode_noalloc",
                      "int4_matmul_select", "int4_device_status", "int4_selftest_wait_timeout",
                      "int4_version"):
@@ -145,6 +154,58 @@ def unpack_int4(packed: torch.Tensor, K: int) -> torch.Tensor:
     with torch.cuda.device(packed.device):
         _check(lib().int4_unpack(packed.data_ptr(), K, N, out.data_ptr(), _stream(packed)))
     return out
+
+
+def dequantize_int4(packed: torch.Tensor, scales: torch.Tensor, K: int, group: int = 128,
+                    dtype: torch.dtype = torch.bfloat16, *,
+                    zeros: torch.Tensor | None = None) -> torch.Tensor:
+    """w_hat = q * s (or (q - z) * s with the affine scheme's `zeros`) as a
+    dense [N, K] tensor of `dtype`, rounded to nearest even."""
+    _need_cuda("packed", packed)
+    _need_cuda("scales", scales)
+    if packed.dtype != torch.uint8 or packed.dim() != 2 or packed.shape[1] != (K + 1) // 2:
+        raise ValueError("packed must be uint8 [N, ceil(K/2)]")
+    N = packed.shape[0]
+    if group < 1 or scales.dtype != torch.float16 or tuple(scales.shape) != (N, -(-K // group)):
+        raise ValueError("scales must be float16 [N, ceil(K/group)]")
+    if dtype not in _DTYPE_CODE:
+        raise TypeError("dtype must be float32, bfloat16 or float16")
+    if scales.device != packed.device:
+        raise ValueError("scales must be on packed's device")
+    if zeros is not None:
+        _need_cuda("zeros", zeros)
+        if zeros.dtype != torch.uint8 or zeros.shape != scales.shape or zeros.device != packed.device:
+            raise ValueError("zeros must be uint8 [N, ceil(K/group)] on packed's device")
+    out = torch.empty((N, K), dtype=dtype, device=packed.device)
+    with torch.cuda.device(packed.device):
+        if zeros is None:
+            _check(lib().int4_dequantize(packed.data_ptr(), scales.data_ptr(), K, int(group), N,
+                                         out.data_ptr(), _DTYPE_CODE[dtype], _stream(packed)))
+        else:
+            _check(lib().int4_dequantize_affine(packed.data_ptr(), scales.data_ptr(),
+                                                zeros.data_ptr(), K, int(group), N, out.data_ptr(),
+                                                _DTYPE_CODE[dtype], _stream(packed)))
+    return out
+
+
+def quantize_int4_affine(w: torch.Tensor, group: int = 128):
+    """The asymmetric variant: w [N, K] -> (packed uint8 [N, ceil(K/2)] of
+    unsigned codes, scales fp16 [N, G], zeros uint8 [N, G], K)."""
+    _need_cuda("w", w)
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    if w.dtype not in _DTYPE_CODE:
+        raise TypeError("w must be float32, bfloat16 or float16")
+    N, K = w.shape
+    G = -(-K // group) if group >= 1 else 0
+    packed = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((N, max(G, 0)), dtype=torch.float16, device=w.device)
+    zeros = torch.empty((N, max(G, 0)), dtype=torch.uint8, device=w.device)
+    with torch.cuda.device(w.device):
+        _check(lib().int4_quantize_affine(w.data_ptr(), _DTYPE_CODE[w.dtype], N, K, int(group),
+                                          packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+                                          _stream(w)))
+    return packed, scales, zeros, K
 
 
 def _matmul_operands(x, packed, scales, K: int, group: int, out=None):
@@ -215,15 +276,27 @@ def _workspace_for(x: torch.Tensor, nbytes: int) -> torch.Tensor | None:
 
 
 def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: int,
-                group: int = 128, *, path: int = PATH_AUTO, out: torch.Tensor | None = None,
-                workspace: torch.Tensor | bool | None = None):
+                group: int = 128, *, zeros: torch.Tensor | None = None,
+                bias: torch.Tensor | None = None, relu: bool = False, path: int = PATH_AUTO,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | bool | None = None):
     """y = x @ dequantize(W).T as float32 [M, N]; x is [M, K] fp32/bf16/fp16.
 
-    `workspace`: None uses a zero-filled workspace the binding keeps per device
-    and stream; a uint8 CUDA tensor (zero-filled before its first use, at
-    least matmul_workspace_size bytes) is used as given; False runs the
-    schedule that needs no workspace (the C entry int4_matmul)."""
+    `zeros` (uint8 [N, G]): the affine scheme's zero points (codes from
+    quantize_int4_affine); `bias` (float32 [N]) and `relu` apply to each
+    output before it is stored.  `workspace`: None uses a zero-filled
+    workspace the binding keeps per device and stream; a uint8 CUDA tensor
+    (zero-filled before its first use, at least matmul_workspace_size bytes)
+    is used as given; False runs the schedule that needs no workspace (the C
+    entry int4_matmul)."""
     M, N = _matmul_operands(x, packed, scales, K, group, out)
+    if zeros is not None:
+        _need_cuda("zeros", zeros)
+        if zeros.dtype != torch.uint8 or zeros.shape != scales.shape or zeros.device != x.device:
+            raise ValueError("zeros must be uint8 [N, ceil(K/group)] on x's device")
+    if bias is not None:
+        _need_cuda("bias", bias)
+        if bias.dtype != torch.float32 or tuple(bias.shape) != (N,) or bias.device != x.device:
+            raise ValueError("bias must be float32 [N] on x's device")
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=x.device)
     L = _lib if _lib is not None else lib()
@@ -239,9 +312,16 @@ def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: 
             if workspace.dtype != torch.uint8 or workspace.device != x.device:
                 raise ValueError("workspace must be a uint8 tensor on x's device")
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
-        _check(L.int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
-                                  scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
-                                  int(path), ws_ptr, ws_bytes, _stream(x)))
+        if zeros is None and bias is None and not relu:
+            _check(L.int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
+                                      scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
+                                      int(path), ws_ptr, ws_bytes, _stream(x)))
+        else:
+            _check(L.int4_matmul_ex(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
+                                    scales.data_ptr(), None if zeros is None else zeros.data_ptr(),
+                                    K, int(group), M, N, None if bias is None else bias.data_ptr(),
+                                    EPI_RELU if relu else 0, out.data_ptr(), int(path), ws_ptr,
+                                    ws_bytes, _stream(x)))
     return out
 
 
@@ -300,3 +380,8 @@ def selftest_wait_timeout(spins: int, device=None) -> None:
     with torch.cuda.device(dev):
         _check(lib().int4_selftest_wait_timeout(
             int(spins), ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+from .module import Int4Linear  # noqa: E402  (uses the functions above)
+
+__all__.append("Int4Linear")

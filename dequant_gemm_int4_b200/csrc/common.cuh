@@ -35,6 +35,20 @@ struct Elem<__half> {
   }
 };
 
+// What the matmul kernels do to an output before storing it: add the output
+// column's bias (fp32 [N], optional), then ReLU (max(v, 0), NaN kept), as the
+// linear layer of the page "Build a Blockwise INT4 Inference Engine", steps 3
+// and 4 (x @ W_dq^T + bias, then ReLU).
+struct Epilogue {
+  const float* bias = nullptr;
+  int relu = 0;
+  __device__ __forceinline__ float apply(float v, int64_t n) const {
+    if (bias != nullptr) v += __ldg(bias + n);
+    if (relu != 0 && v < 0.0f) v = 0.0f;
+    return v;
+  }
+};
+
 // Kernels whose bounded waits give up OR a bit into the library's
 // device-side status word; its address comes from status_word().
 __device__ __forceinline__ void report_status(uint32_t* status, uint32_t bit) {

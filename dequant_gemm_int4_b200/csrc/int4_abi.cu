@@ -148,6 +148,63 @@ int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* 
   return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_unpack");
 }
 
+int int4_quantize_affine(const void* w, int32_t w_dtype, int64_t N, int64_t K, int32_t group,
+                         uint8_t* packed, uint16_t* scales, uint8_t* zeros, void* stream) {
+  if (!int4lib::dtype_ok(w_dtype)) return int4lib::fail(INT4_ERR_DTYPE, "int4_quantize_affine: unknown w_dtype");
+  if (N < 0 || K < 1 || group < 1)
+    return int4lib::fail(INT4_ERR_ARG, "int4_quantize_affine: need N >= 0, K >= 1, group >= 1");
+  if (!int4lib::mul_ok(N, K)) return int4lib::fail(INT4_ERR_ARG, "int4_quantize_affine: N*K too large");
+  if (N == 0) return INT4_OK;
+  if (!w || !packed || !scales || !zeros)
+    return int4lib::fail(INT4_ERR_ARG, "int4_quantize_affine: null pointer");
+  const DType t = static_cast<DType>(w_dtype);
+  if (!int4lib::aligned(w, int4lib::dtype_size(t)) || !int4lib::aligned(scales, 2))
+    return int4lib::fail(INT4_ERR_ALIGN, "int4_quantize_affine: w or scales not aligned to its element size");
+  const cudaError_t e = int4lib::launch_quantize_affine(w, t, N, K, group, packed, scales, zeros,
+                                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_quantize_affine");
+}
+
+static int dequantize_common(const char* name, const uint8_t* packed, const uint16_t* scales,
+                             const uint8_t* zeros, bool need_zeros, int64_t K, int32_t group,
+                             int64_t N, void* out, int32_t out_dtype, void* stream) {
+  char msg[160];
+  if (!int4lib::dtype_ok(out_dtype)) {
+    std::snprintf(msg, sizeof msg, "%s: unknown out_dtype", name);
+    return int4lib::fail(INT4_ERR_DTYPE, msg);
+  }
+  if (N < 0 || K < 1 || group < 1 || !int4lib::mul_ok(N, K)) {
+    std::snprintf(msg, sizeof msg, "%s: need N >= 0, K >= 1, group >= 1 and N*K below 2^62", name);
+    return int4lib::fail(INT4_ERR_ARG, msg);
+  }
+  if (N == 0) return INT4_OK;
+  if (!packed || !scales || !out || (need_zeros && !zeros)) {
+    std::snprintf(msg, sizeof msg, "%s: null pointer", name);
+    return int4lib::fail(INT4_ERR_ARG, msg);
+  }
+  const DType t = static_cast<DType>(out_dtype);
+  if (!int4lib::aligned(out, int4lib::dtype_size(t)) || !int4lib::aligned(scales, 2)) {
+    std::snprintf(msg, sizeof msg, "%s: out or scales not aligned to its element size", name);
+    return int4lib::fail(INT4_ERR_ALIGN, msg);
+  }
+  const cudaError_t e = int4lib::launch_dequantize(packed, scales, need_zeros ? zeros : nullptr, K,
+                                                   group, N, out, t, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, name);
+}
+
+int int4_dequantize_affine(const uint8_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                           int64_t K, int32_t group, int64_t N, void* out, int32_t out_dtype,
+                           void* stream) {
+  return dequantize_common("int4_dequantize_affine", packed, scales, zeros, true, K, group, N, out,
+                           out_dtype, stream);
+}
+
+int int4_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t K, int32_t group,
+                    int64_t N, void* out, int32_t out_dtype, void* stream) {
+  return dequantize_common("int4_dequantize", packed, scales, nullptr, false, K, group, N, out,
+                           out_dtype, stream);
+}
+
 static int matmul_check(const void* x, int32_t x_dtype, const uint8_t* packed,
                         const uint16_t* scales, int64_t K, int32_t group, int64_t M, int64_t N,
                         const float* y) {
@@ -172,29 +229,36 @@ static int matmul_choose(DType t, int64_t K, int32_t group, int64_t M, int64_t N
   return INT4_PATH_SIMT;
 }
 
-int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
-                     int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+int int4_matmul_ex(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                   const uint8_t* zeros, int64_t K, int32_t group, int64_t M, int64_t N,
+                   const float* bias, int32_t flags, float* y, int32_t path, void* workspace,
+                   size_t workspace_bytes, void* stream) {
   const int rc = matmul_check(x, x_dtype, packed, scales, K, group, M, N, y);
   if (rc != INT4_OK || M == 0 || N == 0) return rc;
+  if ((flags & ~INT4_EPI_RELU) != 0) return int4lib::fail(INT4_ERR_ARG, "int4_matmul: unknown flags");
+  if (bias != nullptr && !int4lib::aligned(bias, 4))
+    return int4lib::fail(INT4_ERR_ALIGN, "int4_matmul: bias not 4-byte aligned");
   if (workspace == nullptr && workspace_bytes != 0)
     return int4lib::fail(INT4_ERR_ARG, "int4_matmul: null workspace with a non-zero size");
   if (!int4lib::aligned(workspace, 256))
     return int4lib::fail(INT4_ERR_ALIGN, "int4_matmul: workspace not 256-byte aligned");
   const DType t = static_cast<DType>(x_dtype);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int4lib::Epilogue ep;
+  ep.bias = bias;
+  ep.relu = (flags & INT4_EPI_RELU) ? 1 : 0;
   if (path == INT4_PATH_AUTO) path = matmul_choose(t, K, group, M, N, x, packed);
   cudaError_t e;
   switch (path) {
     case INT4_PATH_SIMT:
-      e = int4lib::launch_matmul_simt(x, t, packed, scales, K, group, M, N, y, s);
+      e = int4lib::launch_matmul_simt(x, t, packed, scales, zeros, K, group, M, N, ep, y, s);
       break;
     case INT4_PATH_DECODE: {
       if (!int4lib::decode_supported(t, K, group, M, N, x, packed))
         return int4lib::fail(INT4_ERR_UNSUPPORTED, "int4_matmul: decode kernel cannot run this shape");
       size_t need = 0;
-      e = int4lib::launch_matmul_decode(x, t, packed, scales, K, group, M, N, y, workspace,
-                                        workspace_bytes, s, &need);
+      e = int4lib::launch_matmul_decode(x, t, packed, scales, zeros, ep, K, group, M, N, y,
+                                        workspace, workspace_bytes, s, &need);
       if (e == cudaErrorInvalidValue && need > 0) {
         char msg[200];
         std::snprintf(msg, sizeof msg,
@@ -208,12 +272,19 @@ int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, cons
     case INT4_PATH_PREFILL:
       if (!int4lib::prefill_supported(t, K, group, M, N, x, packed))
         return int4lib::fail(INT4_ERR_UNSUPPORTED, "int4_matmul: tensor-core kernel cannot run this shape");
-      e = int4lib::launch_matmul_prefill(x, t, packed, scales, K, group, M, N, y, s);
+      e = int4lib::launch_matmul_prefill(x, t, packed, scales, zeros, ep, K, group, M, N, y, s);
       break;
     default:
       return int4lib::fail(INT4_ERR_ARG, "int4_matmul: unknown path");
   }
   return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_matmul");
+}
+
+int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                     int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return int4_matmul_ex(x, x_dtype, packed, scales, nullptr, K, group, M, N, nullptr, 0, y, path,
+                        workspace, workspace_bytes, stream);
 }
 
 int int4_matmul(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,

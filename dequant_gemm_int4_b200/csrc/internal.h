@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace int4lib {
 
 enum class DType : int { F32 = 0, BF16 = 1, F16 = 2 };
@@ -22,13 +24,23 @@ cudaError_t launch_wait_timeout_selftest(uint32_t spins, cudaStream_t stream);
 // quantize.cu
 cudaError_t launch_quantize(const void* w, DType wt, int64_t N, int64_t K, int group,
                             uint8_t* packed, uint16_t* scales, cudaStream_t stream);
+// quantize_affine.cu: the asymmetric variant (unsigned codes, zero points).
+cudaError_t launch_quantize_affine(const void* w, DType wt, int64_t N, int64_t K, int group,
+                                   uint8_t* packed, uint16_t* scales, uint8_t* zeros,
+                                   cudaStream_t stream);
 // unpack.cu
 cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out,
                           cudaStream_t stream);
+// dequantize.cu: w_hat = q * s (zeros == nullptr) or (q - z) * s, rounded to
+// the output type.
+cudaError_t launch_dequantize(const uint8_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                              int64_t K, int group, int64_t N, void* out, DType ot,
+                              cudaStream_t stream);
 // matmul_simt.cu
 cudaError_t launch_matmul_simt(const void* x, DType xt, const uint8_t* packed,
-                               const uint16_t* scales, int64_t K, int group, int64_t M,
-                               int64_t N, float* y, cudaStream_t stream);
+                               const uint16_t* scales, const uint8_t* zeros, int64_t K, int group,
+                               int64_t M, int64_t N, const Epilogue& ep, float* y,
+                               cudaStream_t stream);
 // matmul_decode.cu
 bool decode_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                       const uint8_t* packed);
@@ -41,9 +53,10 @@ cudaError_t decode_workspace_size(DType xt, int64_t K, int group, int64_t M, int
 // before its first use, 256-byte aligned) must hold decode_workspace_size
 // bytes, else cudaErrorInvalidValue with *need set.
 cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
-                                 const uint16_t* scales, int64_t K, int group, int64_t M,
-                                 int64_t N, float* y, void* workspace, size_t workspace_bytes,
-                                 cudaStream_t stream, size_t* need);
+                                 const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
+                                 int64_t K, int group, int64_t M, int64_t N, float* y,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                                 size_t* need);
 // The same decode matmul with its scratch in the library's fixed device
 // array (no allocation).  cudaErrorInvalidValue with *need set: the array is
 // too small for this call.
@@ -58,8 +71,9 @@ cudaError_t reset_split_counters();
 bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                        const uint8_t* packed);
 cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
-                                  const uint16_t* scales, int64_t K, int group, int64_t M,
-                                  int64_t N, float* y, cudaStream_t stream);
+                                  const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
+                                  int64_t K, int group, int64_t M, int64_t N, float* y,
+                                  cudaStream_t stream);
 
 int num_sms();  // SM count of the current device (cached per device)
 

@@ -123,10 +123,13 @@ template <typename TX>
 struct Cvt;
 template <>
 struct Cvt<__nv_bfloat16> {
-  static constexpr uint32_t kMagic = 0x43084308u;
-  __device__ __forceinline__ static uint32_t sub(uint32_t a) {
+  static constexpr uint32_t kMagic = 0x43084308u;  // 128 + 8 in each half (the XOR flips the sign bit)
+  static constexpr uint32_t kBase = 0x43004300u;   // 128 in each half (unsigned codes)
+  // The subtrahend for unsigned codes with zero point z: 128 + z in each half.
+  __device__ __forceinline__ static uint32_t zero_bias(uint32_t z) { return (0x4300u + z) * 0x00010001u; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t a, uint32_t b = 0x43084308u) {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x43084308u));
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -140,10 +143,12 @@ struct Cvt<__nv_bfloat16> {
 };
 template <>
 struct Cvt<__half> {
-  static constexpr uint32_t kMagic = 0x64086408u;
-  __device__ __forceinline__ static uint32_t sub(uint32_t a) {
+  static constexpr uint32_t kMagic = 0x64086408u;  // 1024 + 8 in each half
+  static constexpr uint32_t kBase = 0x64006400u;   // 1024 in each half
+  __device__ __forceinline__ static uint32_t zero_bias(uint32_t z) { return (0x6400u + z) * 0x00010001u; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t a, uint32_t b = 0x64086408u) {
     uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x64086408u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
   }
   __device__ __forceinline__ static void mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -157,15 +162,19 @@ struct Cvt<__half> {
 };
 
 // Word w = 8 consecutive k (nibbles e0..e7 at bits 4i).  p[i] = (e_i, e_{i+4})
-// as bf16x2 / f16x2: ((w >> 4i) & 0x000F000F) ^ magic, minus the bias.
-template <typename TX>
-__device__ __forceinline__ void expand(uint32_t w, uint32_t (&p)[4]) {
+// as bf16x2 / f16x2: ((w >> 4i) & 0x000F000F) ^ magic, minus the bias.  For
+// unsigned codes (the asymmetric scheme, ASYM) the XOR leaves the nibble as
+// it is and `zb` = zero_bias(z) subtracts 128 + z (1024 + z), so p holds
+// q - z exactly.
+template <typename TX, bool ASYM = false>
+__device__ __forceinline__ void expand(uint32_t w, uint32_t (&p)[4], uint32_t zb = Cvt<TX>::kMagic) {
+  constexpr uint32_t kx = ASYM ? Cvt<TX>::kBase : Cvt<TX>::kMagic;
   const uint32_t v[4] = {w, w >> 4, w >> 8, w >> 12};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(v[i]), "r"(0x000F000Fu), "r"(Cvt<TX>::kMagic));
-    p[i] = Cvt<TX>::sub(r);
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(v[i]), "r"(0x000F000Fu), "r"(kx));
+    p[i] = Cvt<TX>::sub(r, ASYM ? zb : Cvt<TX>::kMagic);
   }
 }
 
@@ -254,10 +263,11 @@ struct DLayout {
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-template <typename TX, int NT, int GPB>
+template <typename TX, int NT, int GPB, bool ASYM>
 __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-    const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
+    const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
+    float* __restrict__ y, int64_t K, int group, int G, int M,
     int64_t N, int KB, int64_t U, int P, int64_t gran, float* __restrict__ partials,
     uint32_t* __restrict__ counters, uint32_t* status) {
   using L = DLayout<NT>;
@@ -377,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
       const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
       const int64_t row0 = r * kRowsPerCta;
       const uint16_t* sp[kTiles][2];
+      const uint8_t* zp[kTiles][2];
 #pragma unroll
       for (int t = 0; t < kTiles; ++t)
 #pragma unroll
@@ -384,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           int64_t gr = row0 + rg * 16 * kTiles + 16 * t + tile_row<GPB>(g) + 8 * h;
           if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
           sp[t][h] = scales + gr * G;
+          zp[t][h] = ASYM ? zeros + gr * G : nullptr;
         }
       float tot[kTiles][NT][4];
 #pragma unroll
@@ -436,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
         // are needed, as raw fp16 bits (two per register for group 64); group
         // 32 loads them at use, to stay within registers.
         uint32_t sraw[kTiles][2];
+        uint32_t zraw[kTiles][2];  // zero points of the block's groups, one byte each
         if (GPB <= 2) {
           const int gi0 = (GPB == 1) ? ((bpg == 1) ? kb : kb / bpg) : kb * 2;
 #pragma unroll
@@ -445,6 +458,20 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
               uint32_t r = (gi0 < G) ? __ldg(sp[t][h] + gi0) : 0u;
               if (GPB == 2) r |= (gi0 + 1 < G) ? static_cast<uint32_t>(__ldg(sp[t][h] + gi0 + 1)) << 16 : 0u;
               sraw[t][h] = r;
+            }
+        }
+        if (ASYM) {
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t r = 0u;
+#pragma unroll
+              for (int a = 0; a < GPB; ++a) {
+                const int gi = (GPB == 1) ? ((bpg == 1) ? kb : kb / bpg) : kb * GPB + a;
+                r |= (gi < G) ? static_cast<uint32_t>(__ldg(zp[t][h] + gi)) << (8 * a) : 0u;
+              }
+              zraw[t][h] = r;
             }
         }
         float acc[kTiles][NT][4];
@@ -467,8 +494,14 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
 #pragma unroll
           for (int t = 0; t < kTiles; ++t) {
             uint32_t pa[4], pb[4];
-            expand<TX>(wv[t][0][j], pa);
-            expand<TX>(wv[t][1][j], pb);
+            if (ASYM) {
+              const int a = (GPB == 1) ? 0 : (GPB == 2 ? (j >> 1) : j);  // the word's group in the block
+              expand<TX, true>(wv[t][0][j], pa, Cvt<TX>::zero_bias((zraw[t][0] >> (8 * a)) & 0xFFu));
+              expand<TX, true>(wv[t][1][j], pb, Cvt<TX>::zero_bias((zraw[t][1] >> (8 * a)) & 0xFFu));
+            } else {
+              expand<TX>(wv[t][0][j], pa);
+              expand<TX>(wv[t][1][j], pb);
+            }
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               Cvt<TX>::mma(acc[t][nt], pa[0], pb[0], pa[1], pb[1], xf[nt].x, xf[nt].y);
@@ -533,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
           const int tw = (e >> 7) / NT;  // rg * kTiles + t
           const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
           const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
-          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
         }
       }
       ptx::bar_sync(1, kConsumers * 32);  // red is rewritten by the next segment
@@ -570,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
             const int tw = (e >> 7) / NT;
             const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
             const int64_t row = row0 + tw * 16 + tile_row<GPB>(ln >> 2) + ((i < 2) ? 0 : 8);
-            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
           }
           if (cw == 0 && lane == 0) counters[p_first] = 0u;
         }
@@ -853,6 +886,14 @@ __device__ __forceinline__ bool record_flagged(uint32_t a) {
   return (f.x | f.y | f.z | f.w) != 0u;
 }
 
+// Bytes q - z (int8, in [-15, 15]) of the four unsigned codes held one per
+// byte in `q` (each 0..15), for zero point z (zz = z in every byte): with
+// q | 0x80 the per-byte subtraction cannot borrow (128 + q - z >= 113), and
+// flipping bit 7 back leaves the two's-complement q - z.
+__device__ __forceinline__ uint32_t affine_bytes(uint32_t q, uint32_t zz) {
+  return ((q | 0x80808080u) - zz) ^ 0x80808080u;
+}
+
 // One 128-k block (kb) of a flagged record, on the 16-bit warp MMA with x as
 // stored, read from global memory (L2 holds it): the nibbles are expanded to
 // bf16/fp16 and paired with x as in decode_kernel, so every product is exact
@@ -862,10 +903,11 @@ __device__ __forceinline__ bool record_flagged(uint32_t a) {
 // row, and the even lanes add them (times the scale) to their totals.  wr
 // holds words 4c .. 4c + 3 of rows g and g + 8 of each tile.  All 32 lanes
 // call it together.
-template <typename TX, int NP, int kTiles>
+template <typename TX, int NP, int kTiles, bool ASYM>
 __device__ __forceinline__ void block_fallback(const TX* __restrict__ x, int64_t K, int M, int kb,
                                                int g, int c, const uint4 (&wr)[kTiles][2],
                                                const float (&sa)[kTiles], const float (&sb)[kTiles],
+                                               const uint32_t (&za)[kTiles], const uint32_t (&zb)[kTiles],
                                                float (&tot)[kTiles][NP][2]) {
   constexpr int NTB = (2 * NP + 7) / 8;  // 16-bit MMA n-tiles (8 batch rows each)
   float acc[kTiles][NTB][4];
@@ -892,8 +934,8 @@ __device__ __forceinline__ void block_fallback(const TX* __restrict__ x, int64_t
       const uint32_t w0[4] = {wr[t][0].x, wr[t][0].y, wr[t][0].z, wr[t][0].w};
       const uint32_t w1[4] = {wr[t][1].x, wr[t][1].y, wr[t][1].z, wr[t][1].w};
       uint32_t pa[4], pb[4];
-      expand<TX>(w0[j], pa);
-      expand<TX>(w1[j], pb);
+      expand<TX, ASYM>(w0[j], pa, ASYM ? Cvt<TX>::zero_bias(za[t]) : Cvt<TX>::kMagic);
+      expand<TX, ASYM>(w1[j], pb, ASYM ? Cvt<TX>::zero_bias(zb[t]) : Cvt<TX>::kMagic);
 #pragma unroll
       for (int nb = 0; nb < NTB; ++nb) {
         Cvt<TX>::mma(acc[t][nb], pa[0], pb[0], pa[1], pb[1], xf[nb].x, xf[nb].y);
@@ -924,11 +966,12 @@ __device__ __forceinline__ void block_fallback(const TX* __restrict__ x, int64_t
 // decode_kernel.  Each stage carries the digit records of its two blocks:
 // converted in the CTA from the stage's x tile (FUSE), or one bulk copy of
 // the records x_digits_kernel wrote.
-template <typename TX, int NP, bool FUSE>
+template <typename TX, int NP, bool FUSE, bool ASYM>
 __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>::kMinBlocks) decode_i8_kernel(
     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
     const TX* __restrict__ x, const uint8_t* __restrict__ rec,
-    const uint16_t* __restrict__ scales, float* __restrict__ y, int64_t K, int group, int G, int M,
+    const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
+    float* __restrict__ y, int64_t K, int group, int G, int M,
     int64_t N, int KB, int64_t U, int P, int64_t gran, float* __restrict__ partials,
     uint32_t* __restrict__ counters, uint32_t* status) {
   using S = I8Shape<NP, FUSE>;
@@ -1095,7 +1138,8 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
     // weighs 2^16 more, which they fold into their scale.
     const uint32_t fofs = xrec + static_cast<uint32_t>(NP * kDigitTile + 4 * (c >> 1));
     const uint32_t flagofs = xrec + static_cast<uint32_t>(NP * kDigitTile + kRecFlags);
-    const float lane_mul = (c & 1) ? 65536.0f : 1.0f;
+    // Affine codes enter the MMA as q - z, not 16 q: 16 times the factor.
+    const float lane_mul = ((c & 1) ? 65536.0f : 1.0f) * (ASYM ? 16.0f : 1.0f);
     const int bpg = group / 128;
     int gs = 0;
     for (int64_t u = u_begin; u < u_end;) {
@@ -1104,6 +1148,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
       const int bhi = static_cast<int>((u_end - r * KB < KB) ? u_end - r * KB : KB);
       const int64_t row0 = r * kRowsPerCta;
       const uint16_t* sp[kTiles][2];
+      const uint8_t* zp[kTiles][2];
 #pragma unroll
       for (int t = 0; t < kTiles; ++t)
 #pragma unroll
@@ -1111,6 +1156,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
           int64_t gr = row0 + rg * 16 * kTiles + 16 * t + tile_row<1>(g) + 8 * h;
           if (gr >= N) gr = N - 1;  // never written; keeps the scale load in bounds
           sp[t][h] = scales + gr * G;
+          zp[t][h] = ASYM ? zeros + gr * G : nullptr;
         }
       float tot[kTiles][NP][2];
 #pragma unroll
@@ -1121,26 +1167,34 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
       // queue): a block's work is shorter than a load's latency.
       constexpr int kAhead = INT4_DECODE_I8_SCALE_AHEAD;
       uint16_t sraw[kAhead][kTiles][2];
-      auto load_scales = [&](int kb, uint16_t (&dst)[kTiles][2]) {
+      uint8_t zraw[kAhead][kTiles][2];
+      auto load_scales = [&](int kb, uint16_t (&dst)[kTiles][2], uint8_t (&zdst)[kTiles][2]) {
         const int gi = (bpg == 1) ? kb : kb / bpg;
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           dst[t][0] = __ldg(sp[t][0] + gi);
           dst[t][1] = __ldg(sp[t][1] + gi);
+          if (ASYM) {
+            zdst[t][0] = __ldg(zp[t][0] + gi);
+            zdst[t][1] = __ldg(zp[t][1] + gi);
+          }
         }
       };
 #pragma unroll
       for (int q = 0; q < kAhead; ++q)
-        if (blo + bs + q * kSK < bhi) load_scales(blo + bs + q * kSK, sraw[q]);
+        if (blo + bs + q * kSK < bhi) load_scales(blo + bs + q * kSK, sraw[q], zraw[q]);
       bool ok = true;
       for (int kb_stage = blo; kb_stage < bhi; kb_stage += kSK, ++gs) {
         const int s = gs % kStages;
         const int kb = kb_stage + bs;
         float sa[kTiles], sb[kTiles];
+        uint32_t za[kTiles], zb[kTiles];
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           sa[t] = f16_bits_to_float(sraw[0][t][0]);
           sb[t] = f16_bits_to_float(sraw[0][t][1]);
+          za[t] = ASYM ? zraw[0][t][0] : 0u;
+          zb[t] = ASYM ? zraw[0][t][1] : 0u;
         }
 #pragma unroll
         for (int q = 0; q + 1 < kAhead; ++q)
@@ -1148,8 +1202,10 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
           for (int t = 0; t < kTiles; ++t) {
             sraw[q][t][0] = sraw[q + 1][t][0];
             sraw[q][t][1] = sraw[q + 1][t][1];
+            zraw[q][t][0] = zraw[q + 1][t][0];
+            zraw[q][t][1] = zraw[q + 1][t][1];
           }
-        if (kb + kAhead * kSK < bhi) load_scales(kb + kAhead * kSK, sraw[kAhead - 1]);
+        if (kb + kAhead * kSK < bhi) load_scales(kb + kAhead * kSK, sraw[kAhead - 1], zraw[kAhead - 1]);
         ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&full[s]), (gs / kStages) & 1, wc));
         if (ok && S::kFuse)
           ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&ready[s]), (gs / kStages) & 1, wc));
@@ -1166,7 +1222,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
           if (__builtin_expect(record_flagged<NP>(st + flagofs), 0)) {
             // Some batch row's x does not fit its digits exactly: the whole
             // block runs on the 16-bit MMA with x as stored.
-            block_fallback<TX, NP, kTiles>(x, K, M, kb, g, c, wr, sa, sb, tot);
+            block_fallback<TX, NP, kTiles, ASYM>(x, K, M, kb, g, c, wr, sa, sb, za, zb, tot);
           } else {
             // A fragments of the block's four MMAs (k32 each): rows g and
             // g + 8, low nibbles (shifted) in k slots 0..15, high nibbles in
@@ -1178,10 +1234,18 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
               const uint32_t w1[4] = {wr[t][1].x, wr[t][1].y, wr[t][1].z, wr[t][1].w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                a[t][j][0] = (w0[j] << 4) & 0xF0F0F0F0u;
-                a[t][j][1] = (w1[j] << 4) & 0xF0F0F0F0u;
-                a[t][j][2] = w0[j] & 0xF0F0F0F0u;
-                a[t][j][3] = w1[j] & 0xF0F0F0F0u;
+                if (ASYM) {
+                  const uint32_t zza = za[t] * 0x01010101u, zzb = zb[t] * 0x01010101u;
+                  a[t][j][0] = affine_bytes(w0[j] & 0x0F0F0F0Fu, zza);
+                  a[t][j][1] = affine_bytes(w1[j] & 0x0F0F0F0Fu, zzb);
+                  a[t][j][2] = affine_bytes((w0[j] >> 4) & 0x0F0F0F0Fu, zza);
+                  a[t][j][3] = affine_bytes((w1[j] >> 4) & 0x0F0F0F0Fu, zzb);
+                } else {
+                  a[t][j][0] = (w0[j] << 4) & 0xF0F0F0F0u;
+                  a[t][j][1] = (w1[j] << 4) & 0xF0F0F0F0u;
+                  a[t][j][2] = w0[j] & 0xF0F0F0F0u;
+                  a[t][j][3] = w1[j] & 0xF0F0F0F0u;
+                }
               }
             }
             float sal[kTiles], sbl[kTiles];
@@ -1240,7 +1304,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
           }
           const int m = 2 * nt + mp;
           const int64_t row = row0 + tw * 16 + tile_row<1>(gq) + 8 * hh;
-          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+          if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
         }
       }
       ptx::bar_sync(1, kConsumers * 32);
@@ -1270,7 +1334,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
             const int m = 2 * (rest_i % NP) + mp;
             const int tw = rest_i / NP;
             const int64_t row = row0 + tw * 16 + tile_row<1>(gq) + 8 * hh;
-            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+            if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
           }
           if (cw == 0 && lane == 0) counters[p_first] = 0u;
         }
@@ -1310,10 +1374,11 @@ EncodeTiledFn encode_fn() {
 constexpr int kSmallWarps = 8;
 constexpr int kSmallCtasPerSm = 3;
 
-template <typename TX, int NT>
+template <typename TX, int NT, bool ASYM>
 __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_small_kernel(
     const TX* __restrict__ x, const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
-    float* __restrict__ y, int64_t K, int group, int G, int M, int64_t N, int KB) {
+    const uint8_t* __restrict__ zeros, Epilogue ep, float* __restrict__ y, int64_t K, int group,
+    int G, int M, int64_t N, int KB) {
   __shared__ float red[kSmallWarps * NT * 4 * 32];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -1326,6 +1391,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
   const uint8_t* wb = packed + rb * Kp + 16 * c;
   const uint16_t* sa_row = scales + ra * G;
   const uint16_t* sb_row = scales + rb * G;
+  const uint8_t* za_row = ASYM ? zeros + ra * G : nullptr;
+  const uint8_t* zb_row = ASYM ? zeros + rb * G : nullptr;
   float tot[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -1336,6 +1403,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
     // kStep blocks per step, all loads issued before any use.
     uint4 ua[kStep], ub[kStep], xf4[kStep][4][NT];
     uint32_t sraw[kStep][2];
+    uint32_t zraw[kStep][2];
 #pragma unroll
     for (int q = 0; q < kStep; ++q) {
       const int kb = kb0 + kSmallWarps * q;
@@ -1346,6 +1414,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
       const int gi = static_cast<int>(static_cast<int64_t>(kc) * 128 / group);
       sraw[q][0] = __ldg(sa_row + gi);
       sraw[q][1] = __ldg(sb_row + gi);
+      zraw[q][0] = ASYM ? __ldg(za_row + gi) : 0u;
+      zraw[q][1] = ASYM ? __ldg(zb_row + gi) : 0u;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int n = g + 8 * nt;
@@ -1365,11 +1435,13 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+      const uint32_t zba = ASYM ? Cvt<TX>::zero_bias(zraw[q][0]) : Cvt<TX>::kMagic;
+      const uint32_t zbb = ASYM ? Cvt<TX>::zero_bias(zraw[q][1]) : Cvt<TX>::kMagic;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t pa[4], pb[4];
-        expand<TX>(wva[j], pa);
-        expand<TX>(wvb[j], pb);
+        expand<TX, ASYM>(wva[j], pa, zba);
+        expand<TX, ASYM>(wvb[j], pb, zbb);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const uint4 xf = pair_x(xf4[q][j][nt]);
@@ -1404,22 +1476,23 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
     const int nt = e >> 7;
     const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
     const int64_t row = row0 + (ln >> 2) + ((i < 2) ? 0 : 8);
-    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = sum;
+    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
   }
 }
 
-template <typename TX>
-cudaError_t launch_small(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                         int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+template <typename TX, bool ASYM>
+cudaError_t launch_small(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                         const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                         int64_t N, float* y, cudaStream_t stream) {
   const int G = static_cast<int>((K + group - 1) / group);
   const int KB = static_cast<int>((K + 127) / 128);
   const unsigned grid = static_cast<unsigned>((N + 15) / 16);
   if (M <= 8)
-    decode_small_kernel<TX, 1><<<grid, kSmallWarps * 32, 0, stream>>>(x, packed, scales, y, K, group, G,
-                                                                       static_cast<int>(M), N, KB);
+    decode_small_kernel<TX, 1, ASYM><<<grid, kSmallWarps * 32, 0, stream>>>(
+        x, packed, scales, zeros, ep, y, K, group, G, static_cast<int>(M), N, KB);
   else
-    decode_small_kernel<TX, 2><<<grid, kSmallWarps * 32, 0, stream>>>(x, packed, scales, y, K, group, G,
-                                                                       static_cast<int>(M), N, KB);
+    decode_small_kernel<TX, 2, ASYM><<<grid, kSmallWarps * 32, 0, stream>>>(
+        x, packed, scales, zeros, ep, y, K, group, G, static_cast<int>(M), N, KB);
   return cudaGetLastError();
 }
 
@@ -1588,11 +1661,14 @@ void plan_runs(int occ, int rows, int64_t K, int64_t N, bool may_split, DecodePl
   pl->split = last_split;
 }
 
-// Arguments of one decode call.
+// Arguments of one decode call (zeros: the asymmetric scheme's zero points,
+// or nullptr for the symmetric scheme).
 struct DecodeArgs {
   const void* x;
   const uint8_t* packed;
   const uint16_t* scales;
+  const uint8_t* zeros;
+  Epilogue ep;
   int64_t K;
   int group;
   int64_t M;
@@ -1607,7 +1683,7 @@ bool fits(const DecodeNeed& n, const DecodeScratch* sc) {
          n.records <= sc->record_cap;
 }
 
-template <typename TX, int NT, int GPB>
+template <typename TX, int NT, int GPB, bool ASYM>
 cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& pl, float* partials,
                           uint32_t* counters) {
   using L = DLayout<NT>;
@@ -1641,20 +1717,20 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& pl, float* part
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  decode_kernel<TX, NT, GPB><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, a.stream>>>(
-      tw, tx, a.scales, a.y, a.K, a.group, G, static_cast<int>(a.M), a.N, pl.KB, pl.U,
+  decode_kernel<TX, NT, GPB, ASYM><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, a.stream>>>(
+      tw, tx, a.scales, a.zeros, a.ep, a.y, a.K, a.group, G, static_cast<int>(a.M), a.N, pl.KB, pl.U,
       static_cast<int>(pl.P), pl.gran, partials, counters, status);
   return cudaGetLastError();
 }
 
 // The 16-bit decode kernel: plan, scratch need and (if `launch`) the launch.
-template <typename TX, int NT, int GPB>
+template <typename TX, int NT, int GPB, bool ASYM>
 cudaError_t run_bf(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
                    bool launch) {
   constexpr int kPer = kRowGroups * Tiles<NT>::kTiles * NT * 4 * 32;  // outputs of a tile
   static std::atomic<int> occ_cache[64];
   int occ = 0;
-  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_kernel<TX, NT, GPB>),
+  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_kernel<TX, NT, GPB, ASYM>),
                                    kThreads, DLayout<NT>::kAlloc, occ_cache, &occ);
   if (e != cudaSuccess) return e;
   DecodePlan pl;
@@ -1667,11 +1743,11 @@ cudaError_t run_bf(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, D
   *need = n;
   if (!launch) return cudaSuccess;
   if (!fits(n, sc)) return cudaErrorInvalidValue;
-  return launch_decode<TX, NT, GPB>(a, pl, pl.split ? sc->partials : nullptr,
+  return launch_decode<TX, NT, GPB, ASYM>(a, pl, pl.split ? sc->partials : nullptr,
                                     pl.split ? sc->counters : nullptr);
 }
 
-template <typename TX, int NP, bool FUSE>
+template <typename TX, int NP, bool FUSE, bool ASYM>
 cudaError_t launch_decode_i8(const DecodeArgs& a, const DecodePlan& pl, float* partials,
                              uint32_t* counters, uint8_t* records) {
   using S = I8Shape<NP, FUSE>;
@@ -1732,20 +1808,21 @@ cudaError_t launch_decode_i8(const DecodeArgs& a, const DecodePlan& pl, float* p
   cfg.stream = a.stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE>, tw, tx, x,
-                            static_cast<const uint8_t*>(records), a.scales, a.y, a.K, a.group, G,
+  return cudaLaunchKernelEx(&cfg, decode_i8_kernel<TX, NP, FUSE, ASYM>, tw, tx, x,
+                            static_cast<const uint8_t*>(records), a.scales, a.zeros, a.ep, a.y, a.K,
+                            a.group, G,
                             static_cast<int>(a.M), a.N, pl.KB, pl.U, static_cast<int>(pl.P),
                             pl.gran, partials, counters, status);
 }
 
 // The integer decode kernel: plan, scratch need and (if `launch`) the launch.
-template <typename TX, int NP, bool FUSE>
+template <typename TX, int NP, bool FUSE, bool ASYM>
 cudaError_t run_i8(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
                    bool launch) {
   using S = I8Shape<NP, FUSE>;
   static std::atomic<int> occ_cache[64];
   int occ = 0;
-  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_i8_kernel<TX, NP, FUSE>),
+  cudaError_t e = kernel_occupancy(reinterpret_cast<const void*>(decode_i8_kernel<TX, NP, FUSE, ASYM>),
                                    S::kThreads, S::kAlloc, occ_cache, &occ);
   if (e != cudaSuccess) return e;
   DecodePlan pl;
@@ -1759,7 +1836,7 @@ cudaError_t run_i8(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, D
   *need = n;
   if (!launch) return cudaSuccess;
   if (!fits(n, sc)) return cudaErrorInvalidValue;
-  return launch_decode_i8<TX, NP, FUSE>(a, pl, pl.split ? sc->partials : nullptr,
+  return launch_decode_i8<TX, NP, FUSE, ASYM>(a, pl, pl.split ? sc->partials : nullptr,
                                         pl.split ? sc->counters : nullptr,
                                         S::kFuse ? nullptr : sc->records);
 }
@@ -1768,38 +1845,42 @@ cudaError_t run_i8(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, D
 // (the split schedule and, at M > 2 with groups of whole 128-k blocks, the
 // integer kernel with digit records); without it the runs cover whole tiles
 // and such batches take the 16-bit kernel.
-template <typename TX>
+template <typename TX, bool ASYM>
 cudaError_t run_decode(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
                        bool launch) {
   if (small_applies(a.K, a.group, a.N)) {
     *need = DecodeNeed{};
     if (!launch) return cudaSuccess;
-    return launch_small(static_cast<const TX*>(a.x), a.packed, a.scales, a.K, a.group, a.M, a.N,
-                        a.y, a.stream);
+    return launch_small<TX, ASYM>(static_cast<const TX*>(a.x), a.packed, a.scales, a.zeros, a.ep,
+                                  a.K, a.group, a.M, a.N, a.y, a.stream);
   }
   if (a.group % 128 == 0) {
-    if (a.M <= kFuseMaxM) return run_i8<TX, 1, true>(a, scratch, sc, need, launch);
+    if (a.M <= kFuseMaxM) return run_i8<TX, 1, true, ASYM>(a, scratch, sc, need, launch);
     if (!scratch) {
-      if (a.M <= 8) return run_bf<TX, 1, 1>(a, scratch, sc, need, launch);
-      return run_bf<TX, 2, 1>(a, scratch, sc, need, launch);
+      if (a.M <= 8) return run_bf<TX, 1, 1, ASYM>(a, scratch, sc, need, launch);
+      return run_bf<TX, 2, 1, ASYM>(a, scratch, sc, need, launch);
     }
-    if (a.M <= 2) return run_i8<TX, 1, false>(a, scratch, sc, need, launch);
-    if (a.M <= 4) return run_i8<TX, 2, false>(a, scratch, sc, need, launch);
-    if (a.M <= 8) return run_i8<TX, 4, false>(a, scratch, sc, need, launch);
-    return run_i8<TX, 8, false>(a, scratch, sc, need, launch);
+    if (a.M <= 2) return run_i8<TX, 1, false, ASYM>(a, scratch, sc, need, launch);
+    if (a.M <= 4) return run_i8<TX, 2, false, ASYM>(a, scratch, sc, need, launch);
+    if (a.M <= 8) return run_i8<TX, 4, false, ASYM>(a, scratch, sc, need, launch);
+    return run_i8<TX, 8, false, ASYM>(a, scratch, sc, need, launch);
   }
   if (a.M <= 8) {
-    if (a.group == 64) return run_bf<TX, 1, 2>(a, scratch, sc, need, launch);
-    return run_bf<TX, 1, 4>(a, scratch, sc, need, launch);
+    if (a.group == 64) return run_bf<TX, 1, 2, ASYM>(a, scratch, sc, need, launch);
+    return run_bf<TX, 1, 4, ASYM>(a, scratch, sc, need, launch);
   }
-  if (a.group == 64) return run_bf<TX, 2, 2>(a, scratch, sc, need, launch);
-  return run_bf<TX, 2, 4>(a, scratch, sc, need, launch);
+  if (a.group == 64) return run_bf<TX, 2, 2, ASYM>(a, scratch, sc, need, launch);
+  return run_bf<TX, 2, 4, ASYM>(a, scratch, sc, need, launch);
 }
 
 cudaError_t run_decode_any(DType xt, const DecodeArgs& a, bool scratch, const DecodeScratch* sc,
                            DecodeNeed* need, bool launch) {
-  if (xt == DType::BF16) return run_decode<__nv_bfloat16>(a, scratch, sc, need, launch);
-  return run_decode<__half>(a, scratch, sc, need, launch);
+  const bool asym = a.zeros != nullptr;
+  if (xt == DType::BF16)
+    return asym ? run_decode<__nv_bfloat16, true>(a, scratch, sc, need, launch)
+                : run_decode<__nv_bfloat16, false>(a, scratch, sc, need, launch);
+  return asym ? run_decode<__half, true>(a, scratch, sc, need, launch)
+              : run_decode<__half, false>(a, scratch, sc, need, launch);
 }
 
 size_t need_total_bytes(const DecodeNeed& n) {
@@ -1824,7 +1905,8 @@ size_t decode_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 cudaError_t decode_workspace_size(DType xt, int64_t K, int group, int64_t M, int64_t N,
                                   size_t* bytes) {
-  const DecodeArgs a{nullptr, nullptr, nullptr, K, group, M, N, nullptr, nullptr};
+  // The need does not depend on the scheme or the epilogue.
+  const DecodeArgs a{nullptr, nullptr, nullptr, nullptr, Epilogue{}, K, group, M, N, nullptr, nullptr};
   DecodeNeed n;
   const cudaError_t e = run_decode_any(xt, a, true, nullptr, &n, false);
   if (e != cudaSuccess) return e;
@@ -1833,10 +1915,11 @@ cudaError_t decode_workspace_size(DType xt, int64_t K, int group, int64_t M, int
 }
 
 cudaError_t launch_matmul_decode(const void* x, DType xt, const uint8_t* packed,
-                                 const uint16_t* scales, int64_t K, int group, int64_t M,
-                                 int64_t N, float* y, void* workspace, size_t workspace_bytes_given,
-                                 cudaStream_t stream, size_t* need) {
-  const DecodeArgs a{x, packed, scales, K, group, M, N, y, stream};
+                                 const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
+                                 int64_t K, int group, int64_t M, int64_t N, float* y,
+                                 void* workspace, size_t workspace_bytes_given, cudaStream_t stream,
+                                 size_t* need) {
+  const DecodeArgs a{x, packed, scales, zeros, ep, K, group, M, N, y, stream};
   if (workspace == nullptr && workspace_bytes_given == 0) {
     DecodeNeed n;
     return run_decode_any(xt, a, false, nullptr, &n, true);
@@ -1859,7 +1942,7 @@ cudaError_t launch_matmul_decode_noalloc(const void* x, DType xt, const uint8_t*
   float* base = nullptr;
   cudaError_t e = noalloc_scratch(&base);
   if (e != cudaSuccess) return e;
-  const DecodeArgs a{x, packed, scales, K, group, M, N, y, stream};
+  const DecodeArgs a{x, packed, scales, nullptr, Epilogue{}, K, group, M, N, y, stream};
   const DecodeScratch sc = noalloc_regions(base);
   DecodeNeed n;
   e = run_decode_any(xt, a, true, &sc, &n, true);

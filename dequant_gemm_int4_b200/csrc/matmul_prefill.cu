@@ -40,6 +40,14 @@ constexpr int kBN = 128;      // weight rows per tile (MMA M)
 constexpr int kKS = 64;       // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = 4;
 constexpr int kThreads = 512;
+// Raster: the grid walks runs of kGroupM activation-row tiles, all weight-row
+// tiles of a run before the next (activation tile fastest).  A run's x tiles
+// (8 x 4 MB at K = 8192) stay in L2 while the weight tiles stream past, and
+// each weight tile is read once per run instead of once per x tile.
+#ifndef INT4_PREFILL_GROUP_M
+#define INT4_PREFILL_GROUP_M 8
+#endif
+constexpr int kGroupM = INT4_PREFILL_GROUP_M;
 constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
 
 struct Barriers {
@@ -80,25 +88,32 @@ struct Nib;
 template <>
 struct Nib<__nv_bfloat16> {
   static constexpr uint32_t kMagic = 0x43084308u;  // bf16 128 in each half, nibble sign bit flipped
-  __device__ __forceinline__ static uint32_t sub(uint32_t a) {
+  static constexpr uint32_t kBase = 0x43004300u;   // bf16 128 in each half (unsigned codes)
+  __device__ __forceinline__ static uint32_t zero_bias(uint32_t z) { return (0x4300u + z) * 0x00010001u; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t a, uint32_t b) {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x43084308u));  // - 136
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));  // - 136, or - (128 + z)
     return d;
   }
 };
 template <>
 struct Nib<__half> {
   static constexpr uint32_t kMagic = 0x64086408u;  // fp16 1024 in each half
-  __device__ __forceinline__ static uint32_t sub(uint32_t a) {
+  static constexpr uint32_t kBase = 0x64006400u;
+  __device__ __forceinline__ static uint32_t zero_bias(uint32_t z) { return (0x6400u + z) * 0x00010001u; }
+  __device__ __forceinline__ static uint32_t sub(uint32_t a, uint32_t b) {
     uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(0x64086408u));  // - 1032
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));  // - 1032, or - (1024 + z)
     return d;
   }
 };
 
-// 4 packed bytes (8 consecutive k) -> 8 bf16/fp16 in natural k order.
-template <typename TX>
-__device__ __forceinline__ uint4 expand8(uint32_t w) {
+// 4 packed bytes (8 consecutive k) -> 8 bf16/fp16 in natural k order: q
+// (two's-complement nibbles), or q - z for unsigned codes (ASYM, zb =
+// zero_bias(z)).
+template <typename TX, bool ASYM>
+__device__ __forceinline__ uint4 expand8(uint32_t w, uint32_t zb) {
+  constexpr uint32_t kx = ASYM ? Nib<TX>::kBase : Nib<TX>::kMagic;
   const uint32_t ws = w >> 4;
   uint32_t o[4];
 #pragma unroll
@@ -107,8 +122,8 @@ __device__ __forceinline__ uint4 expand8(uint32_t w) {
     const uint32_t sel = static_cast<uint32_t>(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12));
     const uint32_t t = __byte_perm(w, ws, sel);
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(t), "r"(0x000F000Fu), "r"(Nib<TX>::kMagic));
-    o[j] = Nib<TX>::sub(r);
+    asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(t), "r"(0x000F000Fu), "r"(kx));
+    o[j] = Nib<TX>::sub(r, ASYM ? zb : Nib<TX>::kMagic);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -144,11 +159,11 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <typename TX, int BM>
+template <typename TX, int BM, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_p,
-    const uint16_t* __restrict__ scales, float* __restrict__ y, int M, int N, int K, int group,
-    int G, uint32_t* status) {
+    const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
+    float* __restrict__ y, int M, int N, int K, int group, int G, uint32_t* status) {
   using L = Layout<BM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -159,8 +174,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN;
-  const int m0 = blockIdx.y * BM;
+  int n0, m0;
+  {
+    const int num_n = (N + kBN - 1) / kBN, num_m = (M + BM - 1) / BM;
+    const int per_run = kGroupM * num_n;
+    const int run = static_cast<int>(blockIdx.x) / per_run;
+    const int first_m = run * kGroupM;
+    const int gm = (num_m - first_m < kGroupM) ? num_m - first_m : kGroupM;
+    const int r = static_cast<int>(blockIdx.x) - run * per_run;
+    n0 = (r / gm) * kBN;
+    m0 = (first_m + r % gm) * BM;
+  }
   const int nstages = (K + kKS - 1) / kKS;
 
   const uint32_t sA = ptx::smem_u32(smem + L::offA);
@@ -255,9 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int t = threadIdx.x - 128;
     const int swz = t & 7;
     const int first = (t >> 2) & 1;  // rotates the two 16-byte reads to avoid bank conflicts
+    const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G : nullptr;
     for (int it = 0; it < nstages; ++it) {
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1;
+      // The stage's zero point (a stage lies inside one group).
+      const uint32_t zb = ASYM ? Nib<TX>::zero_bias(__ldg(zrow + (it * kKS) / group)) : 0u;
       if (!wait_bar(bar(&bars->full_tma[s]), ph, wc)) break;
       const uint32_t prow = sP + s * L::kP + t * 32;
       const uint4 va = ptx::lds128(prow + 16 * first);
@@ -267,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
       const uint32_t arow = sA + s * L::kA + t * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) ptx::sts128(arow + ((c ^ swz) << 4), expand8<TX>(wds[c]));
+      for (int c = 0; c < 8; ++c) ptx::sts128(arow + ((c ^ swz) << 4), expand8<TX, ASYM>(wds[c], zb));
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(bar(&bars->full_a[s]));
     }
@@ -312,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
 #pragma unroll
       for (int j = 0; j < kCols; ++j) {
         const int m = mbase + j;
-        if (m < M) y[static_cast<int64_t>(m) * N + n] = acc[j];
+        if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j], n);
       }
     }
   }
@@ -343,9 +370,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <typename TX, int BM>
-cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales, int64_t K,
-                      int group, int64_t M, int64_t N, float* y, cudaStream_t stream) {
+template <typename TX, int BM, bool ASYM>
+cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                      const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                      int64_t N, float* y, cudaStream_t stream) {
   using L = Layout<BM>;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
@@ -376,12 +404,12 @@ cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = prefill_kernel<TX, BM>;
+  auto kern = prefill_kernel<TX, BM, ASYM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN), static_cast<unsigned>((M + BM - 1) / BM));
+  const dim3 grid(static_cast<unsigned>(((N + kBN - 1) / kBN) * ((M + BM - 1) / BM)));
   const int G = static_cast<int>((K + group - 1) / group);
-  kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, y, static_cast<int>(M),
+  kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, zeros, ep, y, static_cast<int>(M),
                                               static_cast<int>(N), static_cast<int>(K), group, G,
                                               status);
   return cudaGetLastError();
@@ -397,18 +425,28 @@ bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, con
   if (K > (1LL << 30) || M > (1LL << 30) || N > (1LL << 30)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0 || reinterpret_cast<uintptr_t>(packed) % 16 != 0)
     return false;
-  if ((M + 255) / 256 > 65535) return false;
+  if (((N + kBN - 1) / kBN) * ((M + 255) / 256) > 0x7FFFFFFFLL) return false;
   return true;
 }
 
+template <typename TX>
+static cudaError_t launch_prefill_tx(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                                     const uint8_t* zeros, const Epilogue& ep, int64_t K, int group,
+                                     int64_t M, int64_t N, float* y, cudaStream_t stream) {
+  if (zeros != nullptr)
+    return launch_bm<TX, 256, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  return launch_bm<TX, 256, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, stream);
+}
+
 cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
-                                  const uint16_t* scales, int64_t K, int group, int64_t M,
-                                  int64_t N, float* y, cudaStream_t stream) {
+                                  const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
+                                  int64_t K, int group, int64_t M, int64_t N, float* y,
+                                  cudaStream_t stream) {
   if (xt == DType::BF16)
-    return launch_bm<__nv_bfloat16, 256>(static_cast<const __nv_bfloat16*>(x), packed, scales, K,
-                                         group, M, N, y, stream);
-  return launch_bm<__half, 256>(static_cast<const __half*>(x), packed, scales, K, group, M, N, y,
-                                stream);
+    return launch_prefill_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, zeros, ep, K,
+                             group, M, N, y, stream);
+  return launch_prefill_tx(static_cast<const __half*>(x), packed, scales, zeros, ep, K, group, M, N,
+                           y, stream);
 }
 
 }  // namespace int4lib

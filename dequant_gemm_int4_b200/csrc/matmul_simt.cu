@@ -15,7 +15,10 @@
 //
 // This is the correctness kernel for shapes and dtypes the tensor-core kernels
 // do not take; it tiles 64 weight rows x 16 activation rows per block with a
-// 32-wide K step staged through shared memory.
+// 32-wide K step staged through shared memory.  For the asymmetric scheme of
+// the page "Build a Blockwise INT4 Inference Engine" (step 2) the staged codes
+// are unsigned and the group's zero point is subtracted at use (q - z is an
+// exact small integer too); the optional bias and ReLU apply at the store.
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,11 +31,11 @@ constexpr int BM = 16;   // activation rows per block
 constexpr int BK = 32;   // k per shared-memory step
 constexpr int TM = 4;    // activation rows per thread (BM / (256 / BN))
 
-template <typename TX>
+template <typename TX, bool ASYM>
 __global__ void __launch_bounds__(256) matmul_simt_kernel(
     const TX* __restrict__ x, const uint8_t* __restrict__ packed,
-    const uint16_t* __restrict__ scales, int64_t K, int group, int G, int64_t M, int64_t N,
-    float* __restrict__ y) {
+    const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, int64_t K, int group,
+    int G, int64_t M, int64_t N, Epilogue ep, float* __restrict__ y) {
   __shared__ float xs[BM][BK + 1];
   __shared__ int8_t qs[BN][BK + 4];
 
@@ -52,6 +55,7 @@ __global__ void __launch_bounds__(256) matmul_simt_kernel(
     part[i] = 0.0f;
   }
   float cur_scale = 0.0f;
+  float cur_zero = 0.0f;
 
   for (int64_t k0 = 0; k0 < K; k0 += BK) {
     // Stage x[m0 : m0+16, k0 : k0+32] as fp32 (zeros outside the matrix).
@@ -70,9 +74,14 @@ __global__ void __launch_bounds__(256) matmul_simt_kernel(
         const int64_t k = k0 + c0 + j;  // even
         uint32_t byte = 0;
         if (nr < N && k < K) byte = __ldg(packed + nr * Kp + (k >> 1));
-        qs[r][c0 + j] = static_cast<int8_t>(static_cast<int32_t>(byte << 28) >> 28);
-        qs[r][c0 + j + 1] =
-            (k + 1 < K) ? static_cast<int8_t>(static_cast<int32_t>(byte << 24) >> 28) : 0;
+        if (ASYM) {
+          qs[r][c0 + j] = static_cast<int8_t>(byte & 0xFu);
+          qs[r][c0 + j + 1] = (k + 1 < K) ? static_cast<int8_t>(byte >> 4) : 0;
+        } else {
+          qs[r][c0 + j] = static_cast<int8_t>(static_cast<int32_t>(byte << 28) >> 28);
+          qs[r][c0 + j + 1] =
+              (k + 1 < K) ? static_cast<int8_t>(static_cast<int32_t>(byte << 24) >> 28) : 0;
+        }
       }
     }
     __syncthreads();
@@ -88,8 +97,9 @@ __global__ void __launch_bounds__(256) matmul_simt_kernel(
           part[i] = 0.0f;
         }
         cur_scale = (n < N) ? f16_bits_to_float(__ldg(scales + n * G + k / group)) : 0.0f;
+        if (ASYM) cur_zero = (n < N) ? static_cast<float>(__ldg(zeros + n * G + k / group)) : 0.0f;
       }
-      const float q = static_cast<float>(qs[tn][c]);
+      const float q = static_cast<float>(qs[tn][c]) - cur_zero;  // exact
 #pragma unroll
       for (int i = 0; i < TM; ++i) part[i] = fmaf(xs[tm * TM + i][c], q, part[i]);
     }
@@ -99,15 +109,28 @@ __global__ void __launch_bounds__(256) matmul_simt_kernel(
   for (int i = 0; i < TM; ++i) {
     acc[i] += static_cast<double>(part[i]) * static_cast<double>(cur_scale);
     const int64_t m = m0 + tm * TM + i;
-    if (m < M && n < N) y[m * N + n] = static_cast<float>(acc[i]);
+    if (m < M && n < N) y[m * N + n] = ep.apply(static_cast<float>(acc[i]), n);
   }
+}
+
+template <typename TX>
+void launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales, const uint8_t* zeros,
+               int64_t K, int group, int G, int64_t M, int64_t N, const Epilogue& ep, float* y,
+               dim3 grid, cudaStream_t stream) {
+  if (zeros != nullptr)
+    matmul_simt_kernel<TX, true><<<grid, 256, 0, stream>>>(x, packed, scales, zeros, K, group, G, M,
+                                                           N, ep, y);
+  else
+    matmul_simt_kernel<TX, false><<<grid, 256, 0, stream>>>(x, packed, scales, nullptr, K, group, G,
+                                                            M, N, ep, y);
 }
 
 }  // namespace
 
 cudaError_t launch_matmul_simt(const void* x, DType xt, const uint8_t* packed,
-                               const uint16_t* scales, int64_t K, int group, int64_t M,
-                               int64_t N, float* y, cudaStream_t stream) {
+                               const uint16_t* scales, const uint8_t* zeros, int64_t K, int group,
+                               int64_t M, int64_t N, const Epilogue& ep, float* y,
+                               cudaStream_t stream) {
   const int G = static_cast<int>((K + group - 1) / group);
   const int64_t gx = (N + BN - 1) / BN;
   const int64_t gy = (M + BM - 1) / BM;
@@ -115,16 +138,16 @@ cudaError_t launch_matmul_simt(const void* x, DType xt, const uint8_t* packed,
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
   switch (xt) {
     case DType::F32:
-      matmul_simt_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(x), packed,
-                                                          scales, K, group, G, M, N, y);
+      launch_tx(static_cast<const float*>(x), packed, scales, zeros, K, group, G, M, N, ep, y, grid,
+                stream);
       break;
     case DType::BF16:
-      matmul_simt_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(x), packed, scales, K, group, G, M, N, y);
+      launch_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, zeros, K, group, G, M, N, ep,
+                y, grid, stream);
       break;
     case DType::F16:
-      matmul_simt_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(x), packed,
-                                                           scales, K, group, G, M, N, y);
+      launch_tx(static_cast<const __half*>(x), packed, scales, zeros, K, group, G, M, N, ep, y,
+                grid, stream);
       break;
   }
   return cudaGetLastError();

@@ -1,0 +1,256 @@
+// Asymmetric (affine) 4-bit quantization with per-group zero points (sm_100a).
+//
+// Follows step 2 of the page "Build a Blockwise INT4 Inference Engine": per
+// row and K-group, scale = (max - min) / 15, zero point = clip(round(-min /
+// scale), 0, 15), q = clip(round(w / scale + zero point), 0, 15).  Layout as
+// the symmetric scheme's: the unsigned code of element 2j in the low nibble
+// of byte j (zero pad nibble for odd K), fp16 scales [N, G], and uint8 zero
+// points [N, G].  Rounding convention, in the page's order of operations:
+// d = fp32(max - min), s = fp16_RNE(fp32(d / 15)); with sf = fp32(s),
+// z = clip(rint(fp32(-min / sf)), 0, 15) and q = clip(rint(fp32(fp32(w / sf)
+// + z)), 0, 15), every division an IEEE fp32 division and rint half to even.
+// A zero scale (a constant group, or a range that underflows fp16) codes the
+// group as q = 0, z = 0.
+//
+// HBM-bound like the symmetric quantizer: a warp takes a window of 256
+// consecutive weights of one row (8 per lane, one 16- or 32-byte load),
+// reduces the group's min and max with shuffles over its group / 8 lanes and
+// stores 4 packed bytes per lane; any other shape takes a two-kernel general
+// path (scales and zero points, then one thread per packed byte).
+#include "common.cuh"
+#include "internal.h"
+
+namespace int4lib {
+
+namespace {
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+    v[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<__half>(const __half* p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = f16_bits_to_float(w[i] & 0xFFFFu);
+    v[2 * i + 1] = f16_bits_to_float(w[i] >> 16);
+  }
+}
+
+struct Affine {
+  float sf;       // the scale, read back from fp16
+  float zf;       // the zero point as a float (an integer 0..15)
+  uint32_t bits;  // the fp16 scale
+  uint32_t z;
+};
+
+// Scale and zero point of a group with extremes mn <= mx.
+__device__ __forceinline__ Affine affine_params(float mn, float mx) {
+  Affine a;
+  const float d = __fsub_rn(mx, mn);
+  const float s32 = __fdiv_rn(d, 15.0f);
+  a.bits = __half_as_ushort(__float2half_rn(s32));
+  a.sf = f16_bits_to_float(a.bits);
+  a.zf = 0.0f;
+  if (a.sf != 0.0f) {
+    const float t = rintf(__fdiv_rn(-mn, a.sf));
+    a.zf = fminf(fmaxf(t, 0.0f), 15.0f);
+  }
+  a.z = static_cast<uint32_t>(a.zf);
+  return a;
+}
+
+__device__ __forceinline__ Affine affine_from_stored(uint16_t bits, uint8_t z) {
+  Affine a;
+  a.bits = bits;
+  a.sf = f16_bits_to_float(bits);
+  a.z = z;
+  a.zf = static_cast<float>(z);
+  return a;
+}
+
+// The unsigned code of v: clip(rint(fp32(fp32(v / sf) + z)), 0, 15); 0 when
+// the scale is 0.
+__device__ __forceinline__ uint32_t affine_code(float v, const Affine& a) {
+  if (a.sf == 0.0f) return 0u;
+  const float u = __fadd_rn(__fdiv_rn(v, a.sf), a.zf);
+  return static_cast<uint32_t>(fminf(fmaxf(rintf(u), 0.0f), 15.0f));
+}
+
+// Fast path: K % 8 == 0, group = 8 LPG with LPG a power of two <= 32, w
+// 16-byte aligned, packed 4-byte aligned.  Windows (256 weights of one row)
+// are numbered row-major; each warp takes a contiguous range of them.
+template <typename T, int LPG>
+__global__ void __launch_bounds__(256) quantize_affine_window_kernel(
+    const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
+    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  const int64_t wbeg = warp * per;
+  const int64_t wend = (wbeg + per < total_windows) ? wbeg + per : total_windows;
+  if (wbeg >= wend) return;
+  int64_t row = wbeg / windows_per_row;
+  int64_t win = wbeg - row * windows_per_row;
+  for (int64_t wi = wbeg; wi < wend; ++wi) {
+    const int64_t k0 = win * 256 + 8 * lane;
+    const bool active = k0 < K;
+    float v[8];
+    if (active) {
+      load8<T>(w + row * K + k0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    float mn = active ? v[0] : __int_as_float(0x7F800000);   // +inf
+    float mx = active ? v[0] : __int_as_float(0xFF800000);   // -inf
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+      mn = fminf(mn, active ? v[i] : mn);
+      mx = fmaxf(mx, active ? v[i] : mx);
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (active) {
+      const Affine a = affine_params(mn, mx);
+      uint32_t word = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word |= affine_code(v[i], a) << (4 * i);
+      *reinterpret_cast<uint32_t*>(packed + row * (K >> 1) + (k0 >> 1)) = word;
+      if ((lane & (LPG - 1)) == 0) {
+        const int64_t gi = row * G + k0 / (8 * LPG);
+        scales[gi] = static_cast<uint16_t>(a.bits);
+        zeros[gi] = static_cast<uint8_t>(a.z);
+      }
+    }
+    if (++win == windows_per_row) {
+      win = 0;
+      ++row;
+    }
+  }
+}
+
+// General path, step 1: one thread per (row, group).
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_affine_params_kernel(
+    const T* __restrict__ w, int64_t N, int64_t K, int group, int G, uint16_t* __restrict__ scales,
+    uint8_t* __restrict__ zeros) {
+  const int64_t total = N * G;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx / G;
+    const int64_t k0 = (idx - n * G) * group;
+    const int64_t k1 = (k0 + group < K) ? k0 + group : K;
+    float mn = Elem<T>::load(w + n * K + k0), mx = mn;
+    for (int64_t k = k0 + 1; k < k1; ++k) {
+      const float v = Elem<T>::load(w + n * K + k);
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+    const Affine a = affine_params(mn, mx);
+    scales[idx] = static_cast<uint16_t>(a.bits);
+    zeros[idx] = static_cast<uint8_t>(a.z);
+  }
+}
+
+// General path, step 2: one thread per packed byte, from the stored scale
+// and zero point.
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_affine_pack_kernel(
+    const T* __restrict__ w, int64_t N, int64_t K, int group, int G,
+    const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros,
+    uint8_t* __restrict__ packed) {
+  const int64_t Kp = (K + 1) >> 1;
+  const int64_t total = N * Kp;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = idx / Kp;
+    const int64_t k = 2 * (idx - n * Kp);
+    const int64_t g0 = n * G + k / group;
+    uint32_t byte = affine_code(Elem<T>::load(w + n * K + k), affine_from_stored(scales[g0], zeros[g0]));
+    if (k + 1 < K) {
+      const int64_t g1 = n * G + (k + 1) / group;
+      byte |= affine_code(Elem<T>::load(w + n * K + k + 1), affine_from_stored(scales[g1], zeros[g1]))
+              << 4;
+    }
+    packed[idx] = static_cast<uint8_t>(byte);
+  }
+}
+
+template <typename T, int LPG>
+cudaError_t launch_window(const T* w, int64_t N, int64_t K, int G, uint8_t* packed,
+                          uint16_t* scales, uint8_t* zeros, cudaStream_t stream) {
+  const int64_t wpr = (K + 255) / 256;
+  const int64_t total = N * wpr;
+  const int grid = resident_grid(quantize_affine_window_kernel<T, LPG>, (total + 7) / 8);
+  quantize_affine_window_kernel<T, LPG><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed,
+                                                                  scales, zeros);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* packed,
+                         uint16_t* scales, uint8_t* zeros, cudaStream_t stream) {
+  const int G = static_cast<int>((K + group - 1) / group);
+  const bool fast = K % 8 == 0 && reinterpret_cast<uintptr_t>(w) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(packed) % 4 == 0;
+  if (fast) {
+    switch (group) {
+      case 8: return launch_window<T, 1>(w, N, K, G, packed, scales, zeros, stream);
+      case 16: return launch_window<T, 2>(w, N, K, G, packed, scales, zeros, stream);
+      case 32: return launch_window<T, 4>(w, N, K, G, packed, scales, zeros, stream);
+      case 64: return launch_window<T, 8>(w, N, K, G, packed, scales, zeros, stream);
+      case 128: return launch_window<T, 16>(w, N, K, G, packed, scales, zeros, stream);
+      case 256: return launch_window<T, 32>(w, N, K, G, packed, scales, zeros, stream);
+      default: break;
+    }
+  }
+  quantize_affine_params_kernel<T><<<resident_grid(quantize_affine_params_kernel<T>, (N * G + 255) / 256),
+                                     256, 0, stream>>>(w, N, K, group, G, scales, zeros);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t Kp = (K + 1) / 2;
+  quantize_affine_pack_kernel<T><<<resident_grid(quantize_affine_pack_kernel<T>, (N * Kp + 255) / 256),
+                                   256, 0, stream>>>(w, N, K, group, G, scales, zeros, packed);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_affine(const void* w, DType wt, int64_t N, int64_t K, int group,
+                                   uint8_t* packed, uint16_t* scales, uint8_t* zeros,
+                                   cudaStream_t stream) {
+  switch (wt) {
+    case DType::F32:
+      return launch_typed(static_cast<const float*>(w), N, K, group, packed, scales, zeros, stream);
+    case DType::BF16:
+      return launch_typed(static_cast<const __nv_bfloat16*>(w), N, K, group, packed, scales, zeros,
+                          stream);
+    case DType::F16:
+      return launch_typed(static_cast<const __half*>(w), N, K, group, packed, scales, zeros, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace int4lib

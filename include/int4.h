@@ -103,6 +103,28 @@ int int4_quantize(const void* w, int32_t w_dtype, int64_t N, int64_t K, int32_t 
 int int4_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* out, void* stream);
 
 /*
+ * int4_dequantize - the dequantized weights w_hat = q * s, as a dense matrix.
+ *
+ * Pages: "Building a pure-Python INT4 transformer weight quantizer with
+ * block-wise per-channel scaling", section 5 (w_hat = q * s per block), and
+ * the drill, whose hidden suite checks the matmul "against a full
+ * dequantization"; "Quantizing a Language Model From Scratch" runs its model
+ * on such fake-quantized weights.  out[n, k] = RNE_out( q[n, k] * s[n, k /
+ * group] ): the product is exact in fp32 and rounded once, to nearest even,
+ * to out_dtype (fp32 output is exact; fp16 output overflows to +-inf where
+ * |q s| > 65504).  Bit-exact.  It is the first half of the unfused
+ * dequantize-then-GEMM design the fused int4_matmul replaces; it is not used
+ * by int4_matmul.
+ *
+ * packed    [N, ceil(K/2)] device input; any alignment.
+ * scales    [N, ceil(K/group)] fp16 bits; 2-byte aligned.
+ * out       [N, K] device output of out_dtype; alignment: its element size.
+ * out_dtype INT4_DTYPE_F32 / _BF16 / _F16.
+ */
+int int4_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t K, int32_t group,
+                    int64_t N, void* out, int32_t out_dtype, void* stream);
+
+/*
  * int4_matmul - weight-only dequantizing matmul y = x @ dequantize(W)^T.
  *
  * Page: the drill's int4_matmul(x, packed, scales, K, group) -> float32
@@ -199,6 +221,68 @@ int int4_matmul_ws(const void* x, int32_t x_dtype, const uint8_t* packed, const 
 int int4_matmul_path(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
                      int64_t K, int32_t group, int64_t M, int64_t N, float* y, int32_t path,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * int4_quantize_affine - the asymmetric variant: per-group scale and zero
+ * point, unsigned codes.
+ *
+ * Page: "Build a Blockwise INT4 Inference Engine", step 2 (blockwise
+ * quantization with per-group scales and zero-points); "Quantizing a
+ * Language Model From Scratch" (affine quantization, x' = S (x_q - Z)).  For
+ * row n and group g (the real columns of [g*group, (g+1)*group)):
+ *   mn, mx = min and max of w over the group (exact)
+ *   s      = fp16_RNE( fp32( fp32(mx - mn) / 15 ) )      (IEEE fp32 ops)
+ *   z      = clamp( rint_half_even( fp32(-mn / fp32(s)) ), 0, 15 )
+ *   q[n,k] = clamp( rint_half_even( fp32( fp32(w / fp32(s)) + z ) ), 0, 15 )
+ *   s == 0 (a constant group, or a range that underflows fp16): q = 0, z = 0
+ *   packed[n, j] = q[n,2j] | (q[n,2j+1] << 4) (unsigned nibbles, element 2j
+ *   in the low nibble as in int4_quantize; an odd K pads a zero nibble)
+ * Bit-exact under this convention.  w_hat = (q - z) s; a zero weight in a
+ * group whose range spans 0 is coded exactly.  Precondition: w finite with
+ * (mx - mn) / 15 below 65520 in every group.
+ *
+ * w [N, K] (w_dtype, aligned to its element size); packed [N, ceil(K/2)];
+ * scales [N, G] fp16 bits (2-byte aligned); zeros [N, G] uint8.
+ */
+int int4_quantize_affine(const void* w, int32_t w_dtype, int64_t N, int64_t K, int32_t group,
+                         uint8_t* packed, uint16_t* scales, uint8_t* zeros, void* stream);
+
+/*
+ * int4_dequantize_affine - w_hat = (q - z) * s rounded once, to nearest even,
+ * to out_dtype (int4_dequantize for the asymmetric variant; the same
+ * arguments plus the zero points [N, G] uint8).
+ */
+int int4_dequantize_affine(const uint8_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                           int64_t K, int32_t group, int64_t N, void* out, int32_t out_dtype,
+                           void* stream);
+
+/* Epilogue flags of int4_matmul_ex. */
+#define INT4_EPI_RELU 1  /* y = max(y, 0) after the bias (NaN stays NaN) */
+
+/*
+ * int4_matmul_ex - int4_matmul_path with the asymmetric scheme and a fused
+ * epilogue.
+ *
+ * Pages: "Build a Blockwise INT4 Inference Engine", step 3 (the fused kernel
+ * computes D = relu(A @ dequantize(Q)) with dequantize = (q - zp) * scale)
+ * and step 4 (the layer computes x @ W_dq^T + bias, then ReLU).
+ *   y[m, n] = epilogue( sum_g s[n, g] * sum_{k in g} x[m, k] * (q[n, k] - z[n, g]) )
+ *   epilogue(v) = v + bias[n] (if bias), then max(., 0) (if INT4_EPI_RELU)
+ * zeros   NULL: the symmetric scheme of int4_matmul (two's-complement codes,
+ *         z = 0); else [N, ceil(K/group)] uint8 zero points and unsigned
+ *         codes from int4_quantize_affine.  Every kernel subtracts z from the
+ *         codes before the products, so each group's sum stays exact where
+ *         int4_matmul's does, and the accuracy bound of int4_matmul holds with
+ *         w_hat = (q - z) s.
+ * bias    NULL or [N] fp32, 4-byte aligned; added in fp32 (one rounding).
+ * flags   0 or INT4_EPI_RELU.
+ * The other arguments, the kernel choice, the workspace rules and the
+ * stream ordering are those of int4_matmul_path.
+ */
+int int4_matmul_ex(const void* x, int32_t x_dtype, const uint8_t* packed, const uint16_t* scales,
+                   const uint8_t* zeros, int64_t K, int32_t group, int64_t M, int64_t N,
+                   const float* bias, int32_t flags, float* y, int32_t path, void* workspace,
+                   size_t workspace_bytes, void* stream);
 
 /* Allocation-free decode matmul.  The pages have no counterpart: this entry
  * exists for callers that must not allocate device memory during the call,

@@ -608,3 +608,50 @@ def test_decode_split_scratch_grows_between_shapes(M):
         cols = np.unique(np.random.default_rng(N).integers(0, N, 256))
         assert_matmul_close(y1, x, packed, scales, K, 128, TOL_HALF, cols=cols)
     assert q4.device_status() == q4.OK
+
+
+# ---------------------------------------------------------------------------
+# int4_dequantize: w_hat = q * s rounded once to the output type
+# ---------------------------------------------------------------------------
+def _oracle_w_hat_as(packed, scales, K, group, dtype):
+    """The oracle's exact w_hat (fp64; every value is exact in fp32), rounded to
+    nearest even into `dtype` by the library-independent casts of NumPy and
+    PyTorch on the CPU."""
+    w64 = oracle.dequantize_int4(packed.cpu().numpy(), scales.cpu().numpy(), K, group)
+    w32 = w64.astype(np.float32)
+    assert np.array_equal(w32.astype(np.float64), w64)
+    return torch.from_numpy(w32).to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("N, K, group", [
+    (16, 259, 128), (64, 4096, 128), (33, 1024, 32), (7, 96, 48), (5, 1001, 7), (300, 768, 64),
+    (2, 16, 16), (1, 1, 1),
+])
+def test_dequantize_bit_exact(dtype, N, K, group):
+    packed, scales, _ = _quantized(N, K, group, seed=N * K, dist="student_t3", zero_group_frac=0.05)
+    w_hat = q4.dequantize_int4(packed, scales, K, group, dtype=dtype)
+    assert w_hat.dtype == dtype and tuple(w_hat.shape) == (N, K)
+    ref = _oracle_w_hat_as(packed, scales, K, group, dtype)
+    got = w_hat.cpu()
+    assert torch.equal(got.view(torch.int16 if dtype != torch.float32 else torch.int32),
+                       ref.view(torch.int16 if dtype != torch.float32 else torch.int32))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_dequantize_every_code_and_extreme_scales(dtype):
+    """All 256 bytes (every code pair, -8 included) under scales spanning the
+    fp16 range: subnormal scales, 1, and 65504 (where -8 * s overflows fp16
+    to -inf), on the fast and the general kernel."""
+    sc = [2.0 ** -24, 2.0 ** -14 * 1.5, 0.1, 1.0, 3.0, 1024.0, 65504.0, 0.0]
+    for K, group in [(512, 64), (510, 51)]:       # flat kernel; general kernel
+        N = len(sc)
+        packed = (torch.arange(N * ((K + 1) // 2)) % 256).to(torch.uint8).view(N, -1).to(DEV)
+        G = -(-K // group)
+        scales = torch.tensor(sc, dtype=torch.float16)[:, None].repeat(1, G).to(DEV)
+        w_hat = q4.dequantize_int4(packed, scales, K, group, dtype=dtype).cpu()
+        ref = _oracle_w_hat_as(packed, scales, K, group, dtype)
+        itype = torch.int16 if dtype != torch.float32 else torch.int32
+        assert torch.equal(w_hat.view(itype), ref.view(itype))
+        if dtype == torch.float16:
+            assert bool(torch.isinf(w_hat[6]).any())

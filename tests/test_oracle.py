@@ -25,34 +25,7 @@ def _load(name):
         return json.load(f)
 
 
-# ---------------------------------------------------------------------------
-# Exact rational rounding to a binary floating-point format (IEEE-754
-# round-to-nearest, ties-to-even), written from the definition.  It is the
-# independent route used below to check NumPy's fp32 division and its
-# fp32 -> fp16 cast inside the oracle.
-# ---------------------------------------------------------------------------
-FP32 = (24, -126, 127)   # significand bits (with the hidden bit), emin, emax
-FP16 = (11, -14, 15)
-
-
-def round_to_format(value: Fraction, fmt) -> Fraction:
-    mant, emin, emax = fmt
-    if value == 0:
-        return Fraction(0)
-    sign = -1 if value < 0 else 1
-    a = abs(value)
-    e = a.numerator.bit_length() - a.denominator.bit_length()
-    while Fraction(2) ** e > a:
-        e -= 1
-    while Fraction(2) ** (e + 1) <= a:
-        e += 1
-    e = max(e, emin)                       # subnormals share emin's quantum
-    quantum = Fraction(2) ** (e - mant + 1)
-    r = round(a / quantum)                 # Fraction rounding: half to even
-    val = r * quantum
-    if val >= Fraction(2) ** (emax + 1):
-        return Fraction(sign) * Fraction(10**400)   # stands for infinity
-    return sign * val
+from exact_fp import FP16, FP32, round_to_format  # noqa: E402
 
 
 def exact_scale(m: float) -> float:
