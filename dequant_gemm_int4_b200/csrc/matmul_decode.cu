@@ -100,6 +100,9 @@ namespace {
 #ifndef INT4_DECODE_I8_SCALE_AHEAD
 #define INT4_DECODE_I8_SCALE_AHEAD 1
 #endif
+#ifndef INT4_DECODE_L2_AHEAD
+#define INT4_DECODE_L2_AHEAD 0  // integer kernel: stages beyond the ring whose weights are prefetched into L2
+#endif
 constexpr int kSK = INT4_DECODE_SK;                // 128-wide K blocks per stage (even)
 constexpr int kFuseMaxM = INT4_DECODE_I8_FUSE_MAX_M;  // batch rows the in-kernel x conversion serves
 constexpr int kSub = kSK / 2;                      // 256-k sub-tiles per stage (one copy each)
@@ -702,17 +705,6 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const float (&v)[8]) {
   return mb;
 }
 
-// Whether x 2^p is an integer, i.e. whether the lowest set bit of x's
-// significand sits at or above 2^-p (x finite).
-__device__ __forceinline__ bool digits_exact(float xv, int p) {
-  const uint32_t b = __float_as_uint(xv) & 0x7FFFFFFFu;
-  if (b == 0u) return true;
-  const int E = static_cast<int>(b >> 23);
-  const uint32_t sig = E != 0 ? ((b & 0x7FFFFFu) | 0x800000u) : b;
-  const int lsb = (E != 0 ? E : 1) - 150 + (__ffs(static_cast<int>(sig)) - 1);  // x = sig 2^(..)
-  return lsb + p >= 0;
-}
-
 // The digits of one word of a block: ev[i] / od[i] hold digit i of the
 // word's even / odd k (one byte each, k order), f the block's factor
 // 2^(e-33), and `inexact` whether some value of the word is not an integer
@@ -740,11 +732,14 @@ __device__ __forceinline__ void word_digits(const float (&v)[8], uint32_t amax_b
     const float s2 = __uint_as_float(static_cast<uint32_t>(p2 + 127) << 23);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int vi = __float2int_rn((v[i] * s1) * s2);
+      // t = x 2^p: exact unless it underflows, which can only happen for p < 0
+      // and leaves |t| < 2^-126, never a non-zero integer (hence the guard).
+      const float t = (v[i] * s1) * s2;
+      const int vi = __float2int_rn(t);
       // Balanced base-256 digits: the bytes of v + 0x808080 with the low three
       // flipped back by 128.
       dd[i] = (static_cast<uint32_t>(vi) + 0x808080u) ^ 0x808080u;
-      inexact |= !digits_exact(v[i], p);
+      inexact |= (rintf(t) != t) | ((t == 0.0f) & (v[i] != 0.0f));
     }
     f = __uint_as_float(static_cast<uint32_t>(e - 33 + 127) << 23);
   }
@@ -1078,6 +1073,30 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
     if (lane == 0) {
       int gs = 0;
       bool ok = true;
+      // A second cursor over the run, INT4_DECODE_L2_AHEAD stages beyond the
+      // ring (the first kStages stages were prefetched before the dependency
+      // wait): each issued stage asks L2 to prefetch the weights of that
+      // later stage, more bytes in flight without more shared memory.
+      constexpr int kAheadL2 = INT4_DECODE_L2_AHEAD;
+      int64_t pu = u_begin, pr = u_begin / KB;
+      int pkb = static_cast<int>(u_begin - pr * KB);
+      int pbhi = static_cast<int>((u_end - pr * KB < KB) ? u_end - pr * KB : KB);
+      auto pf_advance = [&]() {
+        pkb += kSK;
+        if (pkb >= pbhi) {
+          pu = pr * KB + pbhi;
+          pr = pu / KB;
+          pkb = static_cast<int>(pu - pr * KB);
+          pbhi = static_cast<int>((u_end - pr * KB < KB) ? u_end - pr * KB : KB);
+        }
+      };
+      if (kAheadL2 > 0) {
+        for (int j = 0; j < kStages && pu < u_end; ++j) pf_advance();   // prefetched at the start
+        for (int j = 0; j < kAheadL2 - 1 && pu < u_end; ++j) {
+          ptx::tma_prefetch_2d(&tm_w, pkb * 64, static_cast<int32_t>(pr * kRowsPerCta));
+          pf_advance();
+        }
+      }
       for (int64_t u = u_begin; ok && u < u_end;) {
         const int64_t r = u / KB;
         const int blo = static_cast<int>(u - r * KB);
@@ -1085,6 +1104,10 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
         const int32_t row0 = static_cast<int32_t>(r * kRowsPerCta);
         for (int kb = blo; kb < bhi; kb += kSK, ++gs) {
           const int s = gs % kStages;
+          if (kAheadL2 > 0 && pu < u_end) {
+            ptx::tma_prefetch_2d(&tm_w, pkb * 64, static_cast<int32_t>(pr * kRowsPerCta));
+            pf_advance();
+          }
           if (!wait_bar(ptx::smem_u32(&empty[s]), ((gs / kStages) & 1) ^ 1u, wc)) {
             ok = false;
             break;
@@ -1219,6 +1242,21 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
             wr[t][0] = ptx::lds128(st + wofs[t][0]);
             wr[t][1] = ptx::lds128(st + wofs[t][1]);
           }
+          // At NP == 1 the block's digit fragments and factors are loaded
+          // with the weights and the flags, before the test that branches on
+          // the flags, so that all of these loads are in flight together.
+          constexpr bool kHoist = NP == 1;
+          constexpr int NPH = kHoist ? NP : 1;
+          uint4 hb01[NPH], hb23[NPH];
+          float hfct[NPH];
+          if (kHoist) {
+#pragma unroll
+            for (int nt = 0; nt < NPH; ++nt) {
+              hb01[nt] = ptx::lds128(st + bofs[0] + nt * kDigitTile);
+              hb23[nt] = ptx::lds128(st + bofs[1] + nt * kDigitTile);
+              hfct[nt] = __uint_as_float(ptx::lds32(st + fofs + nt * 8));
+            }
+          }
           if (__builtin_expect(record_flagged<NP>(st + flagofs), 0)) {
             // Some batch row's x does not fit its digits exactly: the whole
             // block runs on the 16-bit MMA with x as stored.
@@ -1256,9 +1294,9 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
             }
 #pragma unroll
             for (int nt = 0; nt < NP; ++nt) {
-              const uint4 b01 = ptx::lds128(st + bofs[0] + nt * kDigitTile);
-              const uint4 b23 = ptx::lds128(st + bofs[1] + nt * kDigitTile);
-              const float fct = __uint_as_float(ptx::lds32(st + fofs + nt * 8));
+              const uint4 b01 = kHoist ? hb01[kHoist ? nt : 0] : ptx::lds128(st + bofs[0] + nt * kDigitTile);
+              const uint4 b23 = kHoist ? hb23[kHoist ? nt : 0] : ptx::lds128(st + bofs[1] + nt * kDigitTile);
+              const float fct = kHoist ? hfct[kHoist ? nt : 0] : __uint_as_float(ptx::lds32(st + fofs + nt * 8));
 #pragma unroll
               for (int t = 0; t < kTiles; ++t) {
                 int acc[4] = {0, 0, 0, 0};

@@ -5,25 +5,41 @@
 // dequantizing matmul" (problem statement), computed one K group at a time
 // with the group's scale applied to each output before the fp32 running sum.
 //
-// One CTA computes a 128 (weight rows n) x BM (activation rows m) tile of y^T
-// with tcgen05 MMAs (kind::f16, fp32 accumulation in tensor memory):
-//   warp 0      TMA producer: per 64-wide K stage, the packed weights
-//               [128 rows x 32 bytes] and x [BM rows x 64] (128-byte swizzle)
+// A persistent CTA per SM walks output tiles of 128 weight rows (n) x 192
+// activation rows (m), computed with tcgen05 MMAs (kind::f16, fp32
+// accumulation in tensor memory) whose A operand -- the dequantized weights --
+// is read from tensor memory, not shared memory:
+//   warp 0      TMA producer: per 64-wide K stage, x [192 rows x 64] (128-byte
+//               swizzle, the MMA's B operand) and the packed weights
+//               [128 rows x 32 bytes], into a 4-stage shared-memory ring
 //   warps 4-7   dequantizers: thread t expands weight row t of the stage from
 //               nibbles to bf16/fp16 (exact: 128 + u or 1024 + u minus 136 or
-//               1032) into the A tile, K-major with the 128-byte swizzle
-//   warp 1      MMA issuer: D_g = A_g * X_g^T into one of two TMEM partial
-//               buffers (128 lanes x BM columns), one buffer per K group
-//   warps 8-15  epilogue: for every group, load the group's partial from TMEM,
-//               multiply by s[n, g] (one scale per TMEM lane = weight row) and
-//               add into fp32 registers; finally store y.
-// TMEM lane = weight row n, so the per-(column, group) scale of the page is a
-// single register per thread.  Stages flow through full/empty mbarriers; the
-// two TMEM partial buffers let the tensor core run group g+1 while the
-// epilogue drains group g.  Every wait is bounded in time: a wait that gives
-// up sets an abort flag and the status word, every role leaves its loop,
-// outstanding copies and MMAs are drained (again with a bound) and TMEM is
-// freed before the CTA exits.
+//               1032, or minus 128 + z for the asymmetric scheme's unsigned
+//               codes) and stores it with tcgen05.st into TMEM lane t, one of
+//               four 32-column A stages
+//   warp 1      MMA issuer: D_g = A_g * X_g^T, 16 k per MMA, into one of two
+//               TMEM accumulators (128 lanes x 192 columns), one per K group;
+//               a group may span stages (group 128) or share one (group 32)
+//   warps 8-15  epilogue: per group, load the group's accumulator from TMEM,
+//               multiply by s[n, g] (TMEM lane = weight row: one scale per
+//               thread) and add into fp32 registers (packed FMAs); at the end
+//               of a tile, add the bias, apply ReLU and store y.
+// TMEM: columns [0, 384) the two accumulators, [384, 512) the A stages.
+// Shared memory then carries only x (written by TMA, read by the MMA) and the
+// packed bytes, about 14 KB per 16-k MMA step against 25 KB with A staged in
+// shared memory; with one MMA of 128 x 192 x 16 every 96 cycles that is the
+// difference between shared-memory bandwidth (128 B per cycle) binding below
+// two thirds of the tensor rate and binding near nine tenths of it.  The two
+// accumulators let the tensor core run group g + 1 (or the next tile's first
+// group) while the epilogue drains group g or stores a finished tile.
+//
+// Tiles are visited in runs of kGroupM activation tiles, all weight tiles of
+// a run before the next, so a run's x tiles stay in L2 while the weight tiles
+// stream past (each weight tile is read from DRAM once per run).
+//
+// Every wait is bounded in time: a wait that gives up sets an abort flag and
+// the status word, every role leaves its loops, outstanding copies and MMAs
+// are drained (again with a bound) and TMEM is freed before the CTA exits.
 #include <cuda.h>
 
 #include <mutex>
@@ -36,50 +52,49 @@ namespace int4lib {
 
 namespace {
 
-constexpr int kBN = 128;      // weight rows per tile (MMA M)
+constexpr int kBN = 128;      // weight rows per tile (MMA M, TMEM lanes)
+constexpr int kBM = 192;      // activation rows per tile (MMA N)
 constexpr int kKS = 64;       // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = 4;
 constexpr int kThreads = 512;
-// Raster: the grid walks runs of kGroupM activation-row tiles, all weight-row
-// tiles of a run before the next (activation tile fastest).  A run's x tiles
-// (8 x 4 MB at K = 8192) stay in L2 while the weight tiles stream past, and
-// each weight tile is read once per run instead of once per x tile.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColA = 2 * kBM;          // first column of the A stages
+constexpr uint32_t kColsA = kKS / 2;         // 32-bit columns per A stage
+static_assert(kColA + kStages * kColsA <= kTmemCols, "accumulators and A stages fit TMEM");
+constexpr int kEpiCols = kBM / 2;            // accumulator columns per epilogue thread
+constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
 #ifndef INT4_PREFILL_GROUP_M
 #define INT4_PREFILL_GROUP_M 8
 #endif
-constexpr int kGroupM = INT4_PREFILL_GROUP_M;
-constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
+constexpr int kGroupM = INT4_PREFILL_GROUP_M;  // activation tiles per raster run
 
 struct Barriers {
-  uint64_t full_tma[kStages];   // TMA bytes of stage s landed
-  uint64_t full_a[kStages];     // dequantized A tile of stage s written
-  uint64_t empty[kStages];      // MMAs reading stage s finished
-  uint64_t tmem_full[2];        // group partial in TMEM buffer b complete
-  uint64_t tmem_empty[2];       // epilogue finished reading buffer b
+  uint64_t full[kStages];       // TMA bytes of stage s landed
+  uint64_t afull[kStages];      // dequantized A of stage s written to TMEM
+  uint64_t empty[kStages];      // MMAs reading stage s (x and A) finished
+  uint64_t tmem_full[2];        // group accumulator b complete
+  uint64_t tmem_empty[2];       // epilogue finished reading accumulator b
   uint64_t drain;               // abort path: all issued MMAs finished
 };
 
-template <int BM>
 struct Layout {
-  static constexpr int kA = kBN * kKS * 2;  // 16 KB
-  static constexpr int kX = BM * kKS * 2;   // 32 KB at BM = 256
+  static constexpr int kX = kBM * kKS * 2;  // 24 KB
   static constexpr int kP = kBN * kKS / 2;  // 4 KB
-  static constexpr int offA = 0;
-  static constexpr int offX = offA + kStages * kA;
+  static constexpr int offX = 0;
   static constexpr int offP = offX + kStages * kX;
   static constexpr int offBar = offP + kStages * kP;
   static constexpr int offMisc = offBar + static_cast<int>(sizeof(Barriers));
   static constexpr int kBytes = offMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
-  static constexpr uint32_t kTmemCols = 2 * BM;
 };
+static_assert(Layout::kX % 1024 == 0, "x stages keep the 1024-byte swizzle alignment");
 
 // Instruction descriptor, kind::f16: D fp32, A/B bf16 (1) or fp16 (0),
-// both K-major, N = BM, M = 128.
-template <typename TX, int BM>
+// both K-major, N = kBM, M = kBN.
+template <typename TX>
 __device__ __forceinline__ constexpr uint32_t make_idesc() {
   constexpr uint32_t ab = std::is_same<TX, __nv_bfloat16>::value ? 1u : 0u;
-  return (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(BM >> 3) << 17) |
+  return (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(kBM >> 3) << 17) |
          (static_cast<uint32_t>(kBN >> 4) << 24);
 }
 
@@ -108,14 +123,13 @@ struct Nib<__half> {
   }
 };
 
-// 4 packed bytes (8 consecutive k) -> 8 bf16/fp16 in natural k order: q
-// (two's-complement nibbles), or q - z for unsigned codes (ASYM, zb =
-// zero_bias(z)).
+// 4 packed bytes (8 consecutive k) -> 8 bf16/fp16 in natural k order, two per
+// 32-bit word (the lower k in the low half): q (two's-complement nibbles), or
+// q - z for unsigned codes (ASYM, zb = zero_bias(z)).
 template <typename TX, bool ASYM>
-__device__ __forceinline__ uint4 expand8(uint32_t w, uint32_t zb) {
+__device__ __forceinline__ void expand8(uint32_t w, uint32_t zb, uint32_t* o) {
   constexpr uint32_t kx = ASYM ? Nib<TX>::kBase : Nib<TX>::kMagic;
   const uint32_t ws = w >> 4;
-  uint32_t o[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     // byte j low nibble -> bits 0..3, byte j high nibble -> bits 16..19
@@ -125,7 +139,6 @@ __device__ __forceinline__ uint4 expand8(uint32_t w, uint32_t zb) {
     asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(r) : "r"(t), "r"(0x000F000Fu), "r"(kx));
     o[j] = Nib<TX>::sub(r, ASYM ? zb : Nib<TX>::kMagic);
   }
-  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 struct WaitCtx {
@@ -159,12 +172,23 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <typename TX, int BM, bool ASYM>
+// Origin (first weight row, first activation row) of tile T in the raster.
+__device__ __forceinline__ void tile_origin(int T, int num_n, int num_m, int& n0, int& m0) {
+  const int per_run = kGroupM * num_n;
+  const int run = T / per_run;
+  const int first_m = run * kGroupM;
+  const int gm = (num_m - first_m < kGroupM) ? num_m - first_m : kGroupM;
+  const int r = T - run * per_run;
+  n0 = (r / gm) * kBN;
+  m0 = (first_m + r % gm) * kBM;
+}
+
+template <typename TX, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_p,
     const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
     float* __restrict__ y, int M, int N, int K, int group, int G, uint32_t* status) {
-  using L = Layout<BM>;
+  using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -174,28 +198,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int n0, m0;
-  {
-    const int num_n = (N + kBN - 1) / kBN, num_m = (M + BM - 1) / BM;
-    const int per_run = kGroupM * num_n;
-    const int run = static_cast<int>(blockIdx.x) / per_run;
-    const int first_m = run * kGroupM;
-    const int gm = (num_m - first_m < kGroupM) ? num_m - first_m : kGroupM;
-    const int r = static_cast<int>(blockIdx.x) - run * per_run;
-    n0 = (r / gm) * kBN;
-    m0 = (first_m + r % gm) * BM;
-  }
+  const int num_n = (N + kBN - 1) / kBN;
+  const int num_m = (M + kBM - 1) / kBM;
+  const int num_tiles = num_n * num_m;
   const int nstages = (K + kKS - 1) / kKS;
 
-  const uint32_t sA = ptx::smem_u32(smem + L::offA);
   const uint32_t sX = ptx::smem_u32(smem + L::offX);
   const uint32_t sP = ptx::smem_u32(smem + L::offP);
   auto bar = [&](uint64_t* b) { return ptx::smem_u32(b); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      ptx::mbar_init(bar(&bars->full_tma[s]), 1);
-      ptx::mbar_init(bar(&bars->full_a[s]), 128);
+      ptx::mbar_init(bar(&bars->full[s]), 1);
+      ptx::mbar_init(bar(&bars->afull[s]), 128);
       ptx::mbar_init(bar(&bars->empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -209,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     ptx::prefetch_tmap(&tm_p);
   }
   if (warp == 2) {
-    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), L::kTmemCols);
+    ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -218,54 +233,72 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const uint32_t tmem_base = *tmem_holder;
   const WaitCtx wc{abort_flag, status};
 
+  // Register split (per thread): 32 for the producer and MMA warps, 96 for
+  // the dequantizers, 192 for the epilogue; 4*32*32 + 4*32*96 + 8*32*192 =
+  // 65536, the 512 threads x 128 registers the CTA is launched with.
   if (warp < 4) {
-    ptx::regs_dec<24>();
+    ptx::regs_dec<32>();
     if (warp == 0 && lane == 0) {
       // ---------------- TMA producer ----------------
-      int it = 0;
-      for (; it < nstages; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!wait_bar(bar(&bars->empty[s]), ph ^ 1u, wc)) break;
-        ptx::mbar_arrive_expect_tx(bar(&bars->full_tma[s]), L::kX + L::kP);
-        ptx::tma_load_2d(sX + s * L::kX, &tm_x, it * kKS, m0, bar(&bars->full_tma[s]));
-        ptx::tma_load_2d(sP + s * L::kP, &tm_p, it * (kKS / 2), n0, bar(&bars->full_tma[s]));
+      int gs = 0;  // stages issued (ring slot and phase)
+      bool ok = true;
+      for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
+        int n0, m0;
+        tile_origin(T, num_n, num_m, n0, m0);
+        for (int it = 0; it < nstages; ++it, ++gs) {
+          const int s = gs % kStages;
+          if (!wait_bar(bar(&bars->empty[s]), ((gs / kStages) & 1) ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar(&bars->full[s]), L::kX + L::kP);
+          ptx::tma_load_2d(sX + s * L::kX, &tm_x, it * kKS, m0, bar(&bars->full[s]));
+          ptx::tma_load_2d(sP + s * L::kP, &tm_p, it * (kKS / 2), n0, bar(&bars->full[s]));
+        }
       }
       if (*abort_flag) {
         // Let every issued copy land before the CTA's shared memory goes away.
-        const int first = it - kStages > 0 ? it - kStages : 0;
-        for (int j = first; j < it; ++j)
-          drain_bar(bar(&bars->full_tma[j % kStages]), (j / kStages) & 1);
+        const int first = gs - kStages > 0 ? gs - kStages : 0;
+        for (int j = first; j < gs; ++j) drain_bar(bar(&bars->full[j % kStages]), (j / kStages) & 1);
       }
     } else if (warp == 1 && lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = make_idesc<TX, BM>();
-      int gi = 0;
-      for (int it = 0; it < nstages; ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        const int k0 = it * kKS;
-        const bool first_of_group = (k0 % group) == 0;
-        const bool last_of_group = ((k0 + kKS) % group) == 0 || (k0 + kKS) >= K;
-        const int buf = gi & 1;
-        if (first_of_group) {
-          if (!wait_bar(bar(&bars->tmem_empty[buf]), ((gi >> 1) & 1) ^ 1u, wc)) break;
+      constexpr uint32_t idesc = make_idesc<TX>();
+      int gs = 0;
+      uint32_t gc = 0;  // groups started (accumulator and phase)
+      bool ok = true;
+      for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
+        for (int it = 0; ok && it < nstages; ++it, ++gs) {
+          const int s = gs % kStages;
+          const uint32_t ph = (gs / kStages) & 1;
+          if (!wait_bar(bar(&bars->full[s]), ph, wc) || !wait_bar(bar(&bars->afull[s]), ph, wc)) {
+            ok = false;
+            break;
+          }
           ptx::tc_fence_after();
-        }
-        if (!wait_bar(bar(&bars->full_tma[s]), ph, wc)) break;
-        if (!wait_bar(bar(&bars->full_a[s]), ph, wc)) break;
-        ptx::tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(buf * BM);
 #pragma unroll
-        for (int kk = 0; kk < kKS / 16; ++kk) {
-          const uint64_t ad = ptx::sw128_kmajor_desc(sA + s * L::kA + kk * 32);
-          const uint64_t bd = ptx::sw128_kmajor_desc(sX + s * L::kX + kk * 32);
-          ptx::umma_f16(d, ad, bd, idesc, (first_of_group && kk == 0) ? 0u : 1u);
-        }
-        ptx::umma_commit(bar(&bars->empty[s]));
-        if (last_of_group) {
-          ptx::umma_commit(bar(&bars->tmem_full[buf]));
-          ++gi;
+          for (int kk = 0; kk < kKS / 16; ++kk) {
+            const int k = it * kKS + 16 * kk;
+            if (k >= K) break;
+            const bool first = (k % group) == 0;
+            const bool last = ((k + 16) % group) == 0 || k + 16 >= K;
+            const uint32_t buf = gc & 1u;
+            if (first) {
+              if (!wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)) {
+                ok = false;
+                break;
+              }
+              ptx::tc_fence_after();
+            }
+            const uint64_t bd = ptx::sw128_kmajor_desc(sX + s * L::kX + kk * 32);
+            ptx::umma_f16_tmem_a(tmem_base + buf * kBM, tmem_base + kColA + s * kColsA + kk * 8, bd,
+                                 idesc, first ? 0u : 1u);
+            if (last) {
+              ptx::umma_commit(bar(&bars->tmem_full[buf]));
+              ++gc;
+            }
+          }
+          ptx::umma_commit(bar(&bars->empty[s]));
         }
       }
       if (*abort_flag) {
@@ -274,72 +307,108 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       }
     }
   } else if (warp < 8) {
-    ptx::regs_dec<72>();
-    // ---------------- dequantizers: thread t owns weight row t ----------------
+    ptx::regs_dec<96>();
+    // ---------------- dequantizers: thread t owns weight row t (TMEM lane t) ----------------
     const int t = threadIdx.x - 128;
-    const int swz = t & 7;
-    const int first = (t >> 2) & 1;  // rotates the two 16-byte reads to avoid bank conflicts
-    const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G : nullptr;
-    for (int it = 0; it < nstages; ++it) {
-      const int s = it % kStages;
-      const uint32_t ph = (it / kStages) & 1;
-      // The stage's zero point (a stage lies inside one group).
-      const uint32_t zb = ASYM ? Nib<TX>::zero_bias(__ldg(zrow + (it * kKS) / group)) : 0u;
-      if (!wait_bar(bar(&bars->full_tma[s]), ph, wc)) break;
-      const uint32_t prow = sP + s * L::kP + t * 32;
-      const uint4 va = ptx::lds128(prow + 16 * first);
-      const uint4 vb = ptx::lds128(prow + 16 * (first ^ 1));
-      const uint4 lo = first ? vb : va;
-      const uint4 hi = first ? va : vb;
-      const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-      const uint32_t arow = sA + s * L::kA + t * 128;
+    const int first_half = (t >> 2) & 1;  // rotates the two 16-byte reads to avoid bank conflicts
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    int gs = 0;
+    bool ok = true;
+    for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
+      int n0, m0;
+      tile_origin(T, num_n, num_m, n0, m0);
+      const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G
+                                 : nullptr;
+      for (int it = 0; it < nstages; ++it, ++gs) {
+        const int s = gs % kStages;
+        // The zero points of the stage's two 32-k halves (one group, or two
+        // for group 32), loaded before the wait.
+        uint32_t zb0 = 0u, zb1 = 0u;
+        if (ASYM) {
+          const int g0 = (it * kKS) / group;
+          const int g1 = (it * kKS + 32) / group;
+          zb0 = Nib<TX>::zero_bias(__ldg(zrow + g0));
+          zb1 = Nib<TX>::zero_bias(__ldg(zrow + (g1 < G ? g1 : G - 1)));
+        }
+        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), (gs / kStages) & 1, wc))) {
+          ok = false;
+          break;
+        }
+        const uint32_t prow = sP + s * L::kP + t * 32;
+        const uint4 va = ptx::lds128(prow + 16 * first_half);
+        const uint4 vb = ptx::lds128(prow + 16 * (first_half ^ 1));
+        const uint4 lo = first_half ? vb : va;
+        const uint4 hi = first_half ? va : vb;
+        const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const uint32_t acol = tmem_base + lane_base + kColA + s * kColsA;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) ptx::sts128(arow + ((c ^ swz) << 4), expand8<TX, ASYM>(wds[c], zb));
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(bar(&bars->full_a[s]));
+        for (int h = 0; h < 2; ++h) {
+          uint32_t o[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) expand8<TX, ASYM>(wds[4 * h + c], h ? zb1 : zb0, o + 4 * c);
+          ptx::tmem_st_32x32b_x16(acol + 16 * h, o);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(&bars->afull[s]));
+      }
     }
   } else {
-    ptx::regs_inc<208>();
+    ptx::regs_inc<192>();
     // ---------------- epilogue: lane quarter q, column half h ----------------
     const int q = warp & 3;
     const int h = (warp - 8) >> 2;
     const int row = 32 * q + lane;
-    const int n = n0 + row;
-    constexpr int kCols = BM / 2;
-    float acc[kCols];
-#pragma unroll
-    for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
-    const uint16_t* srow = scales + static_cast<int64_t>(n < N ? n : 0) * G;
-    float s_next = (n < N) ? f16_bits_to_float(__ldg(srow)) : 0.0f;
+    uint32_t gc = 0;
     bool ok = true;
-    for (int gi = 0; gi < G; ++gi) {
-      const int buf = gi & 1;
-      const float sc = s_next;
-      if (gi + 1 < G && n < N) s_next = f16_bits_to_float(__ldg(srow + gi + 1));
-      if (!wait_bar(bar(&bars->tmem_full[buf]), (gi >> 1) & 1, wc)) {
-        ok = false;
-        break;
+    for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
+      int n0, m0;
+      tile_origin(T, num_n, num_m, n0, m0);
+      const int n = n0 + row;
+      float2 acc[kEpiCols / 2];
+#pragma unroll
+      for (int j = 0; j < kEpiCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      const uint16_t* srow = scales + static_cast<int64_t>(n < N ? n : N - 1) * G;
+      float s_next = f16_bits_to_float(__ldg(srow));
+      for (int gi = 0; gi < G; ++gi, ++gc) {
+        const uint32_t buf = gc & 1u;
+        const float sc = s_next;
+        if (gi + 1 < G) s_next = f16_bits_to_float(__ldg(srow + gi + 1));
+        if (!wait_bar(bar(&bars->tmem_full[buf]), (gc >> 1) & 1u, wc)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const float2 sc2 = make_float2(sc, sc);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * kBM +
+                               static_cast<uint32_t>(h * kEpiCols);
+#pragma unroll
+        for (int c = 0; c < kEpiCols; c += 32) {
+          uint32_t r0[16], r1[16];
+          ptx::tmem_ld_32x32b_x16(taddr + c, r0);
+          ptx::tmem_ld_32x32b_x16(taddr + c + 16, r1);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            acc[c / 2 + j] = __ffma2_rn(
+                make_float2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), sc2,
+                acc[c / 2 + j]);
+            acc[c / 2 + 8 + j] = __ffma2_rn(
+                make_float2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), sc2,
+                acc[c / 2 + 8 + j]);
+          }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(&bars->tmem_empty[buf]));
       }
-      ptx::tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) +
-                             static_cast<uint32_t>(buf * BM + h * kCols);
+      if (ok && n < N) {
+        const int mbase = m0 + h * kEpiCols;
 #pragma unroll
-      for (int c = 0; c < kCols; c += 16) {
-        uint32_t r[16];
-        ptx::tmem_ld_32x32b_x16(taddr + c, r);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(__uint_as_float(r[j]), sc, acc[c + j]);
-      }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(&bars->tmem_empty[buf]));
-    }
-    if (ok && n < N) {
-      const int mbase = m0 + h * kCols;
-#pragma unroll
-      for (int j = 0; j < kCols; ++j) {
-        const int m = mbase + j;
-        if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j], n);
+        for (int j = 0; j < kEpiCols / 2; ++j) {
+          const int m = mbase + 2 * j;
+          if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j].x, n);
+          if (m + 1 < M) y[static_cast<int64_t>(m + 1) * N + n] = ep.apply(acc[j].y, n);
+        }
       }
     }
   }
@@ -348,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   __syncthreads();
   if (warp == 2) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, L::kTmemCols);
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -370,11 +439,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <typename TX, int BM, bool ASYM>
-cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                      const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
-                      int64_t N, float* y, cudaStream_t stream) {
-  using L = Layout<BM>;
+template <typename TX, bool ASYM>
+cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                         const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                         int64_t N, float* y, cudaStream_t stream) {
+  using L = Layout;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   uint32_t* status = status_word();
@@ -383,7 +452,7 @@ cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {kKS, BM};
+    const cuuint32_t box[2] = {kKS, kBM};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
                                        ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -404,15 +473,26 @@ cudaError_t launch_bm(const TX* x, const uint8_t* packed, const uint16_t* scales
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = prefill_kernel<TX, BM, ASYM>;
+  auto kern = prefill_kernel<TX, ASYM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(((N + kBN - 1) / kBN) * ((M + BM - 1) / BM)));
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  const int64_t sms = num_sms();
+  const dim3 grid(static_cast<unsigned>(tiles < sms ? tiles : sms));  // persistent: one CTA per SM
   const int G = static_cast<int>((K + group - 1) / group);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, zeros, ep, y, static_cast<int>(M),
                                               static_cast<int>(N), static_cast<int>(K), group, G,
                                               status);
   return cudaGetLastError();
+}
+
+template <typename TX>
+cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                      const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                      int64_t N, float* y, cudaStream_t stream) {
+  if (zeros != nullptr)
+    return launch_typed<TX, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  return launch_typed<TX, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, stream);
 }
 
 }  // namespace
@@ -421,21 +501,12 @@ bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, con
                        const uint8_t* packed) {
   if (xt == DType::F32) return false;
   if (M < 1 || N < 1 || K < 1) return false;
-  if (K % 32 != 0 || group % kKS != 0) return false;
+  if (K % 32 != 0 || group % 32 != 0) return false;
   if (K > (1LL << 30) || M > (1LL << 30) || N > (1LL << 30)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0 || reinterpret_cast<uintptr_t>(packed) % 16 != 0)
     return false;
-  if (((N + kBN - 1) / kBN) * ((M + 255) / 256) > 0x7FFFFFFFLL) return false;
+  if (((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM) > 0x7FFFFFFFLL) return false;
   return true;
-}
-
-template <typename TX>
-static cudaError_t launch_prefill_tx(const TX* x, const uint8_t* packed, const uint16_t* scales,
-                                     const uint8_t* zeros, const Epilogue& ep, int64_t K, int group,
-                                     int64_t M, int64_t N, float* y, cudaStream_t stream) {
-  if (zeros != nullptr)
-    return launch_bm<TX, 256, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
-  return launch_bm<TX, 256, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, stream);
 }
 
 cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
@@ -443,10 +514,10 @@ cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed
                                   int64_t K, int group, int64_t M, int64_t N, float* y,
                                   cudaStream_t stream) {
   if (xt == DType::BF16)
-    return launch_prefill_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, zeros, ep, K,
-                             group, M, N, y, stream);
-  return launch_prefill_tx(static_cast<const __half*>(x), packed, scales, zeros, ep, K, group, M, N,
-                           y, stream);
+    return launch_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, zeros, ep, K, group, M,
+                     N, y, stream);
+  return launch_tx(static_cast<const __half*>(x), packed, scales, zeros, ep, K, group, M, N, y,
+                   stream);
 }
 
 }  // namespace int4lib

@@ -67,3 +67,30 @@ def assert_matmul_close(y, x, packed, scales, K, group, c, rows=None, cols=None)
         f"matmul error {err[worst]:.3e} > bound {bound[worst]:.3e} at {worst} "
         f"(y={yn[worst]:.6e}, ref={y_ref[worst]:.6e})")
     return float((err / np.maximum(bound, 1e-300)).max())
+
+
+def assert_matmul_lines(y, x, packed, scales, K, group, c, rows, cols, chunk=4096):
+    """Whole lines of y against the oracle: every column of the sampled rows
+    `rows` and every row of the sampled columns `cols`, the oracle computed
+    over chunks of weight rows (so full-size matrices fit in host memory)."""
+    xn_rows = to_np(x.index_select(0, torch.as_tensor(rows, device=x.device))).astype(np.float64)
+    pn_all = packed.cpu().numpy()
+    sn_all = scales.cpu().numpy()
+    y_rows = y.index_select(0, torch.as_tensor(rows, device=y.device)).cpu().numpy()
+    N = pn_all.shape[0]
+    worst = 0.0
+    for n0 in range(0, N, chunk):
+        n1 = min(n0 + chunk, N)
+        ref = oracle.int4_matmul_ref(xn_rows, pn_all[n0:n1], sn_all[n0:n1], K, group)
+        bound = oracle.matmul_error_bound(xn_rows, pn_all[n0:n1], sn_all[n0:n1], K, group, c)
+        err = np.abs(y_rows[:, n0:n1].astype(np.float64) - ref)
+        assert (err <= bound).all(), f"rows: error above the bound in columns {n0}..{n1}"
+        worst = max(worst, float((err / np.maximum(bound, 1e-300)).max()))
+    xn = to_np(x).astype(np.float64)
+    ci = torch.as_tensor(cols, device=y.device)
+    y_cols = y.index_select(1, ci).cpu().numpy().astype(np.float64)
+    ref = oracle.int4_matmul_ref(xn, pn_all[cols], sn_all[cols], K, group)
+    bound = oracle.matmul_error_bound(xn, pn_all[cols], sn_all[cols], K, group, c)
+    err = np.abs(y_cols - ref)
+    assert (err <= bound).all(), "columns: error above the bound"
+    return max(worst, float((err / np.maximum(bound, 1e-300)).max()))

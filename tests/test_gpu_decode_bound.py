@@ -61,7 +61,8 @@ def _adversarial_x(M, K, dtype):
     big, tiny = ADVERSARIAL[dtype]
     x = torch.full((M, K), tiny, dtype=torch.float64)
     x[:, ::128] = big                       # the block's largest value, on a zero weight
-    x *= (2.0 ** -torch.arange(M, dtype=torch.float64))[:, None]   # rows at other scales
+    # Rows at other scales (powers of two, within fp16's normal range).
+    x *= (2.0 ** -(torch.arange(M, dtype=torch.float64) % 4))[:, None]
     return x.to(dtype).to(DEV)
 
 

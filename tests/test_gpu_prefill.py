@@ -1,7 +1,9 @@
 """GPU parity of the tcgen05 tensor-core matmul (the prefill path) against
 the CPU oracle: |y - y_ref| <= 4e-3 * sum|x||w_hat| for bf16/fp16 x, on
-shapes with ragged M, N and K tails, partial last groups, zero groups and
-the full-size prefill workloads (sampled outputs)."""
+shapes with ragged M, N and K tails, partial last groups, zero groups,
+groups of 32 (two per pipeline stage) and of 96 (spanning stages), more
+tiles than SMs, and the full-size prefill workloads (whole rows and columns
+of y)."""
 
 import numpy as np
 import pytest
@@ -9,7 +11,7 @@ import torch
 
 import dequant_gemm_int4_b200 as q4
 import oracle
-from gpu_util import TOL_HALF, assert_matmul_close
+from gpu_util import TOL_HALF, assert_matmul_close, assert_matmul_lines
 from workloads import PREFILL_LINEARS, make_activations, make_weights
 
 pytestmark = pytest.mark.gpu
@@ -50,6 +52,8 @@ def test_prefill_smallest_tile():
     (256, 128, 128, 128), (256, 128, 1024, 128), (512, 256, 512, 64), (300, 200, 256, 128),
     (17, 130, 192, 64), (1000, 77, 4096, 128), (256, 128, 96, 64), (256, 128, 8224, 128),
     (513, 385, 640, 128), (64, 1000, 2048, 256), (257, 129, 3072, 3072),
+    (300, 200, 96, 32), (500, 300, 1056, 32), (192, 128, 2016, 96), (1024, 2304, 768, 32),
+    (2048, 2048, 512, 64), (4000, 1000, 256, 32),   # more tiles than SMs: several per CTA
 ])
 def test_prefill_shapes(dtype, M, N, K, group):
     _run(M, N, K, group, dtype, seed=M + N + K)
@@ -89,12 +93,34 @@ def test_prefill_matches_decode_and_simt():
 def test_prefill_is_the_automatic_choice_for_large_m():
     assert q4.matmul_select(torch.bfloat16, 8192, 128, 2048, 8192) == q4.PATH_PREFILL
     assert q4.matmul_select(torch.float16, 768, 64, 1024, 2304) == q4.PATH_PREFILL
+    assert q4.matmul_select(torch.float16, 768, 32, 1024, 2304) == q4.PATH_PREFILL
+
+
+def test_prefill_group_32_one_hot_is_exact():
+    """Group 32: two groups per 64-k stage, each with its own accumulator."""
+    N, K, group = 256, 256, 32
+    packed, scales, _ = _quantized(N, K, group, 5, "student_t3", 0.2)
+    w_hat = oracle.dequantize_int4(packed.cpu().numpy(), scales.cpu().numpy(), K, group)
+    ks = [0, 31, 32, 33, 63, 64, 95, 96, 200, 255]
+    x = torch.zeros(192, K, device=DEV, dtype=torch.float16)
+    for i, k in enumerate(ks):
+        x[i, k] = 1.0
+    y = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL).cpu().numpy()
+    for i, k in enumerate(ks):
+        assert np.array_equal(y[i].astype(np.float64), w_hat[:, k]), k
 
 
 @pytest.mark.parametrize("layer", PREFILL_LINEARS, ids=lambda l: l.name)
 @pytest.mark.parametrize("M", [2048, 8192])
-def test_prefill_full_size_sampled(layer, M):
+def test_prefill_full_size_whole_rows_and_columns(layer, M):
+    """The full-size prefill workloads: every output of 16 random activation
+    rows (first and last included) and of 16 random weight rows."""
     rng = np.random.default_rng(M + layer.N)
     rows = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 14)]))
-    cols = np.unique(np.concatenate([[0, layer.N - 1], rng.integers(0, layer.N, 254)]))
-    _run(M, layer.N, layer.K, layer.group, torch.bfloat16, seed=4, rows=rows, cols=cols)
+    cols = np.unique(np.concatenate([[0, layer.N - 1], rng.integers(0, layer.N, 14)]))
+    packed, scales, _ = _quantized(layer.N, layer.K, layer.group, 5)
+    x = make_activations(M, layer.K, seed=6, device=DEV, dtype=torch.bfloat16)
+    assert q4.matmul_select(torch.bfloat16, layer.K, layer.group, M, layer.N) == q4.PATH_PREFILL
+    y = q4.int4_matmul(x, packed, scales, layer.K, layer.group)
+    assert q4.device_status() == q4.OK
+    assert_matmul_lines(y, x, packed, scales, layer.K, layer.group, TOL_HALF, rows, cols)
