@@ -385,6 +385,55 @@ def unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks, reps: int = 5):
     return rows
 
 
+def variant_rows(dev, w, xd, xp, flush_l2, peaks, reps: int = 5):
+    """The asymmetric (zero-point) variant and the fused bias + ReLU epilogue
+    on the bench's matrix, each timed per call with CUDA events after an L2
+    flush: affine quantize (GB/s on its bytes: bf16 w in, packed codes, fp16
+    scales and uint8 zero points out), affine decode M = 1 and prefill
+    M = 8192, and the symmetric decode and prefill with bias + ReLU."""
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            flush_l2()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / reps
+
+    Kp, G = K_W // 2, K_W // GROUP
+    packed_a, scales_a, zeros_a, _ = q4.quantize_int4_affine(w, GROUP)
+    ms = timed(lambda: q4.quantize_int4_affine(w, GROUP))
+    qbytes = N_W * K_W * 2 + N_W * Kp + 3 * N_W * G
+    rows = {"affine_quantize": {"ms": ms, "GB/s": qbytes / (ms * 1e-3) / 1e9,
+                                "frac": qbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+    packed, scales, _ = q4.quantize_int4(w, GROUP)
+    bias = torch.randn(N_W, generator=torch.Generator().manual_seed(0)).to(dev)
+    yd = torch.empty((xd.shape[0], N_W), dtype=torch.float32, device=dev)
+    for name, kw, pk, sc in (("affine_decode", {"zeros": zeros_a}, packed_a, scales_a),
+                             ("bias_relu_decode", {"bias": bias, "relu": True}, packed, scales)):
+        ms = timed(lambda: q4.int4_matmul(xd, pk, sc, K_W, GROUP, out=yd, **kw))
+        gbs = N_W * Kp / (ms * 1e-3) / 1e9
+        rows[name] = {"ms": ms, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                      "timing": "single call after an L2 flush (the launch inside the events)"}
+    if xp is not None:
+        yp = torch.empty((xp.shape[0], N_W), dtype=torch.float32, device=dev)
+        for name, kw, pk, sc in (("affine_prefill", {"zeros": zeros_a}, packed_a, scales_a),
+                                 ("bias_relu_prefill", {"bias": bias, "relu": True}, packed, scales)):
+            ms = timed(lambda: q4.int4_matmul(xp, pk, sc, K_W, GROUP, out=yp, **kw))
+            tf = 2 * xp.shape[0] * N_W * K_W / (ms * 1e-3) / 1e12
+            rows[name] = {"ms": ms, "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"]}
+    return rows
+
+
 def run_ours(args):
     import torch
 
@@ -546,6 +595,9 @@ def run_ours(args):
     unfused = None
     if not args.no_unfused and not args.only:
         unfused = unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks)
+    variants = None
+    if not args.no_variants and not args.only and w is not None:
+        variants = variant_rows(dev, w, xd, xp, flush_l2, peaks)
 
     # End to end through the public Python API: pinned host x in, y out.
     e2e = None
@@ -594,7 +646,8 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "flushed before every row (256 MiB write, then 256 MiB read of another buffer); the decode row's back-to-back calls read distinct weight copies (940 MB > L2)",
                    "parallelism": f"replicas x{world}"},
-        "rows": rows, "decode_llama7b": shape_rows, "unfused": unfused, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "rows": rows, "decode_llama7b": shape_rows, "unfused": unfused, "variants": variants,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * sum(launches_per_step[n] for n in order),
         "wall_ms_timed_region": wall_ms,
     }
@@ -613,15 +666,25 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the affine-variant and bias+ReLU epilogue rows")
     ap.add_argument("--no-unfused", action="store_true",
                     help="skip the dequantize-then-GEMM comparison rows")
     ap.add_argument("--no-shapes", action="store_true",
                     help="skip the decode rows at the Llama-7B-shaped linears")
     ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,
                     help="run one kernel of the step only (for profiling); no e2e or CPU baseline")
+    ap.add_argument("--shape", default=None, metavar="N,K,M",
+                    help="with --only: a smaller weight matrix N x K (and prefill batch M) for "
+                         "profiler captures that must stay a few GB on the device")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.shape is not None:
+        if not args.only:
+            ap.error("--shape is for single-kernel profiling runs (--only)")
+        global N_W, K_W, M_PREFILL
+        N_W, K_W, M_PREFILL = (int(v) for v in args.shape.split(","))
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -314,6 +314,11 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
     ptx::prefetch_tmap(&tm_x);
   }
   __syncthreads();
+  // Launched as a programmatic dependent of what precedes it on the stream:
+  // the set-up above overlaps that kernel's tail; every thread waits for it
+  // to complete before reading an input or writing an output.
+  ptx::launch_dependents();
+  ptx::grid_dependency_wait();
 
   const int c = lane & 3;
   const int g = lane >> 2;
@@ -1431,6 +1436,17 @@ __global__ void __launch_bounds__(kSmallWarps * 32, kSmallCtasPerSm) decode_smal
   const uint16_t* sb_row = scales + rb * G;
   const uint8_t* za_row = ASYM ? zeros + ra * G : nullptr;
   const uint8_t* zb_row = ASYM ? zeros + rb * G : nullptr;
+  // Launched as a programmatic dependent of what precedes it on the stream:
+  // ask L2 for the weight lines of this warp's first step (L2 is coherent, so
+  // lines the earlier kernel still writes are read fresh after the wait), let
+  // the next kernel start its own set-up, then wait for the earlier kernel
+  // before reading any input or writing y.
+  if (warp < KB) {
+    ptx::prefetch_l2(wa + static_cast<int64_t>(warp) * 64);
+    ptx::prefetch_l2(wb + static_cast<int64_t>(warp) * 64);
+  }
+  ptx::launch_dependents();
+  ptx::grid_dependency_wait();
   float tot[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -1524,14 +1540,20 @@ cudaError_t launch_small(const TX* x, const uint8_t* packed, const uint16_t* sca
                          int64_t N, float* y, cudaStream_t stream) {
   const int G = static_cast<int>((K + group - 1) / group);
   const int KB = static_cast<int>((K + 127) / 128);
-  const unsigned grid = static_cast<unsigned>((N + 15) / 16);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((N + 15) / 16));
+  cfg.blockDim = dim3(kSmallWarps * 32);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (M <= 8)
-    decode_small_kernel<TX, 1, ASYM><<<grid, kSmallWarps * 32, 0, stream>>>(
-        x, packed, scales, zeros, ep, y, K, group, G, static_cast<int>(M), N, KB);
-  else
-    decode_small_kernel<TX, 2, ASYM><<<grid, kSmallWarps * 32, 0, stream>>>(
-        x, packed, scales, zeros, ep, y, K, group, G, static_cast<int>(M), N, KB);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, decode_small_kernel<TX, 1, ASYM>, x, packed, scales, zeros, ep,
+                              y, K, group, G, static_cast<int>(M), N, KB);
+  return cudaLaunchKernelEx(&cfg, decode_small_kernel<TX, 2, ASYM>, x, packed, scales, zeros, ep, y,
+                            K, group, G, static_cast<int>(M), N, KB);
 }
 
 // Small matrices: 16-row tiles that fit one wave, K a multiple of 128 (so
@@ -1755,10 +1777,19 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& pl, float* part
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  decode_kernel<TX, NT, GPB, ASYM><<<static_cast<unsigned>(pl.P), kThreads, L::kAlloc, a.stream>>>(
-      tw, tx, a.scales, a.zeros, a.ep, a.y, a.K, a.group, G, static_cast<int>(a.M), a.N, pl.KB, pl.U,
-      static_cast<int>(pl.P), pl.gran, partials, counters, status);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.P));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::kAlloc;
+  cfg.stream = a.stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<TX, NT, GPB, ASYM>, tw, tx, a.scales, a.zeros, a.ep,
+                            a.y, a.K, a.group, G, static_cast<int>(a.M), a.N, pl.KB, pl.U,
+                            static_cast<int>(pl.P), pl.gran, partials, counters, status);
 }
 
 // The 16-bit decode kernel: plan, scratch need and (if `launch`) the launch.

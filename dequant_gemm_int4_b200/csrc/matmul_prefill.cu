@@ -16,7 +16,7 @@
 //               nibbles to bf16/fp16 (exact: 128 + u or 1024 + u minus 136 or
 //               1032, or minus 128 + z for the asymmetric scheme's unsigned
 //               codes) and stores it with tcgen05.st into TMEM lane t, one of
-//               four 32-column A stages
+//               a ring of 32-column A slots
 //   warp 1      MMA issuer: D_g = A_g * X_g^T, 16 k per MMA, into one of two
 //               TMEM accumulators (128 lanes x 192 columns), one per K group;
 //               a group may span stages (group 128) or share one (group 32)
@@ -52,36 +52,60 @@ namespace int4lib {
 
 namespace {
 
+#ifndef INT4_PREFILL_A_TMEM
+#define INT4_PREFILL_A_TMEM 0  // 1: dequantized A in tensor memory (tcgen05.st), else shared memory
+#endif
+#ifndef INT4_PREFILL_BM
+#define INT4_PREFILL_BM (INT4_PREFILL_A_TMEM ? 192 : 256)
+#endif
+#ifndef INT4_PREFILL_STAGES
+#define INT4_PREFILL_STAGES 4
+#endif
+#ifndef INT4_PREFILL_A_STAGES
+#define INT4_PREFILL_A_STAGES 4
+#endif
 constexpr int kBN = 128;      // weight rows per tile (MMA M, TMEM lanes)
-constexpr int kBM = 192;      // activation rows per tile (MMA N)
+constexpr int kBM = INT4_PREFILL_BM;  // activation rows per tile (MMA N)
 constexpr int kKS = 64;       // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int kStages = 4;
+constexpr int kStages = INT4_PREFILL_STAGES;    // shared-memory ring (x and packed bytes)
+constexpr int kAStages = INT4_PREFILL_A_STAGES;  // TMEM ring of dequantized A
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColA = 2 * kBM;          // first column of the A stages
+constexpr bool kATmem = INT4_PREFILL_A_TMEM != 0;
+constexpr uint32_t kColA = 2 * kBM;          // first column of the A stages (A in TMEM)
 constexpr uint32_t kColsA = kKS / 2;         // 32-bit columns per A stage
-static_assert(kColA + kStages * kColsA <= kTmemCols, "accumulators and A stages fit TMEM");
+static_assert(kColA + (kATmem ? kAStages * kColsA : 0) <= kTmemCols,
+              "accumulators (and A stages) fit TMEM");
+static_assert(kATmem || kAStages == kStages, "A in shared memory lives in the stage ring");
+static_assert(kBM % 64 == 0, "the epilogue reads 32 columns at a time per column half");
+static_assert(kAStages <= kStages, "an A slot is reused no sooner than its shared-memory stage");
 constexpr int kEpiCols = kBM / 2;            // accumulator columns per epilogue thread
 constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
 #ifndef INT4_PREFILL_GROUP_M
 #define INT4_PREFILL_GROUP_M 8
 #endif
 constexpr int kGroupM = INT4_PREFILL_GROUP_M;  // activation tiles per raster run
+#ifndef INT4_PREFILL_PERSISTENT
+#define INT4_PREFILL_PERSISTENT 1  // 1: one CTA per SM walks the tiles; 0: one CTA per tile
+#endif
 
 struct Barriers {
   uint64_t full[kStages];       // TMA bytes of stage s landed
-  uint64_t afull[kStages];      // dequantized A of stage s written to TMEM
-  uint64_t empty[kStages];      // MMAs reading stage s (x and A) finished
+  uint64_t empty[kStages];      // MMAs reading stage s (x) finished
+  uint64_t afull[kAStages];     // dequantized A of slot a written to TMEM
+  uint64_t aempty[kAStages];    // MMAs reading A slot a finished
   uint64_t tmem_full[2];        // group accumulator b complete
   uint64_t tmem_empty[2];       // epilogue finished reading accumulator b
   uint64_t drain;               // abort path: all issued MMAs finished
 };
 
 struct Layout {
-  static constexpr int kX = kBM * kKS * 2;  // 24 KB
+  static constexpr int kX = kBM * kKS * 2;  // 24 KB at N = 192
   static constexpr int kP = kBN * kKS / 2;  // 4 KB
+  static constexpr int kA = kATmem ? 0 : kBN * kKS * 2;  // 16 KB: A tiles in shared memory
   static constexpr int offX = 0;
-  static constexpr int offP = offX + kStages * kX;
+  static constexpr int offA = offX + kStages * kX;
+  static constexpr int offP = offA + kStages * kA;
   static constexpr int offBar = offP + kStages * kP;
   static constexpr int offMisc = offBar + static_cast<int>(sizeof(Barriers));
   static constexpr int kBytes = offMisc + 16;
@@ -204,14 +228,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int nstages = (K + kKS - 1) / kKS;
 
   const uint32_t sX = ptx::smem_u32(smem + L::offX);
+  const uint32_t sA = ptx::smem_u32(smem + L::offA);
   const uint32_t sP = ptx::smem_u32(smem + L::offP);
   auto bar = [&](uint64_t* b) { return ptx::smem_u32(b); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       ptx::mbar_init(bar(&bars->full[s]), 1);
-      ptx::mbar_init(bar(&bars->afull[s]), 128);
       ptx::mbar_init(bar(&bars->empty[s]), 1);
+    }
+    for (int a = 0; a < kAStages; ++a) {
+      ptx::mbar_init(bar(&bars->afull[a]), 128);
+      ptx::mbar_init(bar(&bars->aempty[a]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(&bars->tmem_full[b]), 1);
@@ -268,20 +296,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       uint32_t gc = 0;  // groups started (accumulator and phase)
       bool ok = true;
       for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
+        // Position of the next MMA's k inside its group, kept incrementally:
+        // this single thread issues every MMA, and a division per MMA would
+        // cost more than the MMA itself.
+        int gpos = 0;
         for (int it = 0; ok && it < nstages; ++it, ++gs) {
           const int s = gs % kStages;
           const uint32_t ph = (gs / kStages) & 1;
-          if (!wait_bar(bar(&bars->full[s]), ph, wc) || !wait_bar(bar(&bars->afull[s]), ph, wc)) {
+          const int as = gs % kAStages;
+          if (!wait_bar(bar(&bars->full[s]), ph, wc) ||
+              !wait_bar(bar(&bars->afull[as]), (gs / kAStages) & 1, wc)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
+          const uint64_t bd0 = ptx::sw128_kmajor_desc(sX + s * L::kX);
+          const uint64_t ad0 = kATmem ? 0ull : ptx::sw128_kmajor_desc(sA + as * L::kA);
 #pragma unroll
           for (int kk = 0; kk < kKS / 16; ++kk) {
             const int k = it * kKS + 16 * kk;
             if (k >= K) break;
-            const bool first = (k % group) == 0;
-            const bool last = ((k + 16) % group) == 0 || k + 16 >= K;
+            const bool first = gpos == 0;
+            gpos += 16;
+            const bool last = gpos == group || k + 16 >= K;
+            if (gpos == group) gpos = 0;
             const uint32_t buf = gc & 1u;
             if (first) {
               if (!wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)) {
@@ -290,15 +328,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
               }
               ptx::tc_fence_after();
             }
-            const uint64_t bd = ptx::sw128_kmajor_desc(sX + s * L::kX + kk * 32);
-            ptx::umma_f16_tmem_a(tmem_base + buf * kBM, tmem_base + kColA + s * kColsA + kk * 8, bd,
-                                 idesc, first ? 0u : 1u);
+            // +32 bytes along K is +2 in the descriptor's address field.
+            const uint64_t bd = bd0 + static_cast<uint64_t>(2 * kk);
+            if (kATmem)
+              ptx::umma_f16_tmem_a(tmem_base + buf * kBM, tmem_base + kColA + as * kColsA + kk * 8,
+                                   bd, idesc, first ? 0u : 1u);
+            else
+              ptx::umma_f16(tmem_base + buf * kBM, ad0 + static_cast<uint64_t>(2 * kk), bd, idesc,
+                            first ? 0u : 1u);
             if (last) {
               ptx::umma_commit(bar(&bars->tmem_full[buf]));
               ++gc;
             }
           }
           ptx::umma_commit(bar(&bars->empty[s]));
+          ptx::umma_commit(bar(&bars->aempty[as]));
         }
       }
       if (*abort_flag) {
@@ -330,7 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
           zb0 = Nib<TX>::zero_bias(__ldg(zrow + g0));
           zb1 = Nib<TX>::zero_bias(__ldg(zrow + (g1 < G ? g1 : G - 1)));
         }
-        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), (gs / kStages) & 1, wc))) {
+        const int as = gs % kAStages;
+        // The stage's bytes have landed, and the MMAs that read this A slot
+        // kAStages stages ago have finished.
+        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), (gs / kStages) & 1, wc) &&
+                                         wait_bar(bar(&bars->aempty[as]), ((gs / kAStages) & 1) ^ 1u, wc))) {
           ok = false;
           break;
         }
@@ -340,17 +388,31 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         const uint4 lo = first_half ? vb : va;
         const uint4 hi = first_half ? va : vb;
         const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        const uint32_t acol = tmem_base + lane_base + kColA + s * kColsA;
+        if (kATmem) {
+          const uint32_t acol = tmem_base + lane_base + kColA + as * kColsA;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t o[16];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t o[16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) expand8<TX, ASYM>(wds[4 * h + c], h ? zb1 : zb0, o + 4 * c);
-          ptx::tmem_st_32x32b_x16(acol + 16 * h, o);
+            for (int c = 0; c < 4; ++c) expand8<TX, ASYM>(wds[4 * h + c], h ? zb1 : zb0, o + 4 * c);
+            ptx::tmem_st_32x32b_x16(acol + 16 * h, o);
+          }
+          ptx::tmem_st_wait();
+          ptx::tc_fence_before();
+        } else {
+          // Row t of the K-major A tile, 128-byte swizzle: 16-byte chunk c at
+          // (c ^ (t & 7)).
+          const uint32_t arow = sA + as * L::kA + t * 128;
+          const int swz = t & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+            expand8<TX, ASYM>(wds[c], c < 4 ? zb0 : zb1, o);
+            ptx::sts128(arow + ((c ^ swz) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          }
+          ptx::fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
         }
-        ptx::tmem_st_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(bar(&bars->afull[s]));
+        ptx::mbar_arrive(bar(&bars->afull[as]));
       }
     }
   } else {
@@ -478,7 +540,8 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   const int64_t sms = num_sms();
-  const dim3 grid(static_cast<unsigned>(tiles < sms ? tiles : sms));  // persistent: one CTA per SM
+  const int64_t ctas = INT4_PREFILL_PERSISTENT ? (tiles < sms ? tiles : sms) : tiles;
+  const dim3 grid(static_cast<unsigned>(ctas));  // persistent: one CTA per SM
   const int G = static_cast<int>((K + group - 1) / group);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, zeros, ep, y, static_cast<int>(M),
                                               static_cast<int>(N), static_cast<int>(K), group, G,

@@ -117,6 +117,11 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t c0
                : "memory");
 }
 
+// Ask L2 to fetch the 128-byte line holding `p` (no register written).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
+}
+
 // Untiled bulk copy global -> shared, completing on an mbarrier: both
 // addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

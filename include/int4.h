@@ -163,9 +163,9 @@ int int4_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t K, in
  * of CTAs and runs the integer kernel at every M, which is faster when the
  * row tiles do not fill the GPU evenly.
  *
- * Stream ordering: the decode kernels for groups that are a multiple of 128
- * launch with programmatic stream serialization and wait for the preceding
- * work on `stream` before touching memory, so ordinary stream order holds.
+ * Stream ordering: the decode kernels (M <= 16, bf16/fp16 x) launch with
+ * programmatic stream serialization and wait for the preceding work on
+ * `stream` before touching memory, so ordinary stream order holds.
  * They also signal dependents early: a kernel that the caller launches after
  * them with programmatic stream serialization must execute
  * griddepcontrol.wait (cudaGridDependencySynchronize) before it reads y.
@@ -290,8 +290,8 @@ int int4_matmul_ex(const void* x, int32_t x_dtype, const uint8_t* packed, const 
  * latency-critical path that must not enter an allocator (whose calls can
  * block, synchronize or fail under memory pressure).
  *
- * Computes what int4_matmul computes on its decode path (same kernels, same
- * result bits), with the partial tiles of the split (4 MiB: one wave of up to
+ * Computes what int4_matmul_ws computes on its decode path (same kernels, same
+ * split, same result bits), with the partial tiles of the split (4 MiB: one wave of up to
  * 512 CTAs), their arrival counters (2 KiB) and the integer digits of x
  * (4 MiB: K up to 64384 at M = 16, 246528 at M <= 4; not used at M <= 2) kept
  * in a fixed library-owned device array instead of per-stream scratch.  It calls no cudaMalloc, cudaFree or other
