@@ -5,33 +5,39 @@
 // dequantizing matmul" (problem statement), computed one K group at a time
 // with the group's scale applied to each output before the fp32 running sum.
 //
-// A persistent CTA per SM walks output tiles of 128 weight rows (n) x 192
+// A persistent CTA per SM walks output tiles of 128 weight rows (n) x 256
 // activation rows (m), computed with tcgen05 MMAs (kind::f16, fp32
-// accumulation in tensor memory) whose A operand -- the dequantized weights --
-// is read from tensor memory, not shared memory:
-//   warp 0      TMA producer: per 64-wide K stage, x [192 rows x 64] (128-byte
+// accumulation in tensor memory):
+//   warp 0      TMA producer: per 64-wide K stage, x [256 rows x 64] (128-byte
 //               swizzle, the MMA's B operand) and the packed weights
 //               [128 rows x 32 bytes], into a 4-stage shared-memory ring
 //   warps 4-7   dequantizers: thread t expands weight row t of the stage from
 //               nibbles to bf16/fp16 (exact: 128 + u or 1024 + u minus 136 or
 //               1032, or minus 128 + z for the asymmetric scheme's unsigned
-//               codes) and stores it with tcgen05.st into TMEM lane t, one of
-//               a ring of 32-column A slots
+//               codes) into row t of the stage's K-major A tile (128-byte
+//               swizzle) in shared memory
 //   warp 1      MMA issuer: D_g = A_g * X_g^T, 16 k per MMA, into one of two
-//               TMEM accumulators (128 lanes x 192 columns), one per K group;
-//               a group may span stages (group 128) or share one (group 32)
+//               TMEM accumulators (128 lanes x 256 columns), one per K group;
+//               a group may span stages (group 128) or share one (group 32).
+//               The whole warp runs the loop and one elected lane issues, so
+//               every value the MMAs take stays warp-uniform: issued from a
+//               lone lane the same loop left the tensor core idle between
+//               MMAs for a fifth of the time.
 //   warps 8-15  epilogue: per group, load the group's accumulator from TMEM,
 //               multiply by s[n, g] (TMEM lane = weight row: one scale per
 //               thread) and add into fp32 registers (packed FMAs); at the end
 //               of a tile, add the bias, apply ReLU and store y.
-// TMEM: columns [0, 384) the two accumulators, [384, 512) the A stages.
-// Shared memory then carries only x (written by TMA, read by the MMA) and the
-// packed bytes, about 14 KB per 16-k MMA step against 25 KB with A staged in
-// shared memory; with one MMA of 128 x 192 x 16 every 96 cycles that is the
-// difference between shared-memory bandwidth (128 B per cycle) binding below
-// two thirds of the tensor rate and binding near nine tenths of it.  The two
-// accumulators let the tensor core run group g + 1 (or the next tile's first
-// group) while the epilogue drains group g or stores a finished tile.
+// TMEM: the two accumulators fill its 512 columns.  They let the tensor core
+// run group g + 1 (or the next tile's first group) while the epilogue drains
+// group g or stores a finished tile.
+//
+// Per 16-k MMA step shared memory carries A (4 KB) and x (8 KB) to the tensor
+// core, plus the dequantizers' 4 KB and the copy engine's 8 KB of writes:
+// about 190 bytes per cycle at the full tensor rate against 128 the SM's
+// shared memory delivers, so this one-CTA form is bound near two thirds of
+// the tensor peak.  Holding A in tensor memory instead (tcgen05.st from the
+// dequantizers, MMAs reading A from TMEM, 192-row tiles to make room) cuts
+// the bytes but measured slower.
 //
 // Tiles are visited in runs of kGroupM activation tiles, all weight tiles of
 // a run before the next, so a run's x tiles stay in L2 while the weight tiles
@@ -52,33 +58,17 @@ namespace int4lib {
 
 namespace {
 
-#ifndef INT4_PREFILL_A_TMEM
-#define INT4_PREFILL_A_TMEM 0  // 1: dequantized A in tensor memory (tcgen05.st), else shared memory
-#endif
-#ifndef INT4_PREFILL_BM
-#define INT4_PREFILL_BM (INT4_PREFILL_A_TMEM ? 192 : 256)
-#endif
 #ifndef INT4_PREFILL_STAGES
 #define INT4_PREFILL_STAGES 4
 #endif
-#ifndef INT4_PREFILL_A_STAGES
-#define INT4_PREFILL_A_STAGES 4
-#endif
 constexpr int kBN = 128;      // weight rows per tile (MMA M, TMEM lanes)
-constexpr int kBM = INT4_PREFILL_BM;  // activation rows per tile (MMA N)
+constexpr int kBM = 256;      // activation rows per tile (MMA N)
 constexpr int kKS = 64;       // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = INT4_PREFILL_STAGES;    // shared-memory ring (x and packed bytes)
-constexpr int kAStages = INT4_PREFILL_A_STAGES;  // TMEM ring of dequantized A
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-constexpr bool kATmem = INT4_PREFILL_A_TMEM != 0;
-constexpr uint32_t kColA = 2 * kBM;          // first column of the A stages (A in TMEM)
-constexpr uint32_t kColsA = kKS / 2;         // 32-bit columns per A stage
-static_assert(kColA + (kATmem ? kAStages * kColsA : 0) <= kTmemCols,
-              "accumulators (and A stages) fit TMEM");
-static_assert(kATmem || kAStages == kStages, "A in shared memory lives in the stage ring");
+static_assert(2 * kBM <= kTmemCols, "two accumulators fit TMEM");
 static_assert(kBM % 64 == 0, "the epilogue reads 32 columns at a time per column half");
-static_assert(kAStages <= kStages, "an A slot is reused no sooner than its shared-memory stage");
 constexpr int kEpiCols = kBM / 2;            // accumulator columns per epilogue thread
 constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
 #ifndef INT4_PREFILL_GROUP_M
@@ -92,8 +82,7 @@ constexpr int kGroupM = INT4_PREFILL_GROUP_M;  // activation tiles per raster ru
 struct Barriers {
   uint64_t full[kStages];       // TMA bytes of stage s landed
   uint64_t empty[kStages];      // MMAs reading stage s (x) finished
-  uint64_t afull[kAStages];     // dequantized A of slot a written to TMEM
-  uint64_t aempty[kAStages];    // MMAs reading A slot a finished
+  uint64_t afull[kStages];      // dequantized A of stage s written
   uint64_t tmem_full[2];        // group accumulator b complete
   uint64_t tmem_empty[2];       // epilogue finished reading accumulator b
   uint64_t drain;               // abort path: all issued MMAs finished
@@ -102,7 +91,7 @@ struct Barriers {
 struct Layout {
   static constexpr int kX = kBM * kKS * 2;  // 24 KB at N = 192
   static constexpr int kP = kBN * kKS / 2;  // 4 KB
-  static constexpr int kA = kATmem ? 0 : kBN * kKS * 2;  // 16 KB: A tiles in shared memory
+  static constexpr int kA = kBN * kKS * 2;  // 16 KB: dequantized A
   static constexpr int offX = 0;
   static constexpr int offA = offX + kStages * kX;
   static constexpr int offP = offA + kStages * kA;
@@ -237,10 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       ptx::mbar_init(bar(&bars->full[s]), 1);
       ptx::mbar_init(bar(&bars->empty[s]), 1);
     }
-    for (int a = 0; a < kAStages; ++a) {
-      ptx::mbar_init(bar(&bars->afull[a]), 128);
-      ptx::mbar_init(bar(&bars->aempty[a]), 1);
-    }
+    for (int s = 0; s < kStages; ++s) ptx::mbar_init(bar(&bars->afull[s]), 128);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(&bars->tmem_full[b]), 1);
       ptx::mbar_init(bar(&bars->tmem_empty[b]), 256);
@@ -289,73 +275,86 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         const int first = gs - kStages > 0 ? gs - kStages : 0;
         for (int j = first; j < gs; ++j) drain_bar(bar(&bars->full[j % kStages]), (j / kStages) & 1);
       }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
+      // The whole warp waits and keeps the books; the elected lane issues the
+      // MMAs and commits.  The bookkeeping between MMAs shows up directly in
+      // the tensor rate, so the position inside the K group is tracked once
+      // per 64-k stage when groups are whole stages (one test per four MMAs),
+      // else once per 32-k half (groups of 32, 96, ...), never per MMA and
+      // never by division.
+      const bool leader = ptx::elect_one();
       constexpr uint32_t idesc = make_idesc<TX>();
+      const int span = group % kKS == 0 ? kKS : kKS / 2;  // k per bookkeeping step
       int gs = 0;
       uint32_t gc = 0;  // groups started (accumulator and phase)
       bool ok = true;
       for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
-        // Position of the next MMA's k inside its group, kept incrementally:
-        // this single thread issues every MMA, and a division per MMA would
-        // cost more than the MMA itself.
-        int gpos = 0;
+        int gpos = 0;  // k offset of the next step inside its group
         for (int it = 0; ok && it < nstages; ++it, ++gs) {
           const int s = gs % kStages;
           const uint32_t ph = (gs / kStages) & 1;
-          const int as = gs % kAStages;
-          if (!wait_bar(bar(&bars->full[s]), ph, wc) ||
-              !wait_bar(bar(&bars->afull[as]), (gs / kAStages) & 1, wc)) {
+          if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), ph, wc) &&
+                                           wait_bar(bar(&bars->afull[s]), ph, wc))) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint64_t bd0 = ptx::sw128_kmajor_desc(sX + s * L::kX);
-          const uint64_t ad0 = kATmem ? 0ull : ptx::sw128_kmajor_desc(sA + as * L::kA);
-#pragma unroll
-          for (int kk = 0; kk < kKS / 16; ++kk) {
-            const int k = it * kKS + 16 * kk;
-            if (k >= K) break;
+          const uint64_t ad0 = ptx::sw128_kmajor_desc(sA + s * L::kA);
+          const int rem = K - it * kKS;  // k left in this tile's K (a multiple of 32)
+          // One bookkeeping step: MMAs kk0 .. kk0 + nk - 1 of the stage, all in
+          // one K group (K and the group are multiples of 32).
+          auto step = [&](int kk0, int nk) -> bool {
             const bool first = gpos == 0;
-            gpos += 16;
-            const bool last = gpos == group || k + 16 >= K;
+            gpos += span;
+            const bool last = gpos == group || 16 * (kk0 + nk) >= rem;
             if (gpos == group) gpos = 0;
             const uint32_t buf = gc & 1u;
             if (first) {
-              if (!wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)) {
-                ok = false;
-                break;
-              }
+              if (!__all_sync(0xffffffffu,
+                            wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)))
+              return false;
               ptx::tc_fence_after();
             }
-            // +32 bytes along K is +2 in the descriptor's address field.
-            const uint64_t bd = bd0 + static_cast<uint64_t>(2 * kk);
-            if (kATmem)
-              ptx::umma_f16_tmem_a(tmem_base + buf * kBM, tmem_base + kColA + as * kColsA + kk * 8,
-                                   bd, idesc, first ? 0u : 1u);
-            else
-              ptx::umma_f16(tmem_base + buf * kBM, ad0 + static_cast<uint64_t>(2 * kk), bd, idesc,
-                            first ? 0u : 1u);
-            if (last) {
-              ptx::umma_commit(bar(&bars->tmem_full[buf]));
-              ++gc;
+            if (leader) {
+              const uint32_t d = tmem_base + buf * kBM;
+#pragma unroll
+              for (int j = 0; j < kKS / 16; ++j) {
+                if (j < nk) {
+                  // +32 bytes along K is +2 in a descriptor's address field.
+                  const uint64_t dk = static_cast<uint64_t>(2 * (kk0 + j));
+                  ptx::umma_f16(d, ad0 + dk, bd0 + dk, idesc, (first && j == 0) ? 0u : 1u);
+                }
+              }
+              if (last) ptx::umma_commit(bar(&bars->tmem_full[buf]));
             }
+            __syncwarp();
+            if (last) ++gc;
+            return true;
+          };
+          if (span == kKS) {
+            ok = step(0, rem >= kKS ? kKS / 16 : rem / 16);
+          } else {
+            ok = step(0, 2);
+            if (ok && rem > kKS / 2) ok = step(2, 2);
           }
-          ptx::umma_commit(bar(&bars->empty[s]));
-          ptx::umma_commit(bar(&bars->aempty[as]));
+          if (!ok) break;
+          if (leader) ptx::umma_commit(bar(&bars->empty[s]));
+          __syncwarp();
         }
       }
       if (*abort_flag) {
-        ptx::umma_commit(bar(&bars->drain));
+        if (leader) ptx::umma_commit(bar(&bars->drain));
+        __syncwarp();
         drain_bar(bar(&bars->drain), 0);
       }
     }
   } else if (warp < 8) {
     ptx::regs_dec<96>();
-    // ---------------- dequantizers: thread t owns weight row t (TMEM lane t) ----------------
+    // ---------------- dequantizers: thread t owns weight row t ----------------
     const int t = threadIdx.x - 128;
     const int first_half = (t >> 2) & 1;  // rotates the two 16-byte reads to avoid bank conflicts
-    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     int gs = 0;
     bool ok = true;
     for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
@@ -374,11 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
           zb0 = Nib<TX>::zero_bias(__ldg(zrow + g0));
           zb1 = Nib<TX>::zero_bias(__ldg(zrow + (g1 < G ? g1 : G - 1)));
         }
-        const int as = gs % kAStages;
-        // The stage's bytes have landed, and the MMAs that read this A slot
-        // kAStages stages ago have finished.
-        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), (gs / kStages) & 1, wc) &&
-                                         wait_bar(bar(&bars->aempty[as]), ((gs / kAStages) & 1) ^ 1u, wc))) {
+        // The stage's bytes have landed, which also means the MMAs that read
+        // its A tile kStages stages ago have finished: the producer refilled
+        // the stage only after they released it.
+        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), (gs / kStages) & 1, wc))) {
           ok = false;
           break;
         }
@@ -388,31 +386,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         const uint4 lo = first_half ? vb : va;
         const uint4 hi = first_half ? va : vb;
         const uint32_t wds[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        if (kATmem) {
-          const uint32_t acol = tmem_base + lane_base + kColA + as * kColsA;
+        // Row t of the K-major A tile, 128-byte swizzle: 16-byte chunk c at
+        // (c ^ (t & 7)).
+        const uint32_t arow = sA + s * L::kA + t * 128;
+        const int swz = t & 7;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t o[16];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) expand8<TX, ASYM>(wds[4 * h + c], h ? zb1 : zb0, o + 4 * c);
-            ptx::tmem_st_32x32b_x16(acol + 16 * h, o);
-          }
-          ptx::tmem_st_wait();
-          ptx::tc_fence_before();
-        } else {
-          // Row t of the K-major A tile, 128-byte swizzle: 16-byte chunk c at
-          // (c ^ (t & 7)).
-          const uint32_t arow = sA + as * L::kA + t * 128;
-          const int swz = t & 7;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[4];
-            expand8<TX, ASYM>(wds[c], c < 4 ? zb0 : zb1, o);
-            ptx::sts128(arow + ((c ^ swz) << 4), make_uint4(o[0], o[1], o[2], o[3]));
-          }
-          ptx::fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[4];
+          expand8<TX, ASYM>(wds[c], c < 4 ? zb0 : zb1, o);
+          ptx::sts128(arow + ((c ^ swz) << 4), make_uint4(o[0], o[1], o[2], o[3]));
         }
-        ptx::mbar_arrive(bar(&bars->afull[as]));
+        ptx::fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
+        ptx::mbar_arrive(bar(&bars->afull[s]));
       }
     }
   } else {
