@@ -54,10 +54,10 @@ DECODE_COPIES = 8
 # sha256 of that source file and is reported as null once the file changes.
 KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
-    "prefill": (3_925_588_000 + 920_221_696, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
-                "009294f3ae9d1c445ad32b0380ace3d8f9cb911804642ade540a76cdcf693f64"),
-    "decode": (125_485_312 + 3_899_904, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
-               "f3ac46c0847c0e41bb556fe66ffc7f43a78eba80f11968fcbb4f105fd034a952"),
+    "prefill": (769_880_000 + 914_330_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
+                "e59d0e58a38a386849973b6323a1eb61886b801e716eb19aacdc62973f8c9bb0"),
+    "decode": (125_434_624 + 4_626_688, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
+               "178d4852998a2a29a2efcc14e285759e676798d29112d05fa6ce6942d811fe84"),
     "quantize": (469_856_256 + 104_254_208, "dequant_gemm_int4_b200/csrc/quantize.cu",
                  "24a51fde9c6ea1afd8a159345f565f16441d8a085e241e8e6d8d123c71573f57"),
     "unpack": (117_453_056 + 182_672_128, "dequant_gemm_int4_b200/csrc/unpack.cu",
