@@ -54,8 +54,8 @@ DECODE_COPIES = 8
 # sha256 of that source file and is reported as null once the file changes.
 KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
-    "prefill": (769_880_000 + 914_330_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
-                "e59d0e58a38a386849973b6323a1eb61886b801e716eb19aacdc62973f8c9bb0"),
+    "prefill": (846_660_000 + 913_850_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
+                "3255ba0a6114629d9acd7863f190894e9234e5b0e940ff374c652cef4e8eaae7"),
     "decode": (125_434_624 + 4_626_688, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
                "178d4852998a2a29a2efcc14e285759e676798d29112d05fa6ce6942d811fe84"),
     "quantize": (469_856_256 + 104_254_208, "dequant_gemm_int4_b200/csrc/quantize.cu",
@@ -269,6 +269,8 @@ def run_reference(args):
 # rate; launch gaps only) and launched call by call from the host.
 DECODE_SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]
 DECODE_MS = (1, 4, 16)
+PREFILL_SHAPES = [(8192, 8192), (28672, 8192)]
+PREFILL_MS = (2048, 8192)
 
 
 def decode_shape_rows(dev, peaks, reps: int = 10):
@@ -334,6 +336,56 @@ def decode_shape_rows(dev, peaks, reps: int = 10):
                 "us_per_call_host_launched": host_us,
                 "path": q4.matmul_select(torch.bfloat16, K, GROUP, M, N), "copies": ncopy}
         del copies
+    return rows
+
+
+def prefill_shape_rows(dev, peaks, reps: int = 3, windows: int = 5):
+    """The configured prefill workloads W [8192, 8192] and [28672, 8192], group
+    128, bf16 x at M = 2048 and 8192: per call, the median of `windows` event
+    windows of `reps` back-to-back calls."""
+    import statistics
+
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+    from workloads import make_activations, make_weights
+
+    L = q4.lib()
+    rows = {}
+    for N, K in PREFILL_SHAPES:
+        w = make_weights(N, K, seed=4, device=dev, dtype=torch.float32)
+        packed, scales, _ = q4.quantize_int4(w, GROUP)
+        del w
+        for M in PREFILL_MS:
+            x = make_activations(M, K, seed=M, device=dev, dtype=torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+
+            def run():
+                sp = torch.cuda.current_stream(dev).cuda_stream
+                rc = L.int4_matmul_ws(x.data_ptr(), 1, packed.data_ptr(), scales.data_ptr(), K, GROUP,
+                                      M, N, y.data_ptr(), None, 0, sp)
+                if rc != 0:
+                    raise RuntimeError(f"INT4 library error {rc}: {L.int4_last_error()}")
+
+            for _ in range(2):
+                run()
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(windows):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(reps):
+                    run()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) / reps)
+            ms = statistics.median(times)
+            tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+            rows[f"{N}x{K}_m{M}"] = {"ms": ms, "TFLOP/s": tf, "frac": tf / peaks["bf16_tflops"],
+                                     "path": q4.matmul_select(torch.bfloat16, K, GROUP, M, N)}
+            del x, y
+        del packed, scales
     return rows
 
 
@@ -590,8 +642,10 @@ def run_ours(args):
     roof["traffic"] = _traffic(dom)
 
     shape_rows = None
+    prefill_rows = None
     if not args.no_shapes and not args.only:
         shape_rows = decode_shape_rows(dev, peaks)
+        prefill_rows = prefill_shape_rows(dev, peaks)
     unfused = None
     if not args.no_unfused and not args.only:
         unfused = unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks)
@@ -646,7 +700,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "flushed before every row (256 MiB write, then 256 MiB read of another buffer); the decode row's back-to-back calls read distinct weight copies (940 MB > L2)",
                    "parallelism": f"replicas x{world}"},
-        "rows": rows, "decode_llama7b": shape_rows, "unfused": unfused, "variants": variants,
+        "rows": rows, "decode_llama7b": shape_rows, "prefill_shapes": prefill_rows, "unfused": unfused, "variants": variants,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * sum(launches_per_step[n] for n in order),
         "wall_ms_timed_region": wall_ms,
@@ -671,7 +725,7 @@ def main():
     ap.add_argument("--no-unfused", action="store_true",
                     help="skip the dequantize-then-GEMM comparison rows")
     ap.add_argument("--no-shapes", action="store_true",
-                    help="skip the decode rows at the Llama-7B-shaped linears")
+                    help="skip the rows at the other configured shapes (Llama-7B decode, prefill)")
     ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,
                     help="run one kernel of the step only (for profiling); no e2e or CPU baseline")
     ap.add_argument("--shape", default=None, metavar="N,K,M",

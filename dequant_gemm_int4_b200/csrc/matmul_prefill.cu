@@ -313,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
             const uint32_t buf = gc & 1u;
             if (first) {
               if (!__all_sync(0xffffffffu,
-                            wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)))
-              return false;
+                              wait_bar(bar(&bars->tmem_empty[buf]), ((gc >> 1) & 1u) ^ 1u, wc)))
+                return false;
               ptx::tc_fence_after();
             }
             if (leader) {
@@ -421,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         const uint32_t buf = gc & 1u;
         const float sc = s_next;
         if (gi + 1 < G) s_next = f16_bits_to_float(__ldg(srow + gi + 1));
-        if (!wait_bar(bar(&bars->tmem_full[buf]), (gc >> 1) & 1u, wc)) {
+        // Warp-uniform, as the warp-wide TMEM loads below require.
+        if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->tmem_full[buf]), (gc >> 1) & 1u, wc))) {
           ok = false;
           break;
         }
