@@ -31,13 +31,14 @@
 // run group g + 1 (or the next tile's first group) while the epilogue drains
 // group g or stores a finished tile.
 //
-// Per 16-k MMA step shared memory carries A (4 KB) and x (8 KB) to the tensor
-// core, plus the dequantizers' 4 KB and the copy engine's 8 KB of writes:
-// about 190 bytes per cycle at the full tensor rate against 128 the SM's
-// shared memory delivers, so this one-CTA form is bound near two thirds of
-// the tensor peak.  Holding A in tensor memory instead (tcgen05.st from the
-// dequantizers, MMAs reading A from TMEM, 192-row tiles to make room) cuts
-// the bytes but measured slower.
+// The kernel runs at about two thirds of the tensor peak, and what holds it
+// there is the hand-offs.  The MMA issuer spends about a third of its time
+// waiting: most on the epilogue freeing an accumulator, then on the
+// dequantizers and on the copies.  Shared memory, at about 190 bytes per
+// 16-k step against 128 per cycle, is busy but not saturated.  Holding A in
+// tensor memory instead (tcgen05.st from the dequantizers, MMAs reading A
+// from TMEM, 192-row tiles to make room) cuts those bytes but measured
+// slower.
 //
 // Tiles are visited in runs of kGroupM activation tiles, all weight tiles of
 // a run before the next, so a run's x tiles stay in L2 while the weight tiles
