@@ -272,7 +272,8 @@ int int4_matmul_ex(const void* x, int32_t x_dtype, const uint8_t* packed, const 
     case INT4_PATH_PREFILL:
       if (!int4lib::prefill_supported(t, K, group, M, N, x, packed))
         return int4lib::fail(INT4_ERR_UNSUPPORTED, "int4_matmul: tensor-core kernel cannot run this shape");
-      e = int4lib::launch_matmul_prefill(x, t, packed, scales, zeros, ep, K, group, M, N, y, s);
+      e = int4lib::launch_matmul_prefill(x, t, packed, scales, zeros, ep, K, group, M, N, y,
+                                         workspace, workspace_bytes, s);
       break;
     default:
       return int4lib::fail(INT4_ERR_ARG, "int4_matmul: unknown path");
@@ -313,7 +314,13 @@ int int4_matmul_workspace_size(int32_t x_dtype, int64_t K, int32_t group, int64_
   if (M == 0 || N == 0) return INT4_OK;
   const DType t = static_cast<DType>(x_dtype);
   static const uint8_t* const kAligned = reinterpret_cast<const uint8_t*>(static_cast<uintptr_t>(256));
-  if (matmul_choose(t, K, group, M, N, kAligned, kAligned) != INT4_PATH_DECODE) return INT4_OK;
+  const int path = matmul_choose(t, K, group, M, N, kAligned, kAligned);
+  if (path == INT4_PATH_PREFILL) {
+    // Non-zero only when the split of K pays (fewer tiles than SMs).
+    *bytes = int4lib::prefill_workspace_size(K, group, M, N);
+    return INT4_OK;
+  }
+  if (path != INT4_PATH_DECODE) return INT4_OK;
   const cudaError_t e = int4lib::decode_workspace_size(t, K, group, M, N, bytes);
   return e == cudaSuccess ? INT4_OK : int4lib::fail_cuda(e, "int4_matmul_workspace_size");
 }

@@ -70,10 +70,18 @@ cudaError_t reset_split_counters();
 // matmul_prefill.cu
 bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, const void* x,
                        const uint8_t* packed);
+// With a workspace of prefill_workspace_size bytes (when that is non-zero:
+// fewer tiles than SMs), K is split into pieces whose fp32 sums a second
+// kernel adds; a smaller or null workspace runs the call unsplit.  The sums
+// start kWorkspaceCounterBytes into the workspace: a workspace also serves
+// decode calls, whose layout begins with arrival counters that every call
+// must find zero (1024 counters of 4 bytes in matmul_decode.cu).
 cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
                                   const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
                                   int64_t K, int group, int64_t M, int64_t N, float* y,
-                                  cudaStream_t stream);
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+size_t prefill_workspace_size(int64_t K, int group, int64_t M, int64_t N);
+constexpr size_t kWorkspaceCounterBytes = 4096;
 
 int num_sms();  // SM count of the current device (cached per device)
 

@@ -49,7 +49,9 @@
 // are drained (again with a bound) and TMEM is freed before the CTA exits.
 #include <cuda.h>
 
+#include <cstring>
 #include <mutex>
+#include <numeric>
 
 #include "common.cuh"
 #include "internal.h"
@@ -197,11 +199,38 @@ __device__ __forceinline__ void tile_origin(int T, int num_n, int num_m, int& n0
   m0 = (first_m + r % gm) * kBM;
 }
 
+// Work unit u: piece u % ksplit of tile u / ksplit.  A tile's K is cut into
+// ksplit pieces of whole chunks of `spc` stages (spc * 64 k: a common
+// multiple of the group and the stage), so each piece starts and ends on a
+// group boundary; pieces of one tile are adjacent units.
+struct Unit {
+  int n0, m0;    // tile origin
+  int piece;
+  int it0, it1;  // stages [it0, it1)
+  int g0, g1;    // K groups [g0, g1)
+};
+__device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int ksplit, int nchunks, int spc,
+                                        int nstages, int K, int group) {
+  Unit w;
+  const int T = u / ksplit;
+  w.piece = u - T * ksplit;
+  tile_origin(T, num_n, num_m, w.n0, w.m0);
+  const int c0 = w.piece * nchunks / ksplit;
+  const int c1 = (w.piece + 1) * nchunks / ksplit;
+  w.it0 = c0 * spc;
+  w.it1 = c1 * spc < nstages ? c1 * spc : nstages;
+  w.g0 = (w.it0 * kKS) / group;
+  const int kend = w.it1 * kKS < K ? w.it1 * kKS : K;
+  w.g1 = (kend + group - 1) / group;
+  return w;
+}
+
 template <typename TX, bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_p,
     const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
-    float* __restrict__ y, int M, int N, int K, int group, int G, uint32_t* status) {
+    float* __restrict__ y, int M, int N, int K, int group, int G, int ksplit, int spc,
+    float* __restrict__ ypart, uint32_t* status) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -216,6 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int num_m = (M + kBM - 1) / kBM;
   const int num_tiles = num_n * num_m;
   const int nstages = (K + kKS - 1) / kKS;
+  const int nchunks = (nstages + spc - 1) / spc;
+  const int num_units = num_tiles * ksplit;
 
   const uint32_t sX = ptx::smem_u32(smem + L::offX);
   const uint32_t sA = ptx::smem_u32(smem + L::offA);
@@ -257,10 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       // ---------------- TMA producer ----------------
       int gs = 0;  // stages issued (ring slot and phase)
       bool ok = true;
-      for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
-        int n0, m0;
-        tile_origin(T, num_n, num_m, n0, m0);
-        for (int it = 0; it < nstages; ++it, ++gs) {
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+        const int n0 = w.n0, m0 = w.m0;
+        for (int it = w.it0; it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
           if (!wait_bar(bar(&bars->empty[s]), ((gs / kStages) & 1) ^ 1u, wc)) {
             ok = false;
@@ -290,9 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       int gs = 0;
       uint32_t gc = 0;  // groups started (accumulator and phase)
       bool ok = true;
-      for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
-        int gpos = 0;  // k offset of the next step inside its group
-        for (int it = 0; ok && it < nstages; ++it, ++gs) {
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+        int gpos = 0;  // k offset of the next step inside its group (a piece starts a group)
+        for (int it = w.it0; ok && it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
           const uint32_t ph = (gs / kStages) & 1;
           if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->full[s]), ph, wc) &&
@@ -358,12 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int first_half = (t >> 2) & 1;  // rotates the two 16-byte reads to avoid bank conflicts
     int gs = 0;
     bool ok = true;
-    for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
-      int n0, m0;
-      tile_origin(T, num_n, num_m, n0, m0);
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+      const int n0 = w.n0;
       const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G
                                  : nullptr;
-      for (int it = 0; it < nstages; ++it, ++gs) {
+      for (int it = w.it0; it < w.it1; ++it, ++gs) {
         const int s = gs % kStages;
         // The zero points of the stage's two 32-k halves (one group, or two
         // for group 32), loaded before the wait.
@@ -409,19 +441,19 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int row = 32 * q + lane;
     uint32_t gc = 0;
     bool ok = true;
-    for (int T = blockIdx.x; ok && T < num_tiles; T += gridDim.x) {
-      int n0, m0;
-      tile_origin(T, num_n, num_m, n0, m0);
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+      const int n0 = w.n0, m0 = w.m0;
       const int n = n0 + row;
       float2 acc[kEpiCols / 2];
 #pragma unroll
       for (int j = 0; j < kEpiCols / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
       const uint16_t* srow = scales + static_cast<int64_t>(n < N ? n : N - 1) * G;
-      float s_next = f16_bits_to_float(__ldg(srow));
-      for (int gi = 0; gi < G; ++gi, ++gc) {
+      float s_next = w.g0 < w.g1 ? f16_bits_to_float(__ldg(srow + w.g0)) : 0.0f;
+      for (int gi = w.g0; gi < w.g1; ++gi, ++gc) {
         const uint32_t buf = gc & 1u;
         const float sc = s_next;
-        if (gi + 1 < G) s_next = f16_bits_to_float(__ldg(srow + gi + 1));
+        if (gi + 1 < w.g1) s_next = f16_bits_to_float(__ldg(srow + gi + 1));
         // Warp-uniform, as the warp-wide TMEM loads below require.
         if (!__all_sync(0xffffffffu, wait_bar(bar(&bars->tmem_full[buf]), (gc >> 1) & 1u, wc))) {
           ok = false;
@@ -452,11 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       }
       if (ok && n < N) {
         const int mbase = m0 + h * kEpiCols;
+        if (ypart == nullptr) {
 #pragma unroll
-        for (int j = 0; j < kEpiCols / 2; ++j) {
-          const int m = mbase + 2 * j;
-          if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j].x, n);
-          if (m + 1 < M) y[static_cast<int64_t>(m + 1) * N + n] = ep.apply(acc[j].y, n);
+          for (int j = 0; j < kEpiCols / 2; ++j) {
+            const int m = mbase + 2 * j;
+            if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j].x, n);
+            if (m + 1 < M) y[static_cast<int64_t>(m + 1) * N + n] = ep.apply(acc[j].y, n);
+          }
+        } else {
+          // A piece of a split K: its fp32 sums, added in piece order (and
+          // the epilogue applied) by prefill_reduce_kernel.
+          float* yp = ypart + static_cast<int64_t>(w.piece) * M * N;
+#pragma unroll
+          for (int j = 0; j < kEpiCols / 2; ++j) {
+            const int m = mbase + 2 * j;
+            if (m < M) yp[static_cast<int64_t>(m) * N + n] = acc[j].x;
+            if (m + 1 < M) yp[static_cast<int64_t>(m + 1) * N + n] = acc[j].y;
+          }
         }
       }
     }
@@ -488,10 +532,58 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// y = epilogue(sum over pieces p of ypart[p]), adding the pieces in order.
+__global__ void __launch_bounds__(256) prefill_reduce_kernel(const float* __restrict__ ypart, int ksplit,
+                                                             int64_t MN, int64_t N, Epilogue ep,
+                                                             float* __restrict__ y) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < MN;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v = __ldcs(ypart + i);
+    for (int p = 1; p < ksplit; ++p) v += __ldcs(ypart + static_cast<int64_t>(p) * MN + i);
+    y[i] = ep.apply(v, static_cast<int>(i % N));
+  }
+}
+
+// How many K pieces to cut each tile into.  With fewer tiles than SMs the
+// machine idles; more pieces fill it, at the price of writing and re-reading
+// the pieces' fp32 sums.  The estimate (calibrated on B200): waves of units
+// times a unit's time -- its share of the tile's stages at about 0.6 us per
+// 64-k stage of a 128 x 256 tile, plus about 3 us to start and finish a
+// unit -- plus, when split, the partial sums' round trip through HBM and
+// about 1 us for the adding kernel.
+struct SplitPlan {
+  int ksplit = 1;
+  int spc = 1;  // stages per chunk: a common multiple of the group and the 64-k stage
+};
+SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N) {
+  SplitPlan p;
+  const int64_t g64 = std::gcd(static_cast<int64_t>(group), static_cast<int64_t>(kKS));
+  p.spc = static_cast<int>(group / g64);  // lcm(group, 64) / 64
+  const int64_t nstages = (K + kKS - 1) / kKS;
+  const int64_t nchunks = (nstages + p.spc - 1) / p.spc;
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  const int64_t sms = num_sms();
+  if (tiles >= sms || nchunks < 2) return p;
+  const double stage_us = 0.6, unit_us = 3.0, reduce_us = 1.0, hbm_bytes_per_us = 6.0e6;
+  const double tile_us = static_cast<double>(nstages) * stage_us;
+  double best = 0.0;
+  for (int64_t k = 1; k <= 8 && k <= nchunks; ++k) {
+    const double waves = static_cast<double>((tiles * k + sms - 1) / sms);
+    const double t = waves * (tile_us / static_cast<double>(k) + unit_us) +
+                     (k > 1 ? static_cast<double>(k) * M * N * 8 / hbm_bytes_per_us + reduce_us : 0.0);
+    if (k == 1 || t < best) {
+      best = t;
+      p.ksplit = static_cast<int>(k);
+    }
+  }
+  return p;
+}
+
 template <typename TX, bool ASYM>
 cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* scales,
                          const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
-                         int64_t N, float* y, cudaStream_t stream) {
+                         int64_t N, float* y, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
   using L = Layout;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
@@ -525,24 +617,44 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
   auto kern = prefill_kernel<TX, ASYM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  // Split K only when the caller's workspace holds the pieces' sums (past
+  // the counters a decode call keeps at its start).
+  SplitPlan sp = plan_split(K, group, M, N);
+  const size_t part_bytes = static_cast<size_t>(sp.ksplit) * M * N * sizeof(float);
+  if (sp.ksplit > 1 &&
+      (workspace == nullptr || workspace_bytes < kWorkspaceCounterBytes + part_bytes))
+    sp.ksplit = 1;
+  float* ypart = sp.ksplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                          kWorkspaceCounterBytes)
+                               : nullptr;
+  const int64_t units = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM) * sp.ksplit;
   const int64_t sms = num_sms();
-  const int64_t ctas = INT4_PREFILL_PERSISTENT ? (tiles < sms ? tiles : sms) : tiles;
+  const int64_t ctas = INT4_PREFILL_PERSISTENT ? (units < sms ? units : sms) : units;
   const dim3 grid(static_cast<unsigned>(ctas));  // persistent: one CTA per SM
   const int G = static_cast<int>((K + group - 1) / group);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, zeros, ep, y, static_cast<int>(M),
                                               static_cast<int>(N), static_cast<int>(K), group, G,
-                                              status);
+                                              sp.ksplit, sp.spc, ypart, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || ypart == nullptr) return e;
+  const int64_t MN = M * N;
+  int64_t blocks = (MN + 255) / 256;
+  if (blocks > 8 * sms) blocks = 8 * sms;
+  prefill_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(ypart, sp.ksplit, MN, N,
+                                                                         ep, y);
   return cudaGetLastError();
 }
 
 template <typename TX>
 cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales,
                       const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
-                      int64_t N, float* y, cudaStream_t stream) {
+                      int64_t N, float* y, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
   if (zeros != nullptr)
-    return launch_typed<TX, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
-  return launch_typed<TX, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, stream);
+    return launch_typed<TX, true>(x, packed, scales, zeros, ep, K, group, M, N, y, workspace,
+                                  workspace_bytes, stream);
+  return launch_typed<TX, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, workspace,
+                                 workspace_bytes, stream);
 }
 
 }  // namespace
@@ -562,12 +674,18 @@ bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, con
 cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed,
                                   const uint16_t* scales, const uint8_t* zeros, const Epilogue& ep,
                                   int64_t K, int group, int64_t M, int64_t N, float* y,
-                                  cudaStream_t stream) {
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (xt == DType::BF16)
     return launch_tx(static_cast<const __nv_bfloat16*>(x), packed, scales, zeros, ep, K, group, M,
-                     N, y, stream);
+                     N, y, workspace, workspace_bytes, stream);
   return launch_tx(static_cast<const __half*>(x), packed, scales, zeros, ep, K, group, M, N, y,
-                   stream);
+                   workspace, workspace_bytes, stream);
+}
+
+size_t prefill_workspace_size(int64_t K, int group, int64_t M, int64_t N) {
+  const SplitPlan sp = plan_split(K, group, M, N);
+  return sp.ksplit > 1 ? kWorkspaceCounterBytes + static_cast<size_t>(sp.ksplit) * M * N * sizeof(float)
+                       : 0;
 }
 
 }  // namespace int4lib

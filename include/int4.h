@@ -188,10 +188,15 @@ int int4_matmul_workspace_size(int32_t x_dtype, int64_t K, int32_t group, int64_
  *
  * Same contract and result bounds as int4_matmul.  The library allocates
  * nothing: `workspace` holds the decode kernels' scratch (arrival counters,
- * partial tiles of the split, and the integer digits of x at M > 2).
+ * partial tiles of the split, and the integer digits of x at M > 2), or the
+ * tensor-core kernel's partial sums of a split K.
  *   - workspace_bytes must be at least int4_matmul_workspace_size(...) for
  *     this problem, else INT4_ERR_ARG (nothing launched).  workspace == NULL
- *     with workspace_bytes == 0 selects the schedule of int4_matmul.
+ *     with workspace_bytes == 0 selects the schedule of int4_matmul.  On the
+ *     tensor-core path (M > 16) the workspace is optional: when the matrix
+ *     has fewer 128 x 256 tiles than the device has SMs, a workspace of the
+ *     queried size lets the call split K into pieces whose fp32 sums a second
+ *     kernel adds in piece order; a smaller or NULL one runs it unsplit.
  *   - workspace must be 256-byte aligned (INT4_ERR_ALIGN) and zero-filled
  *     before its first use; every call leaves its counters zero again, so a
  *     workspace can serve any number of calls, of any shape, that are

@@ -120,12 +120,18 @@ def test_workspace_size_rejects_bad_arguments(L):
     assert q(1, 1 << 40, 128, 1 << 30, 8192, ctypes.byref(out)) == q4.ERR_ARG
     # Paths that use no scratch need no workspace, and need no GPU to say so.
     for args in [(0, 4096, 128, 1, 8192),        # fp32 x: the CUDA-core kernel
-                 (1, 4096, 128, 64, 8192),       # M > 16: the tensor-core kernel
+                 (1, 4096, 128, 8192, 8192),     # the tensor-core kernel with tiles to spare
                  (1, 4100, 128, 1, 8192),        # K % 32 != 0
                  (1, 4096, 128, 0, 8192)]:       # empty
         out.value = 123
         assert q(*args, ctypes.byref(out)) == q4.OK
         assert out.value == 0
+    # The tensor-core kernel with fewer tiles (64) than SMs splits K into
+    # pieces whose fp32 sums live in the workspace, past 4 KB of counters
+    # (148 SMs assumed without a device).
+    out.value = 0
+    assert q(1, 4096, 128, 64, 8192, ctypes.byref(out)) == q4.OK
+    assert out.value > 4096 and (out.value - 4096) % (64 * 8192 * 4) == 0
 
 
 def test_noalloc_rejects_what_the_decode_kernels_cannot_run(L):

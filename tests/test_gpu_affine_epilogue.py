@@ -131,8 +131,10 @@ PATHS = [
     (3, 9000, 2048, 64, q4.PATH_DECODE, None),       # 16-bit kernel, group 64
     (12, 5000, 2048, 32, q4.PATH_DECODE, None),      # 16-bit kernel, group 32
     (4, 2048, 4096, 128, q4.PATH_DECODE, None),      # small-matrix kernel
-    (256, 512, 1024, 128, q4.PATH_PREFILL, None),    # tensor-core kernel
+    (256, 512, 1024, 128, q4.PATH_PREFILL, None),    # tensor-core kernel, K split (4 tiles)
     (300, 384, 2048, 64, q4.PATH_PREFILL, None),
+    (300, 384, 2048, 64, q4.PATH_PREFILL, False),    # tensor-core kernel, whole K
+    (1024, 768, 3072, 32, q4.PATH_PREFILL, None),    # groups of 32, K split
     (7, 100, 259, 128, q4.PATH_SIMT, None),          # CUDA-core kernel (odd K)
 ]
 

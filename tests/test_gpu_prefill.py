@@ -124,3 +124,52 @@ def test_prefill_full_size_whole_rows_and_columns(layer, M):
     y = q4.int4_matmul(x, packed, scales, layer.K, layer.group)
     assert q4.device_status() == q4.OK
     assert_matmul_lines(y, x, packed, scales, layer.K, layer.group, TOL_HALF, rows, cols)
+
+
+@pytest.mark.parametrize("M, N, K, group, dtype", [
+    (64, 4096, 4096, 128, torch.bfloat16),     # 32 tiles: K split in pieces
+    (1024, 768, 3072, 32, torch.float16),      # distilgpt2 mlp c_proj shape, groups of 32
+    (100, 1000, 2016, 96, torch.bfloat16),     # group 96: pieces of 3 stages, ragged M and N
+    (256, 11008, 4096, 128, torch.bfloat16),   # 86 tiles: the estimate keeps it whole
+])
+def test_prefill_split_k_matches_oracle_and_unsplit(M, N, K, group, dtype):
+    """With fewer tiles than SMs the binding's workspace lets the kernel cut
+    K into pieces of whole groups, added in piece order by a second kernel:
+    the same bound as the unsplit call, and the same bits on every call."""
+    packed, scales, _ = _quantized(N, K, group, 13, "student_t3", 0.05)
+    x = make_activations(M, K, seed=14, device=DEV, dtype=dtype)
+    need = q4.matmul_workspace_size(dtype, K, group, M, N)
+    y_split = q4.int4_matmul(x, packed, scales, K, group)
+    y_plain = q4.int4_matmul(x, packed, scales, K, group, workspace=False)
+    assert q4.device_status() == q4.OK
+    cols = None if N <= 2048 else np.unique(np.random.default_rng(N).integers(0, N, 400))
+    assert_matmul_close(y_split, x, packed, scales, K, group, TOL_HALF, cols=cols)
+    assert_matmul_close(y_plain, x, packed, scales, K, group, TOL_HALF, cols=cols)
+    assert torch.equal(y_split, q4.int4_matmul(x, packed, scales, K, group))   # deterministic
+    if need == 0:
+        assert torch.equal(y_split, y_plain)
+
+
+def test_prefill_split_workspace_query():
+    # 32 tiles on a device of 148 SMs: split; 7168 tiles: never.
+    assert q4.matmul_workspace_size(torch.bfloat16, 4096, 128, 64, 4096) > 0
+    assert q4.matmul_workspace_size(torch.bfloat16, 8192, 128, 8192, 28672) == 0
+
+
+def test_split_prefill_leaves_decode_counters_alone():
+    """One workspace serves both kernels: the split's partial sums lie past
+    the arrival counters a decode call expects to find zero."""
+    K, group = 4096, 128
+    packed, scales, _ = _quantized(11008, K, group, 15)
+    need = max(q4.matmul_workspace_size(torch.bfloat16, K, group, 4, 11008),
+               q4.matmul_workspace_size(torch.bfloat16, K, group, 64, 4096))
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    xd = make_activations(4, K, seed=16, device=DEV, dtype=torch.bfloat16)
+    y0 = q4.int4_matmul(xd, packed, scales, K, group, workspace=ws)
+    pk2, sc2, _ = _quantized(4096, K, group, 17)
+    xp = make_activations(64, K, seed=18, device=DEV, dtype=torch.bfloat16)
+    yp = q4.int4_matmul(xp, pk2, sc2, K, group, workspace=ws)
+    assert_matmul_close(yp, xp, pk2, sc2, K, group, TOL_HALF)
+    y1 = q4.int4_matmul(xd, packed, scales, K, group, workspace=ws)
+    assert q4.device_status() == q4.OK
+    assert torch.equal(y0, y1)
