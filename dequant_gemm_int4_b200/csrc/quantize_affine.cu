@@ -56,21 +56,50 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&v)[8]) {
 
 struct Affine {
   float sf;       // the scale, read back from fp16
+  float r;        // 1 / sf correctly rounded (0 when sf is 0)
   float zf;       // the zero point as a float (an integer 0..15)
   uint32_t bits;  // the fp16 scale
   uint32_t z;
 };
 
+// fp32(v / sf), correctly rounded, from r = RN(1 / sf): q = RN(v r) is within
+// one ulp of the quotient, the residual v - q sf is exact by FMA, and
+// RN(q + residual r) is the correctly rounded quotient (Markstein's theorem
+// for a correctly rounded reciprocal; the test suite compares the codes with
+// the IEEE division bit for bit).  Quotients of 2^100 or more, and an
+// infinite scale, take the IEEE division, where the residual could overflow.  The residual is exact
+// whenever the quotient is 1/4 or more (then |v| >= 2^-26, sf being at least
+// 2^-24); a smaller quotient cannot move rint(quotient + z), exact or not.
+__device__ __forceinline__ float div_by_scale(float v, float sf, float r) {
+  const float q = __fmul_rn(v, r);
+  if (!(fabsf(q) < 0x1p100f) || r == 0.0f) return __fdiv_rn(v, sf);  // huge, or sf = +inf
+  const float e = __fmaf_rn(-q, sf, v);
+  return __fmaf_rn(e, r, q);
+}
+
+// fp32(d / 15), correctly rounded, for finite d >= 0: Markstein's step with
+// the constant c = RN(1/15) (q0 = d c, exact residual d - 15 q0 by FMA,
+// q0 + residual c).  Where the residual could round (d subnormal), the
+// quotient lies far below the smallest fp16 subnormal and the scale is 0
+// either way.  The test suite compares the scales with the IEEE division on
+// every fp32 mantissa of the binades that matter.
+__device__ __forceinline__ float div15_rn(float d) {
+  const float c = 0.0666666701f;  // fp32 nearest to 1/15
+  const float q0 = __fmul_rn(d, c);
+  const float e = __fmaf_rn(-15.0f, q0, d);
+  return __fmaf_rn(e, c, q0);
+}
+
 // Scale and zero point of a group with extremes mn <= mx.
 __device__ __forceinline__ Affine affine_params(float mn, float mx) {
   Affine a;
   const float d = __fsub_rn(mx, mn);
-  const float s32 = __fdiv_rn(d, 15.0f);
-  a.bits = __half_as_ushort(__float2half_rn(s32));
+  a.bits = __half_as_ushort(__float2half_rn(div15_rn(d)));
   a.sf = f16_bits_to_float(a.bits);
+  a.r = a.sf != 0.0f ? __frcp_rn(a.sf) : 0.0f;
   a.zf = 0.0f;
   if (a.sf != 0.0f) {
-    const float t = rintf(__fdiv_rn(-mn, a.sf));
+    const float t = rintf(div_by_scale(-mn, a.sf, a.r));
     a.zf = fminf(fmaxf(t, 0.0f), 15.0f);
   }
   a.z = static_cast<uint32_t>(a.zf);
@@ -81,6 +110,7 @@ __device__ __forceinline__ Affine affine_from_stored(uint16_t bits, uint8_t z) {
   Affine a;
   a.bits = bits;
   a.sf = f16_bits_to_float(bits);
+  a.r = a.sf != 0.0f ? __frcp_rn(a.sf) : 0.0f;
   a.z = z;
   a.zf = static_cast<float>(z);
   return a;
@@ -90,8 +120,21 @@ __device__ __forceinline__ Affine affine_from_stored(uint16_t bits, uint8_t z) {
 // the scale is 0.
 __device__ __forceinline__ uint32_t affine_code(float v, const Affine& a) {
   if (a.sf == 0.0f) return 0u;
-  const float u = __fadd_rn(__fdiv_rn(v, a.sf), a.zf);
+  const float u = __fadd_rn(div_by_scale(v, a.sf, a.r), a.zf);
   return static_cast<uint32_t>(fminf(fmaxf(rintf(u), 0.0f), 15.0f));
+}
+
+// The same code for a group whose every |v| * r stays below 2^99 (checked
+// once per group), with a finite non-zero scale: the quotient by Markstein's
+// step with no overflow test, the clamp before the rounding (the same
+// result: the bounds are integers), and rint as the exact addition of
+// 1.5 * 2^23, whose low mantissa bits then hold the code.
+__device__ __forceinline__ uint32_t affine_code_fast(float v, const Affine& a) {
+  const float q = __fmul_rn(v, a.r);
+  const float e = __fmaf_rn(-q, a.sf, v);
+  const float u = __fadd_rn(__fmaf_rn(e, a.r, q), a.zf);
+  const float uc = fminf(fmaxf(u, 0.0f), 15.0f);
+  return __float_as_uint(__fadd_rn(uc, 12582912.0f)) & 0xFu;
 }
 
 // Fast path: K % 8 == 0, group = 8 LPG with LPG a power of two <= 32, w
@@ -110,15 +153,28 @@ __global__ void __launch_bounds__(256) quantize_affine_window_kernel(
   if (wbeg >= wend) return;
   int64_t row = wbeg / windows_per_row;
   int64_t win = wbeg - row * windows_per_row;
+  // The next window's weights are loaded while this one is coded, so that
+  // every warp keeps two loads in flight.
+  auto load_window = [&](int64_t r, int64_t wn, float (&dst)[8]) {
+    const int64_t k = wn * 256 + 8 * lane;
+    if (k < K) {
+      load8<T>(w + r * K + k, dst);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = 0.0f;
+    }
+  };
+  float vnext[8];
+  load_window(row, win, vnext);
   for (int64_t wi = wbeg; wi < wend; ++wi) {
     const int64_t k0 = win * 256 + 8 * lane;
     const bool active = k0 < K;
     float v[8];
-    if (active) {
-      load8<T>(w + row * K + k0, v);
-    } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    for (int i = 0; i < 8; ++i) v[i] = vnext[i];
+    if (wi + 1 < wend) {
+      const bool wrap = win + 1 == windows_per_row;
+      load_window(wrap ? row + 1 : row, wrap ? 0 : win + 1, vnext);
     }
     float mn = active ? v[0] : __int_as_float(0x7F800000);   // +inf
     float mx = active ? v[0] : __int_as_float(0xFF800000);   // -inf
@@ -135,8 +191,15 @@ __global__ void __launch_bounds__(256) quantize_affine_window_kernel(
     if (active) {
       const Affine a = affine_params(mn, mx);
       uint32_t word = 0u;
+      const bool fast = a.sf != 0.0f && a.r != 0.0f &&
+                        __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), a.r) < 0x1p99f;
+      if (fast) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) word |= affine_code(v[i], a) << (4 * i);
+        for (int i = 0; i < 8; ++i) word |= affine_code_fast(v[i], a) << (4 * i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= affine_code(v[i], a) << (4 * i);
+      }
       *reinterpret_cast<uint32_t*>(packed + row * (K >> 1) + (k0 >> 1)) = word;
       if ((lane & (LPG - 1)) == 0) {
         const int64_t gi = row * G + k0 / (8 * LPG);

@@ -77,6 +77,68 @@ def test_quantize_affine_bit_exact(dtype, N, K, group):
     assert np.array_equal(packed.cpu().numpy(), p_ref)
 
 
+def _tie_weights(N, K, group, seed):
+    """fp32 weights whose quotients w / s + z fall on, and one ulp either side
+    of, the half-integers k + 1/2 that rint rounds to even: each group gets
+    its extremes first, then values (k + 1/2 - z) s for its own scale s and
+    zero point z, kept inside the extremes."""
+    rng = np.random.default_rng(seed)
+    w = np.zeros((N, K), dtype=np.float32)
+    for n in range(N):
+        for g0 in range(0, K, group):
+            g1 = min(g0 + group, K)
+            a = np.float32(rng.uniform(0.01, 1.0))    # -min
+            b = np.float32(rng.uniform(0.01, 1.0))    # max
+            s = np.float32(np.float16(np.float32(b + a) / np.float32(15)))
+            z = float(np.clip(np.rint(np.float32(a / s)), 0, 15))
+            vals = [np.float32(-a), np.float32(b)]
+            for j in range(g1 - g0 - 2):
+                t = np.float32((rng.integers(0, 15) + 0.5 - z) * float(s))
+                t = [t, np.nextafter(t, np.float32(np.inf)), np.nextafter(t, np.float32(-np.inf))][j % 3]
+                vals.append(np.float32(min(max(t, -a), b)))
+            w[n, g0:g1] = np.array(vals[: g1 - g0], dtype=np.float32)
+    return torch.from_numpy(w).to(DEV)
+
+
+@pytest.mark.parametrize("exponents", [(0,), (-23, -25), ("subnormal",), (19,)])
+def test_affine_scale_division_exhaustive_over_mantissas(exponents):
+    """fp16(fp32(d / 15)) on every fp32 mantissa of the given binades (and on
+    every subnormal): groups of two weights {0, d} have the range d, and the
+    kernel's division by the constant 15 must equal the IEEE division the
+    oracle uses, bit for bit.  The binades cover the fp16 subnormal and
+    overflow boundaries of the scale."""
+    mant = np.arange(1 << 23, dtype=np.uint32)
+    parts = []
+    for e in exponents:
+        if e == "subnormal":
+            parts.append(mant.view(np.float32))
+        else:
+            parts.append(((np.uint32(e + 127) << 23) | mant).view(np.float32))
+    d = np.concatenate(parts)
+    w = np.zeros((1, 2 * d.size), dtype=np.float32)
+    w[0, 1::2] = d
+    wt = torch.from_numpy(w).to(DEV)
+    packed, scales, zeros, _ = q4.quantize_int4_affine(wt, 2)
+    p_ref, s_ref, z_ref, _ = oracle.quantize_uint4_affine(w, 2)
+    got = scales.cpu().view(torch.int16).numpy().view(np.uint16)[0]
+    bad = np.flatnonzero(got != s_ref.view(np.uint16)[0])
+    assert bad.size == 0, f"{bad.size} scales differ, first d = {d[bad[0]]!r}"
+    assert np.array_equal(zeros.cpu().numpy(), z_ref)
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+
+
+@pytest.mark.parametrize("N, K, group", [(24, 4096, 128), (16, 1024, 32), (9, 1000, 100)])
+def test_quantize_affine_ties_bit_exact(N, K, group):
+    """Quotients on and next to the rounding ties: the codes must be those of
+    the IEEE division, bit for bit."""
+    w = _tie_weights(N, K, group, seed=N + K + group)
+    packed, scales, zeros, _ = q4.quantize_int4_affine(w, group)
+    p_ref, s_ref, z_ref, _ = _oracle_affine(w, group)
+    assert np.array_equal(scales.cpu().view(torch.int16).numpy().view(np.uint16), s_ref.view(np.uint16))
+    assert np.array_equal(zeros.cpu().numpy(), z_ref)
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
 @pytest.mark.parametrize("N, K, group", [(64, 4096, 128), (33, 1000, 40), (16, 512, 32)])
 def test_dequantize_affine_bit_exact(dtype, N, K, group):
