@@ -94,6 +94,9 @@ namespace {
 #ifndef INT4_DECODE_SMALL
 #define INT4_DECODE_SMALL 1
 #endif
+#ifndef INT4_DECODE_FLAT
+#define INT4_DECODE_FLAT 1
+#endif
 #ifndef INT4_DECODE_I8_TILES
 #define INT4_DECODE_I8_TILES 2
 #endif
@@ -1563,6 +1566,330 @@ bool small_applies(int64_t K, int group, int64_t N) {
   return (N + 15) / 16 <= static_cast<int64_t>(kSmallCtasPerSm) * num_sms();
 }
 
+// ---------------- matrices that fit in shared memory ----------------
+// Decode for matrices whose 16-row tiles all fit in shared memory at once
+// (one wave, each tile's packed rows resident in its CTA): right after the
+// dependency wait, every CTA issues bulk copies of its whole tile (row by
+// row, in chunks of kFlatChunk bytes of each row, one barrier per chunk) and,
+// for M <= 2 when it fits, of x, and loads the tile's scales into shared
+// memory, so the whole matrix is requested in one round trip and the loop
+// over K reads shared memory only.  W warps split K as in
+// decode_small_kernel (warp w takes 128-k blocks w, w + W, ...), with the
+// small kernel's arithmetic per block; the warps' partials are added in warp
+// order.
+#ifndef INT4_FLAT_PDL_LATE
+#define INT4_FLAT_PDL_LATE 1  // let the next kernel launch only after this CTA's loop
+#endif
+#ifndef INT4_FLAT_CHUNK
+#define INT4_FLAT_CHUNK 2048
+#endif
+constexpr int kFlatChunk = INT4_FLAT_CHUNK;  // bytes of each row per copy chunk (a multiple of 64)
+
+// Row stride of the resident tile: Kp, padded so that the quarter warp's
+// 16-byte loads of rows g and g + 1 fall in different banks.
+__host__ __device__ constexpr int64_t flat_row_stride(int64_t Kp) {
+  return Kp % 128 == 0 ? Kp + 64 : Kp;
+}
+
+// Shared-memory layout of a CTA: the tile's rows, x (if staged), the tile's
+// scales [16, G] (and zero points), the barriers (chunks, then x).
+struct FlatLayout {
+  int64_t rstride, off_x, off_s, off_z, off_bar, bytes;
+  int nch;
+};
+__host__ __device__ inline FlatLayout flat_layout(int64_t K, int G, int M, bool xs, bool asym) {
+  FlatLayout L;
+  const int64_t Kp = K / 2;
+  L.rstride = flat_row_stride(Kp);
+  L.nch = static_cast<int>((Kp + kFlatChunk - 1) / kFlatChunk);
+  L.off_x = 16 * L.rstride;
+  L.off_s = L.off_x + (xs ? static_cast<int64_t>(M) * K * 2 : 0);
+  L.off_z = L.off_s + (16 * static_cast<int64_t>(G) * 2 + 15) / 16 * 16;
+  L.off_bar = L.off_z + (asym ? (16 * static_cast<int64_t>(G) + 15) / 16 * 16 : 0);
+  L.bytes = L.off_bar + 8 * (L.nch + 1);
+  return L;
+}
+
+template <typename TX, int NT, bool ASYM, int W, bool XS>
+__global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
+    const TX* __restrict__ x, const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
+    const uint8_t* __restrict__ zeros, Epilogue ep, float* __restrict__ y, int64_t K, int group,
+    int G, int M, int64_t N, int KB, uint32_t* status) {
+  static_assert(!XS || NT == 1, "x is staged for M <= 2 only");
+  extern __shared__ __align__(16) uint8_t tile_smem[];
+  __shared__ float red[W * NT * 4 * 32];
+  __shared__ uint32_t abort_word;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int64_t Kp = K / 2;
+  const FlatLayout L = flat_layout(K, G, M, XS, ASYM);
+  const int nch = L.nch;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tile_smem + L.off_bar);  // chunks, then x
+  const uint32_t tbase = ptx::smem_u32(tile_smem);
+  uint16_t* s_sc = reinterpret_cast<uint16_t*>(tile_smem + L.off_s);
+  uint8_t* s_z = tile_smem + L.off_z;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 16;
+  const int rows = static_cast<int>(N - row0 < 16 ? N - row0 : 16);
+  const WaitCtx wc{&abort_word, status};
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nch + (XS ? 1 : 0); ++i) ptx::mbar_init(ptx::smem_u32(&bars[i]), 1);
+    abort_word = 0u;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  // Launched as a programmatic dependent of what precedes it on the stream:
+  // the set-up above overlaps that kernel's tail; nothing is read before the
+  // wait.  The next kernel is let in only after this CTA's loop: its CTAs,
+  // small enough to sit beside these ones while they wait for this grid,
+  // took issue slots from the loop (4096 x 4096 at M = 1: 8.3 against
+  // 6.2 us per call back to back).
+  if (!INT4_FLAT_PDL_LATE) ptx::launch_dependents();
+  ptx::grid_dependency_wait();
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < nch; ++i) {
+        const int64_t off = static_cast<int64_t>(i) * kFlatChunk;
+        const int64_t cb = Kp - off < kFlatChunk ? Kp - off : kFlatChunk;
+        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&bars[i]), static_cast<uint32_t>(rows * cb));
+      }
+      if (XS) {
+        const uint32_t xb = static_cast<uint32_t>(static_cast<int64_t>(M) * K * 2);
+        ptx::mbar_arrive_expect_tx(ptx::smem_u32(&bars[nch]), xb);
+        ptx::bulk_load(tbase + static_cast<uint32_t>(L.off_x), x, xb, ptx::smem_u32(&bars[nch]));
+      }
+    }
+    __syncwarp();
+    // Chunk-major order: every row's first chunk is requested first.
+    for (int i = lane; i < rows * nch; i += 32) {
+      const int r = i % rows, ch = i / rows;
+      const int64_t off = static_cast<int64_t>(ch) * kFlatChunk;
+      const int64_t cb = Kp - off < kFlatChunk ? Kp - off : kFlatChunk;
+      ptx::bulk_load(tbase + static_cast<uint32_t>(r * L.rstride + off), packed + (row0 + r) * Kp + off,
+                     static_cast<uint32_t>(cb), ptx::smem_u32(&bars[ch]));
+    }
+  }
+  // The tile's scales (and zero points): rows*G contiguous values.
+  for (int i = threadIdx.x; i < rows * G; i += blockDim.x) {
+    s_sc[i] = __ldg(scales + row0 * G + i);
+    if (ASYM) s_z[i] = __ldg(zeros + row0 * G + i);
+  }
+  __syncthreads();
+  // Rows past N are never copied; their (stale) words and scales only reach
+  // outputs that are not stored.
+  const uint32_t wa = tbase + static_cast<uint32_t>(g * L.rstride + 16 * c);
+  const uint32_t wb = tbase + static_cast<uint32_t>((g + 8) * L.rstride + 16 * c);
+  float tot[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tot[nt][i] = 0.0f;
+  // x fragments of block kb from global memory (L2-resident), one block ahead.
+  auto load_x = [&](int kb, uint4 (&xf)[4][NT]) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int n = g + 8 * nt;
+      const TX* xp = x + static_cast<int64_t>(n < M ? n : 0) * K + static_cast<int64_t>(kb) * 128 + 32 * c;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        xf[j][nt] = (n < M) ? __ldg(reinterpret_cast<const uint4*>(xp + 8 * j)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  uint4 xc[4][NT], xn[4][NT];
+  bool ok = true;
+  if (XS) {
+    ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&bars[nch]), 0u, wc));
+  } else if (warp < KB) {
+    load_x(warp, xc);
+  }
+  const int n0 = g < M ? g : 0;  // staged x: this lane's batch row
+  for (int kb = warp; ok && kb < KB; kb += W) {
+    if (XS) {
+      const uint32_t xs = tbase + static_cast<uint32_t>(L.off_x + (static_cast<int64_t>(n0) * K + kb * 128 + 32 * c) * 2);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) xc[j][0] = g < M ? ptx::lds128(xs + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
+    } else if (kb + W < KB) {
+      load_x(kb + W, xn);
+    }
+    const int ch = (kb * 64) / kFlatChunk;
+    ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&bars[ch]), 0u, wc));
+    if (!ok) break;
+    const int gi = static_cast<int>(static_cast<int64_t>(kb) * 128 / group);
+    const uint4 ua = ptx::lds128(wa + kb * 64);
+    const uint4 ub = ptx::lds128(wb + kb * 64);
+    const uint32_t wva[4] = {ua.x, ua.y, ua.z, ua.w};
+    const uint32_t wvb[4] = {ub.x, ub.y, ub.z, ub.w};
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+    const uint32_t zba = ASYM ? Cvt<TX>::zero_bias(s_z[g * G + gi]) : Cvt<TX>::kMagic;
+    const uint32_t zbb = ASYM ? Cvt<TX>::zero_bias(s_z[(g + 8) * G + gi]) : Cvt<TX>::kMagic;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t pa[4], pb[4];
+      expand<TX, ASYM>(wva[j], pa, zba);
+      expand<TX, ASYM>(wvb[j], pb, zbb);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4 xf = pair_x(xc[j][nt]);
+        Cvt<TX>::mma(acc[nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
+        Cvt<TX>::mma(acc[nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
+      }
+    }
+    const float sa = f16_bits_to_float(s_sc[g * G + gi]);
+    const float sb = f16_bits_to_float(s_sc[(g + 8) * G + gi]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      tot[nt][0] = fmaf(acc[nt][0], sa, tot[nt][0]);
+      tot[nt][1] = fmaf(acc[nt][1], sa, tot[nt][1]);
+      tot[nt][2] = fmaf(acc[nt][2], sb, tot[nt][2]);
+      tot[nt][3] = fmaf(acc[nt][3], sb, tot[nt][3]);
+    }
+    if (!XS) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) xc[j][nt] = xn[j][nt];
+    }
+  }
+  if (INT4_FLAT_PDL_LATE) ptx::launch_dependents();
+  // Warps' partials summed in warp order.
+  constexpr int kPerWarp = NT * 4 * 32;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) red[warp * kPerWarp + (nt * 4 + i) * 32 + lane] = tot[nt][i];
+  __syncthreads();
+  if (abort_word != 0u) {
+    // A wait gave up: let the copies in flight land before the CTA's
+    // shared memory is released, and store nothing.
+    if (threadIdx.x == 0)
+      for (int i = 0; i < nch + (XS ? 1 : 0); ++i) drain_bar(ptx::smem_u32(&bars[i]), 0u);
+    return;
+  }
+  for (int e = threadIdx.x; e < kPerWarp; e += blockDim.x) {
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) sum += red[w * kPerWarp + e];
+    const int ln = e & 31;
+    const int i = (e >> 5) & 3;
+    const int nt = e >> 7;
+    const int m = nt * 8 + 2 * (ln & 3) + (i & 1);
+    const int64_t row = row0 + (ln >> 2) + ((i < 2) ? 0 : 8);
+    if (m < M && row < N) y[static_cast<int64_t>(m) * N + row] = ep.apply(sum, row);
+  }
+}
+
+// CTAs per SM of one shared-memory decode kernel for a layout of `bytes`
+// bytes, queried once per device and size.
+template <typename TX, int NT, bool ASYM, int W, bool XS>
+int flat_occupancy(int64_t bytes) {
+  constexpr int kMaxDevices = 64;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  static thread_local int64_t last_bytes[kMaxDevices] = {};
+  static thread_local int last_occ[kMaxDevices] = {};
+  if (last_bytes[dev] == bytes) return last_occ[dev];
+  int occ = 0;
+  // The opt-in is the device's limit less the kernel's static shared memory,
+  // the same for every shape, so concurrent callers agree.
+  const void* fn = reinterpret_cast<const void*>(decode_flat_kernel<TX, NT, ASYM, W, XS>);
+  int optin = 0;
+  cudaFuncAttributes fa;
+  bool failed = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+                cudaFuncGetAttributes(&fa, fn) != cudaSuccess;
+  if (!failed) {
+    const int64_t max_dyn = static_cast<int64_t>(optin) - static_cast<int64_t>(fa.sharedSizeBytes);
+    if (bytes <= max_dyn)
+      failed = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(max_dyn)) !=
+                   cudaSuccess ||
+               cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, W * 32, static_cast<size_t>(bytes)) !=
+                   cudaSuccess;
+  }
+  if (failed) {
+    occ = 0;
+    (void)cudaGetLastError();  // a refused query only rules this kernel out
+  }
+  last_bytes[dev] = bytes;
+  last_occ[dev] = occ;
+  return occ;
+}
+
+// Kernel choice for a shape: warps per CTA (8, else 4) and whether x is
+// staged (M <= 2, preferred), the first whose tiles fit one wave; 0 when
+// none does (the shape then takes another decode kernel).
+constexpr int kFlatXs = 0x100;
+
+template <typename TX, int NT, bool ASYM, int W, bool XS>
+bool flat_fits(int64_t K, int G, int M, int64_t tiles) {
+  const int64_t bytes = flat_layout(K, G, M, XS, ASYM).bytes;
+  return tiles <= static_cast<int64_t>(flat_occupancy<TX, NT, ASYM, W, XS>(bytes)) * num_sms();
+}
+
+template <typename TX, bool ASYM>
+int flat_choice(int64_t K, int group, int64_t M, int64_t N) {
+  if (!INT4_DECODE_FLAT || group % 128 != 0 || K % 128 != 0 || M > 16) return 0;
+  // Where the integer kernel would convert x inside its CTAs (M <= 2 on a
+  // matrix too tall for the small-matrix kernel), it is faster: its
+  // arithmetic takes a quarter of the instructions per weight.
+  if (M <= kFuseMaxM && !small_applies(K, group, N)) return 0;
+  const int G = static_cast<int>(K / group + (K % group != 0));
+  const int64_t tiles = (N + 15) / 16;
+  const int m = static_cast<int>(M);
+  if (M <= 8) {
+    if (M <= 2 && flat_fits<TX, 1, ASYM, 8, true>(K, G, m, tiles)) return 8 | kFlatXs;
+    if (flat_fits<TX, 1, ASYM, 8, false>(K, G, m, tiles)) return 8;
+    if (M <= 2 && flat_fits<TX, 1, ASYM, 4, true>(K, G, m, tiles)) return 4 | kFlatXs;
+    if (flat_fits<TX, 1, ASYM, 4, false>(K, G, m, tiles)) return 4;
+    return 0;
+  }
+  if (flat_fits<TX, 2, ASYM, 8, false>(K, G, m, tiles)) return 8;
+  if (flat_fits<TX, 2, ASYM, 4, false>(K, G, m, tiles)) return 4;
+  return 0;
+}
+
+template <typename TX, int NT, bool ASYM, int W, bool XS>
+cudaError_t launch_flat_w(const TX* x, const uint8_t* packed, const uint16_t* scales,
+                          const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                          int64_t N, float* y, cudaStream_t stream) {
+  uint32_t* status = status_word();
+  if (status == nullptr) return cudaErrorInvalidSymbol;
+  const int G = static_cast<int>((K + group - 1) / group);
+  const int KB = static_cast<int>((K + 127) / 128);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((N + 15) / 16));
+  cfg.blockDim = dim3(W * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(flat_layout(K, G, static_cast<int>(M), XS, ASYM).bytes);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_flat_kernel<TX, NT, ASYM, W, XS>, x, packed, scales, zeros, ep,
+                            y, K, group, G, static_cast<int>(M), N, KB, status);
+}
+
+template <typename TX, bool ASYM>
+cudaError_t launch_flat(int choice, const TX* x, const uint8_t* packed, const uint16_t* scales,
+                        const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                        int64_t N, float* y, cudaStream_t stream) {
+  const bool xs = (choice & kFlatXs) != 0;
+  const int w = choice & 0xFF;
+  if (M <= 8) {
+    if (w == 8)
+      return xs ? launch_flat_w<TX, 1, ASYM, 8, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+                : launch_flat_w<TX, 1, ASYM, 8, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+    return xs ? launch_flat_w<TX, 1, ASYM, 4, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+              : launch_flat_w<TX, 1, ASYM, 4, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  }
+  return w == 8 ? launch_flat_w<TX, 2, ASYM, 8, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+                : launch_flat_w<TX, 2, ASYM, 4, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+}
+
+
 // ---------------- host side: scratch, schedule, launch ----------------
 // A decode call may need device scratch: one arrival counter per CTA (zero
 // when the call starts; every call leaves its counters zero), two partial-
@@ -1917,6 +2244,12 @@ cudaError_t run_i8(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, D
 template <typename TX, bool ASYM>
 cudaError_t run_decode(const DecodeArgs& a, bool scratch, const DecodeScratch* sc, DecodeNeed* need,
                        bool launch) {
+  if (const int fw = flat_choice<TX, ASYM>(a.K, a.group, a.M, a.N)) {
+    *need = DecodeNeed{};
+    if (!launch) return cudaSuccess;
+    return launch_flat<TX, ASYM>(fw, static_cast<const TX*>(a.x), a.packed, a.scales, a.zeros, a.ep,
+                                 a.K, a.group, a.M, a.N, a.y, a.stream);
+  }
   if (small_applies(a.K, a.group, a.N)) {
     *need = DecodeNeed{};
     if (!launch) return cudaSuccess;

@@ -186,13 +186,15 @@ def _check(y, x, packed, scales, zeros, K, group, c, bias=None, relu=False, cols
 # Shapes per kernel path: (M, N, K, group, path, workspace)
 PATHS = [
     (1, 28672, 4096, 128, q4.PATH_DECODE, None),     # integer kernel, x converted in the CTA
-    (2, 11008, 4096, 256, q4.PATH_DECODE, None),
-    (5, 11008, 4096, 128, q4.PATH_DECODE, None),     # integer kernel, x digit records
+    (2, 18000, 4096, 256, q4.PATH_DECODE, None),
+    (5, 18000, 4096, 128, q4.PATH_DECODE, None),     # integer kernel, x digit records
     (16, 9000, 2048, 128, q4.PATH_DECODE, None),
-    (4, 11008, 4096, 128, q4.PATH_DECODE, False),    # no workspace: the 16-bit kernel
+    (4, 18000, 4096, 128, q4.PATH_DECODE, False),    # no workspace: the 16-bit kernel
     (3, 9000, 2048, 64, q4.PATH_DECODE, None),       # 16-bit kernel, group 64
     (12, 5000, 2048, 32, q4.PATH_DECODE, None),      # 16-bit kernel, group 32
-    (4, 2048, 4096, 128, q4.PATH_DECODE, None),      # small-matrix kernel
+    (4, 2048, 4096, 128, q4.PATH_DECODE, None),      # resident-tile kernel
+    (16, 4096, 11008, 128, q4.PATH_DECODE, None),    # resident-tile kernel, two n-tiles
+    (3, 2048, 32768, 128, q4.PATH_DECODE, None),     # small-matrix kernel (rows too long)
     (256, 512, 1024, 128, q4.PATH_PREFILL, None),    # tensor-core kernel, K split (4 tiles)
     (300, 384, 2048, 64, q4.PATH_PREFILL, None),
     (300, 384, 2048, 64, q4.PATH_PREFILL, False),    # tensor-core kernel, whole K

@@ -83,8 +83,9 @@ def _block_integer_form(x64, K):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M", [1, 2, 4, 16])
 @pytest.mark.parametrize("mode", ["workspace", "no_workspace", "noalloc"])
-def test_decode_bound_with_large_x_on_zero_weights(dtype, M, mode):
-    N, K, group = 8192, 2048, 128
+@pytest.mark.parametrize("N", [8192, 20000])   # M > 2: resident tiles, then the integer kernel
+def test_decode_bound_with_large_x_on_zero_weights(dtype, M, mode, N):
+    K, group = 2048, 128
     assert q4.matmul_select(dtype, K, group, M, N) == q4.PATH_DECODE
     packed, scales, _ = _weights_off_the_block_start(N, K, group)
     x = _adversarial_x(M, K, dtype)
@@ -106,11 +107,12 @@ def test_decode_bound_with_large_x_on_zero_weights(dtype, M, mode):
 
 
 @pytest.mark.parametrize("M", [1, 2, 5, 16])
-def test_decode_blocks_flagged_in_some_rows_only(M):
+@pytest.mark.parametrize("N", [9000, 20000])   # M > 2: resident tiles, then the integer kernel
+def test_decode_blocks_flagged_in_some_rows_only(M, N):
     """Only some batch rows of some blocks are wide; every row of such a block
     takes the 16-bit products, the other blocks stay on the integer form, and
     the whole output meets the bound."""
-    N, K, group = 9000, 4096, 256
+    K, group = 4096, 256
     packed, scales, _ = q4.quantize_int4(
         make_weights(N, K, seed=31, device=DEV, dtype=torch.float32, dist="student_t3",
                      zero_group_frac=0.02, group=group), group)
@@ -126,10 +128,12 @@ def test_decode_blocks_flagged_in_some_rows_only(M):
     assert_matmul_close(y, x, packed, scales, K, group, TOL_HALF, cols=cols)
 
 
-def test_decode_silu_like_activations():
+@pytest.mark.parametrize("N", [11008, 18000])
+def test_decode_silu_like_activations(N):
     """Activations shaped like a gated MLP's (x sigmoid(x) of wide normals):
-    values down to about 1e-12 next to values near 20 in the same block."""
-    N, K, group, M = 11008, 4096, 128, 4
+    values down to about 1e-12 next to values near 20 in the same block, on
+    the resident-tile kernel (N = 11008) and the integer one (N = 18000)."""
+    K, group, M = 4096, 128, 4
     packed, scales, _ = q4.quantize_int4(
         make_weights(N, K, seed=5, device=DEV, dtype=torch.float32), group)
     z = make_activations(M, K, seed=8, device=DEV, dtype=torch.float32) * 8.0
@@ -153,7 +157,7 @@ def _call_ws(x, packed, scales, K, group, y, ws, nbytes):
 
 @pytest.mark.parametrize("M, N, K, group", [
     (1, 28672, 8192, 128),    # split tiles, x converted in the matmul
-    (4, 11008, 4096, 128),    # split tiles and x digit records
+    (4, 18000, 4096, 128),    # split tiles and x digit records
     (16, 20000, 4096, 128),
     (3, 9000, 2048, 64),      # the 16-bit kernel, split
 ])
@@ -184,8 +188,8 @@ def test_workspace_size_is_enforced_and_sufficient(M, N, K, group):
 
 
 @pytest.mark.parametrize("M, N, K, group", [
-    (1, 28672, 8192, 128), (2, 11008, 4096, 128), (4, 11008, 4096, 128), (16, 20000, 4096, 128),
-    (8, 9000, 2048, 64), (12, 5000, 2048, 32), (1, 4096, 4096, 128),
+    (1, 28672, 8192, 128), (2, 18000, 4096, 128), (4, 18000, 4096, 128), (16, 20000, 4096, 128),
+    (8, 9000, 2048, 64), (12, 5000, 2048, 32), (1, 4096, 4096, 128), (4, 11008, 4096, 128),
 ])
 def test_matmul_without_workspace(M, N, K, group):
     """int4_matmul (no workspace): runs of whole row tiles, and at M > 2 the
@@ -211,8 +215,8 @@ def test_matmul_without_workspace(M, N, K, group):
 def test_workspace_shared_by_shapes_on_one_stream():
     """One zero-filled workspace, large enough for every call, serves calls of
     different shapes (different CTA counts and regions) back to back."""
-    shapes = [(1, 28672, 8192, 128), (16, 20000, 4096, 128), (4, 11008, 4096, 128),
-              (2, 9000, 12288, 128), (3, 9000, 2048, 64)]
+    shapes = [(1, 28672, 8192, 128), (16, 20000, 4096, 128), (4, 18000, 4096, 128),
+              (2, 9000, 12288, 128), (3, 9000, 2048, 64), (1, 4096, 4096, 128)]
     need = max(q4.matmul_workspace_size(torch.bfloat16, K, g, M, N) for M, N, K, g in shapes)
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     cases = []

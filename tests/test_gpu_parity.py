@@ -332,6 +332,11 @@ def test_matmul_tiny_case_fp32():
     (3, 300, 4096, 64), (9, 200, 1024, 32), (1, 2304, 768, 32), (1, 768, 3072, 64),
     (16, 77, 8224, 128), (5, 1000, 2048, 256), (2, 64, 96, 32), (7, 129, 160, 32),
     (12, 33, 640, 64), (1, 1, 32, 32),
+    (4, 18000, 4096, 128),   # too tall for resident tiles: the integer kernel
+    (1, 2048, 32768, 128),   # rows too long for resident tiles: the small-matrix kernel
+    (9, 1500, 40960, 256),
+    (16, 11000, 4096, 128),  # resident tiles, 4 warps per tile, ragged last tile
+    (5, 1001, 2048, 512),
 ])
 def test_matmul_paths(path, dtype, M, N, K, group):
     packed, scales, _ = _quantized(N, K, group, seed=M + N + K)
@@ -401,6 +406,8 @@ def test_matmul_decode_is_deterministic_and_matches_simt():
     (8, 1000, 12288, 128),   # ragged last tile, runs cross tile boundaries
     (2, 37, 4096, 256),      # a single short tile, group spanning two blocks
     (5, 6000, 1024, 128),    # many tiles, runs of whole tiles plus boundary pieces
+    (4, 20000, 2048, 128),   # the integer kernel with digit records, split runs
+    (1, 30001, 1024, 256),   # the integer kernel, x converted in the CTA, ragged
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_matmul_decode_split_tiles(M, N, K, group, dtype):
@@ -447,11 +454,11 @@ def _wide_range_x(M, K, dtype, seed, outlier=2.0 ** 12, tiny=2.0 ** -14):
     return x.to(dtype).to(DEV)
 
 
-# Decode kernels by matrix height: N = 512 fits one wave of 16-row tiles and
-# takes the small-matrix kernel (bf16 expansion); N = 8192 takes the integer
-# tensor-core kernel (x as digits: converted in the CTA at M <= 2, by the
-# digits kernel above).
-DECODE_KERNEL_N = [512, 8192]
+# Decode kernels by matrix height: N = 512 keeps its packed tiles resident
+# in shared memory (bf16 expansion); N = 20000 takes the integer tensor-core
+# kernel (x as digits: converted in the CTA at M <= 2, by the digits kernel
+# above).
+DECODE_KERNEL_N = [512, 20000]
 
 
 def _cols(N, seed):

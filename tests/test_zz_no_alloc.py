@@ -17,11 +17,12 @@ DEV = "cuda"
 
 @pytest.mark.parametrize("M, N, K, group, dtype", [
     (1, 28672, 8192, 128, torch.bfloat16),   # partial tiles at most run ends
-    (4, 4096, 4096, 128, torch.bfloat16),    # the small-matrix kernel: no scratch at all
-    (4, 11008, 4096, 128, torch.bfloat16),   # x digits (two n-tiles) and split tiles
+    (4, 4096, 4096, 128, torch.bfloat16),    # resident tiles: no scratch at all
+    (1, 2048, 32768, 128, torch.bfloat16),   # the small-matrix kernel: no scratch at all
+    (4, 18000, 4096, 128, torch.bfloat16),   # x digits (two n-tiles) and split tiles
     (8, 28672, 4096, 128, torch.bfloat16),   # x digits (four n-tiles), 64-row tiles
     (16, 20000, 4096, 128, torch.bfloat16),  # x digits in the static array
-    (2, 11008, 4096, 256, torch.float16),    # x converted inside the matmul
+    (2, 18000, 4096, 256, torch.float16),    # x converted inside the matmul
     (16, 1000, 12288, 64, torch.float16),    # 64-row tiles, ragged last tile
     (3, 37, 4096, 32, torch.bfloat16),       # a single short tile
 ])
