@@ -57,8 +57,8 @@ KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
     "prefill": (805_800_000 + 914_570_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
                 "7ef3d9ac2d504ffa33065761b2ba66b252ebe2512b521d94f19c78000af6ad93"),
-    "decode": (125_434_624 + 4_626_688, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
-               "178d4852998a2a29a2efcc14e285759e676798d29112d05fa6ce6942d811fe84"),
+    "decode": (125_550_000 + 3_400_000, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
+               "796f562ceeeee2604aedc6feabc2f31bf88accadb46ae8d096833e85fec80aa7"),
     "quantize": (469_856_256 + 104_254_208, "dequant_gemm_int4_b200/csrc/quantize.cu",
                  "24a51fde9c6ea1afd8a159345f565f16441d8a085e241e8e6d8d123c71573f57"),
     "unpack": (117_453_056 + 182_672_128, "dequant_gemm_int4_b200/csrc/unpack.cu",
