@@ -390,6 +390,154 @@ def prefill_shape_rows(dev, peaks, reps: int = 3, windows: int = 5):
     return rows
 
 
+DISTILGPT2_SHAPES = [(2304, 768), (3072, 768), (768, 3072)]
+DISTILGPT2_GROUPS = (32, 64)
+DISTILGPT2_M_PREFILL = 1024
+BULK_QUANT = [((28672, 8192), (32, 64)), ((8192, 28673), (32, 64, 128))]
+DECODE_GROUPS = (32, 64)
+
+
+def _graph_us(fn, reps: int, calls: int) -> float:
+    """Per-call device time of `fn` (calls launches) replayed from a CUDA graph."""
+    import torch
+
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * calls)
+
+
+def config_rows(dev, peaks, flush_l2, reps: int = 5):
+    """The other configured workloads, each timed on its own after the step:
+    the distilgpt2-shaped linears (groups 32 and 64, fp16 x; M = 1 decode back
+    to back over weight copies that exceed L2, from a CUDA graph, and M = 1024
+    prefill back to back, its operands L2-resident), the bulk quantize and
+    unpack at groups 32 and 64 and odd K (each call after an L2 flush, median
+    of `reps`), and the group-32/64 decode kernel on W [28672, 8192] at M = 1."""
+    import statistics
+
+    import torch
+
+    import dequant_gemm_int4_b200 as q4
+    from workloads import make_activations, make_weights
+
+    L = q4.lib()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    sp = lambda: torch.cuda.current_stream(dev).cuda_stream  # noqa: E731
+
+    def call(rc):
+        if rc != 0:
+            raise RuntimeError(f"INT4 library error {rc}: {L.int4_last_error()}")
+
+    def decode_us(x, copies, K, g, M, N, xcode):
+        nb = q4.matmul_workspace_size(x.dtype, K, g, M, N, dev)
+        ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device=dev)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+
+        def run():
+            for pk, sc in copies:
+                call(L.int4_matmul_ws(x.data_ptr(), xcode, pk.data_ptr(), sc.data_ptr(), K, g, M, N,
+                                      y.data_ptr(), ws.data_ptr(), ws.numel(), sp()))
+        return _graph_us(run, 10, len(copies))
+
+    def flushed_ms(fn):
+        times = []
+        for _ in range(reps):
+            flush_l2()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    out = {"distilgpt2": {}, "bulk_quantize": {}, "decode_groups": {}}
+    f16 = q4.DTYPE_F16
+    for N, K in DISTILGPT2_SHAPES:
+        w = make_weights(N, K, seed=N + K, device=dev, dtype=torch.float32)
+        for g in DISTILGPT2_GROUPS:
+            packed, scales, _ = q4.quantize_int4(w, g)
+            per_copy = packed.numel() + 2 * scales.numel()
+            ncopy = max(2, -(-3 * l2 // per_copy))
+            copies = [(packed, scales)] + [(packed.clone(), scales.clone()) for _ in range(ncopy - 1)]
+            x1 = make_activations(1, K, seed=1, device=dev, dtype=torch.float16)
+            us = decode_us(x1, copies, K, g, 1, N, f16)
+            gbs = N * (K // 2) / (us * 1e-6) / 1e9
+            del copies
+            M = DISTILGPT2_M_PREFILL
+            xp = make_activations(M, K, seed=2, device=dev, dtype=torch.float16)
+            yp = torch.empty((M, N), dtype=torch.float32, device=dev)
+            nb = q4.matmul_workspace_size(torch.float16, K, g, M, N, dev)
+            wsp = torch.zeros(max(nb, 256), dtype=torch.uint8, device=dev)
+            pus = _graph_us(lambda: call(L.int4_matmul_ws(xp.data_ptr(), f16, packed.data_ptr(),
+                                                          scales.data_ptr(), K, g, M, N, yp.data_ptr(),
+                                                          wsp.data_ptr(), wsp.numel(), sp())), 20, 1)
+            tf = 2.0 * M * N * K / (pus * 1e-6) / 1e12
+            out["distilgpt2"][f"{N}x{K}_g{g}"] = {
+                "decode_m1_us": us, "decode_m1_GB/s": gbs, "decode_m1_frac": gbs / peaks["hbm_gbs"],
+                "decode_copies": ncopy, "decode_path": q4.matmul_select(torch.float16, K, g, 1, N),
+                f"prefill_m{M}_us": pus, f"prefill_m{M}_TFLOP/s": tf,
+                f"prefill_m{M}_frac": tf / peaks["bf16_tflops"],
+                "prefill_path": q4.matmul_select(torch.float16, K, g, M, N),
+                "timing": "graph replay; decode over weight copies beyond L2, prefill operands L2-resident"}
+            del packed, scales, xp, yp, wsp
+        del w
+    for (N, K), groups in BULK_QUANT:
+        w = make_weights(N, K, seed=17, device=dev, dtype=torch.bfloat16, dist="student_t3",
+                         zero_group_frac=0.01, group=32)
+        Kp = (K + 1) // 2
+        packed = torch.empty((N, Kp), dtype=torch.uint8, device=dev)
+        unpacked = torch.empty((N, K), dtype=torch.int8, device=dev)
+        for g in groups:
+            G = -(-K // g)
+            scales = torch.empty((N, G), dtype=torch.float16, device=dev)
+            qms = flushed_ms(lambda: call(L.int4_quantize(w.data_ptr(), q4.DTYPE_BF16, N, K, g,
+                                                          packed.data_ptr(), scales.data_ptr(), sp())))
+            ums = flushed_ms(lambda: call(L.int4_unpack(packed.data_ptr(), K, N, unpacked.data_ptr(), sp())))
+            qb = N * K * 2 + N * Kp + 2 * N * G
+            ub = N * Kp + N * K
+            out["bulk_quantize"][f"{N}x{K}_g{g}"] = {
+                "quantize_ms": qms, "quantize_GB/s": qb / (qms * 1e-3) / 1e9,
+                "quantize_frac": qb / (qms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "unpack_ms": ums, "unpack_GB/s": ub / (ums * 1e-3) / 1e9,
+                "unpack_frac": ub / (ums * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "timing": "single call after an L2 flush, median"}
+            del scales
+        del w, packed, unpacked
+    N, K = N_W, K_W
+    w = make_weights(N, K, seed=5, device=dev, dtype=torch.bfloat16, dist="student_t3",
+                     zero_group_frac=0.01, group=32)
+    x = make_activations(1, K, seed=7, device=dev, dtype=torch.bfloat16)
+    for g in DECODE_GROUPS:
+        packed, scales, _ = q4.quantize_int4(w, g)
+        per_copy = packed.numel() + 2 * scales.numel()
+        ncopy = max(2, -(-3 * l2 // per_copy))
+        copies = [(packed, scales)] + [(packed.clone(), scales.clone()) for _ in range(ncopy - 1)]
+        us = decode_us(x, copies, K, g, 1, N, q4.DTYPE_BF16)
+        gbs = N * (K // 2) / (us * 1e-6) / 1e9
+        out["decode_groups"][f"{N}x{K}_g{g}_m1"] = {
+            "us_per_call": us, "GB/s": gbs, "frac": gbs / peaks["hbm_gbs"], "copies": ncopy,
+            "timing": "cuda graph replay over weight copies beyond L2"}
+        del copies, packed, scales
+    del w
+    return out
+
+
 def unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks, reps: int = 5):
     """The unfused design the fused matmul replaces, as context: the library's
     int4_dequantize to a bf16 w_hat [N, K], then a cuBLAS bf16 GEMM (torch)
@@ -678,9 +826,11 @@ def run_ours(args):
 
     shape_rows = None
     prefill_rows = None
+    cfg_rows = None
     if not args.no_shapes and not args.only:
         shape_rows = decode_shape_rows(dev, peaks)
         prefill_rows = prefill_shape_rows(dev, peaks)
+        cfg_rows = config_rows(dev, peaks, flush_l2)
     unfused = None
     if not args.no_unfused and not args.only:
         unfused = unfused_rows(dev, packed, scales, xd, xp, flush_l2, peaks)
@@ -735,7 +885,8 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "flushed before every row (256 MiB write, then 256 MiB read of another buffer); the decode row's back-to-back calls read distinct weight copies (3.9 GB > L2)",
                    "parallelism": f"replicas x{world}"},
-        "rows": rows, "decode_llama7b": shape_rows, "prefill_shapes": prefill_rows, "unfused": unfused, "variants": variants,
+        "rows": rows, "decode_llama7b": shape_rows, "prefill_shapes": prefill_rows, "configs": cfg_rows,
+        "unfused": unfused, "variants": variants,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         "gpu_launches": args.steps * sum(launches_per_step[n] for n in order),
         "wall_ms_timed_region": wall_ms,
@@ -760,7 +911,7 @@ def main():
     ap.add_argument("--no-unfused", action="store_true",
                     help="skip the dequantize-then-GEMM comparison rows")
     ap.add_argument("--no-shapes", action="store_true",
-                    help="skip the rows at the other configured shapes (Llama-7B decode, prefill)")
+                    help="skip the rows at the other configured shapes (Llama-7B decode, prefill, distilgpt2, bulk quantize, group-32/64 decode)")
     ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,
                     help="run one kernel of the step only (for profiling); no e2e or CPU baseline")
     ap.add_argument("--shape", default=None, metavar="N,K,M",

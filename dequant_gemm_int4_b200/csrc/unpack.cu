@@ -56,99 +56,53 @@ __global__ void __launch_bounds__(256) unpack_flat_kernel(const uint8_t* __restr
   }
 }
 
-// Any K and alignment: a lane takes NB packed bytes (2 NB outputs), a warp a
-// window of 64 NB outputs of one row.  A lane takes its aligned NB-byte
-// chunk of the packed byte range, the next lane's chunk by shuffle,
-// funnel-shifts by the row's byte offset, expands the nibbles and writes
-// them with aligned word stores (store_segment).
-#ifndef INT4_UNPACK_ANY_BYTES
-#define INT4_UNPACK_ANY_BYTES 8
-#endif
-// packed bytes per lane: 8 measured faster than 16 (2.1 against 1.2 TB/s on
-// W [8192, 28673]), whose eight clipped word stores per lane cost more than
-// the halved window count saves.
-constexpr int kUnpackAnyBytes = INT4_UNPACK_ANY_BYTES;
-
-template <int NB>
-__device__ __forceinline__ void load_packed_chunk(const uint8_t* base, int64_t c, int64_t nbytes,
-                                                  uint32_t (&w)[NB / 4]) {
-  if (NB == 8) {
-    const uint2 v = load_chunk8(base, c, nbytes);
-    w[0] = v.x;
-    w[1] = v.y;
-  } else {
-    const uint4 v = load_chunk16(base, c, nbytes);
-    w[0] = v.x;
-    w[1] = v.y;
-    w[NB / 4 > 2 ? 2 : 0] = v.z;
-    w[NB / 4 > 3 ? 3 : 0] = v.w;
-  }
+// Any K and alignment, row by row (blockIdx.y walks the rows): output row r
+// is the byte range [o_r, o_r + K) with o_r = oshift + r K from the 16-byte
+// aligned `obase`.  A thread writes one aligned 16-byte chunk that lies
+// inside the row: its outputs are nibbles col .. col + 15 of packed row r;
+// the thread loads the two aligned 8-byte words around them (its neighbours
+// read the same words, from L1), shifts the pair by the byte and nibble
+// offset, expands the 16 nibbles and stores them with one 16-byte store.  The
+// row's bytes before its first and after its last whole chunk (fewer than 16
+// at each end) are written byte by byte, so neighbouring rows never write the
+// same byte.
+__device__ __forceinline__ uint8_t unpack_byte(const uint8_t* pbase, int64_t prow, int64_t col) {
+  const uint32_t byte = pbase[prow + (col >> 1)];
+  return static_cast<uint8_t>(sext4((col & 1) ? (byte >> 4) : (byte & 0xFu)));
 }
 
-template <int NB>
-__global__ void __launch_bounds__(256) unpack_any_kernel(const uint8_t* __restrict__ pbase,
-                                                        int64_t pshift, int64_t pbytes, int64_t K,
-                                                        int64_t windows_per_row, int64_t total_windows,
-                                                        uint8_t* __restrict__ obase, int64_t oshift) {
-  static_assert(NB == 8 || NB == 16, "8- or 16-byte chunks");
-  constexpr int NW = NB / 4;     // packed words per lane
-  constexpr int WOUT = 64 * NB;  // outputs per window
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t per = (total_windows + nwarps - 1) / nwarps;
-  int64_t wi = warp * per;
-  const int64_t wend = (wi + per < total_windows) ? wi + per : total_windows;
-  if (wi >= wend) return;
+__global__ void __launch_bounds__(256) unpack_rows_kernel(
+    const uint8_t* __restrict__ pbase, int64_t pshift, int64_t pbytes, int64_t N, int64_t K,
+    uint8_t* __restrict__ obase, int64_t oshift) {
   const int64_t Kp = (K + 1) >> 1;
-  int64_t row = wi / windows_per_row;
-  int64_t col = wi - row * windows_per_row;
-
-  // The next window's chunk is loaded while the current one is expanded.
-  auto fetch = [&](int64_t r, int64_t cl, uint32_t (&own)[NW], uint32_t (&extra)[NW]) {
-    const int64_t c = (pshift + r * Kp + cl * (32 * NB) + lane * NB) / NB;
-    load_packed_chunk<NB>(pbase, c, pbytes, own);
-    if (lane == 31) {
-      load_packed_chunk<NB>(pbase, c + 1, pbytes, extra);
-    } else {
-#pragma unroll
-      for (int j = 0; j < NW; ++j) extra[j] = 0u;
+  for (int64_t r = blockIdx.y; r < N; r += gridDim.y) {
+    const int64_t o0 = oshift + r * K;      // row start, bytes from obase
+    const int64_t cA = (o0 + 15) >> 4;      // first whole chunk
+    const int64_t cB = (o0 + K) >> 4;       // one past the last whole chunk
+    const int64_t prow = pshift + r * Kp;   // packed row start, bytes from pbase
+    for (int64_t c = cA + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < cB;
+         c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t col = 16 * c - o0;
+      const int64_t B = prow + (col >> 1);
+      const uint32_t sh = static_cast<uint32_t>(B & 7) * 8u + static_cast<uint32_t>(col & 1) * 4u;
+      const uint2 l = load_chunk8(pbase, B >> 3, pbytes);
+      const uint2 h = load_chunk8(pbase, (B >> 3) + 1, pbytes);
+      const uint64_t lo = (static_cast<uint64_t>(l.y) << 32) | l.x;
+      const uint64_t hi = (static_cast<uint64_t>(h.y) << 32) | h.x;
+      const uint64_t v = sh == 0u ? lo : (lo >> sh) | (hi << (64u - sh));
+      const uint2 x = expand_word(static_cast<uint32_t>(v));
+      const uint2 y = expand_word(static_cast<uint32_t>(v >> 32));
+      reinterpret_cast<uint4*>(obase)[c] = make_uint4(x.x, x.y, y.x, y.y);
     }
-  };
-  uint32_t own[NW], extra[NW];
-  fetch(row, col, own, extra);
-  for (; wi < wend;) {
-    uint32_t win[2 * NW];
-#pragma unroll
-    for (int j = 0; j < NW; ++j) win[j] = own[j];
-    uint32_t cur_extra[NW];
-#pragma unroll
-    for (int j = 0; j < NW; ++j) cur_extra[j] = extra[j];
-    const int boff = static_cast<int>((pshift + row * Kp + col * (32 * NB) + lane * NB) & (NB - 1));
-    const int64_t crow = row, ccol = col;
-    if (++col == windows_per_row) {
-      col = 0;
-      ++row;
+    if (blockIdx.x == 0 && threadIdx.x < 32) {
+      // The ends: [o0, 16 cA) and [16 cB, o0 + K), or the whole row when it
+      // holds no whole chunk.
+      const int64_t head_end = (cA < cB) ? 16 * cA - o0 : K;
+      const int64_t tail_beg = (cA < cB) ? 16 * cB - o0 : K;
+      const int i = threadIdx.x;
+      for (int64_t col = i; col < head_end; col += 32) obase[o0 + col] = unpack_byte(pbase, prow, col);
+      for (int64_t col = tail_beg + i; col < K; col += 32) obase[o0 + col] = unpack_byte(pbase, prow, col);
     }
-    if (++wi < wend) fetch(row, col, own, extra);
-#pragma unroll
-    for (int j = 0; j < NW; ++j) {
-      const uint32_t nx = __shfl_down_sync(0xffffffffu, win[j], 1);
-      win[NW + j] = (lane == 31) ? cur_extra[j] : nx;
-    }
-    uint32_t bw[NW];
-    byte_shift_words<2 * NW, NW>(win, boff, bw);
-    uint32_t o[2 * NW];
-#pragma unroll
-    for (int j = 0; j < NW; ++j) {
-      const uint2 e = expand_word(bw[j]);
-      o[2 * j] = e.x;
-      o[2 * j + 1] = e.y;
-    }
-    const int64_t rowo = oshift + crow * K;
-    const int64_t f0 = rowo + ccol * WOUT;
-    const int64_t hi = (f0 + WOUT < rowo + K) ? f0 + WOUT : rowo + K;
-    store_segment<2 * NW>(obase, f0, f0, hi, o, lane);
   }
 }
 
@@ -166,18 +120,18 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t K, int64_t N, int8_t* o
     unpack_flat_kernel<<<static_cast<int>(grid), 256, 0, stream>>>(packed, total, out);
     return cudaGetLastError();
   }
-  constexpr int NB = kUnpackAnyBytes;
   const uintptr_t pa = reinterpret_cast<uintptr_t>(packed);
-  const uint8_t* pbase = reinterpret_cast<const uint8_t*>(pa & ~static_cast<uintptr_t>(NB - 1));
-  const int64_t pshift = static_cast<int64_t>(pa & (NB - 1));
+  const uint8_t* pbase = reinterpret_cast<const uint8_t*>(pa & ~static_cast<uintptr_t>(7));
+  const int64_t pshift = static_cast<int64_t>(pa & 7);
   const uintptr_t oa = reinterpret_cast<uintptr_t>(out);
-  uint8_t* obase = reinterpret_cast<uint8_t*>(oa & ~static_cast<uintptr_t>(3));
-  const int64_t oshift = static_cast<int64_t>(oa & 3);
-  const int64_t wpr = (K + 64 * NB - 1) / (64 * NB);
-  const int64_t total = N * wpr;
-  const int grid = resident_grid(unpack_any_kernel<NB>, (total + 31) / 32);
-  unpack_any_kernel<NB><<<grid, 256, 0, stream>>>(
-      pbase, pshift, pshift + N * ((K + 1) / 2), K, wpr, total, obase, oshift);
+  uint8_t* obase = reinterpret_cast<uint8_t*>(oa & ~static_cast<uintptr_t>(15));
+  const int64_t oshift = static_cast<int64_t>(oa & 15);
+  // Blocks per row cover its whole chunks (K / 16 + 1 at most); the rows go
+  // to blockIdx.y, up to the grid's limit, then stride.
+  const int64_t bx = (K / 16 + 1 + 255) / 256;
+  const int64_t by = N < 65535 ? N : 65535;
+  unpack_rows_kernel<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by)), 256, 0, stream>>>(
+      pbase, pshift, pshift + N * ((K + 1) / 2), N, K, obase, oshift);
   return cudaGetLastError();
 }
 

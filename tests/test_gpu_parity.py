@@ -290,6 +290,21 @@ def test_unpack_random_bytes(N, K):
     assert np.array_equal(q.cpu().numpy(), oracle.unpack_int4(packed.cpu().numpy(), K))
 
 
+def test_unpack_full_size_odd_k_every_row():
+    """The bulk-quantize workload's odd-K matrix [8192, 28673]: every output
+    byte against the oracle, compared in row chunks on the host."""
+    N, K = 8192, 28673
+    Kp = (K + 1) // 2
+    g = torch.Generator(device=DEV)
+    g.manual_seed(28673)
+    packed = torch.randint(0, 256, (N, Kp), generator=g, device=DEV, dtype=torch.int32).to(torch.uint8)
+    q = q4.unpack_int4(packed, K)
+    for r0 in range(0, N, 1024):
+        got = q[r0:r0 + 1024].cpu().numpy()
+        want = oracle.unpack_int4(packed[r0:r0 + 1024].cpu().numpy(), K)
+        assert np.array_equal(got, want), r0
+
+
 def test_unpack_all_256_bytes_and_minus_eight():
     packed = torch.arange(256, device=DEV, dtype=torch.int32).to(torch.uint8).view(1, 256)
     q = q4.unpack_int4(packed, 512).cpu().numpy()[0]
