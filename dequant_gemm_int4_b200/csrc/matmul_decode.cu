@@ -1585,10 +1585,12 @@ bool small_applies(int64_t K, int group, int64_t N) {
 #endif
 constexpr int kFlatChunk = INT4_FLAT_CHUNK;  // bytes of each row per copy chunk (a multiple of 64)
 
-// Row stride of the resident tile: Kp, padded so that the quarter warp's
-// 16-byte loads of rows g and g + 1 fall in different banks.
-__host__ __device__ constexpr int64_t flat_row_stride(int64_t Kp) {
-  return Kp % 128 == 0 ? Kp + 64 : Kp;
+// Row stride of the resident tile: Kp (a multiple of 64) padded so that the
+// lanes of one shared-memory wavefront hit distinct banks: the row stride in
+// words is 16, 8 or 4 modulo 32 for the 16-, 8- and 4-byte weight loads of
+// groups of whole blocks, of 64 and of 32 (GPB = 1, 2, 4 groups per block).
+__host__ __device__ constexpr int64_t flat_row_stride(int64_t Kp, int gpb) {
+  return Kp + ((128 + 64 / gpb) - Kp % 128) % 128;
 }
 
 // Shared-memory layout of a CTA: the tile's rows, x (if staged), the tile's
@@ -1597,10 +1599,10 @@ struct FlatLayout {
   int64_t rstride, off_x, off_s, off_z, off_bar, bytes;
   int nch;
 };
-__host__ __device__ inline FlatLayout flat_layout(int64_t K, int G, int M, bool xs, bool asym) {
+__host__ __device__ inline FlatLayout flat_layout(int64_t K, int G, int M, bool xs, bool asym, int gpb) {
   FlatLayout L;
   const int64_t Kp = K / 2;
-  L.rstride = flat_row_stride(Kp);
+  L.rstride = flat_row_stride(Kp, gpb);
   L.nch = static_cast<int>((Kp + kFlatChunk - 1) / kFlatChunk);
   L.off_x = 16 * L.rstride;
   L.off_s = L.off_x + (xs ? static_cast<int64_t>(M) * K * 2 : 0);
@@ -1610,7 +1612,7 @@ __host__ __device__ inline FlatLayout flat_layout(int64_t K, int G, int M, bool 
   return L;
 }
 
-template <typename TX, int NT, bool ASYM, int W, bool XS>
+template <typename TX, int NT, bool ASYM, int W, bool XS, int GPB>
 __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
     const TX* __restrict__ x, const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
     const uint8_t* __restrict__ zeros, Epilogue ep, float* __restrict__ y, int64_t K, int group,
@@ -1623,7 +1625,7 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int64_t Kp = K / 2;
-  const FlatLayout L = flat_layout(K, G, M, XS, ASYM);
+  const FlatLayout L = flat_layout(K, G, M, XS, ASYM, GPB);
   const int nch = L.nch;
   uint64_t* bars = reinterpret_cast<uint64_t*>(tile_smem + L.off_bar);  // chunks, then x
   const uint32_t tbase = ptx::smem_u32(tile_smem);
@@ -1677,8 +1679,11 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
   __syncthreads();
   // Rows past N are never copied; their (stale) words and scales only reach
   // outputs that are not stored.
-  const uint32_t wa = tbase + static_cast<uint32_t>(g * L.rstride + 16 * c);
-  const uint32_t wb = tbase + static_cast<uint32_t>((g + 8) * L.rstride + 16 * c);
+  // Lane (g, c) reads words word_index<GPB>(c, j), j = 0..3, of rows g and
+  // g + 8 of each block, so that word j of the four lanes of a quad lies in
+  // one group; its x fragments are the same words of x.
+  const uint32_t wa = tbase + static_cast<uint32_t>(g * L.rstride);
+  const uint32_t wb = tbase + static_cast<uint32_t>((g + 8) * L.rstride);
   float tot[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -1689,10 +1694,11 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int n = g + 8 * nt;
-      const TX* xp = x + static_cast<int64_t>(n < M ? n : 0) * K + static_cast<int64_t>(kb) * 128 + 32 * c;
+      const TX* xp = x + static_cast<int64_t>(n < M ? n : 0) * K + static_cast<int64_t>(kb) * 128;
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        xf[j][nt] = (n < M) ? __ldg(reinterpret_cast<const uint4*>(xp + 8 * j)) : make_uint4(0u, 0u, 0u, 0u);
+        xf[j][nt] = (n < M) ? __ldg(reinterpret_cast<const uint4*>(xp + 8 * word_index<GPB>(c, j)))
+                            : make_uint4(0u, 0u, 0u, 0u);
     }
   };
   uint4 xc[4][NT], xn[4][NT];
@@ -1705,47 +1711,72 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
   const int n0 = g < M ? g : 0;  // staged x: this lane's batch row
   for (int kb = warp; ok && kb < KB; kb += W) {
     if (XS) {
-      const uint32_t xs = tbase + static_cast<uint32_t>(L.off_x + (static_cast<int64_t>(n0) * K + kb * 128 + 32 * c) * 2);
+      const uint32_t xs = tbase + static_cast<uint32_t>(L.off_x + (static_cast<int64_t>(n0) * K + kb * 128) * 2);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) xc[j][0] = g < M ? ptx::lds128(xs + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
+      for (int j = 0; j < 4; ++j)
+        xc[j][0] = g < M ? ptx::lds128(xs + 16 * word_index<GPB>(c, j)) : make_uint4(0u, 0u, 0u, 0u);
     } else if (kb + W < KB) {
       load_x(kb + W, xn);
     }
     const int ch = (kb * 64) / kFlatChunk;
     ok = __all_sync(0xffffffffu, wait_bar(ptx::smem_u32(&bars[ch]), 0u, wc));
     if (!ok) break;
-    const int gi = static_cast<int>(static_cast<int64_t>(kb) * 128 / group);
-    const uint4 ua = ptx::lds128(wa + kb * 64);
-    const uint4 ub = ptx::lds128(wb + kb * 64);
-    const uint32_t wva[4] = {ua.x, ua.y, ua.z, ua.w};
-    const uint32_t wvb[4] = {ub.x, ub.y, ub.z, ub.w};
-    float acc[NT][4];
+    uint32_t wva[4], wvb[4];
+    if (GPB == 1) {
+      const uint4 ua = ptx::lds128(wa + kb * 64 + 16 * c);
+      const uint4 ub = ptx::lds128(wb + kb * 64 + 16 * c);
+      wva[0] = ua.x; wva[1] = ua.y; wva[2] = ua.z; wva[3] = ua.w;
+      wvb[0] = ub.x; wvb[1] = ub.y; wvb[2] = ub.z; wvb[3] = ub.w;
+    } else if (GPB == 2) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int h = 0; h < 2; ++h) {
+        const uint2 ua = ptx::lds64(wa + kb * 64 + 4 * (8 * h + 2 * c));
+        const uint2 ub = ptx::lds64(wb + kb * 64 + 4 * (8 * h + 2 * c));
+        wva[2 * h] = ua.x; wva[2 * h + 1] = ua.y;
+        wvb[2 * h] = ub.x; wvb[2 * h + 1] = ub.y;
+      }
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-    const uint32_t zba = ASYM ? Cvt<TX>::zero_bias(s_z[g * G + gi]) : Cvt<TX>::kMagic;
-    const uint32_t zbb = ASYM ? Cvt<TX>::zero_bias(s_z[(g + 8) * G + gi]) : Cvt<TX>::kMagic;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t pa[4], pb[4];
-      expand<TX, ASYM>(wva[j], pa, zba);
-      expand<TX, ASYM>(wvb[j], pb, zbb);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint4 xf = pair_x(xc[j][nt]);
-        Cvt<TX>::mma(acc[nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
-        Cvt<TX>::mma(acc[nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
+      for (int j = 0; j < 4; ++j) {
+        wva[j] = ptx::lds32(wa + kb * 64 + 4 * (4 * j + c));
+        wvb[j] = ptx::lds32(wb + kb * 64 + 4 * (4 * j + c));
       }
     }
-    const float sa = f16_bits_to_float(s_sc[g * G + gi]);
-    const float sb = f16_bits_to_float(s_sc[(g + 8) * G + gi]);
+    // One accumulator per group of the block (GPB of them), each scaled by
+    // its group's scale and added in order.
+    constexpr int kJPer = 4 / GPB;  // words j per group
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      tot[nt][0] = fmaf(acc[nt][0], sa, tot[nt][0]);
-      tot[nt][1] = fmaf(acc[nt][1], sa, tot[nt][1]);
-      tot[nt][2] = fmaf(acc[nt][2], sb, tot[nt][2]);
-      tot[nt][3] = fmaf(acc[nt][3], sb, tot[nt][3]);
+    for (int sg = 0; sg < GPB; ++sg) {
+      const int gi = GPB == 1 ? static_cast<int>(static_cast<int64_t>(kb) * 128 / group) : kb * GPB + sg;
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+      const uint32_t zba = ASYM ? Cvt<TX>::zero_bias(s_z[g * G + gi]) : Cvt<TX>::kMagic;
+      const uint32_t zbb = ASYM ? Cvt<TX>::zero_bias(s_z[(g + 8) * G + gi]) : Cvt<TX>::kMagic;
+#pragma unroll
+      for (int jj = 0; jj < kJPer; ++jj) {
+        const int j = sg * kJPer + jj;
+        uint32_t pa[4], pb[4];
+        expand<TX, ASYM>(wva[j], pa, zba);
+        expand<TX, ASYM>(wvb[j], pb, zbb);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4 xf = pair_x(xc[j][nt]);
+          Cvt<TX>::mma(acc[nt], pa[0], pb[0], pa[1], pb[1], xf.x, xf.y);
+          Cvt<TX>::mma(acc[nt], pa[2], pb[2], pa[3], pb[3], xf.z, xf.w);
+        }
+      }
+      const float sa = f16_bits_to_float(s_sc[g * G + gi]);
+      const float sb = f16_bits_to_float(s_sc[(g + 8) * G + gi]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        tot[nt][0] = fmaf(acc[nt][0], sa, tot[nt][0]);
+        tot[nt][1] = fmaf(acc[nt][1], sa, tot[nt][1]);
+        tot[nt][2] = fmaf(acc[nt][2], sb, tot[nt][2]);
+        tot[nt][3] = fmaf(acc[nt][3], sb, tot[nt][3]);
+      }
     }
     if (!XS) {
 #pragma unroll
@@ -1784,7 +1815,7 @@ __global__ void __launch_bounds__(W * 32, W == 8 ? 2 : 5) decode_flat_kernel(
 
 // CTAs per SM of one shared-memory decode kernel for a layout of `bytes`
 // bytes, queried once per device and size.
-template <typename TX, int NT, bool ASYM, int W, bool XS>
+template <typename TX, int NT, bool ASYM, int W, bool XS, int GPB>
 int flat_occupancy(int64_t bytes) {
   constexpr int kMaxDevices = 64;
   int dev = 0;
@@ -1795,7 +1826,7 @@ int flat_occupancy(int64_t bytes) {
   int occ = 0;
   // The opt-in is the device's limit less the kernel's static shared memory,
   // the same for every shape, so concurrent callers agree.
-  const void* fn = reinterpret_cast<const void*>(decode_flat_kernel<TX, NT, ASYM, W, XS>);
+  const void* fn = reinterpret_cast<const void*>(decode_flat_kernel<TX, NT, ASYM, W, XS, GPB>);
   int optin = 0;
   cudaFuncAttributes fa;
   bool failed = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
@@ -1822,35 +1853,48 @@ int flat_occupancy(int64_t bytes) {
 // none does (the shape then takes another decode kernel).
 constexpr int kFlatXs = 0x100;
 
-template <typename TX, int NT, bool ASYM, int W, bool XS>
+template <typename TX, int NT, bool ASYM, int W, bool XS, int GPB>
 bool flat_fits(int64_t K, int G, int M, int64_t tiles) {
-  const int64_t bytes = flat_layout(K, G, M, XS, ASYM).bytes;
-  return tiles <= static_cast<int64_t>(flat_occupancy<TX, NT, ASYM, W, XS>(bytes)) * num_sms();
+  const int64_t bytes = flat_layout(K, G, M, XS, ASYM, GPB).bytes;
+  return tiles <= static_cast<int64_t>(flat_occupancy<TX, NT, ASYM, W, XS, GPB>(bytes)) * num_sms();
+}
+
+template <typename TX, bool ASYM, int GPB>
+int flat_choice_g(int64_t K, int G, int m, int64_t tiles) {
+  if (m <= 8) {
+    if (m <= 2 && flat_fits<TX, 1, ASYM, 8, true, GPB>(K, G, m, tiles)) return 8 | kFlatXs;
+    if (flat_fits<TX, 1, ASYM, 8, false, GPB>(K, G, m, tiles)) return 8;
+    if (m <= 2 && flat_fits<TX, 1, ASYM, 4, true, GPB>(K, G, m, tiles)) return 4 | kFlatXs;
+    if (flat_fits<TX, 1, ASYM, 4, false, GPB>(K, G, m, tiles)) return 4;
+    return 0;
+  }
+  if (flat_fits<TX, 2, ASYM, 8, false, GPB>(K, G, m, tiles)) return 8;
+  // Four warps with a group per word at M > 8 spill, and lose to the
+  // pipelined 16-bit kernel (W [11008, 4096], group 32, M = 16: 25.3
+  // against 22.2 us).
+  if (GPB == 1 && flat_fits<TX, 2, ASYM, 4, false, GPB>(K, G, m, tiles)) return 4;
+  return 0;
 }
 
 template <typename TX, bool ASYM>
 int flat_choice(int64_t K, int group, int64_t M, int64_t N) {
-  if (!INT4_DECODE_FLAT || group % 128 != 0 || K % 128 != 0 || M > 16) return 0;
+  if (!INT4_DECODE_FLAT || K % 128 != 0 || M > 16) return 0;
+  if (!(group == 32 || group == 64 || group % 128 == 0)) return 0;
   // Where the integer kernel would convert x inside its CTAs (M <= 2 on a
   // matrix too tall for the small-matrix kernel), it is faster: its
   // arithmetic takes a quarter of the instructions per weight.
-  if (M <= kFuseMaxM && !small_applies(K, group, N)) return 0;
+  if (group % 128 == 0 && M <= kFuseMaxM && !small_applies(K, group, N)) return 0;
   const int G = static_cast<int>(K / group + (K % group != 0));
   const int64_t tiles = (N + 15) / 16;
   const int m = static_cast<int>(M);
-  if (M <= 8) {
-    if (M <= 2 && flat_fits<TX, 1, ASYM, 8, true>(K, G, m, tiles)) return 8 | kFlatXs;
-    if (flat_fits<TX, 1, ASYM, 8, false>(K, G, m, tiles)) return 8;
-    if (M <= 2 && flat_fits<TX, 1, ASYM, 4, true>(K, G, m, tiles)) return 4 | kFlatXs;
-    if (flat_fits<TX, 1, ASYM, 4, false>(K, G, m, tiles)) return 4;
-    return 0;
-  }
-  if (flat_fits<TX, 2, ASYM, 8, false>(K, G, m, tiles)) return 8;
-  if (flat_fits<TX, 2, ASYM, 4, false>(K, G, m, tiles)) return 4;
-  return 0;
+  const int gpb = group == 32 ? 4 : group == 64 ? 2 : 1;
+  const int c = gpb == 4   ? flat_choice_g<TX, ASYM, 4>(K, G, m, tiles)
+                : gpb == 2 ? flat_choice_g<TX, ASYM, 2>(K, G, m, tiles)
+                           : flat_choice_g<TX, ASYM, 1>(K, G, m, tiles);
+  return c == 0 ? 0 : c | (gpb << 12);
 }
 
-template <typename TX, int NT, bool ASYM, int W, bool XS>
+template <typename TX, int NT, bool ASYM, int W, bool XS, int GPB>
 cudaError_t launch_flat_w(const TX* x, const uint8_t* packed, const uint16_t* scales,
                           const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
                           int64_t N, float* y, cudaStream_t stream) {
@@ -1864,31 +1908,41 @@ cudaError_t launch_flat_w(const TX* x, const uint8_t* packed, const uint16_t* sc
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>((N + 15) / 16));
   cfg.blockDim = dim3(W * 32);
-  cfg.dynamicSmemBytes = static_cast<size_t>(flat_layout(K, G, static_cast<int>(M), XS, ASYM).bytes);
+  cfg.dynamicSmemBytes = static_cast<size_t>(flat_layout(K, G, static_cast<int>(M), XS, ASYM, GPB).bytes);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_flat_kernel<TX, NT, ASYM, W, XS>, x, packed, scales, zeros, ep,
+  return cudaLaunchKernelEx(&cfg, decode_flat_kernel<TX, NT, ASYM, W, XS, GPB>, x, packed, scales, zeros, ep,
                             y, K, group, G, static_cast<int>(M), N, KB, status);
 }
 
-template <typename TX, bool ASYM>
-cudaError_t launch_flat(int choice, const TX* x, const uint8_t* packed, const uint16_t* scales,
-                        const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
-                        int64_t N, float* y, cudaStream_t stream) {
+template <typename TX, bool ASYM, int GPB>
+cudaError_t launch_flat_g(int choice, const TX* x, const uint8_t* packed, const uint16_t* scales,
+                          const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                          int64_t N, float* y, cudaStream_t stream) {
   const bool xs = (choice & kFlatXs) != 0;
   const int w = choice & 0xFF;
   if (M <= 8) {
     if (w == 8)
-      return xs ? launch_flat_w<TX, 1, ASYM, 8, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
-                : launch_flat_w<TX, 1, ASYM, 8, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
-    return xs ? launch_flat_w<TX, 1, ASYM, 4, true>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
-              : launch_flat_w<TX, 1, ASYM, 4, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+      return xs ? launch_flat_w<TX, 1, ASYM, 8, true, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+                : launch_flat_w<TX, 1, ASYM, 8, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+    return xs ? launch_flat_w<TX, 1, ASYM, 4, true, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+              : launch_flat_w<TX, 1, ASYM, 4, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
   }
-  return w == 8 ? launch_flat_w<TX, 2, ASYM, 8, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
-                : launch_flat_w<TX, 2, ASYM, 4, false>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  return w == 8 ? launch_flat_w<TX, 2, ASYM, 8, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
+                : launch_flat_w<TX, 2, ASYM, 4, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
 }
 
+// `choice`: flat_choice's value (warps, staged x, groups per block in bits 12+).
+template <typename TX, bool ASYM>
+cudaError_t launch_flat(int choice, const TX* x, const uint8_t* packed, const uint16_t* scales,
+                        const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
+                        int64_t N, float* y, cudaStream_t stream) {
+  const int gpb = choice >> 12;
+  if (gpb == 4) return launch_flat_g<TX, ASYM, 4>(choice, x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  if (gpb == 2) return launch_flat_g<TX, ASYM, 2>(choice, x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  return launch_flat_g<TX, ASYM, 1>(choice, x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+}
 
 // ---------------- host side: scratch, schedule, launch ----------------
 // A decode call may need device scratch: one arrival counter per CTA (zero

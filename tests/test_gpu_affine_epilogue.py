@@ -190,8 +190,10 @@ PATHS = [
     (5, 18000, 4096, 128, q4.PATH_DECODE, None),     # integer kernel, x digit records
     (16, 9000, 2048, 128, q4.PATH_DECODE, None),
     (4, 18000, 4096, 128, q4.PATH_DECODE, False),    # no workspace: the 16-bit kernel
-    (3, 9000, 2048, 64, q4.PATH_DECODE, None),       # 16-bit kernel, group 64
-    (12, 5000, 2048, 32, q4.PATH_DECODE, None),      # 16-bit kernel, group 32
+    (3, 9000, 2048, 64, q4.PATH_DECODE, None),       # resident tiles, group 64
+    (12, 5000, 2048, 32, q4.PATH_DECODE, None),      # resident tiles, group 32
+    (3, 30000, 2048, 64, q4.PATH_DECODE, None),      # 16-bit kernel, group 64
+    (12, 30000, 2048, 32, q4.PATH_DECODE, None),     # 16-bit kernel, group 32
     (4, 2048, 4096, 128, q4.PATH_DECODE, None),      # resident-tile kernel
     (16, 4096, 11008, 128, q4.PATH_DECODE, None),    # resident-tile kernel, two n-tiles
     (3, 2048, 32768, 128, q4.PATH_DECODE, None),     # small-matrix kernel (rows too long)

@@ -159,7 +159,7 @@ def _call_ws(x, packed, scales, K, group, y, ws, nbytes):
     (1, 28672, 8192, 128),    # split tiles, x converted in the matmul
     (4, 18000, 4096, 128),    # split tiles and x digit records
     (16, 20000, 4096, 128),
-    (3, 9000, 2048, 64),      # the 16-bit kernel, split
+    (3, 30000, 2048, 64),     # the 16-bit kernel, split
 ])
 def test_workspace_size_is_enforced_and_sufficient(M, N, K, group):
     need = q4.matmul_workspace_size(torch.bfloat16, K, group, M, N)
@@ -190,6 +190,7 @@ def test_workspace_size_is_enforced_and_sufficient(M, N, K, group):
 @pytest.mark.parametrize("M, N, K, group", [
     (1, 28672, 8192, 128), (2, 18000, 4096, 128), (4, 18000, 4096, 128), (16, 20000, 4096, 128),
     (8, 9000, 2048, 64), (12, 5000, 2048, 32), (1, 4096, 4096, 128), (4, 11008, 4096, 128),
+    (8, 30000, 2048, 64), (2, 30000, 2048, 32),
 ])
 def test_matmul_without_workspace(M, N, K, group):
     """int4_matmul (no workspace): runs of whole row tiles, and at M > 2 the

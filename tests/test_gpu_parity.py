@@ -423,6 +423,8 @@ def test_matmul_decode_is_deterministic_and_matches_simt():
     (5, 6000, 1024, 128),    # many tiles, runs of whole tiles plus boundary pieces
     (4, 20000, 2048, 128),   # the integer kernel with digit records, split runs
     (1, 30001, 1024, 256),   # the integer kernel, x converted in the CTA, ragged
+    (3, 40000, 1024, 64),    # the 16-bit kernel, group 64, split runs
+    (16, 30001, 1024, 32),   # the 16-bit kernel, group 32, 64-row tiles, ragged
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_matmul_decode_split_tiles(M, N, K, group, dtype):

@@ -25,6 +25,7 @@ DEV = "cuda"
     (2, 18000, 4096, 256, torch.float16),    # x converted inside the matmul
     (16, 1000, 12288, 64, torch.float16),    # 64-row tiles, ragged last tile
     (3, 37, 4096, 32, torch.bfloat16),       # a single short tile
+    (16, 30000, 2048, 64, torch.float16),    # the 16-bit kernel, split tiles
 ])
 def test_noalloc_matches_regular_entry(M, N, K, group, dtype):
     w = make_weights(N, K, seed=N + K, device=DEV, dtype=torch.float32, dist="student_t3",
