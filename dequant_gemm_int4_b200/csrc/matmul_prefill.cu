@@ -65,14 +65,12 @@ namespace {
 #define INT4_PREFILL_STAGES 4
 #endif
 constexpr int kBN = 128;      // weight rows per tile (MMA M, TMEM lanes)
-constexpr int kBM = 256;      // activation rows per tile (MMA N)
+// Activation rows per tile (MMA N), a template parameter BM of the kernel:
+// 256, or 128 for problems whose 256-row tiles would leave most SMs idle.
 constexpr int kKS = 64;       // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = INT4_PREFILL_STAGES;    // shared-memory ring (x and packed bytes)
 constexpr int kThreads = 512;
 constexpr uint32_t kTmemCols = 512;
-static_assert(2 * kBM <= kTmemCols, "two accumulators fit TMEM");
-static_assert(kBM % 64 == 0, "the epilogue reads 32 columns at a time per column half");
-constexpr int kEpiCols = kBM / 2;            // accumulator columns per epilogue thread
 constexpr uint64_t kTimeoutNs = 250000000ull;  // 250 ms: far above any legitimate wait
 #ifndef INT4_PREFILL_GROUP_M
 #define INT4_PREFILL_GROUP_M 8
@@ -91,8 +89,12 @@ struct Barriers {
   uint64_t drain;               // abort path: all issued MMAs finished
 };
 
+template <int BM>
 struct Layout {
-  static constexpr int kX = kBM * kKS * 2;  // 24 KB at N = 192
+  static_assert(2 * BM <= static_cast<int>(kTmemCols), "two accumulators fit TMEM");
+  static_assert(BM % 64 == 0, "the epilogue reads 32 columns at a time per column half");
+  static constexpr int kEpiCols = BM / 2;   // accumulator columns per epilogue thread
+  static constexpr int kX = BM * kKS * 2;   // 32 KB at BM = 256
   static constexpr int kP = kBN * kKS / 2;  // 4 KB
   static constexpr int kA = kBN * kKS * 2;  // 16 KB: dequantized A
   static constexpr int offX = 0;
@@ -103,14 +105,15 @@ struct Layout {
   static constexpr int kBytes = offMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
-static_assert(Layout::kX % 1024 == 0, "x stages keep the 1024-byte swizzle alignment");
+static_assert(Layout<128>::kX % 1024 == 0 && Layout<256>::kX % 1024 == 0,
+              "x stages keep the 1024-byte swizzle alignment");
 
 // Instruction descriptor, kind::f16: D fp32, A/B bf16 (1) or fp16 (0),
-// both K-major, N = kBM, M = kBN.
-template <typename TX>
+// both K-major, N = BM, M = kBN.
+template <typename TX, int BM>
 __device__ __forceinline__ constexpr uint32_t make_idesc() {
   constexpr uint32_t ab = std::is_same<TX, __nv_bfloat16>::value ? 1u : 0u;
-  return (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(kBM >> 3) << 17) |
+  return (1u << 4) | (ab << 7) | (ab << 10) | (static_cast<uint32_t>(BM >> 3) << 17) |
          (static_cast<uint32_t>(kBN >> 4) << 24);
 }
 
@@ -189,14 +192,14 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity) {
 }
 
 // Origin (first weight row, first activation row) of tile T in the raster.
-__device__ __forceinline__ void tile_origin(int T, int num_n, int num_m, int& n0, int& m0) {
+__device__ __forceinline__ void tile_origin(int T, int num_n, int num_m, int bm, int& n0, int& m0) {
   const int per_run = kGroupM * num_n;
   const int run = T / per_run;
   const int first_m = run * kGroupM;
   const int gm = (num_m - first_m < kGroupM) ? num_m - first_m : kGroupM;
   const int r = T - run * per_run;
   n0 = (r / gm) * kBN;
-  m0 = (first_m + r % gm) * kBM;
+  m0 = (first_m + r % gm) * bm;
 }
 
 // Work unit u: piece u % ksplit of tile u / ksplit.  A tile's K is cut into
@@ -209,12 +212,12 @@ struct Unit {
   int it0, it1;  // stages [it0, it1)
   int g0, g1;    // K groups [g0, g1)
 };
-__device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int ksplit, int nchunks, int spc,
-                                        int nstages, int K, int group) {
+__device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int bm, int ksplit, int nchunks,
+                                        int spc, int nstages, int K, int group) {
   Unit w;
   const int T = u / ksplit;
   w.piece = u - T * ksplit;
-  tile_origin(T, num_n, num_m, w.n0, w.m0);
+  tile_origin(T, num_n, num_m, bm, w.n0, w.m0);
   const int c0 = w.piece * nchunks / ksplit;
   const int c1 = (w.piece + 1) * nchunks / ksplit;
   w.it0 = c0 * spc;
@@ -225,13 +228,14 @@ __device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int ksplit,
   return w;
 }
 
-template <typename TX, bool ASYM>
+template <typename TX, bool ASYM, int BM>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_p,
     const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
     float* __restrict__ y, int M, int N, int K, int group, int G, int ksplit, int spc,
     float* __restrict__ ypart, uint32_t* status) {
-  using L = Layout;
+  using L = Layout<BM>;
+  constexpr int kEpiCols = L::kEpiCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int num_n = (N + kBN - 1) / kBN;
-  const int num_m = (M + kBM - 1) / kBM;
+  const int num_m = (M + BM - 1) / BM;
   const int num_tiles = num_n * num_m;
   const int nstages = (K + kKS - 1) / kKS;
   const int nchunks = (nstages + spc - 1) / spc;
@@ -289,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       int gs = 0;  // stages issued (ring slot and phase)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+        const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
         const int n0 = w.n0, m0 = w.m0;
         for (int it = w.it0; it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
@@ -316,13 +320,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       // else once per 32-k half (groups of 32, 96, ...), never per MMA and
       // never by division.
       const bool leader = ptx::elect_one();
-      constexpr uint32_t idesc = make_idesc<TX>();
+      constexpr uint32_t idesc = make_idesc<TX, BM>();
       const int span = group % kKS == 0 ? kKS : kKS / 2;  // k per bookkeeping step
       int gs = 0;
       uint32_t gc = 0;  // groups started (accumulator and phase)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+        const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
         int gpos = 0;  // k offset of the next step inside its group (a piece starts a group)
         for (int it = w.it0; ok && it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
               ptx::tc_fence_after();
             }
             if (leader) {
-              const uint32_t d = tmem_base + buf * kBM;
+              const uint32_t d = tmem_base + buf * BM;
 #pragma unroll
               for (int j = 0; j < kKS / 16; ++j) {
                 if (j < nk) {
@@ -391,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     int gs = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+      const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
       const int n0 = w.n0;
       const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G
                                  : nullptr;
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     uint32_t gc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const Unit w = unit_of(u, num_n, num_m, ksplit, nchunks, spc, nstages, K, group);
+      const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
       const int n0 = w.n0, m0 = w.m0;
       const int n = n0 + row;
       float2 acc[kEpiCols / 2];
@@ -461,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         }
         ptx::tc_fence_after();
         const float2 sc2 = make_float2(sc, sc);
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * kBM +
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + buf * BM +
                                static_cast<uint32_t>(h * kEpiCols);
 #pragma unroll
         for (int c = 0; c < kEpiCols; c += 32) {
@@ -544,32 +548,50 @@ __global__ void __launch_bounds__(256) prefill_reduce_kernel(const float* __rest
   }
 }
 
+#ifndef INT4_PREFILL_SMALL_BM
+#define INT4_PREFILL_SMALL_BM 1  // 128-row activation tiles for problems of less than one wave
+#endif
+
+// Activation rows per tile: 128 when the 256-row tiling leaves SMs idle and
+// the 128-row one still fits one wave (twice the CTAs, each with half the
+// MMAs and half the stores of y, which a single CTA per SM issues at about
+// 16 GB/s: 8 us for a 128 x 256 fp32 tile), else 256.
+int choose_bm(int64_t M, int64_t N) {
+  const int64_t sms = num_sms();
+  const int64_t nt = (N + kBN - 1) / kBN;
+  const int64_t t256 = nt * ((M + 255) / 256);
+  const int64_t t128 = nt * ((M + 127) / 128);
+  return (INT4_PREFILL_SMALL_BM && t256 < sms && t128 <= sms) ? 128 : 256;
+}
+
 // How many K pieces to cut each tile into.  With fewer tiles than SMs the
 // machine idles; more pieces fill it, at the price of writing and re-reading
 // the pieces' fp32 sums.  The estimate (calibrated on B200): waves of units
 // times a unit's time -- its share of the tile's stages at about 0.6 us per
-// 64-k stage of a 128 x 256 tile, plus about 3 us to start and finish a
-// unit -- plus, when split, the partial sums' round trip through HBM and
-// about 1 us for the adding kernel.
+// 64-k stage of a 128 x 256 tile (half that at 128 rows), about 3 us to
+// start and finish a unit, and its store of a tile of fp32 sums at about
+// 16 GB/s per SM -- plus, when split, the partial sums' round trip through
+// HBM and about 1 us for the adding kernel.
 struct SplitPlan {
   int ksplit = 1;
   int spc = 1;  // stages per chunk: a common multiple of the group and the 64-k stage
 };
-SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N) {
+SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N, int bm) {
   SplitPlan p;
   const int64_t g64 = std::gcd(static_cast<int64_t>(group), static_cast<int64_t>(kKS));
   p.spc = static_cast<int>(group / g64);  // lcm(group, 64) / 64
   const int64_t nstages = (K + kKS - 1) / kKS;
   const int64_t nchunks = (nstages + p.spc - 1) / p.spc;
-  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + bm - 1) / bm);
   const int64_t sms = num_sms();
   if (tiles >= sms || nchunks < 2) return p;
-  const double stage_us = 0.6, unit_us = 3.0, reduce_us = 1.0, hbm_bytes_per_us = 6.0e6;
+  const double stage_us = 0.6 * bm / 256.0, unit_us = 3.0, reduce_us = 1.0, hbm_bytes_per_us = 6.0e6;
+  const double store_us = static_cast<double>(kBN) * bm * 4 / 16.0e3;
   const double tile_us = static_cast<double>(nstages) * stage_us;
   double best = 0.0;
   for (int64_t k = 1; k <= 8 && k <= nchunks; ++k) {
     const double waves = static_cast<double>((tiles * k + sms - 1) / sms);
-    const double t = waves * (tile_us / static_cast<double>(k) + unit_us) +
+    const double t = waves * (tile_us / static_cast<double>(k) + unit_us + store_us) +
                      (k > 1 ? static_cast<double>(k) * M * N * 8 / hbm_bytes_per_us + reduce_us : 0.0);
     if (k == 1 || t < best) {
       best = t;
@@ -579,12 +601,12 @@ SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N) {
   return p;
 }
 
-template <typename TX, bool ASYM>
+template <typename TX, bool ASYM, int BM>
 cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* scales,
                          const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
                          int64_t N, float* y, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream) {
-  using L = Layout;
+  using L = Layout<BM>;
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return cudaErrorNotSupported;
   uint32_t* status = status_word();
@@ -593,7 +615,7 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
   {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {kKS, kBM};
+    const cuuint32_t box[2] = {kKS, BM};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt = std::is_same<TX, __nv_bfloat16>::value
                                        ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -614,12 +636,12 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = prefill_kernel<TX, ASYM>;
+  auto kern = prefill_kernel<TX, ASYM, BM>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return e;
   // Split K only when the caller's workspace holds the pieces' sums (past
   // the counters a decode call keeps at its start).
-  SplitPlan sp = plan_split(K, group, M, N);
+  SplitPlan sp = plan_split(K, group, M, N, BM);
   const size_t part_bytes = static_cast<size_t>(sp.ksplit) * M * N * sizeof(float);
   if (sp.ksplit > 1 &&
       (workspace == nullptr || workspace_bytes < kWorkspaceCounterBytes + part_bytes))
@@ -627,7 +649,7 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
   float* ypart = sp.ksplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                           kWorkspaceCounterBytes)
                                : nullptr;
-  const int64_t units = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM) * sp.ksplit;
+  const int64_t units = ((N + kBN - 1) / kBN) * ((M + BM - 1) / BM) * sp.ksplit;
   const int64_t sms = num_sms();
   const int64_t ctas = INT4_PREFILL_PERSISTENT ? (units < sms ? units : sms) : units;
   const dim3 grid(static_cast<unsigned>(ctas));  // persistent: one CTA per SM
@@ -650,11 +672,16 @@ cudaError_t launch_tx(const TX* x, const uint8_t* packed, const uint16_t* scales
                       const uint8_t* zeros, const Epilogue& ep, int64_t K, int group, int64_t M,
                       int64_t N, float* y, void* workspace, size_t workspace_bytes,
                       cudaStream_t stream) {
+  const bool small = choose_bm(M, N) == 128;
   if (zeros != nullptr)
-    return launch_typed<TX, true>(x, packed, scales, zeros, ep, K, group, M, N, y, workspace,
-                                  workspace_bytes, stream);
-  return launch_typed<TX, false>(x, packed, scales, nullptr, ep, K, group, M, N, y, workspace,
-                                 workspace_bytes, stream);
+    return small ? launch_typed<TX, true, 128>(x, packed, scales, zeros, ep, K, group, M, N, y, workspace,
+                                              workspace_bytes, stream)
+                 : launch_typed<TX, true, 256>(x, packed, scales, zeros, ep, K, group, M, N, y, workspace,
+                                              workspace_bytes, stream);
+  return small ? launch_typed<TX, false, 128>(x, packed, scales, nullptr, ep, K, group, M, N, y, workspace,
+                                             workspace_bytes, stream)
+               : launch_typed<TX, false, 256>(x, packed, scales, nullptr, ep, K, group, M, N, y, workspace,
+                                             workspace_bytes, stream);
 }
 
 }  // namespace
@@ -667,7 +694,7 @@ bool prefill_supported(DType xt, int64_t K, int group, int64_t M, int64_t N, con
   if (K > (1LL << 30) || M > (1LL << 30) || N > (1LL << 30)) return false;
   if (reinterpret_cast<uintptr_t>(x) % 16 != 0 || reinterpret_cast<uintptr_t>(packed) % 16 != 0)
     return false;
-  if (((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM) > 0x7FFFFFFFLL) return false;
+  if (((N + kBN - 1) / kBN) * ((M + 127) / 128) > 0x7FFFFFFFLL) return false;
   return true;
 }
 
@@ -683,7 +710,7 @@ cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed
 }
 
 size_t prefill_workspace_size(int64_t K, int group, int64_t M, int64_t N) {
-  const SplitPlan sp = plan_split(K, group, M, N);
+  const SplitPlan sp = plan_split(K, group, M, N, choose_bm(M, N));
   return sp.ksplit > 1 ? kWorkspaceCounterBytes + static_cast<size_t>(sp.ksplit) * M * N * sizeof(float)
                        : 0;
 }
