@@ -105,8 +105,19 @@ def _check(rc: int) -> None:
         raise Int4Error(rc, msg.decode() if msg else "")
 
 
+# The current CUDA stream of a device as a raw handle: torch's own accessor
+# when it has one (no Stream object is built), else the public API.
+_raw_stream_fn = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _raw_stream(device_index: int) -> int:
+    if _raw_stream_fn is not None:
+        return _raw_stream_fn(device_index)
+    return torch.cuda.current_stream(device_index).cuda_stream
+
+
 def _stream(t: torch.Tensor):
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    return ctypes.c_void_p(_raw_stream(t.get_device()))
 
 
 def _need_cuda(name: str, t: torch.Tensor) -> None:
@@ -230,11 +241,15 @@ def _matmul_operands(x, packed, scales, K: int, group: int, out=None):
     if out is not None and (not isinstance(out, torch.Tensor) or out.dtype != torch.float32
                             or tuple(out.shape) != (M, N)):
         raise ValueError("out must be float32 [M, N]")
+    dev = None
     for name, t in (("x", x), ("packed", packed), ("scales", scales), ("out", out)):
         if t is None:
             continue
         _need_cuda(name, t)
-        if t.device != x.device:
+        d = t.get_device()
+        if dev is None:
+            dev = d
+        elif d != dev:
             raise ValueError(f"{name} must be on x's device")
     return M, N
 
@@ -262,11 +277,11 @@ _ws_size_cache: dict = {}
 _ws_cache: dict = {}
 
 
-def _workspace_for(x: torch.Tensor, nbytes: int) -> torch.Tensor | None:
+def _workspace_for(x: torch.Tensor, nbytes: int, stream: int | None = None) -> torch.Tensor | None:
     if nbytes == 0:
         return None
-    stream = torch.cuda.current_stream(x.device)
-    key = (x.device.index, stream.cuda_stream)
+    dev = x.get_device()
+    key = (dev, _raw_stream(dev) if stream is None else stream)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
         # torch.zeros runs on the current stream, before the call that uses it.
@@ -289,23 +304,29 @@ def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: 
     is used as given; False runs the schedule that needs no workspace (the C
     entry int4_matmul)."""
     M, N = _matmul_operands(x, packed, scales, K, group, out)
+    dev = x.get_device()
     if zeros is not None:
         _need_cuda("zeros", zeros)
-        if zeros.dtype != torch.uint8 or zeros.shape != scales.shape or zeros.device != x.device:
+        if zeros.dtype != torch.uint8 or zeros.shape != scales.shape or zeros.get_device() != dev:
             raise ValueError("zeros must be uint8 [N, ceil(K/group)] on x's device")
     if bias is not None:
         _need_cuda("bias", bias)
-        if bias.dtype != torch.float32 or tuple(bias.shape) != (N,) or bias.device != x.device:
+        if bias.dtype != torch.float32 or tuple(bias.shape) != (N,) or bias.get_device() != dev:
             raise ValueError("bias must be float32 [N] on x's device")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.float32, device=x.device)
+        out = x.new_empty((M, N), dtype=torch.float32)
     L = _lib if _lib is not None else lib()
-    same_dev = x.device.index == torch.cuda.current_device()
-    with (_nullctx() if same_dev else torch.cuda.device(x.device)):
+    same_dev = dev == torch.cuda.current_device()
+    with (_nullctx() if same_dev else torch.cuda.device(dev)):
+        stream = _raw_stream(dev)
         if workspace is False:
             ws_ptr, ws_bytes = None, 0
         elif workspace is None:
-            ws = _workspace_for(x, matmul_workspace_size(x.dtype, K, group, M, N, x.device))
+            key = (dev, x.dtype, int(K), int(group), int(M), int(N))
+            nb = _ws_size_cache.get(key)
+            if nb is None:
+                nb = matmul_workspace_size(x.dtype, K, group, M, N, x.device)
+            ws = _workspace_for(x, nb, stream)
             ws_ptr, ws_bytes = (ws.data_ptr(), ws.numel()) if ws is not None else (None, 0)
         else:
             _need_cuda("workspace", workspace)
@@ -315,13 +336,13 @@ def int4_matmul(x: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, K: 
         if zeros is None and bias is None and not relu:
             _check(L.int4_matmul_path(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
                                       scales.data_ptr(), K, int(group), M, N, out.data_ptr(),
-                                      int(path), ws_ptr, ws_bytes, _stream(x)))
+                                      int(path), ws_ptr, ws_bytes, stream))
         else:
             _check(L.int4_matmul_ex(x.data_ptr(), _DTYPE_CODE[x.dtype], packed.data_ptr(),
                                     scales.data_ptr(), None if zeros is None else zeros.data_ptr(),
                                     K, int(group), M, N, None if bias is None else bias.data_ptr(),
                                     EPI_RELU if relu else 0, out.data_ptr(), int(path), ws_ptr,
-                                    ws_bytes, _stream(x)))
+                                    ws_bytes, stream))
     return out
 
 
