@@ -443,6 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int q = warp & 3;
     const int h = (warp - 8) >> 2;
     const int row = 32 * q + lane;
+    // y (or the pieces' buffer, which starts 16-byte aligned in the
+    // workspace) takes 16-byte stores when its rows are whole float4s.
+    const bool vec_store = N % 4 == 0 && (reinterpret_cast<uintptr_t>(ypart == nullptr ? y : ypart) & 15) == 0;
     uint32_t gc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
@@ -486,8 +489,41 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         ptx::tc_fence_before();
         ptx::mbar_arrive(bar(&bars->tmem_empty[buf]));
       }
-      if (ok && n < N) {
-        const int mbase = m0 + h * kEpiCols;
+      const int mbase = m0 + h * kEpiCols;
+      float* const dst = ypart == nullptr ? y : ypart + static_cast<int64_t>(w.piece) * M * N;
+      if (ok && vec_store) {
+        // 16-byte stores: a 4 x 4 transpose inside each quad of lanes (two
+        // butterfly steps of shuffles) leaves lane r with activation row
+        // m = 4 b + r of the quad's four consecutive weight rows.  N is a
+        // multiple of 4, so a quad is wholly inside or outside [0, N); every
+        // lane takes part in the shuffles and only inside quads store.
+        const int r = lane & 3;
+        const int nq = n - r;
+        const bool b1 = (r & 2) != 0, b0 = (r & 1) != 0;
+#pragma unroll
+        for (int b = 0; b < kEpiCols / 4; ++b) {
+          float a0 = acc[2 * b].x, a1 = acc[2 * b].y, a2 = acc[2 * b + 1].x, a3 = acc[2 * b + 1].y;
+          {
+            const float s1 = b1 ? a0 : a2, s2 = b1 ? a1 : a3;
+            const float t1 = __shfl_xor_sync(0xffffffffu, s1, 2), t2 = __shfl_xor_sync(0xffffffffu, s2, 2);
+            if (b1) { a0 = t1; a1 = t2; } else { a2 = t1; a3 = t2; }
+          }
+          {
+            const float s1 = b0 ? a0 : a1, s2 = b0 ? a2 : a3;
+            const float t1 = __shfl_xor_sync(0xffffffffu, s1, 1), t2 = __shfl_xor_sync(0xffffffffu, s2, 1);
+            if (b0) { a0 = t1; a2 = t2; } else { a1 = t1; a3 = t2; }
+          }
+          const int m = mbase + 4 * b + r;
+          if (m < M && nq < N) {
+            // Split-K pieces keep their raw sums (the adding kernel applies
+            // the epilogue).
+            const float4 v = ypart == nullptr ? make_float4(ep.apply(a0, nq), ep.apply(a1, nq + 1),
+                                                            ep.apply(a2, nq + 2), ep.apply(a3, nq + 3))
+                                              : make_float4(a0, a1, a2, a3);
+            *reinterpret_cast<float4*>(dst + static_cast<int64_t>(m) * N + nq) = v;
+          }
+        }
+      } else if (ok && n < N) {
         if (ypart == nullptr) {
 #pragma unroll
           for (int j = 0; j < kEpiCols / 2; ++j) {
@@ -498,12 +534,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         } else {
           // A piece of a split K: its fp32 sums, added in piece order (and
           // the epilogue applied) by prefill_reduce_kernel.
-          float* yp = ypart + static_cast<int64_t>(w.piece) * M * N;
 #pragma unroll
           for (int j = 0; j < kEpiCols / 2; ++j) {
             const int m = mbase + 2 * j;
-            if (m < M) yp[static_cast<int64_t>(m) * N + n] = acc[j].x;
-            if (m + 1 < M) yp[static_cast<int64_t>(m + 1) * N + n] = acc[j].y;
+            if (m < M) dst[static_cast<int64_t>(m) * N + n] = acc[j].x;
+            if (m + 1 < M) dst[static_cast<int64_t>(m + 1) * N + n] = acc[j].y;
           }
         }
       }
