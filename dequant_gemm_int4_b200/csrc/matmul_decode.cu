@@ -664,6 +664,11 @@ __global__ void __launch_bounds__(kThreads, INT4_DECODE_MIN_BLOCKS) decode_kerne
 // quarter warp over all banks.
 constexpr int kDigitTile = 1024;
 constexpr int kRecFlags = 64;  // flag bytes of a record, after its factors
+// Per batch row m (records of at most two n-tiles): the block's digit sums
+// C01 = D0 + 256 D1 and C23 = D2 + 256 D3 (D_i = the sum of digit i over the
+// block's k) as two int32 at kRecSums + 8 m; the affine scheme subtracts
+// z C from each pair product.
+constexpr int kRecSums = 96;
 
 __device__ __forceinline__ void transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d,
                                              uint32_t (&o)[4]) {
@@ -755,6 +760,22 @@ __device__ __forceinline__ void word_digits(const float (&v)[8], uint32_t amax_b
   transpose4x4(dd[1], dd[3], dd[5], dd[7], od);
 }
 
+// The block's digit-pair sums (C01, C23) from each lane's digit words ev/od
+// (signed bytes), summed over the half warp.  All 32 lanes call it together.
+__device__ __forceinline__ int2 block_digit_sums(const uint32_t (&ev)[4], const uint32_t (&od)[4]) {
+  int d[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = __dp4a(static_cast<int>(ev[i]), 0x01010101, __dp4a(static_cast<int>(od[i]), 0x01010101, 0));
+  // The pair sums are linear in the digits: reduce them directly.
+  int c01 = d[0] + 256 * d[1], c23 = d[2] + 256 * d[3];
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    c01 += __shfl_xor_sync(0xffffffffu, c01, o);
+    c23 += __shfl_xor_sync(0xffffffffu, c23, o);
+  }
+  return make_int2(c01, c23);
+}
+
 // Whether any lane of this lane's half warp (one block) set `pred`.  All 32
 // lanes must call it together.
 __device__ __forceinline__ bool half_warp_any(bool pred) {
@@ -773,7 +794,7 @@ __device__ __forceinline__ int digit_offset(int m, int i, int h) {
 // memory (row pitch 512 bytes): xs addresses this lane's word h of row 0, rb
 // the block's record.  All 32 lanes call it together (one block per half
 // warp).
-template <typename TX, int R, int NP>
+template <typename TX, int R, int NP, bool SUMS>
 __device__ __forceinline__ void convert_rows(uint32_t xs, uint32_t rb, int h) {
   static_assert(R <= 4, "the flag bytes of the converted rows share one word");
   float v[R][8];
@@ -793,6 +814,10 @@ __device__ __forceinline__ void convert_rows(uint32_t xs, uint32_t rb, int h) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) ptx::sts64(rb + digit_offset(r, i, h), ev[i], od[i]);
     if (h == 0) ptx::sts32(rb + NP * kDigitTile + 4 * r, __float_as_uint(f));
+    if (SUMS) {
+      const int2 cs = block_digit_sums(ev, od);
+      if (h == 0) ptx::sts64(rb + NP * kDigitTile + kRecSums + 8 * r, static_cast<uint32_t>(cs.x), static_cast<uint32_t>(cs.y));
+    }
   }
   // Rows R .. 3 of the word stay zero (rows past M are never written).
   if (h == 0) ptx::sts32(rb + NP * kDigitTile + kRecFlags, flags);
@@ -828,6 +853,7 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const TX* __restrict__ x,
   bool inexact;
   word_digits(v, amax_bits, ev, od, f, inexact);
   const bool flag = half_warp_any(inexact);  // every lane votes, live or not
+  const int2 cs = block_digit_sums(ev, od);   // every lane takes part
   if (!live) return;
   uint8_t* r = rec + b * (static_cast<int64_t>(NP) * kDigitTile + 128);
 #pragma unroll
@@ -836,6 +862,7 @@ __global__ void __launch_bounds__(256) x_digits_kernel(const TX* __restrict__ x,
   if (h == 0) {
     reinterpret_cast<float*>(r + NP * kDigitTile)[m] = f;
     r[NP * kDigitTile + kRecFlags + m] = flag ? 1u : 0u;
+    if (NP <= 2) *reinterpret_cast<int2*>(r + NP * kDigitTile + kRecSums + 8 * m) = cs;
   }
 }
 
@@ -978,6 +1005,9 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
     int64_t N, int KB, int64_t U, int P, int64_t gran, float* __restrict__ partials,
     uint32_t* __restrict__ counters, uint32_t* status) {
   using S = I8Shape<NP, FUSE>;
+  // Affine codes as unsigned q with z times the block's digit sums
+  // subtracted (records of at most two n-tiles carry the sums).
+  constexpr bool kAsymSums = ASYM && NP <= 2;
   constexpr int kTiles = S::kTiles;
   constexpr int kRowsPerCta = S::kRowsPerCta;
   constexpr int kWBytes = S::kWBytes;
@@ -1070,9 +1100,9 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
       const uint32_t xs = st + S::offX + bl * 256 + 16 * h;
       const uint32_t rb = st + kWBytes + bl * kRec;
       if (M == 2)
-        convert_rows<TX, 2, NP>(xs, rb, h);
+        convert_rows<TX, 2, NP, kAsymSums>(xs, rb, h);
       else
-        convert_rows<TX, 1, NP>(xs, rb, h);
+        convert_rows<TX, 1, NP, kAsymSums>(xs, rb, h);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&ready[s]));
     }
@@ -1169,7 +1199,9 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
     // weighs 2^16 more, which they fold into their scale.
     const uint32_t fofs = xrec + static_cast<uint32_t>(NP * kDigitTile + 4 * (c >> 1));
     const uint32_t flagofs = xrec + static_cast<uint32_t>(NP * kDigitTile + kRecFlags);
-    // Affine codes enter the MMA as q - z, not 16 q: 16 times the factor.
+    // This lane's digit-pair sum: batch row 2 nt + c / 2, pair c & 1 (plus 16 nt bytes).
+    const uint32_t sumofs = xrec + static_cast<uint32_t>(NP * kDigitTile + kRecSums + 8 * (c >> 1) + 4 * (c & 1));
+    // Affine codes enter the MMA as q (or q - z), not 16 q: 16 times the factor.
     const float lane_mul = ((c & 1) ? 65536.0f : 1.0f) * (ASYM ? 16.0f : 1.0f);
     const int bpg = group / 128;
     int gs = 0;
@@ -1280,7 +1312,14 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
               const uint32_t w1[4] = {wr[t][1].x, wr[t][1].y, wr[t][1].z, wr[t][1].w};
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
-                if (ASYM) {
+                if (kAsymSums) {
+                  // The unsigned codes q; z times the block's digit sums is
+                  // subtracted from the products below.
+                  a[t][j][0] = w0[j] & 0x0F0F0F0Fu;
+                  a[t][j][1] = w1[j] & 0x0F0F0F0Fu;
+                  a[t][j][2] = (w0[j] >> 4) & 0x0F0F0F0Fu;
+                  a[t][j][3] = (w1[j] >> 4) & 0x0F0F0F0Fu;
+                } else if (ASYM) {
                   const uint32_t zza = za[t] * 0x01010101u, zzb = zb[t] * 0x01010101u;
                   a[t][j][0] = affine_bytes(w0[j] & 0x0F0F0F0Fu, zza);
                   a[t][j][1] = affine_bytes(w1[j] & 0x0F0F0F0Fu, zzb);
@@ -1305,6 +1344,7 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
               const uint4 b01 = kHoist ? hb01[kHoist ? nt : 0] : ptx::lds128(st + bofs[0] + nt * kDigitTile);
               const uint4 b23 = kHoist ? hb23[kHoist ? nt : 0] : ptx::lds128(st + bofs[1] + nt * kDigitTile);
               const float fct = kHoist ? hfct[kHoist ? nt : 0] : __uint_as_float(ptx::lds32(st + fofs + nt * 8));
+              const int csum = kAsymSums ? static_cast<int>(ptx::lds32(st + sumofs + nt * 16)) : 0;
 #pragma unroll
               for (int t = 0; t < kTiles; ++t) {
                 int acc[4] = {0, 0, 0, 0};
@@ -1312,8 +1352,11 @@ __global__ void __launch_bounds__(I8Shape<NP, FUSE>::kThreads, I8Shape<NP, FUSE>
                 mma_s8(acc, a[t][1], b01.z, b01.w);
                 mma_s8(acc, a[t][2], b23.x, b23.y);
                 mma_s8(acc, a[t][3], b23.z, b23.w);
-                const float p0 = static_cast<float>(acc[0] + 256 * acc[1]);
-                const float p1 = static_cast<float>(acc[2] + 256 * acc[3]);
+                // Exact in int32: |q d| sums stay below 2^26, |z C| below 2^26.
+                const float p0 = static_cast<float>(acc[0] + 256 * acc[1] -
+                                                    (kAsymSums ? static_cast<int>(za[t]) * csum : 0));
+                const float p1 = static_cast<float>(acc[2] + 256 * acc[3] -
+                                                    (kAsymSums ? static_cast<int>(zb[t]) * csum : 0));
                 tot[t][nt][0] = fmaf(p0 * fct, sal[t], tot[t][nt][0]);
                 tot[t][nt][1] = fmaf(p1 * fct, sbl[t], tot[t][nt][1]);
               }
