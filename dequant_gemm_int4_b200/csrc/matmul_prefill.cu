@@ -202,24 +202,39 @@ __device__ __forceinline__ void tile_origin(int T, int num_n, int num_m, int bm,
   m0 = (first_m + r % gm) * bm;
 }
 
-// Work unit u: piece u % ksplit of tile u / ksplit.  A tile's K is cut into
-// ksplit pieces of whole chunks of `spc` stages (spc * 64 k: a common
-// multiple of the group and the stage), so each piece starts and ends on a
-// group boundary; pieces of one tile are adjacent units.
+// Work units: units u < full are whole tiles (tile u); the rest are pieces
+// of the remaining (tail) tiles, ksplit per tile: unit full + v is piece
+// v % ksplit of tile full + v / ksplit, and its sums go to slot v of the
+// pieces' buffer.  A tile's K is cut into ksplit pieces of whole chunks of
+// `spc` stages (spc * 64 k: a common multiple of the group and the stage), so
+// each piece starts and ends on a group boundary; pieces of one tile are
+// adjacent units.  With full = 0 every tile is split; with ksplit = 1 none.
 struct Unit {
   int n0, m0;    // tile origin
   int piece;
+  int slot;      // slot in the pieces' buffer, -1 for a whole tile
   int it0, it1;  // stages [it0, it1)
   int g0, g1;    // K groups [g0, g1)
 };
-__device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int bm, int ksplit, int nchunks,
-                                        int spc, int nstages, int K, int group) {
+__device__ __forceinline__ Unit unit_of(int u, int num_n, int num_m, int bm, int full, int ksplit,
+                                        int nchunks, int spc, int nstages, int K, int group) {
   Unit w;
-  const int T = u / ksplit;
-  w.piece = u - T * ksplit;
+  int T, k;
+  if (u < full || ksplit == 1) {
+    T = u;
+    w.piece = 0;
+    w.slot = -1;
+    k = 1;
+  } else {
+    const int v = u - full;
+    T = full + v / ksplit;
+    w.piece = v - (v / ksplit) * ksplit;
+    w.slot = v;
+    k = ksplit;
+  }
   tile_origin(T, num_n, num_m, bm, w.n0, w.m0);
-  const int c0 = w.piece * nchunks / ksplit;
-  const int c1 = (w.piece + 1) * nchunks / ksplit;
+  const int c0 = w.piece * nchunks / k;
+  const int c1 = (w.piece + 1) * nchunks / k;
   w.it0 = c0 * spc;
   w.it1 = c1 * spc < nstages ? c1 * spc : nstages;
   w.g0 = (w.it0 * kKS) / group;
@@ -232,7 +247,7 @@ template <typename TX, bool ASYM, int BM>
 __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_p,
     const uint16_t* __restrict__ scales, const uint8_t* __restrict__ zeros, Epilogue ep,
-    float* __restrict__ y, int M, int N, int K, int group, int G, int ksplit, int spc,
+    float* __restrict__ y, int M, int N, int K, int group, int G, int full, int ksplit, int spc,
     float* __restrict__ ypart, uint32_t* status) {
   using L = Layout<BM>;
   constexpr int kEpiCols = L::kEpiCols;
@@ -250,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
   const int num_tiles = num_n * num_m;
   const int nstages = (K + kKS - 1) / kKS;
   const int nchunks = (nstages + spc - 1) / spc;
-  const int num_units = num_tiles * ksplit;
+  const int num_units = full + (num_tiles - full) * ksplit;
 
   const uint32_t sX = ptx::smem_u32(smem + L::offX);
   const uint32_t sA = ptx::smem_u32(smem + L::offA);
@@ -293,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       int gs = 0;  // stages issued (ring slot and phase)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
+        const Unit w = unit_of(u, num_n, num_m, BM, full, ksplit, nchunks, spc, nstages, K, group);
         const int n0 = w.n0, m0 = w.m0;
         for (int it = w.it0; it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
@@ -326,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
       uint32_t gc = 0;  // groups started (accumulator and phase)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
+        const Unit w = unit_of(u, num_n, num_m, BM, full, ksplit, nchunks, spc, nstages, K, group);
         int gpos = 0;  // k offset of the next step inside its group (a piece starts a group)
         for (int it = w.it0; ok && it < w.it1; ++it, ++gs) {
           const int s = gs % kStages;
@@ -395,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     int gs = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
+      const Unit w = unit_of(u, num_n, num_m, BM, full, ksplit, nchunks, spc, nstages, K, group);
       const int n0 = w.n0;
       const uint8_t* zrow = ASYM ? zeros + static_cast<int64_t>(n0 + t < N ? n0 + t : N - 1) * G
                                  : nullptr;
@@ -443,13 +458,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
     const int q = warp & 3;
     const int h = (warp - 8) >> 2;
     const int row = 32 * q + lane;
-    // y (or the pieces' buffer, which starts 16-byte aligned in the
-    // workspace) takes 16-byte stores when its rows are whole float4s.
-    const bool vec_store = N % 4 == 0 && (reinterpret_cast<uintptr_t>(ypart == nullptr ? y : ypart) & 15) == 0;
+    // y takes 16-byte stores when its rows are whole float4s; the pieces'
+    // slots (128 x BM tile-local, rows of 128 floats) whenever the buffer is
+    // 16-byte aligned.
+    const bool vec_y = N % 4 == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+    const bool vec_p = (reinterpret_cast<uintptr_t>(ypart) & 15) == 0;
     uint32_t gc = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const Unit w = unit_of(u, num_n, num_m, BM, ksplit, nchunks, spc, nstages, K, group);
+      const Unit w = unit_of(u, num_n, num_m, BM, full, ksplit, nchunks, spc, nstages, K, group);
       const int n0 = w.n0, m0 = w.m0;
       const int n = n0 + row;
       float2 acc[kEpiCols / 2];
@@ -490,13 +507,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
         ptx::mbar_arrive(bar(&bars->tmem_empty[buf]));
       }
       const int mbase = m0 + h * kEpiCols;
-      float* const dst = ypart == nullptr ? y : ypart + static_cast<int64_t>(w.piece) * M * N;
-      if (ok && vec_store) {
+      // A piece of a split tile keeps its raw fp32 sums in its slot, tile-
+      // local as [m - m0][n - n0] (rows of kBN floats, edges included); the
+      // adding kernel sums the pieces in order, applies the epilogue and
+      // writes y.
+      const bool piece = w.slot >= 0;
+      float* const slot = piece ? ypart + static_cast<int64_t>(w.slot) * (kBN * BM) : nullptr;
+      if (ok && (piece ? vec_p : vec_y)) {
         // 16-byte stores: a 4 x 4 transpose inside each quad of lanes (two
         // butterfly steps of shuffles) leaves lane r with activation row
         // m = 4 b + r of the quad's four consecutive weight rows.  N is a
-        // multiple of 4, so a quad is wholly inside or outside [0, N); every
-        // lane takes part in the shuffles and only inside quads store.
+        // multiple of 4 (or the slot's rows are 128 floats), so a quad is
+        // wholly inside or outside; every lane takes part in the shuffles.
         const int r = lane & 3;
         const int nq = n - r;
         const bool b1 = (r & 2) != 0, b0 = (r & 1) != 0;
@@ -514,32 +536,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(
             if (b0) { a0 = t1; a2 = t2; } else { a1 = t1; a3 = t2; }
           }
           const int m = mbase + 4 * b + r;
-          if (m < M && nq < N) {
-            // Split-K pieces keep their raw sums (the adding kernel applies
-            // the epilogue).
-            const float4 v = ypart == nullptr ? make_float4(ep.apply(a0, nq), ep.apply(a1, nq + 1),
-                                                            ep.apply(a2, nq + 2), ep.apply(a3, nq + 3))
-                                              : make_float4(a0, a1, a2, a3);
-            *reinterpret_cast<float4*>(dst + static_cast<int64_t>(m) * N + nq) = v;
+          if (piece) {
+            // Rows and columns past M and N are never read back: not stored.
+            if (m < M && nq < N)
+              *reinterpret_cast<float4*>(slot + (m - m0) * kBN + (nq - n0)) = make_float4(a0, a1, a2, a3);
+          } else if (m < M && nq < N) {
+            *reinterpret_cast<float4*>(y + static_cast<int64_t>(m) * N + nq) =
+                make_float4(ep.apply(a0, nq), ep.apply(a1, nq + 1), ep.apply(a2, nq + 2), ep.apply(a3, nq + 3));
+          }
+        }
+      } else if (ok && piece) {
+        if (n < N) {
+#pragma unroll
+          for (int j = 0; j < kEpiCols / 2; ++j) {
+            const int ml = mbase - m0 + 2 * j;
+            if (m0 + ml < M) slot[ml * kBN + row] = acc[j].x;
+            if (m0 + ml + 1 < M) slot[(ml + 1) * kBN + row] = acc[j].y;
           }
         }
       } else if (ok && n < N) {
-        if (ypart == nullptr) {
 #pragma unroll
-          for (int j = 0; j < kEpiCols / 2; ++j) {
-            const int m = mbase + 2 * j;
-            if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j].x, n);
-            if (m + 1 < M) y[static_cast<int64_t>(m + 1) * N + n] = ep.apply(acc[j].y, n);
-          }
-        } else {
-          // A piece of a split K: its fp32 sums, added in piece order (and
-          // the epilogue applied) by prefill_reduce_kernel.
-#pragma unroll
-          for (int j = 0; j < kEpiCols / 2; ++j) {
-            const int m = mbase + 2 * j;
-            if (m < M) dst[static_cast<int64_t>(m) * N + n] = acc[j].x;
-            if (m + 1 < M) dst[static_cast<int64_t>(m + 1) * N + n] = acc[j].y;
-          }
+        for (int j = 0; j < kEpiCols / 2; ++j) {
+          const int m = mbase + 2 * j;
+          if (m < M) y[static_cast<int64_t>(m) * N + n] = ep.apply(acc[j].x, n);
+          if (m + 1 < M) y[static_cast<int64_t>(m + 1) * N + n] = ep.apply(acc[j].y, n);
         }
       }
     }
@@ -571,18 +591,46 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// y = epilogue(sum over pieces p of ypart[p]), adding the pieces in order.
+// y of the split (tail) tiles = epilogue(sum of their pieces' slots, in
+// piece order).  blockIdx.y walks the tail tiles (tile full + t of the
+// raster, its origin computed once per block); a thread takes four
+// consecutive elements li .. li + 3 of the tile, at [m][n] = [li / kBN]
+// [li % kBN] of its pieces' slots t ksplit .. t ksplit + ksplit - 1, with
+// 16-byte loads (and a 16-byte store when y's rows allow).
 __global__ void __launch_bounds__(256) prefill_reduce_kernel(const float* __restrict__ ypart, int ksplit,
-                                                             int64_t MN, int64_t N, Epilogue ep,
-                                                             float* __restrict__ y) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < MN;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float v = __ldcs(ypart + i);
-    for (int p = 1; p < ksplit; ++p) v += __ldcs(ypart + static_cast<int64_t>(p) * MN + i);
-    y[i] = ep.apply(v, static_cast<int>(i % N));
+                                                             int full, int num_n, int num_m, int bm,
+                                                             int M, int N, Epilogue ep, float* __restrict__ y) {
+  const int t = blockIdx.y;
+  int n0, m0;
+  tile_origin(full + t, num_n, num_m, bm, n0, m0);
+  const int per_tile = kBN * bm;
+  const int li = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (li >= per_tile) return;
+  const int m = m0 + (li >> 7), n = n0 + (li & (kBN - 1));
+  if (m >= M || n >= N) return;
+  const float4* p = reinterpret_cast<const float4*>(ypart + static_cast<int64_t>(t) * ksplit * per_tile + li);
+  float4 v = __ldcs(p);
+  for (int q = 1; q < ksplit; ++q) {
+    const float4 u = __ldcs(p + static_cast<int64_t>(q) * (per_tile / 4));
+    v.x += u.x;
+    v.y += u.y;
+    v.z += u.z;
+    v.w += u.w;
+  }
+  float* yr = y + static_cast<int64_t>(m) * N + n;
+  if (n + 3 < N && N % 4 == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0) {
+    *reinterpret_cast<float4*>(yr) = make_float4(ep.apply(v.x, n), ep.apply(v.y, n + 1), ep.apply(v.z, n + 2),
+                                                 ep.apply(v.w, n + 3));
+  } else {
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 4 && n + i < N; ++i) yr[i] = ep.apply(vv[i], n + i);
   }
 }
+static_assert(kBN == 128, "the adding kernel splits a slot index by shifts");
 
+#ifndef INT4_PREFILL_TAIL_SPLIT
+#define INT4_PREFILL_TAIL_SPLIT 1  // cut the tiles of a last partial wave into K pieces
+#endif
 #ifndef INT4_PREFILL_SMALL_BM
 #define INT4_PREFILL_SMALL_BM 1  // 128-row activation tiles for problems of less than one wave
 #endif
@@ -599,17 +647,21 @@ int choose_bm(int64_t M, int64_t N) {
   return (INT4_PREFILL_SMALL_BM && t256 < sms && t128 <= sms) ? 128 : 256;
 }
 
-// How many K pieces to cut each tile into.  With fewer tiles than SMs the
-// machine idles; more pieces fill it, at the price of writing and re-reading
-// the pieces' fp32 sums.  The estimate (calibrated on B200): waves of units
-// times a unit's time -- its share of the tile's stages at about 0.6 us per
-// 64-k stage of a 128 x 256 tile (half that at 128 rows), about 3 us to
-// start and finish a unit, and its store of a tile of fp32 sums at about
-// 16 GB/s per SM -- plus, when split, the partial sums' round trip through
-// HBM and about 1 us for the adding kernel.
+// How to cut the work: whole tiles, except that the tiles of a last,
+// partial wave (all of them when there are fewer tiles than SMs) may be cut
+// into ksplit K pieces, so that the pieces fill that wave.  Pieces write and
+// re-read their fp32 sums and need the adding kernel.  The estimate
+// (calibrated on B200): a unit costs its share of the tile's stages at about
+// 0.6 us per 64-k stage of a 128 x 256 tile (half that at 128 rows), about
+// 3 us to start and finish, and its store of a tile of fp32 sums at about
+// 16 GB/s per SM; whole waves come first, then one wave of the tail's
+// units, then the pieces' round trip through HBM and about 1 us for the
+// adding kernel.
 struct SplitPlan {
   int ksplit = 1;
-  int spc = 1;  // stages per chunk: a common multiple of the group and the 64-k stage
+  int full = 0;   // leading whole-tile units
+  int ntail = 0;  // tiles cut into pieces
+  int spc = 1;    // stages per chunk: a common multiple of the group and the 64-k stage
 };
 SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N, int bm) {
   SplitPlan p;
@@ -619,21 +671,32 @@ SplitPlan plan_split(int64_t K, int group, int64_t M, int64_t N, int bm) {
   const int64_t nchunks = (nstages + p.spc - 1) / p.spc;
   const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + bm - 1) / bm);
   const int64_t sms = num_sms();
-  if (tiles >= sms || nchunks < 2) return p;
+  const int64_t waves = tiles / sms;
+  const int64_t tail = tiles - waves * sms;
+  if (tail == 0 || nchunks < 2 || !INT4_PREFILL_TAIL_SPLIT && waves > 0) return p;
   const double stage_us = 0.6 * bm / 256.0, unit_us = 3.0, reduce_us = 1.0, hbm_bytes_per_us = 6.0e6;
   const double store_us = static_cast<double>(kBN) * bm * 4 / 16.0e3;
   const double tile_us = static_cast<double>(nstages) * stage_us;
-  double best = 0.0;
-  for (int64_t k = 1; k <= 8 && k <= nchunks; ++k) {
-    const double waves = static_cast<double>((tiles * k + sms - 1) / sms);
-    const double t = waves * (tile_us / static_cast<double>(k) + unit_us + store_us) +
-                     (k > 1 ? static_cast<double>(k) * M * N * 8 / hbm_bytes_per_us + reduce_us : 0.0);
-    if (k == 1 || t < best) {
+  const double whole = tile_us + unit_us + store_us;
+  const double tile_bytes = static_cast<double>(kBN) * bm * 4;
+  double best = whole;  // k = 1: the tail as one more wave of whole tiles
+  for (int64_t k = 2; k <= 8 && k <= nchunks && tail * k <= sms; ++k) {
+    const double t = tile_us / static_cast<double>(k) + unit_us + store_us +
+                     static_cast<double>(tail * k) * tile_bytes * 2 / hbm_bytes_per_us + reduce_us;
+    if (t < best) {
       best = t;
       p.ksplit = static_cast<int>(k);
     }
   }
+  if (p.ksplit > 1) {
+    p.full = static_cast<int>(waves * sms);
+    p.ntail = static_cast<int>(tail);
+  }
   return p;
+}
+
+size_t split_bytes(const SplitPlan& sp, int bm) {
+  return sp.ksplit > 1 ? static_cast<size_t>(sp.ntail) * sp.ksplit * kBN * bm * sizeof(float) : 0;
 }
 
 template <typename TX, bool ASYM, int BM>
@@ -677,28 +740,32 @@ cudaError_t launch_typed(const TX* x, const uint8_t* packed, const uint16_t* sca
   // Split K only when the caller's workspace holds the pieces' sums (past
   // the counters a decode call keeps at its start).
   SplitPlan sp = plan_split(K, group, M, N, BM);
-  const size_t part_bytes = static_cast<size_t>(sp.ksplit) * M * N * sizeof(float);
+  const size_t part_bytes = split_bytes(sp, BM);
+  // The pieces' buffer takes 16-byte loads and stores: a workspace too small
+  // or not 16-byte aligned runs the tiles whole.
   if (sp.ksplit > 1 &&
-      (workspace == nullptr || workspace_bytes < kWorkspaceCounterBytes + part_bytes))
-    sp.ksplit = 1;
+      (workspace == nullptr || workspace_bytes < kWorkspaceCounterBytes + part_bytes ||
+       (reinterpret_cast<uintptr_t>(workspace) & 15) != 0))
+    sp = SplitPlan{};
   float* ypart = sp.ksplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                           kWorkspaceCounterBytes)
                                : nullptr;
-  const int64_t units = ((N + kBN - 1) / kBN) * ((M + BM - 1) / BM) * sp.ksplit;
+  const int64_t num_tiles = ((N + kBN - 1) / kBN) * ((M + BM - 1) / BM);
+  const int64_t units = sp.full + (num_tiles - sp.full) * sp.ksplit;
   const int64_t sms = num_sms();
   const int64_t ctas = INT4_PREFILL_PERSISTENT ? (units < sms ? units : sms) : units;
   const dim3 grid(static_cast<unsigned>(ctas));  // persistent: one CTA per SM
   const int G = static_cast<int>((K + group - 1) / group);
   kern<<<grid, kThreads, L::kAlloc, stream>>>(tx, tp, scales, zeros, ep, y, static_cast<int>(M),
                                               static_cast<int>(N), static_cast<int>(K), group, G,
-                                              sp.ksplit, sp.spc, ypart, status);
+                                              sp.full, sp.ksplit, sp.spc, ypart, status);
   e = cudaGetLastError();
   if (e != cudaSuccess || ypart == nullptr) return e;
-  const int64_t MN = M * N;
-  int64_t blocks = (MN + 255) / 256;
-  if (blocks > 8 * sms) blocks = 8 * sms;
-  prefill_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(ypart, sp.ksplit, MN, N,
-                                                                         ep, y);
+  // One thread per four elements of each tail tile.
+  const int64_t bx = (static_cast<int64_t>(kBN) * BM / 4 + 255) / 256;
+  prefill_reduce_kernel<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(sp.ntail)), 256, 0, stream>>>(
+      ypart, sp.ksplit, sp.full, static_cast<int>((N + kBN - 1) / kBN),
+      static_cast<int>((M + BM - 1) / BM), BM, static_cast<int>(M), static_cast<int>(N), ep, y);
   return cudaGetLastError();
 }
 
@@ -745,9 +812,9 @@ cudaError_t launch_matmul_prefill(const void* x, DType xt, const uint8_t* packed
 }
 
 size_t prefill_workspace_size(int64_t K, int group, int64_t M, int64_t N) {
-  const SplitPlan sp = plan_split(K, group, M, N, choose_bm(M, N));
-  return sp.ksplit > 1 ? kWorkspaceCounterBytes + static_cast<size_t>(sp.ksplit) * M * N * sizeof(float)
-                       : 0;
+  const int bm = choose_bm(M, N);
+  const SplitPlan sp = plan_split(K, group, M, N, bm);
+  return sp.ksplit > 1 ? kWorkspaceCounterBytes + split_bytes(sp, bm) : 0;
 }
 
 }  // namespace int4lib

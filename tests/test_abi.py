@@ -127,11 +127,11 @@ def test_workspace_size_rejects_bad_arguments(L):
         assert q(*args, ctypes.byref(out)) == q4.OK
         assert out.value == 0
     # The tensor-core kernel with fewer tiles (64) than SMs splits K into
-    # pieces whose fp32 sums live in the workspace, past 4 KB of counters
-    # (148 SMs assumed without a device).
+    # pieces whose fp32 sums live in the workspace, past 4 KB of counters,
+    # one 128-row tile slot each (148 SMs assumed without a device).
     out.value = 0
     assert q(1, 4096, 128, 64, 8192, ctypes.byref(out)) == q4.OK
-    assert out.value > 4096 and (out.value - 4096) % (64 * 8192 * 4) == 0
+    assert out.value > 4096 and (out.value - 4096) % (128 * 128 * 4) == 0
 
 
 def test_noalloc_rejects_what_the_decode_kernels_cannot_run(L):
