@@ -193,10 +193,11 @@ int int4_matmul_workspace_size(int32_t x_dtype, int64_t K, int32_t group, int64_
  *   - workspace_bytes must be at least int4_matmul_workspace_size(...) for
  *     this problem, else INT4_ERR_ARG (nothing launched).  workspace == NULL
  *     with workspace_bytes == 0 selects the schedule of int4_matmul.  On the
- *     tensor-core path (M > 16) the workspace is optional: when the matrix
- *     has fewer 128 x 256 tiles than the device has SMs, a workspace of the
- *     queried size lets the call split K into pieces whose fp32 sums a second
- *     kernel adds in piece order; a smaller or NULL one runs it unsplit.
+ *     tensor-core path (M > 16) the workspace is optional: when the last
+ *     wave of the matrix's tiles (128 weight rows x 128 or 256 batch rows)
+ *     leaves SMs idle, a workspace of the queried size lets the call split
+ *     the K of that wave's tiles into pieces whose fp32 sums a second kernel
+ *     adds in piece order; a smaller or NULL one runs every tile whole.
  *   - workspace must be 256-byte aligned (INT4_ERR_ALIGN) and zero-filled
  *     before its first use; every call leaves its counters zero again, so a
  *     workspace can serve any number of calls, of any shape, that are
