@@ -1915,7 +1915,9 @@ int flat_choice_g(int64_t K, int G, int m, int64_t tiles) {
   // Four warps with a group per word at M > 8 spill, and lose to the
   // pipelined 16-bit kernel (W [11008, 4096], group 32, M = 16: 25.3
   // against 22.2 us).
-  if (GPB == 1 && flat_fits<TX, 2, ASYM, 4, false, GPB>(K, G, m, tiles)) return 4;
+  if constexpr (GPB == 1) {
+    if (flat_fits<TX, 2, ASYM, 4, false, GPB>(K, G, m, tiles)) return 4;
+  }
   return 0;
 }
 
@@ -1972,8 +1974,12 @@ cudaError_t launch_flat_g(int choice, const TX* x, const uint8_t* packed, const 
     return xs ? launch_flat_w<TX, 1, ASYM, 4, true, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
               : launch_flat_w<TX, 1, ASYM, 4, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
   }
-  return w == 8 ? launch_flat_w<TX, 2, ASYM, 8, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream)
-                : launch_flat_w<TX, 2, ASYM, 4, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  if constexpr (GPB == 1) {
+    if (w == 4)
+      return launch_flat_w<TX, 2, ASYM, 4, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
+  }
+  // (flat_choice picks 4 warps at M > 8 only for groups of whole blocks.)
+  return launch_flat_w<TX, 2, ASYM, 8, false, GPB>(x, packed, scales, zeros, ep, K, group, M, N, y, stream);
 }
 
 // `choice`: flat_choice's value (warps, staged x, groups per block in bits 12+).

@@ -131,6 +131,8 @@ def test_prefill_full_size_whole_rows_and_columns(layer, M):
     (1024, 768, 3072, 32, torch.float16),      # distilgpt2 mlp c_proj shape, groups of 32
     (100, 1000, 2016, 96, torch.bfloat16),     # group 96: pieces of 3 stages, ragged M and N
     (256, 11008, 4096, 128, torch.bfloat16),   # 86 tiles: the estimate keeps it whole
+    (768, 8192, 4096, 128, torch.bfloat16),    # 192 tiles: one whole wave, the other 44 in 3 pieces
+    (700, 9000, 2048, 64, torch.float16),      # ragged tail tiles, groups of 64
 ])
 def test_prefill_split_k_matches_oracle_and_unsplit(M, N, K, group, dtype):
     """With fewer tiles than SMs the binding's workspace lets the kernel cut
