@@ -55,10 +55,10 @@ DECODE_COPIES = 32
 # sha256 of that source file and is reported as null once the file changes.
 KERNEL_TRAFFIC = {
     # kernel: (bytes per launch, source file, sha256 of the source at capture)
-    "prefill": (800_810_000 + 914_920_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
-                "0d6f1de68f76b812ae1475511b89a474c3ce318f1651bc9c59608d8ee88b4676"),
-    "decode": (125_580_000 + 3_180_000, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
-               "e28aa1d3674484c09f95b0767df4ac65107bdbeaf0ceb162fa53682441f965cf"),
+    "prefill": (812_040_000 + 919_400_000, "dequant_gemm_int4_b200/csrc/matmul_prefill.cu",
+                "fb5b9e91a3e50e847a3e16ee33705d4b1cf935874397d6e856b9fded9b268250"),
+    "decode": (125_570_000 + 3_240_000, "dequant_gemm_int4_b200/csrc/matmul_decode.cu",
+               "7a09f42f7ba224b046786c6639e561bd7ffffb659138712f3b01fa51b6273e55"),
     "quantize": (469_856_256 + 104_254_208, "dequant_gemm_int4_b200/csrc/quantize.cu",
                  "24a51fde9c6ea1afd8a159345f565f16441d8a085e241e8e6d8d123c71573f57"),
     "unpack": (117_450_000 + 180_200_000, "dequant_gemm_int4_b200/csrc/unpack.cu",
