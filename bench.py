@@ -124,10 +124,17 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return self
+        # nvidia-smi can take a second to start on a fresh box: wait for its
+        # first sample (or at most 3 s, in case it buffers its output), so
+        # that a short timed region is still sampled.
+        deadline = time.time() + 3.0
+        while self.proc.poll() is None and time.time() < deadline and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
@@ -759,7 +766,6 @@ def run_ours(args):
     # The clock sampler runs from the first warm-up step to the end of the timed
     # steps (the GPU is busy throughout), so short timed regions still get samples.
     with ClockSampler(local) as clk:
-        time.sleep(0.3)  # let nvidia-smi start polling
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
@@ -845,32 +851,67 @@ def run_ours(args):
     if not args.no_variants and not args.only and w is not None:
         variants = variant_rows(dev, w, xd, xp, flush_l2, peaks)
 
-    # End to end through the public Python API: pinned host x in, y out.
+    # End to end through the public Python API, one step of the decode row:
+    # pinned host x in, the DECODE_COPIES layer calls launched from Python
+    # (no graph), every layer's y back to pinned host memory.  Each y is read
+    # back on a copy stream as soon as its call ends, so the reads overlap
+    # the next layers; the step ends when the last read has landed.  A single
+    # call per step (x in, one call, y out) is reported beside it.
     e2e = None
     if not args.no_e2e and not args.only:
         import dequant_gemm_int4_b200 as api
+        layers = [(packed, scales)] + dcopies
         xh = xd.cpu().pin_memory()
-        yh = torch.empty((M_DECODE, N_W), dtype=torch.float32).pin_memory()
-        for _ in range(args.warmup):
+        yh = torch.empty((len(layers), M_DECODE, N_W), dtype=torch.float32).pin_memory()
+        ydev = torch.empty((len(layers), M_DECODE, N_W), dtype=torch.float32, device=dev)
+        copy_stream = torch.cuda.Stream(dev)
+        done = [torch.cuda.Event() for _ in layers]
+
+        def e2e_step():
+            xdev = xh.to(dev, non_blocking=True)
+            for i, (pk, sc) in enumerate(layers):
+                api.int4_matmul(xdev, pk, sc, K_W, GROUP, out=ydev[i])
+                done[i].record(stream)
+                copy_stream.wait_event(done[i])
+                with torch.cuda.stream(copy_stream):
+                    yh[i].copy_(ydev[i], non_blocking=True)
+            stream.wait_stream(copy_stream)
+
+        def single_step():
             y = api.int4_matmul(xh.to(dev, non_blocking=True), packed, scales, K_W, GROUP)
-            yh.copy_(y, non_blocking=True)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        tot = 0.0
-        for _ in range(args.steps):
-            flush_l2()
-            e0.record(stream)
-            y = api.int4_matmul(xh.to(dev, non_blocking=True), packed, scales, K_W, GROUP)
-            yh.copy_(y, non_blocking=True)
-            e1.record(stream)
+            yh[0].copy_(y, non_blocking=True)
+
+        def time_e2e(fn):
+            for _ in range(args.warmup):
+                fn()
             torch.cuda.synchronize()
-            tot += e0.elapsed_time(e1)
-        t = _max_over_ranks(tot / args.steps, world) * 1e-3
-        e2e = {"value": units["decode"]["bytes"] / t / 1e9 * world, "unit": "GB/s",
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            tot = 0.0
+            for _ in range(args.steps):
+                flush_l2()
+                torch.cuda.synchronize()
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1)
+            return _max_over_ranks(tot / args.steps, world) * 1e-3
+
+        t = time_e2e(e2e_step)
+        t1 = time_e2e(single_step)
+        ybytes = M_DECODE * N_W * 4
+        e2e = {"value": units["decode"]["bytes"] * len(layers) / t / 1e9 * world, "unit": "GB/s",
                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-               "d2h_bytes_per_step": yh.numel() * yh.element_size(),
-               "scope": "decode row via the Python API: H2D of x, int4_matmul, D2H of y"}
+               "d2h_bytes_per_step": ybytes * len(layers),
+               "ms_per_step": t * 1e3, "calls_per_step": len(layers),
+               "scope": ("decode row via the Python API: H2D of x, then int4_matmul over the "
+                         f"{len(layers)} weight copies launched from Python, each y read back "
+                         "to pinned host memory on a copy stream"),
+               "single_call": {"value": units["decode"]["bytes"] / t1 / 1e9 * world, "ms": t1 * 1e3,
+                               "h2d_bytes": xh.numel() * xh.element_size(), "d2h_bytes": ybytes,
+                               "scope": "H2D of x, one int4_matmul call, D2H of its y"}}
+        del ydev
 
     if rank != 0:
         if world > 1:
