@@ -47,6 +47,8 @@ WORKLOAD = ("W[28672,8192] bf16 g128: quantize+unpack, decode M=1 (32 calls back
 # then close to the steady state of a decode loop, with the start of the
 # first call and the end of the last spread over 32 calls.
 DECODE_COPIES = 32
+# Layers per read-back of y in the end-to-end step.
+E2E_READBACK = 8
 
 
 # DRAM traffic per launch of each kernel (dram__bytes_read.sum +
@@ -853,10 +855,12 @@ def run_ours(args):
 
     # End to end through the public Python API, one step of the decode row:
     # pinned host x in, the DECODE_COPIES layer calls launched from Python
-    # (no graph), every layer's y back to pinned host memory.  Each y is read
-    # back on a copy stream as soon as its call ends, so the reads overlap
-    # the next layers; the step ends when the last read has landed.  A single
-    # call per step (x in, one call, y out) is reported beside it.
+    # (no graph), every layer's y back to pinned host memory.  The ys are
+    # read back on a copy stream, E2E_READBACK layers at a time as soon as
+    # those calls end, so the reads overlap the next layers (an event between
+    # two calls would also stop the second from starting early, so they come
+    # only every few layers); the step ends when the last read has landed.  A
+    # single call per step (x in, one call, y out) is reported beside it.
     e2e = None
     if not args.no_e2e and not args.only:
         import dequant_gemm_int4_b200 as api
@@ -865,16 +869,18 @@ def run_ours(args):
         yh = torch.empty((len(layers), M_DECODE, N_W), dtype=torch.float32).pin_memory()
         ydev = torch.empty((len(layers), M_DECODE, N_W), dtype=torch.float32, device=dev)
         copy_stream = torch.cuda.Stream(dev)
-        done = [torch.cuda.Event() for _ in layers]
+        batches = [(b, min(b + E2E_READBACK, len(layers))) for b in range(0, len(layers), E2E_READBACK)]
+        done = [torch.cuda.Event() for _ in batches]
 
         def e2e_step():
             xdev = xh.to(dev, non_blocking=True)
-            for i, (pk, sc) in enumerate(layers):
-                api.int4_matmul(xdev, pk, sc, K_W, GROUP, out=ydev[i])
-                done[i].record(stream)
-                copy_stream.wait_event(done[i])
+            for (b0, b1), ev in zip(batches, done):
+                for i in range(b0, b1):
+                    api.int4_matmul(xdev, layers[i][0], layers[i][1], K_W, GROUP, out=ydev[i])
+                ev.record(stream)
+                copy_stream.wait_event(ev)
                 with torch.cuda.stream(copy_stream):
-                    yh[i].copy_(ydev[i], non_blocking=True)
+                    yh[b0:b1].copy_(ydev[b0:b1], non_blocking=True)
             stream.wait_stream(copy_stream)
 
         def single_step():
@@ -906,8 +912,8 @@ def run_ours(args):
                "d2h_bytes_per_step": ybytes * len(layers),
                "ms_per_step": t * 1e3, "calls_per_step": len(layers),
                "scope": ("decode row via the Python API: H2D of x, then int4_matmul over the "
-                         f"{len(layers)} weight copies launched from Python, each y read back "
-                         "to pinned host memory on a copy stream"),
+                         f"{len(layers)} weight copies launched from Python, every y read back "
+                         f"to pinned host memory on a copy stream, {E2E_READBACK} layers at a time"),
                "single_call": {"value": units["decode"]["bytes"] / t1 / 1e9 * world, "ms": t1 * 1e3,
                                "h2d_bytes": xh.numel() * xh.element_size(), "d2h_bytes": ybytes,
                                "scope": "H2D of x, one int4_matmul call, D2H of its y"}}
