@@ -12,11 +12,13 @@
 // A zero scale (a constant group, or a range that underflows fp16) codes the
 // group as q = 0, z = 0.
 //
-// HBM-bound like the symmetric quantizer: a warp takes a window of 256
-// consecutive weights of one row (8 per lane, one 16- or 32-byte load),
-// reduces the group's min and max with shuffles over its group / 8 lanes and
-// stores 4 packed bytes per lane; any other shape takes a two-kernel general
-// path (scales and zero points, then one thread per packed byte).
+// HBM-bound like the symmetric quantizer: a warp takes a window of 512
+// consecutive weights of one row (16 per lane, two 16- or 32-byte loads),
+// reduces the group's min and max with shuffles over its group / 16 lanes,
+// codes the weights two per instruction (float2 arithmetic) and stores 8
+// packed bytes per lane.  Groups of 8 take windows of 256 (8 per lane); any
+// other shape takes a two-kernel general path (scales and zero points, then
+// one thread per packed byte).
 #include "common.cuh"
 #include "internal.h"
 
@@ -137,6 +139,29 @@ __device__ __forceinline__ uint32_t affine_code_fast(float v, const Affine& a) {
   return __float_as_uint(__fadd_rn(uc, 12582912.0f)) & 0xFu;
 }
 
+// affine_code_fast on 16 weights, two per float2 instruction (each component
+// rounds as the scalar operation does): element 2j in the low nibble of
+// byte j, bytes 0..3 in .x and 4..7 in .y.
+__device__ __forceinline__ uint2 affine_codes16_fast(const float (&v)[16], const Affine& a) {
+  const float2 r2 = make_float2(a.r, a.r);
+  const float2 ns2 = make_float2(-a.sf, -a.sf);
+  const float2 z2 = make_float2(a.zf, a.zf);
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  uint32_t word[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 x = make_float2(v[2 * i], v[2 * i + 1]);
+    const float2 q = __fmul2_rn(x, r2);
+    const float2 e = __ffma2_rn(q, ns2, x);  // x - q sf, exact
+    const float2 u = __fadd2_rn(__ffma2_rn(e, r2, q), z2);
+    const float2 uc = make_float2(fminf(fmaxf(u.x, 0.0f), 15.0f), fminf(fmaxf(u.y, 0.0f), 15.0f));
+    const float2 t = __fadd2_rn(uc, magic);
+    const uint32_t byte = (__float_as_uint(t.x) & 0xFu) | ((__float_as_uint(t.y) & 0xFu) << 4);
+    word[i >> 2] |= byte << (8 * (i & 3));
+  }
+  return make_uint2(word[0], word[1]);
+}
+
 // Fast path: K % 8 == 0, group = 8 LPG with LPG a power of two <= 32, w
 // 16-byte aligned, packed 4-byte aligned.  Windows (256 weights of one row)
 // are numbered row-major; each warp takes a contiguous range of them.
@@ -214,6 +239,98 @@ __global__ void __launch_bounds__(256) quantize_affine_window_kernel(
   }
 }
 
+// Wide fast path: K % 16 == 0, group = 16 LPG with LPG a power of two <= 32,
+// w 16-byte aligned, packed 8-byte aligned.  Windows (512 weights of one
+// row, 16 per lane) are numbered row-major; each warp takes a contiguous
+// range of them.  Lanes past the row's end (K not a multiple of 512) take
+// part in the shuffles with neutral extremes and store nothing.
+template <typename T, int LPG>
+__global__ void __launch_bounds__(256) quantize_affine_wide_kernel(
+    const T* __restrict__ w, int64_t K, int G, int64_t windows_per_row, int64_t total_windows,
+    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales, uint8_t* __restrict__ zeros) {
+  constexpr int kGroup = 16 * LPG;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t per = (total_windows + nwarps - 1) / nwarps;
+  const int64_t wbeg = warp * per;
+  const int64_t wend = (wbeg + per < total_windows) ? wbeg + per : total_windows;
+  if (wbeg >= wend) return;
+  int64_t row = wbeg / windows_per_row;
+  int64_t win = wbeg - row * windows_per_row;
+  // The next window's weights are loaded while this one is coded.
+  auto load_window = [&](int64_t r, int64_t wn, float (&dst)[16]) {
+    const int64_t k = wn * 512 + 16 * lane;
+    if (k < K) {
+      float lo[8], hi[8];
+      load8<T>(w + r * K + k, lo);
+      load8<T>(w + r * K + k + 8, hi);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        dst[i] = lo[i];
+        dst[8 + i] = hi[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[i] = 0.0f;
+    }
+  };
+  float vnext[16];
+  load_window(row, win, vnext);
+  for (int64_t wi = wbeg; wi < wend; ++wi) {
+    const int64_t k0 = win * 512 + 16 * lane;
+    const bool active = k0 < K;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = vnext[i];
+    if (wi + 1 < wend) {
+      const bool wrap = win + 1 == windows_per_row;
+      load_window(wrap ? row + 1 : row, wrap ? 0 : win + 1, vnext);
+    }
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      mn = fminf(mn, v[i]);
+      mx = fmaxf(mx, v[i]);
+    }
+    if (!active) {
+      mn = __int_as_float(0x7F800000);  // +inf
+      mx = __int_as_float(0xFF800000);  // -inf
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (active) {
+      const Affine a = affine_params(mn, mx);
+      const bool fast = a.sf != 0.0f && a.r != 0.0f &&
+                        __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), a.r) < 0x1p99f;
+      uint2 word;
+      if (fast) {
+        word = affine_codes16_fast(v, a);
+      } else {
+        word = make_uint2(0u, 0u);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          word.x |= affine_code(v[i], a) << (4 * i);
+          word.y |= affine_code(v[8 + i], a) << (4 * i);
+        }
+      }
+      *reinterpret_cast<uint2*>(packed + row * (K >> 1) + (k0 >> 1)) = word;
+      if ((lane & (LPG - 1)) == 0) {
+        const int64_t gi = row * G + k0 / kGroup;
+        scales[gi] = static_cast<uint16_t>(a.bits);
+        zeros[gi] = static_cast<uint8_t>(a.z);
+      }
+    }
+    if (++win == windows_per_row) {
+      win = 0;
+      ++row;
+    }
+  }
+}
+
 // General path, step 1: one thread per (row, group).
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_affine_params_kernel(
@@ -272,10 +389,34 @@ cudaError_t launch_window(const T* w, int64_t N, int64_t K, int G, uint8_t* pack
   return cudaGetLastError();
 }
 
+template <typename T, int LPG>
+cudaError_t launch_wide(const T* w, int64_t N, int64_t K, int G, uint8_t* packed,
+                        uint16_t* scales, uint8_t* zeros, cudaStream_t stream) {
+  const int64_t wpr = (K + 511) / 512;
+  const int64_t total = N * wpr;
+  const int grid = resident_grid(quantize_affine_wide_kernel<T, LPG>, (total + 7) / 8);
+  quantize_affine_wide_kernel<T, LPG><<<grid, 256, 0, stream>>>(w, K, G, wpr, total, packed,
+                                                                scales, zeros);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_typed(const T* w, int64_t N, int64_t K, int group, uint8_t* packed,
                          uint16_t* scales, uint8_t* zeros, cudaStream_t stream) {
   const int G = static_cast<int>((K + group - 1) / group);
+  const bool wide = K % 16 == 0 && reinterpret_cast<uintptr_t>(w) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(packed) % 8 == 0;
+  if (wide) {
+    switch (group) {
+      case 16: return launch_wide<T, 1>(w, N, K, G, packed, scales, zeros, stream);
+      case 32: return launch_wide<T, 2>(w, N, K, G, packed, scales, zeros, stream);
+      case 64: return launch_wide<T, 4>(w, N, K, G, packed, scales, zeros, stream);
+      case 128: return launch_wide<T, 8>(w, N, K, G, packed, scales, zeros, stream);
+      case 256: return launch_wide<T, 16>(w, N, K, G, packed, scales, zeros, stream);
+      case 512: return launch_wide<T, 32>(w, N, K, G, packed, scales, zeros, stream);
+      default: break;
+    }
+  }
   const bool fast = K % 8 == 0 && reinterpret_cast<uintptr_t>(w) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(packed) % 4 == 0;
   if (fast) {

@@ -66,6 +66,9 @@ def _oracle_affine(w, group):
 @pytest.mark.parametrize("N, K, group", [
     (16, 1024, 128), (40, 4096, 64), (33, 768, 32), (8, 512, 8), (5, 2048, 256), (7, 256, 16),
     (9, 259, 128), (6, 1001, 100), (3, 96, 48), (2, 5, 2), (1, 1, 1),
+    # 16 weights per lane: a partial last group (K % group = 16) and a
+    # partial last window; group 512 (32 lanes per group)
+    (10, 1040, 128), (4, 4112, 512), (3, 1552, 64),
 ])
 def test_quantize_affine_bit_exact(dtype, N, K, group):
     w = _special_affine_weights(N, K, group, seed=N * K + group, dtype=dtype)
@@ -75,6 +78,24 @@ def test_quantize_affine_bit_exact(dtype, N, K, group):
     assert np.array_equal(scales.cpu().view(torch.int16).numpy().view(np.uint16), s_ref.view(np.uint16))
     assert np.array_equal(zeros.cpu().numpy(), z_ref)
     assert np.array_equal(packed.cpu().numpy(), p_ref)
+
+
+@pytest.mark.parametrize("group", [32, 128])
+def test_quantize_affine_full_size_sampled_rows(group):
+    """W [28672, 8192] bf16 (the bench's matrix): 512 rows spread over the
+    matrix, bit-exact against the oracle on those rows (quantization is per
+    row)."""
+    N, K = 28672, 8192
+    w = make_weights(N, K, seed=11, device=DEV, dtype=torch.bfloat16, dist="student_t3",
+                     zero_group_frac=0.01, group=group)
+    packed, scales, zeros, _ = q4.quantize_int4_affine(w, group)
+    rows = np.linspace(0, N - 1, 512).astype(np.int64)
+    idx = torch.as_tensor(rows, device=DEV)
+    p_ref, s_ref, z_ref, _ = _oracle_affine(w.index_select(0, idx), group)
+    assert np.array_equal(scales.index_select(0, idx).cpu().view(torch.int16).numpy().view(np.uint16),
+                          s_ref.view(np.uint16))
+    assert np.array_equal(zeros.index_select(0, idx).cpu().numpy(), z_ref)
+    assert np.array_equal(packed.index_select(0, idx).cpu().numpy(), p_ref)
 
 
 def _tie_weights(N, K, group, seed):
