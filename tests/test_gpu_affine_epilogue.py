@@ -222,6 +222,8 @@ PATHS = [
     (300, 384, 2048, 64, q4.PATH_PREFILL, None),
     (300, 384, 2048, 64, q4.PATH_PREFILL, False),    # tensor-core kernel, whole K
     (1024, 768, 3072, 32, q4.PATH_PREFILL, None),    # groups of 32, K split
+    (16, 3000, 2048, 64, q4.PATH_PREFILL, None),     # tensor-core kernel at M <= 32
+    (5, 1000, 1024, 128, q4.PATH_PREFILL, False),    # the same, whole K
     (7, 100, 259, 128, q4.PATH_SIMT, None),          # CUDA-core kernel (odd K)
 ]
 

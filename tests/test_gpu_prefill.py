@@ -152,6 +152,34 @@ def test_prefill_split_k_matches_oracle_and_unsplit(M, N, K, group, dtype):
         assert torch.equal(y_split, y_plain)
 
 
+@pytest.mark.parametrize("M, N, K, group, dtype", [
+    (1, 4096, 4096, 128, torch.bfloat16),
+    (5, 11008, 4096, 128, torch.float16),
+    (16, 4096, 11008, 128, torch.bfloat16),
+    (16, 768, 3072, 32, torch.float16),        # groups of 32: two per stage
+    (32, 2304, 768, 64, torch.bfloat16),
+    (9, 1000, 2016, 96, torch.bfloat16),       # ragged N, groups spanning stages
+    (16, 300, 96, 32, torch.float16),          # K of one and a half stages
+    (24, 28672, 1024, 128, torch.bfloat16),    # more tiles than SMs
+])
+def test_prefill_small_m(M, N, K, group, dtype):
+    """M <= 32 forced onto the tensor-core kernel (one activation tile, rows
+    past M zero-filled by the copies): with a workspace the tiles of a
+    partial wave may be cut into K pieces, added in piece order; without one
+    they run whole.  Both meet the bound and repeat bit for bit."""
+    packed, scales, _ = _quantized(N, K, group, 21, "student_t3", 0.05)
+    x = make_activations(M, K, seed=22, device=DEV, dtype=dtype)
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device=DEV)
+    y_split = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL, workspace=ws)
+    y_plain = q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL, workspace=False)
+    assert q4.device_status() == q4.OK
+    cols = None if N <= 2048 else np.unique(np.random.default_rng(N).integers(0, N, 500))
+    assert_matmul_close(y_split, x, packed, scales, K, group, TOL_HALF, cols=cols)
+    assert_matmul_close(y_plain, x, packed, scales, K, group, TOL_HALF, cols=cols)
+    assert torch.equal(y_split, q4.int4_matmul(x, packed, scales, K, group, path=q4.PATH_PREFILL,
+                                               workspace=ws))
+
+
 def test_prefill_split_workspace_query():
     """32 tiles on a device of 148 SMs: every tile is split.  7168 tiles: 48
     whole waves, and the 64 tiles of the partial last wave cut in two (one
