@@ -101,6 +101,7 @@ def _row_units():
     scales = 2 * N_W * G
     return {
         "quantize": {"bytes": N_W * K_W * 2 + packed + scales, "bound": "hbm"},
+        "quantize_affine": {"bytes": N_W * K_W * 2 + packed + scales + N_W * G, "bound": "hbm"},
         "unpack": {"bytes": packed + N_W * K_W, "bound": "hbm"},
         "decode": {"bytes": packed, "bytes_total": packed + scales + M_DECODE * K_W * 2 + 4 * M_DECODE * N_W,
                    "bound": "hbm"},
@@ -681,6 +682,8 @@ def run_ours(args):
         yp = torch.empty((M_PREFILL, N_W), dtype=torch.float32, device=dev)
     if "unpack" in order:
         unpacked = torch.empty((N_W, K_W), dtype=torch.int8, device=dev)
+    zeros_q = (torch.empty((N_W, K_W // GROUP), dtype=torch.uint8, device=dev)
+               if "quantize_affine" in order else None)
     # The decode matmul's workspace (zero-filled once; every call leaves it so).
     ws_bytes = q4.matmul_workspace_size(torch.bfloat16, K_W, GROUP, M_DECODE, N_W, dev)
     ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
@@ -709,6 +712,8 @@ def run_ours(args):
         "quantize": lambda: call(L.int4_quantize(w.data_ptr(), 1, N_W, K_W, GROUP, packed.data_ptr(),
                                                  scales.data_ptr(), sp())),
         "unpack": lambda: call(L.int4_unpack(packed.data_ptr(), K_W, N_W, unpacked.data_ptr(), sp())),
+        "quantize_affine": lambda: call(L.int4_quantize_affine(w.data_ptr(), 1, N_W, K_W, GROUP, packed.data_ptr(),
+                                                               scales.data_ptr(), zeros_q.data_ptr(), sp())),
         "decode": lambda: [call(L.int4_matmul_ws(xd.data_ptr(), 1, pk.data_ptr(), sc.data_ptr(), K_W,
                                                   GROUP, M_DECODE, N_W, yd.data_ptr(), ws.data_ptr(),
                                                   ws.numel(), sp()))
@@ -722,7 +727,7 @@ def run_ours(args):
     }
     for pc, sc in dcopies:
         call(L.int4_quantize(w.data_ptr(), 1, N_W, K_W, GROUP, pc.data_ptr(), sc.data_ptr(), sp()))
-    if args.only and args.only != "quantize":
+    if args.only and args.only not in ("quantize", "quantize_affine"):
         # The kernel reads packed weights: quantize them once, outside timing.
         kernels["quantize"]()
         torch.cuda.synchronize()
@@ -732,7 +737,7 @@ def run_ours(args):
     # across CTAs there too; the decode row makes DECODE_COPIES calls, and a
     # single call after it is timed on its own (decode_single).
     launches_per_step = {
-        "quantize": 1, "unpack": 1, "decode": DECODE_COPIES + 1,
+        "quantize": 1, "quantize_affine": 1, "unpack": 1, "decode": DECODE_COPIES + 1,
         # the tensor-core kernel, plus the adding kernel when it splits K
         "prefill": 2 if wsp_bytes > 0 else 1,
     }
@@ -966,8 +971,10 @@ def main():
                     help="skip the dequantize-then-GEMM comparison rows")
     ap.add_argument("--no-shapes", action="store_true",
                     help="skip the rows at the other configured shapes (Llama-7B decode, prefill, distilgpt2, bulk quantize, group-32/64 decode)")
-    ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill"], default=None,
-                    help="run one kernel of the step only (for profiling); no e2e or CPU baseline")
+    ap.add_argument("--only", choices=["quantize", "unpack", "decode", "prefill", "quantize_affine"],
+                    default=None,
+                    help="run one kernel of the step only (for profiling); no e2e or CPU baseline. "
+                         "quantize_affine is the asymmetric variant's quantizer on the same W")
     ap.add_argument("--shape", default=None, metavar="N,K,M",
                     help="with --only: a smaller weight matrix N x K (and prefill batch M) for "
                          "profiler captures that must stay a few GB on the device")
