@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (CPU): the algorithmic units behind every
 throughput it prints, the DRAM-traffic figures tied to the kernel sources
-they were captured on, and the decode row's inputs exceeding L2."""
+they were captured on, the decode row's inputs exceeding L2, and the
+reading of the clock record."""
 
 import hashlib
 import importlib.util
@@ -30,6 +31,8 @@ def test_row_units_are_the_closed_forms(bench):
     assert u["decode"]["bytes"] == packed == 117_440_512
     assert u["decode"]["bytes_total"] == packed + scales + 2 * K + 4 * N
     assert u["prefill"]["flops"] == 2 * Mp * N * K
+    # the affine quantizer also writes one uint8 zero point per (row, group)
+    assert u["quantize_affine"]["bytes"] == u["quantize"]["bytes"] + N * (K // g)
     assert {r["bound"] for r in u.values()} == {"hbm", "tensor"}
 
 
@@ -65,3 +68,35 @@ def test_peaks_fall_back_without_the_measured_file(bench, tmp_path, monkeypatch)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     p = bench._peaks()
     assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16_tflops"] == 1590.0
+
+
+def test_clock_summary_reads_the_samples(bench, tmp_path):
+    """The clock record of a run: the median SM clock of the samples taken
+    under load (idle samples below half the highest are left out), the
+    highest max clock, and every throttle reason seen active."""
+    rows = [
+        "0, 345, 1965, 120.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1965, 1965, 900.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 950.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, [N/A], 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join(rows) + "\n")
+    clk = bench.ClockSampler(0)
+    clk.proc, clk.path = object(), str(path)
+    s = clk.summary()
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 4
+    assert not path.exists()   # the record is removed once read
+
+
+def test_clock_summary_without_samples(bench, tmp_path):
+    path = tmp_path / "clocks.csv"
+    path.write_text("")
+    clk = bench.ClockSampler(0)
+    clk.proc, clk.path = object(), str(path)
+    assert clk.summary()["reasons"] == ["no samples"]
+    clk2 = bench.ClockSampler(0)
+    assert clk2.summary()["reasons"] == ["nvidia-smi unavailable"]
