@@ -862,10 +862,9 @@ def run_ours(args):
     # pinned host x in, the DECODE_COPIES layer calls launched from Python
     # (no graph), every layer's y back to pinned host memory.  The ys are
     # read back on a copy stream, E2E_READBACK layers at a time as soon as
-    # those calls end, so the reads overlap the next layers (an event between
-    # two calls would also stop the second from starting early, so they come
-    # only every few layers); the step ends when the last read has landed.  A
-    # single call per step (x in, one call, y out) is reported beside it.
+    # those calls end, so the reads overlap the next layers; the step ends
+    # when the last read has landed.  A single call per step (x in, one call,
+    # y out) is reported beside it.
     e2e = None
     if not args.no_e2e and not args.only:
         import dequant_gemm_int4_b200 as api

@@ -12,13 +12,15 @@
 // A zero scale (a constant group, or a range that underflows fp16) codes the
 // group as q = 0, z = 0.
 //
-// HBM-bound like the symmetric quantizer: a warp takes a window of 512
+// A warp takes a window of 512
 // consecutive weights of one row (16 per lane, two 16- or 32-byte loads),
 // reduces the group's min and max with shuffles over its group / 16 lanes,
 // codes the weights two per instruction (float2 arithmetic) and stores 8
-// packed bytes per lane.  Groups of 8 take windows of 256 (8 per lane); any
-// other shape takes a two-kernel general path (scales and zero points, then
-// one thread per packed byte).
+// packed bytes per lane.  It reads w once but runs at about half of HBM
+// bandwidth: the ALU pipe (the clamp and the min/max of every weight) bounds
+// it.  Groups of 8 take windows of 256 (8 per lane); any other shape takes a
+// two-kernel general path (scales and zero points, then one thread per
+// packed byte).
 #include "common.cuh"
 #include "internal.h"
 
